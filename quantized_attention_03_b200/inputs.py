@@ -1,0 +1,122 @@
+"""Seeded synthetic workloads (shared by the tests, the benchmark and the CPU oracle).
+
+This module holds none of the method's arithmetic: it only draws random fp16 inputs of
+the shapes and value distributions of the method's target workloads (LLM prefill,
+video-DiT attention with channel outliers in K, long-sequence sweeps, packed varlen).
+
+Recipe (all draws on the CPU from ``torch.Generator().manual_seed(seed)``, in this order):
+
+1. (varlen only) the sequence lengths, ``randint(lo, hi + 1)`` each;
+2. Q, K, V as fp32 standard normals in the layout's shape;
+3. the K channel offset: one length-d vector added to every token of every head. With
+   ``offset_channels = c`` only c channels (``randperm(d)[:c]``) get an offset, drawn
+   after the permutation. ``N(0, s^2)`` is read as variance s^2 (std s);
+4. cast to fp16 (round to nearest even).
+
+The channel offset reproduces the outlier structure that motivates smoothing K: a
+shared per-channel bias across all tokens.
+"""
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass, field
+from typing import Optional, Tuple
+
+import torch
+
+SWEEP_N = (1024, 2048, 4096, 8192, 16384, 32768)
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    seed: int
+    B: int
+    H: int
+    N: int
+    d: int
+    causal: bool
+    offset_std: float
+    offset_channels: Optional[int] = None
+    pv_modes: Tuple[str, ...] = ("fp16",)
+    nseq: int = 0                  # > 0: packed varlen with nseq sequences
+    len_lo: int = 512
+    len_hi: int = 16384
+
+
+def tiny() -> Workload:
+    return Workload("tiny B1 H2 N256 d64 non-causal", 1000, 1, 2, 256, 64, False, 2.0)
+
+
+def llm_prefill() -> Workload:
+    return Workload("LLM causal prefill B4 H32 N4096 d128", 1001, 4, 32, 4096, 128, True, 1.0)
+
+
+def video_dit() -> Workload:
+    return Workload("video-DiT B1 H30 N17550 d64 non-causal", 1002, 1, 30, 17550, 64, False, 3.0,
+                    offset_channels=4, pv_modes=("fp16", "fp8"))
+
+
+def sweep(N: int, d: int, causal: bool) -> Workload:
+    B = max(1, 32768 // N)
+    return Workload(f"sweep B{B} H32 N{N} d{d} {'causal' if causal else 'non-causal'}", 1003,
+                    B, 32, N, d, causal, 1.0)
+
+
+def varlen() -> Workload:
+    return Workload("packed varlen causal 8 seqs H32 d128", 1004, 0, 32, 0, 128, True, 2.0,
+                    pv_modes=("fp8",), nseq=8)
+
+
+def _offset(g: torch.Generator, d: int, std: float, channels: Optional[int]) -> torch.Tensor:
+    if channels is None:
+        return torch.randn(d, generator=g) * std
+    perm = torch.randperm(d, generator=g)[:channels]
+    off = torch.zeros(d)
+    off[perm] = torch.randn(channels, generator=g) * std
+    return off
+
+
+def make_dense(w: Workload, B: Optional[int] = None, N: Optional[int] = None):
+    """fp16 CPU tensors q, k, v of shape [B, H, N, d] (B and N may be overridden)."""
+    B = w.B if B is None else B
+    N = w.N if N is None else N
+    g = torch.Generator().manual_seed(w.seed)
+    shape = (B, w.H, N, w.d)
+    q = torch.randn(shape, generator=g)
+    k = torch.randn(shape, generator=g)
+    v = torch.randn(shape, generator=g)
+    k += _offset(g, w.d, w.offset_std, w.offset_channels)
+    return q.half(), k.half(), v.half()
+
+
+def make_varlen(w: Workload, nseq: Optional[int] = None, len_lo: Optional[int] = None,
+                len_hi: Optional[int] = None, lens=None):
+    """Packed fp16 q, k, v of shape [T, H, d] and int32 cu_seqlens [nseq+1]."""
+    g = torch.Generator().manual_seed(w.seed)
+    nseq = w.nseq if nseq is None else nseq
+    lo = w.len_lo if len_lo is None else len_lo
+    hi = w.len_hi if len_hi is None else len_hi
+    if lens is None:
+        lens = torch.randint(lo, hi + 1, (nseq,), generator=g)
+    else:
+        lens = torch.as_tensor(lens, dtype=torch.int64)
+    cu = torch.zeros(len(lens) + 1, dtype=torch.int32)
+    cu[1:] = torch.cumsum(lens, 0).to(torch.int32)
+    T = int(cu[-1])
+    shape = (T, w.H, w.d)
+    q = torch.randn(shape, generator=g)
+    k = torch.randn(shape, generator=g)
+    v = torch.randn(shape, generator=g)
+    k += _offset(g, w.d, w.offset_std, w.offset_channels)
+    return q.half(), k.half(), v.half(), cu
+
+
+def attention_ops(B: int, H: int, N: int, d: int, causal: bool) -> float:
+    """Operation count of one attention forward: 4 B H N^2 d, halved for causal."""
+    ops = 4.0 * B * H * N * N * d
+    return ops / 2 if causal else ops
+
+
+def varlen_ops(lens, H: int, d: int, causal: bool) -> float:
+    return sum(attention_ops(1, H, int(n), d, causal) for n in lens)

@@ -1,0 +1,239 @@
+"""Pins for the oracle's attention: the fp64 reference and the quantized method.
+
+* fp64 attention vs torch's scaled_dot_product_attention in float64 (library routine);
+  N = 1 gives O = V; identical keys give O = mean(V).
+* The smoothing invariant softmax(QK^T) = softmax(Q(K - mean K)^T) ("SageAttention"
+  article, section 技术方案, paragraph on smoothing K), to ~1e-12 in fp64.
+* The quantized method (same section; "SageAttention2" article, 技术方案 (3)-(4)):
+  a single KV tile reduces the online softmax to a plain softmax over integer scores,
+  recomputed here with a library integer matmul; many tiles agree with one tile up to
+  the FP16 rounding of P; the result tracks fp64 attention on inputs built so that a
+  dropped rescale, a wrong scale index or a transposed operand would fail.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import Layout, PV_FP16, PV_FP8
+
+
+def _rand16(shape, seed, scale=1.0):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal(shape) * scale).astype(np.float16)
+
+
+def _cos(a, b):
+    a = np.asarray(a, np.float64).ravel()
+    b = np.asarray(b, np.float64).ravel()
+    return float(a @ b / (np.linalg.norm(a) * np.linalg.norm(b)))
+
+
+def _rel_l1(a, b):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    return float(np.abs(a - b).sum() / np.abs(b).sum())
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp64_matches_torch_sdpa(causal):
+    B, H, N, d = 2, 3, 70, 16
+    q, k, v = (_rand16((B, H, N, d), s) for s in (1, 2, 3))
+    sm = 1 / math.sqrt(d)
+    got = oracle.attn_fp64(q, k, v, Layout.dense(B, H, N, d), causal, sm)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        *(torch.from_numpy(x.astype(np.float64)) for x in (q, k, v)), is_causal=causal, scale=sm)
+    assert np.allclose(got, ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_fp64_special_cases():
+    d = 8
+    v = _rand16((1, 1, 1, d), 4)
+    q = _rand16((1, 1, 1, d), 5)
+    o = oracle.attn_fp64(q, q, v, Layout.dense(1, 1, 1, d), False, 0.3)
+    assert np.allclose(o, v.astype(np.float64), rtol=0, atol=1e-15)          # N = 1: O = V
+    N = 20
+    q = _rand16((1, 1, N, d), 6)
+    k = np.broadcast_to(_rand16((d,), 7), (1, 1, N, d)).astype(np.float16)
+    v = _rand16((1, 1, N, d), 8)
+    o = oracle.attn_fp64(q, k, v, Layout.dense(1, 1, N, d), False, 0.3)
+    assert np.allclose(o, v.astype(np.float64).mean(axis=2, keepdims=True), atol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_smoothing_invariant_fp64(causal):
+    B, H, N, d = 1, 2, 90, 16
+    q, k, v = (_rand16((B, H, N, d), s) for s in (11, 12, 13))
+    k = (k.astype(np.float64) + np.linspace(-30, 30, d)).astype(np.float16)
+    lay = Layout.dense(B, H, N, d)
+    k64 = k.astype(np.float64)
+    ks = k64 - k64.mean(axis=2, keepdims=True)
+    a = oracle.attn_fp64(q, k64, v, lay, causal, 0.25)
+    b = oracle.attn_fp64(q, ks, v, lay, causal, 0.25)
+    assert np.max(np.abs(a - b)) < 1e-12
+
+
+def _single_tile_reference(z, v, causal, pv_mode, sm, vs=None):
+    """Plain softmax over integer scores for one head (valid when one KV tile holds all
+    keys): S by a library int64 matmul, t in base 2, P rounded once, O = P V / sum p."""
+    qc = z["q_i8"][0, 0].astype(np.int64)
+    kc = z["k_i8"][0, 0].astype(np.int64)
+    N = qc.shape[0]
+    S = qc @ kc.T
+    sq = z["q_scale"][0, 0][np.arange(N) // 128].astype(np.float64)
+    sk = z["k_scale"][0, 0][np.arange(N) // 64].astype(np.float64)
+    t = S * sq[:, None] * sk[None, :] * sm / math.log(2)
+    if causal:
+        t[np.triu_indices(N, 1)] = -np.inf
+    p = np.exp2(t - t.max(axis=1, keepdims=True))
+    if pv_mode == PV_FP16:
+        P = p.astype(np.float16).astype(np.float64)
+        O = P @ v[0, 0].astype(np.float64) / p.sum(axis=1, keepdims=True)
+    else:
+        P = torch.from_numpy(448 * p).to(torch.float32).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+        vv = torch.from_numpy(v[0, 0]).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+        O = P @ vv * vs[0, 0][None, :] / (448 * p.sum(axis=1, keepdims=True))
+    return O.astype(np.float16)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("pv_mode", [PV_FP16, PV_FP8])
+def test_single_tile_equals_plain_softmax(causal, pv_mode):
+    N, d = 200, 32
+    q, k, v = (_rand16((1, 1, N, d), s) for s in (21, 22, 23))
+    k = (k.astype(np.float32) + 2.0).astype(np.float16)
+    lay = Layout.dense(1, 1, N, d)
+    sm = 1 / math.sqrt(d)
+    z = oracle.quant_qk(q, k, lay, True)
+    if pv_mode == PV_FP8:
+        vq, vs = oracle.quant_v_fp8(v, lay)
+    else:
+        vq, vs = v, None
+    got = oracle.attn_quant(z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], vq, vs, lay,
+                            causal, pv_mode, sm, tile_n=256)
+    ref = _single_tile_reference(z, vq, causal, pv_mode, sm, vs)
+    diff = np.abs(got.astype(np.float64) - ref.astype(np.float64))
+    # identical up to fp64 summation order and fp16 output rounding (one fp16 ulp)
+    assert diff.max() <= 2 * np.spacing(np.abs(ref).astype(np.float16)).astype(np.float64).max()
+
+
+def _increasing_scores(N, d, seed):
+    """Scores that grow along the keys, so the running max changes from tile to tile."""
+    q = _rand16((1, 1, N, d), seed)
+    q = (np.abs(q.astype(np.float32)) + 0.5).astype(np.float16)
+    k = _rand16((1, 1, N, d), seed + 1, 0.3).astype(np.float32)
+    k += np.linspace(0, 0.6, N)[:, None]
+    return q, k.astype(np.float16), _rand16((1, 1, N, d), seed + 2)
+
+
+@pytest.mark.parametrize("pv_mode", [PV_FP16, PV_FP8])
+def test_tiles_agree_and_rescale_matters(pv_mode):
+    N, d = 640, 32
+    q, k, v = _increasing_scores(N, d, 30)
+    lay = Layout.dense(1, 1, N, d)
+    sm = 1 / math.sqrt(d)
+    one = oracle.sage_attention(q, k, v, lay, False, True, pv_mode, sm, tile_n=1024)
+    many = oracle.sage_attention(q, k, v, lay, False, True, pv_mode, sm, tile_n=128)
+    exact = oracle.attn_fp64(q, k, v, lay, False, sm)
+    # E4M3 P keeps 3 mantissa bits, so the tile walk moves FP8 results more than FP16
+    assert _cos(many, one) > (0.99999 if pv_mode == PV_FP16 else 0.9995)
+    assert _cos(many, exact) > (0.9999 if pv_mode == PV_FP16 else 0.999)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_quantized_tracks_fp64(causal):
+    B, H, N, d = 1, 2, 384, 64
+    q, k, v = (_rand16((B, H, N, d), s) for s in (41, 42, 43))
+    k = (k.astype(np.float32) + _rand16((d,), 44, 2.0)).astype(np.float16)
+    lay = Layout.dense(B, H, N, d)
+    sm = 1 / math.sqrt(d)
+    exact = oracle.attn_fp64(q, k, v, lay, causal, sm)
+    o16 = oracle.sage_attention(q, k, v, lay, causal, True, PV_FP16, sm)
+    o8 = oracle.sage_attention(q, k, v, lay, causal, True, PV_FP8, sm)
+    assert _cos(o16, exact) > 0.9999 and _rel_l1(o16, exact) < 0.02
+    assert _cos(o8, exact) > 0.999
+
+
+def test_block_scale_indexing():
+    # K blocks of 64 tokens and Q blocks of 128 tokens with distinct magnitudes: the
+    # oracle must track fp64 attention, while the same scores with K scales indexed per
+    # 128 tokens instead of 64 (a plausible slip) must not
+    N, d = 512, 32
+    q, k, v = (_rand16((1, 1, N, d), s) for s in (51, 52, 53))
+    mags = 2.0 ** np.array([-1, 1, 0, 1, -1, 0.5, -0.5, 1])
+    k = (k.astype(np.float64) * mags[np.arange(N) // 64][None, None, :, None]).astype(np.float16)
+    q = (q.astype(np.float64) * (2.0 ** np.array([1, -1, 0, 0.5]))[np.arange(N) // 128][None, None, :, None]).astype(np.float16)
+    lay = Layout.dense(1, 1, N, d)
+    sm = 1 / math.sqrt(d)
+    exact = oracle.attn_fp64(q, k, v, lay, False, sm)
+    o = oracle.sage_attention(q, k, v, lay, False, True, PV_FP16, sm)
+    assert _cos(o, exact) > 0.9995
+    z = oracle.quant_qk(q, k, lay, True)
+    wrong = dict(z)
+    wrong["k_scale"] = z["k_scale"][:, :, np.arange(z["k_scale"].shape[2]) // 2 * 2]
+    slip = _single_tile_reference(wrong, v, False, PV_FP16, sm)
+    assert _cos(slip, exact) < 0.99
+
+
+def test_causal_first_row_and_constant_scores():
+    N, d = 130, 16
+    q, k, v = (_rand16((1, 1, N, d), s) for s in (61, 62, 63))
+    lay = Layout.dense(1, 1, N, d)
+    o = oracle.sage_attention(q, k, v, lay, True, True, PV_FP16, 0.25)
+    assert np.array_equal(o[0, 0, 0], v[0, 0, 0])           # row 0 sees only key 0
+    zq = np.zeros_like(q)                                   # all scores 0: O = mean V
+    o = oracle.sage_attention(zq, k, v, lay, False, True, PV_FP16, 0.25)
+    mean = v.astype(np.float64).mean(axis=2)[0, 0]
+    assert np.max(np.abs(o[0, 0].astype(np.float64) - mean)) <= 1e-3
+
+
+def test_fp8_single_token_is_exact():
+    # N = 1: P = 448 exactly and V / s_v = +-448 exactly, so O = V up to fp32 scale rounding
+    d = 16
+    v = _rand16((1, 1, 1, d), 71)
+    q = _rand16((1, 1, 1, d), 72)
+    o = oracle.sage_attention(q, q, v, Layout.dense(1, 1, 1, d), False, True, PV_FP8, 0.25)
+    assert np.array_equal(o, v)
+
+
+def test_smoothing_helps_with_channel_outliers():
+    # "SageAttention" article, 挑战: channel outliers in K ruin direct INT8 quantization;
+    # smoothing K fixes it
+    N, d = 512, 64
+    q, k, v = (_rand16((1, 1, N, d), s) for s in (81, 82, 83))
+    off = np.zeros(d)
+    off[[3, 17, 40, 55]] = [30.0, -25.0, 40.0, 20.0]
+    k = (k.astype(np.float64) + off).astype(np.float16)
+    lay = Layout.dense(1, 1, N, d)
+    sm = 1 / math.sqrt(d)
+    exact = oracle.attn_fp64(q, k, v, lay, False, sm)
+    smooth = oracle.sage_attention(q, k, v, lay, False, True, PV_FP16, sm)
+    raw = oracle.sage_attention(q, k, v, lay, False, False, PV_FP16, sm)
+    assert _rel_l1(smooth, exact) < 0.5 * _rel_l1(raw, exact)
+
+
+def test_varlen_equals_per_sequence_dense():
+    H, d = 2, 32
+    lens = [70, 200, 129]
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    T = int(cu[-1])
+    q, k, v = (_rand16((T, H, d), s) for s in (91, 92, 93))
+    lay = Layout.packed(cu, H, d)
+    o = oracle.sage_attention(q, k, v, lay, True, True, PV_FP16, 0.2)
+    for s, n in enumerate(lens):
+        sl = slice(cu[s], cu[s + 1])
+        dq, dk, dv = (np.ascontiguousarray(x[sl].transpose(1, 0, 2))[None] for x in (q, k, v))
+        od = oracle.sage_attention(dq, dk, dv, Layout.dense(1, H, n, d), True, True, PV_FP16, 0.2)
+        assert np.array_equal(o[sl].transpose(1, 0, 2), od[0])
+
+
+def test_sampled_rows_match_full():
+    B, H, N, d = 1, 2, 300, 32
+    q, k, v = (_rand16((B, H, N, d), s) for s in (101, 102, 103))
+    lay = Layout.dense(B, H, N, d)
+    full = oracle.sage_attention(q, k, v, lay, True, True, PV_FP16, 0.2)
+    part = oracle.sage_attention(q, k, v, lay, True, True, PV_FP16, 0.2, heads=[(0, 1)], rows=(100, 180))
+    assert np.array_equal(part[0, 1, 100:180], full[0, 1, 100:180])
+    assert np.isnan(part[0, 0]).all() and np.isnan(part[0, 1, :100]).all()

@@ -1,0 +1,176 @@
+/*
+ * sage.h - C ABI of the B200 (sm_100a) SageAttention forward pass (libsage.so).
+ *
+ * The method ("SageAttention: Accurate 8-Bit Attention for Plug-and-play Inference
+ * Acceleration", and the follow-up article on SageAttention2) computes attention
+ * O = softmax(sm_scale * Q K^T) V with:
+ *   1. smooth K: K <- K - mean(K), the mean per channel over the tokens of one head
+ *      ("SageAttention" article, section 技术方案, paragraph on smoothing K; softmax is
+ *      unchanged because q.mean(K) is constant along a row);
+ *   2. per-block INT8 quantization of Q and K with one fp32 scale per block
+ *      (scale = amax/127), blocks of FlashAttention size: 128 Q tokens, 64 K tokens
+ *      (same section, paragraph on per-block INT8 of Q, K);
+ *   3. a fused FlashAttention-style pass: S = Q_i8 K_i8^T with INT32 accumulation,
+ *      dequantized by q_scale*k_scale*sm_scale, online softmax over 128-key tiles, and
+ *      P.V either in FP16 (SAGE_PV_FP16; same section, paragraph on the FP16 PV
+ *      accumulator) or with P and V in FP8 E4M3 (SAGE_PV_FP8; "SageAttention2"
+ *      article, 技术方案 items (3) and (4)), each tile's P.V summed into fp32 registers.
+ *
+ * Conventions for every entry point:
+ *   - fp16 tensors are IEEE binary16, passed as `const void*`/`void*`.
+ *   - Dense layout [B, H, N, d] row-major (the layout of the scaled_dot_product_attention
+ *     call the method replaces). Packed varlen layout [T, H, d] with int32 cu_seqlens
+ *     [nseq+1] ON THE DEVICE: sequence s owns tokens cu_seqlens[s] .. cu_seqlens[s+1]-1;
+ *     every per-head quantity (K mean, blocks, causal mask, V scale) is per sequence.
+ *   - Scales: q_scale [nseq, H, ceil(maxlen/128)], k_scale [nseq, H, ceil(maxlen/64)],
+ *     k_mean and v_scale [nseq, H, d] (dense: nseq = B, maxlen = N).
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library never
+ *     frees or retains them. Tensor pointers must be 16-byte aligned.
+ *   - Head dim d is 64 or 128. sm_scale <= 0 selects 1/sqrt(d). causal is the square
+ *     mask j <= i within each sequence.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *     Nothing synchronizes except sage_get_device_status().
+ *   - Host-detectable argument errors return before anything is enqueued. Errors that
+ *     only the device can see (a bounded wait that timed out, malformed cu_seqlens) set
+ *     a device status word, read and cleared by sage_get_device_status(); the output is
+ *     then undefined. No kernel traps or spins without bound.
+ */
+#ifndef SAGE_H
+#define SAGE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SAGE_API __attribute__((visibility("default")))
+#else
+#define SAGE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SAGE_OK = 0,
+    SAGE_ERR_INVALID_ARG = 1,   /* bad size, null pointer, unknown mode */
+    SAGE_ERR_UNSUPPORTED = 2,   /* valid request this build does not implement (e.g. d) */
+    SAGE_ERR_MISALIGNED = 3,    /* a tensor pointer is not 16-byte aligned */
+    SAGE_ERR_WORKSPACE = 4,     /* workspace missing or smaller than sage_workspace_size() */
+    SAGE_ERR_CUDA = 5,          /* a CUDA runtime call failed (see sage_last_cuda_error) */
+    SAGE_ERR_TIMEOUT = 6,       /* device: a bounded wait inside a kernel gave up */
+    SAGE_ERR_BAD_SEQLENS = 7    /* device: cu_seqlens not monotonic / out of range */
+} sage_status_t;
+
+enum { SAGE_PV_FP16 = 0, SAGE_PV_FP8 = 1 };
+
+/* Opaque CUDA stream (binary-compatible with cudaStream_t). */
+typedef struct CUstream_st *sage_stream_t;
+
+/*
+ * Bytes of scratch the fused entry points need for one call: INT8 codes of Q and K,
+ * their block scales, the K mean (and its fp64 column sums), and in FP8 mode the E4M3
+ * codes of V with their per-channel scales. Dense: nseq = B, max_seqlen = N,
+ * total_tokens = B*N.
+ */
+SAGE_API size_t sage_workspace_size(int nseq, int H, int max_seqlen, int total_tokens, int d,
+                           int pv_mode);
+
+/*
+ * Steps 1-2 on their own (dense): k_mean[b,h,c] = mean over tokens of K[b,h,:,c]
+ * (zeros when smooth_k == 0), q_i8/q_scale = per-128-token INT8 of Q, k_i8/k_scale =
+ * per-64-token INT8 of fp32(K) - k_mean. The K-mean sum is accumulated in fp64 (exact
+ * for |K| N < 2^29) and rounded once to fp32; codes are round-half-even of the fp32
+ * quotient x/scale clamped to [-127, 127]; an all-zero block has scale 0 and codes 0.
+ * Outputs are caller-owned device buffers of the shapes in the conventions above.
+ * Uses a small stream-ordered allocation (cudaMallocAsync) for the fp64 sums.
+ */
+SAGE_API sage_status_t sage_quant_qk(const void *q, const void *k, int8_t *q_i8, float *q_scale,
+                            int8_t *k_i8, float *k_scale, float *k_mean, int B, int H, int N,
+                            int d, int smooth_k, sage_stream_t stream);
+
+/* sage_quant_qk for the packed varlen layout (cu_seqlens on the device; NULL reads the
+ * buffers as dense [nseq, H, max_seqlen, d]). */
+SAGE_API sage_status_t sage_quant_qk_varlen(const void *q, const void *k, const int32_t *cu_seqlens,
+                                   int nseq, int total_tokens, int max_seqlen, int H, int d,
+                                   int8_t *q_i8, float *q_scale, int8_t *k_i8, float *k_scale,
+                                   float *k_mean, int smooth_k, sage_stream_t stream);
+
+/*
+ * V to FP8 E4M3 ("SageAttention2" article, 技术方案 (4)) with one fp32 scale per
+ * channel over all tokens of a head: v_scale = amax/448, v_e4m3 = round-to-nearest-even
+ * saturating E4M3 of the fp32 quotient V/v_scale (same [B,H,N,d] layout, one byte each).
+ */
+SAGE_API sage_status_t sage_quant_v_fp8(const void *v, uint8_t *v_e4m3, float *v_scale, int B, int H,
+                               int N, int d, sage_stream_t stream);
+SAGE_API sage_status_t sage_quant_v_fp8_varlen(const void *v, const int32_t *cu_seqlens, int nseq,
+                                      int total_tokens, int max_seqlen, int H, int d,
+                                      uint8_t *v_e4m3, float *v_scale, sage_stream_t stream);
+
+/*
+ * The whole forward pass (steps 1-3), dense layout: out[B,H,N,d] fp16. pv_mode selects
+ * SAGE_PV_FP16 or SAGE_PV_FP8. Scratch comes from stream-ordered allocation
+ * (cudaMallocAsync/cudaFreeAsync on `stream`).
+ */
+SAGE_API sage_status_t sage_attn_fwd(const void *q, const void *k, const void *v, void *out, int B,
+                            int H, int N, int d, int causal, int smooth_k, int pv_mode,
+                            float sm_scale, sage_stream_t stream);
+
+/* sage_attn_fwd with caller-owned scratch of at least sage_workspace_size() bytes
+ * (256-byte aligned); allocates nothing. */
+SAGE_API sage_status_t sage_attn_fwd_ws(const void *q, const void *k, const void *v, void *out, int B,
+                               int H, int N, int d, int causal, int smooth_k, int pv_mode,
+                               float sm_scale, void *workspace, size_t ws_bytes,
+                               sage_stream_t stream);
+
+/*
+ * The whole forward pass on packed sequences: q, k, v, out are [total_tokens, H, d];
+ * cu_seqlens is int32 [nseq+1] on the device with cu_seqlens[0] = 0 and
+ * cu_seqlens[nseq] = total_tokens; max_seqlen (host) must bound every length (it sizes
+ * the grid, so no device-to-host copy is made). workspace may be NULL (stream-ordered
+ * allocation) or caller-owned scratch of sage_workspace_size() bytes.
+ */
+SAGE_API sage_status_t sage_attn_varlen_fwd(const void *q, const void *k, const void *v, void *out,
+                                   const int32_t *cu_seqlens, int nseq, int total_tokens,
+                                   int max_seqlen, int H, int d, int causal, int smooth_k,
+                                   int pv_mode, float sm_scale, void *workspace,
+                                   size_t ws_bytes, sage_stream_t stream);
+
+/*
+ * Step 3 alone on pre-quantized operands (dense): q_i8/q_scale and k_i8/k_scale as
+ * produced by sage_quant_qk; v is fp16 V (SAGE_PV_FP16, v_scale ignored) or E4M3 codes
+ * with per-channel v_scale (SAGE_PV_FP8). Allocates nothing.
+ */
+SAGE_API sage_status_t sage_attn_fwd_quantized(const int8_t *q_i8, const float *q_scale,
+                                      const int8_t *k_i8, const float *k_scale, const void *v,
+                                      const float *v_scale, void *out, int B, int H, int N,
+                                      int d, int causal, int pv_mode, float sm_scale,
+                                      sage_stream_t stream);
+
+/*
+ * Debug: the integer score tiles S = q_i8 k_i8^T (int32, [B,H,N,N]) exactly as the
+ * attention kernel's tensor-core pass produces them, dumped from tensor memory. Meant
+ * for small N (the output is N^2 per head). Uses stream-ordered scratch for a dummy
+ * pass over V.
+ */
+SAGE_API sage_status_t sage_debug_qk_int32(const int8_t *q_i8, const int8_t *k_i8, int32_t *s_out,
+                                  int B, int H, int N, int d, sage_stream_t stream);
+
+/* Synchronizes `stream`, returns the device status word (SAGE_OK if clean) and clears
+ * it. SAGE_ERR_CUDA if the synchronization itself failed. */
+SAGE_API sage_status_t sage_get_device_status(sage_stream_t stream);
+
+/* Human-readable name of a status code (static storage). */
+SAGE_API const char *sage_status_string(sage_status_t status);
+
+/* cudaError_t value of the last failed CUDA runtime call made by this library. */
+SAGE_API int sage_last_cuda_error(void);
+
+/* ABI version (major*100 + minor). */
+SAGE_API int sage_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAGE_H */

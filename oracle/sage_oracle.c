@@ -156,7 +156,7 @@ void oracle_head_k_mean(const uint16_t *K, int64_t n, int64_t stride, int d, flo
         double s = 0.0;
         for (int64_t t = 0; t < n; t++)
             s += oracle_f16_to_f64(K[t * stride + c]);
-        mu[c] = (float)(s / (double)n);
+        mu[c] = n > 0 ? (float)(s / (double)n) : 0.0f;
     }
 }
 

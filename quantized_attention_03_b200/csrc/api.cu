@@ -1,0 +1,462 @@
+// C-ABI entry points of libsage.so: argument validation, workspace carving and the
+// launch sequence colstats -> quant -> attention on the caller's stream.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstdlib>
+#include <mutex>
+
+#include "sage_common.cuh"
+
+namespace sage {
+namespace {
+
+__device__ int g_status;   // device status word: OR of 1 << sage_status_t
+
+int g_last_cuda_error = 0;
+std::mutex g_mu;
+int *g_status_ptr[64] = {};
+
+sage_status_t cuda_fail(cudaError_t e)
+{
+    g_last_cuda_error = (int)e;
+    if (std::getenv("SAGE_LOG"))
+        std::fprintf(stderr, "sage: CUDA error %d (%s)\n", (int)e, cudaGetErrorString(e));
+    return SAGE_ERR_CUDA;
+}
+
+// Device address of this device's status word (looked up once per device).
+int *status_ptr(sage_status_t *err)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= 64) {
+        *err = cuda_fail(e == cudaSuccess ? cudaErrorInvalidDevice : e);
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_status_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_status);
+        if (e != cudaSuccess) {
+            *err = cuda_fail(e);
+            return nullptr;
+        }
+        g_status_ptr[dev] = static_cast<int *>(p);
+    }
+    *err = SAGE_OK;
+    return g_status_ptr[dev];
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Scratch carved from one buffer, every part 256-byte aligned.
+struct Workspace {
+    int8_t *q_i8 = nullptr, *k_i8 = nullptr;
+    float *q_scale = nullptr, *k_scale = nullptr, *k_mean = nullptr;
+    double *ksum = nullptr;
+    uint32_t *vamax = nullptr;   // adjacent to ksum: one memset clears both
+    uint8_t *v8 = nullptr;
+    float *v_scale = nullptr;
+    size_t stats_bytes = 0;      // bytes of [ksum | vamax]
+    size_t total = 0;
+};
+
+Workspace carve(char *base, int nseq, int H, int maxlen, int total_tokens, int d, int pv_mode)
+{
+    Workspace w;
+    const size_t codes = (size_t)total_tokens * H * d;
+    const size_t nqb = (maxlen + kQBlock - 1) / kQBlock, nkb = (maxlen + kKBlock - 1) / kKBlock;
+    const size_t heads = (size_t)nseq * H;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        char *p = base ? base + off : nullptr;
+        off += align256(bytes);
+        return p;
+    };
+    w.q_i8 = reinterpret_cast<int8_t *>(take(codes));
+    w.k_i8 = reinterpret_cast<int8_t *>(take(codes));
+    w.q_scale = reinterpret_cast<float *>(take(heads * nqb * 4));
+    w.k_scale = reinterpret_cast<float *>(take(heads * nkb * 4));
+    w.k_mean = reinterpret_cast<float *>(take(heads * d * 4));
+    const size_t stats0 = off;
+    w.ksum = reinterpret_cast<double *>(take(heads * d * 8));
+    if (pv_mode == SAGE_PV_FP8) {
+        w.vamax = reinterpret_cast<uint32_t *>(take(heads * d * 4));
+        w.stats_bytes = off - stats0;
+        w.v8 = reinterpret_cast<uint8_t *>(take(codes));
+        w.v_scale = reinterpret_cast<float *>(take(heads * d * 4));
+    } else {
+        w.stats_bytes = off - stats0;
+    }
+    w.total = off;
+    return w;
+}
+
+sage_status_t check_shape(int nseq, int H, int maxlen, int d)
+{
+    if (nseq < 0 || H < 0 || maxlen < 0)
+        return SAGE_ERR_INVALID_ARG;
+    if (d != 64 && d != 128)
+        return SAGE_ERR_UNSUPPORTED;
+    if (H > 65535 || nseq > 65535)
+        return SAGE_ERR_UNSUPPORTED;    // grid y/z limits
+    return SAGE_OK;
+}
+
+float resolve_scale(float sm_scale, int d)
+{
+    return sm_scale > 0.0f ? sm_scale : 1.0f / std::sqrt((float)d);
+}
+
+// Steps 1-3 with the given scratch; q/k/v/out already validated.
+sage_status_t forward(const void *q, const void *k, const void *v, void *out, const SeqLayout &L,
+                      int causal, int smooth_k, int pv_mode, float sm_scale, char *ws,
+                      cudaStream_t st)
+{
+    sage_status_t err;
+    int *status = status_ptr(&err);
+    if (!status)
+        return err;
+    Workspace w = carve(ws, L.nseq, L.H, L.maxlen, L.total, L.d, pv_mode);
+    const bool fp8 = pv_mode == SAGE_PV_FP8;
+    cudaError_t e = cudaMemsetAsync(w.ksum, 0, w.stats_bytes, st);
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    const __half *qh = static_cast<const __half *>(q);
+    const __half *kh = static_cast<const __half *>(k);
+    const __half *vh = static_cast<const __half *>(v);
+    if ((e = launch_colstats(kh, vh, smooth_k ? w.ksum : nullptr, fp8 ? w.vamax : nullptr, L,
+                             status, st)) != cudaSuccess)
+        return cuda_fail(e);
+    if ((e = launch_quant(qh, kh, vh, smooth_k ? w.ksum : nullptr, w.vamax, w.q_i8, w.q_scale,
+                          w.k_i8, w.k_scale, w.k_mean, fp8 ? w.v8 : nullptr, w.v_scale, L, status,
+                          st)) != cudaSuccess)
+        return cuda_fail(e);
+    AttnArgs a{w.q_i8, w.q_scale, w.k_i8, w.k_scale, fp8 ? (const void *)w.v8 : v, w.v_scale,
+               static_cast<__half *>(out), nullptr, causal, pv_mode, resolve_scale(sm_scale, L.d)};
+    sage_status_t herr;
+    if ((e = launch_attention(a, L, status, st, &herr)) != cudaSuccess)
+        return herr != SAGE_OK ? herr : cuda_fail(e);
+    return SAGE_OK;
+}
+
+sage_status_t alloc_ws(size_t bytes, cudaStream_t st, char **p)
+{
+    void *ptr = nullptr;
+    cudaError_t e = cudaMallocAsync(&ptr, bytes ? bytes : 256, st);
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    *p = static_cast<char *>(ptr);
+    return SAGE_OK;
+}
+
+}  // namespace
+}  // namespace sage
+
+using namespace sage;
+
+extern "C" {
+
+size_t sage_workspace_size(int nseq, int H, int max_seqlen, int total_tokens, int d, int pv_mode)
+{
+    if (nseq < 0 || H < 0 || max_seqlen < 0 || total_tokens < 0)
+        return 0;
+    return carve(nullptr, nseq, H, max_seqlen, total_tokens, d, pv_mode).total;
+}
+
+sage_status_t sage_quant_qk(const void *q, const void *k, int8_t *q_i8, float *q_scale,
+                            int8_t *k_i8, float *k_scale, float *k_mean, int B, int H, int N,
+                            int d, int smooth_k, sage_stream_t stream)
+{
+    sage_status_t r = check_shape(B, H, N, d);
+    if (r != SAGE_OK)
+        return r;
+    if (B == 0 || H == 0 || N == 0)
+        return SAGE_OK;
+    if (!q || !k || !q_i8 || !q_scale || !k_i8 || !k_scale || !k_mean)
+        return SAGE_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(q_i8) || !aligned16(k_i8))
+        return SAGE_ERR_MISALIGNED;
+    return sage_quant_qk_varlen(q, k, nullptr, B, B * N, N, H, d, q_i8, q_scale, k_i8, k_scale,
+                                k_mean, smooth_k, stream);
+}
+
+sage_status_t sage_quant_qk_varlen(const void *q, const void *k, const int32_t *cu_seqlens,
+                                   int nseq, int total_tokens, int max_seqlen, int H, int d,
+                                   int8_t *q_i8, float *q_scale, int8_t *k_i8, float *k_scale,
+                                   float *k_mean, int smooth_k, sage_stream_t stream)
+{
+    sage_status_t r = check_shape(nseq, H, max_seqlen, d);
+    if (r != SAGE_OK)
+        return r;
+    if (nseq == 0 || H == 0 || max_seqlen == 0 || total_tokens == 0)
+        return SAGE_OK;
+    if (!q || !k || !q_i8 || !q_scale || !k_i8 || !k_scale || !k_mean || total_tokens < 0)
+        return SAGE_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(q_i8) || !aligned16(k_i8))
+        return SAGE_ERR_MISALIGNED;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    int *status = status_ptr(&r);
+    if (!status)
+        return r;
+    const SeqLayout L = cu_seqlens ? SeqLayout::packed(cu_seqlens, nseq, total_tokens, max_seqlen, H, d)
+                                   : SeqLayout::dense(nseq, H, max_seqlen, d);
+    double *ksum = nullptr;
+    cudaError_t e;
+    if (smooth_k) {
+        void *p = nullptr;
+        if ((e = cudaMallocAsync(&p, (size_t)nseq * H * d * 8, st)) != cudaSuccess)
+            return cuda_fail(e);
+        ksum = static_cast<double *>(p);
+        if ((e = cudaMemsetAsync(ksum, 0, (size_t)nseq * H * d * 8, st)) != cudaSuccess)
+            return cuda_fail(e);
+        if ((e = launch_colstats(static_cast<const __half *>(k), nullptr, ksum, nullptr, L, status,
+                                 st)) != cudaSuccess)
+            return cuda_fail(e);
+    }
+    e = launch_quant(static_cast<const __half *>(q), static_cast<const __half *>(k), nullptr, ksum,
+                     nullptr, q_i8, q_scale, k_i8, k_scale, k_mean, nullptr, nullptr, L, status, st);
+    if (ksum)
+        cudaFreeAsync(ksum, st);
+    return e == cudaSuccess ? SAGE_OK : cuda_fail(e);
+}
+
+sage_status_t sage_quant_v_fp8_varlen(const void *v, const int32_t *cu_seqlens, int nseq,
+                                      int total_tokens, int max_seqlen, int H, int d,
+                                      uint8_t *v_e4m3, float *v_scale, sage_stream_t stream)
+{
+    sage_status_t r = check_shape(nseq, H, max_seqlen, d);
+    if (r != SAGE_OK)
+        return r;
+    if (nseq == 0 || H == 0 || max_seqlen == 0 || total_tokens == 0)
+        return SAGE_OK;
+    if (!v || !v_e4m3 || !v_scale || total_tokens < 0)
+        return SAGE_ERR_INVALID_ARG;
+    if (!aligned16(v) || !aligned16(v_e4m3))
+        return SAGE_ERR_MISALIGNED;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    int *status = status_ptr(&r);
+    if (!status)
+        return r;
+    const SeqLayout L = cu_seqlens ? SeqLayout::packed(cu_seqlens, nseq, total_tokens, max_seqlen, H, d)
+                                   : SeqLayout::dense(nseq, H, max_seqlen, d);
+    void *p = nullptr;
+    const size_t bytes = (size_t)nseq * H * d * 4;
+    cudaError_t e;
+    if ((e = cudaMallocAsync(&p, bytes, st)) != cudaSuccess)
+        return cuda_fail(e);
+    uint32_t *vamax = static_cast<uint32_t *>(p);
+    if ((e = cudaMemsetAsync(vamax, 0, bytes, st)) == cudaSuccess &&
+        (e = launch_colstats(nullptr, static_cast<const __half *>(v), nullptr, vamax, L, status,
+                             st)) == cudaSuccess)
+        e = launch_quant(nullptr, nullptr, static_cast<const __half *>(v), nullptr, vamax, nullptr,
+                         nullptr, nullptr, nullptr, nullptr, v_e4m3, v_scale, L, status, st);
+    cudaFreeAsync(p, st);
+    return e == cudaSuccess ? SAGE_OK : cuda_fail(e);
+}
+
+sage_status_t sage_quant_v_fp8(const void *v, uint8_t *v_e4m3, float *v_scale, int B, int H,
+                               int N, int d, sage_stream_t stream)
+{
+    return sage_quant_v_fp8_varlen(v, nullptr, B, B * N, N, H, d, v_e4m3, v_scale, stream);
+}
+
+}  // extern "C"
+
+namespace sage {
+namespace {
+// Dense (cu_seqlens == nullptr) or packed forward pass with optional caller scratch.
+sage_status_t attn_entry(const void *q, const void *k, const void *v, void *out,
+                         const int32_t *cu_seqlens, int nseq, int total_tokens, int max_seqlen,
+                         int H, int d, int causal, int smooth_k, int pv_mode, float sm_scale,
+                         void *workspace, size_t ws_bytes, sage_stream_t stream)
+{
+    sage_status_t r = check_shape(nseq, H, max_seqlen, d);
+    if (r != SAGE_OK)
+        return r;
+    if (pv_mode != SAGE_PV_FP16 && pv_mode != SAGE_PV_FP8)
+        return SAGE_ERR_INVALID_ARG;
+    if (total_tokens < 0)
+        return SAGE_ERR_INVALID_ARG;
+    if (nseq == 0 || H == 0 || max_seqlen == 0 || total_tokens == 0)
+        return SAGE_OK;
+    if (!q || !k || !v || !out)
+        return SAGE_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+        return SAGE_ERR_MISALIGNED;
+    const size_t need = sage_workspace_size(nseq, H, max_seqlen, total_tokens, d, pv_mode);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const SeqLayout L = cu_seqlens ? SeqLayout::packed(cu_seqlens, nseq, total_tokens, max_seqlen, H, d)
+                                   : SeqLayout::dense(nseq, H, max_seqlen, d);
+    if (workspace != nullptr) {
+        if (ws_bytes < need)
+            return SAGE_ERR_WORKSPACE;
+        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+            return SAGE_ERR_MISALIGNED;
+        return forward(q, k, v, out, L, causal, smooth_k, pv_mode, sm_scale,
+                       static_cast<char *>(workspace), st);
+    }
+    char *ws = nullptr;
+    if ((r = alloc_ws(need, st, &ws)) != SAGE_OK)
+        return r;
+    r = forward(q, k, v, out, L, causal, smooth_k, pv_mode, sm_scale, ws, st);
+    cudaFreeAsync(ws, st);
+    return r;
+}
+}  // namespace
+}  // namespace sage
+
+extern "C" {
+
+sage_status_t sage_attn_varlen_fwd(const void *q, const void *k, const void *v, void *out,
+                                   const int32_t *cu_seqlens, int nseq, int total_tokens,
+                                   int max_seqlen, int H, int d, int causal, int smooth_k,
+                                   int pv_mode, float sm_scale, void *workspace,
+                                   size_t ws_bytes, sage_stream_t stream)
+{
+    if (cu_seqlens == nullptr && nseq > 0 && total_tokens > 0)
+        return SAGE_ERR_INVALID_ARG;
+    return attn_entry(q, k, v, out, cu_seqlens, nseq, total_tokens, max_seqlen, H, d, causal,
+                      smooth_k, pv_mode, sm_scale, workspace, ws_bytes, stream);
+}
+
+sage_status_t sage_attn_fwd_ws(const void *q, const void *k, const void *v, void *out, int B,
+                               int H, int N, int d, int causal, int smooth_k, int pv_mode,
+                               float sm_scale, void *workspace, size_t ws_bytes,
+                               sage_stream_t stream)
+{
+    if (workspace == nullptr && !(B == 0 || H == 0 || N == 0))
+        return SAGE_ERR_WORKSPACE;
+    if (B > 0 && N > 0 && (int64_t)B * N > INT32_MAX)
+        return SAGE_ERR_UNSUPPORTED;
+    return attn_entry(q, k, v, out, nullptr, B, B * N, N, H, d, causal, smooth_k, pv_mode,
+                      sm_scale, workspace, ws_bytes, stream);
+}
+
+sage_status_t sage_attn_fwd(const void *q, const void *k, const void *v, void *out, int B, int H,
+                            int N, int d, int causal, int smooth_k, int pv_mode, float sm_scale,
+                            sage_stream_t stream)
+{
+    if (B > 0 && N > 0 && (int64_t)B * N > INT32_MAX)
+        return SAGE_ERR_UNSUPPORTED;
+    return attn_entry(q, k, v, out, nullptr, B, B * N, N, H, d, causal, smooth_k, pv_mode,
+                      sm_scale, nullptr, 0, stream);
+}
+
+sage_status_t sage_attn_fwd_quantized(const int8_t *q_i8, const float *q_scale,
+                                      const int8_t *k_i8, const float *k_scale, const void *v,
+                                      const float *v_scale, void *out, int B, int H, int N,
+                                      int d, int causal, int pv_mode, float sm_scale,
+                                      sage_stream_t stream)
+{
+    sage_status_t r = check_shape(B, H, N, d);
+    if (r != SAGE_OK)
+        return r;
+    if (pv_mode != SAGE_PV_FP16 && pv_mode != SAGE_PV_FP8)
+        return SAGE_ERR_INVALID_ARG;
+    if (B == 0 || H == 0 || N == 0)
+        return SAGE_OK;
+    if (!q_i8 || !q_scale || !k_i8 || !k_scale || !v || !out ||
+        (pv_mode == SAGE_PV_FP8 && !v_scale))
+        return SAGE_ERR_INVALID_ARG;
+    if (!aligned16(q_i8) || !aligned16(k_i8) || !aligned16(v) || !aligned16(out))
+        return SAGE_ERR_MISALIGNED;
+    int *status = status_ptr(&r);
+    if (!status)
+        return r;
+    const SeqLayout L = SeqLayout::dense(B, H, N, d);
+    AttnArgs a{q_i8, q_scale, k_i8, k_scale, v, v_scale, static_cast<__half *>(out), nullptr,
+               causal, pv_mode, resolve_scale(sm_scale, d)};
+    sage_status_t herr;
+    cudaError_t e = launch_attention(a, L, status, reinterpret_cast<cudaStream_t>(stream), &herr);
+    if (e != cudaSuccess)
+        return herr != SAGE_OK ? herr : cuda_fail(e);
+    return SAGE_OK;
+}
+
+sage_status_t sage_debug_qk_int32(const int8_t *q_i8, const int8_t *k_i8, int32_t *s_out, int B,
+                                  int H, int N, int d, sage_stream_t stream)
+{
+    sage_status_t r = check_shape(B, H, N, d);
+    if (r != SAGE_OK)
+        return r;
+    if (B == 0 || H == 0 || N == 0)
+        return SAGE_OK;
+    if (!q_i8 || !k_i8 || !s_out)
+        return SAGE_ERR_INVALID_ARG;
+    if (!aligned16(q_i8) || !aligned16(k_i8))
+        return SAGE_ERR_MISALIGNED;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    int *status = status_ptr(&r);
+    if (!status)
+        return r;
+    const size_t elems = (size_t)B * H * N * d;
+    const size_t nqb = (N + kQBlock - 1) / kQBlock, nkb = (N + kKBlock - 1) / kKBlock;
+    const size_t sc_bytes = align256((size_t)B * H * (nqb + nkb) * 4);
+    const size_t bytes = sc_bytes + 2 * align256(elems * 2);
+    char *ws = nullptr;
+    if ((r = alloc_ws(bytes, st, &ws)) != SAGE_OK)
+        return r;
+    cudaError_t e = cudaMemsetAsync(ws, 0, bytes, st);   // zero scales and V: P V stays finite
+    if (e == cudaSuccess) {
+        const float *qs = reinterpret_cast<float *>(ws);
+        const float *ks = qs + (size_t)B * H * nqb;
+        const void *vz = ws + sc_bytes;
+        __half *o = reinterpret_cast<__half *>(ws + sc_bytes + align256(elems * 2));
+        AttnArgs a{q_i8, qs, k_i8, ks, vz, nullptr, o, s_out, 0, SAGE_PV_FP16, 1.0f};
+        sage_status_t herr;
+        e = launch_attention(a, SeqLayout::dense(B, H, N, d), status, st, &herr);
+        if (e != cudaSuccess && herr != SAGE_OK) {
+            cudaFreeAsync(ws, st);
+            return herr;
+        }
+    }
+    cudaFreeAsync(ws, st);
+    return e == cudaSuccess ? SAGE_OK : cuda_fail(e);
+}
+
+sage_status_t sage_get_device_status(sage_stream_t stream)
+{
+    cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess)
+        return cuda_fail(e);
+    int v = 0;
+    if ((e = cudaMemcpyFromSymbol(&v, g_status, sizeof(int))) != cudaSuccess)
+        return cuda_fail(e);
+    if (v != 0) {
+        const int zero = 0;
+        if ((e = cudaMemcpyToSymbol(g_status, &zero, sizeof(int))) != cudaSuccess)
+            return cuda_fail(e);
+        for (int b = 1; b < 31; b++)
+            if (v & (1 << b))
+                return static_cast<sage_status_t>(b);
+    }
+    return SAGE_OK;
+}
+
+const char *sage_status_string(sage_status_t s)
+{
+    switch (s) {
+    case SAGE_OK: return "SAGE_OK";
+    case SAGE_ERR_INVALID_ARG: return "SAGE_ERR_INVALID_ARG";
+    case SAGE_ERR_UNSUPPORTED: return "SAGE_ERR_UNSUPPORTED";
+    case SAGE_ERR_MISALIGNED: return "SAGE_ERR_MISALIGNED";
+    case SAGE_ERR_WORKSPACE: return "SAGE_ERR_WORKSPACE";
+    case SAGE_ERR_CUDA: return "SAGE_ERR_CUDA";
+    case SAGE_ERR_TIMEOUT: return "SAGE_ERR_TIMEOUT";
+    case SAGE_ERR_BAD_SEQLENS: return "SAGE_ERR_BAD_SEQLENS";
+    }
+    return "SAGE_ERR_UNKNOWN";
+}
+
+int sage_last_cuda_error(void) { return g_last_cuda_error; }
+
+int sage_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,616 @@
+// K-ATTN: the fused quantized attention pass for sm_100a.
+//
+// Method ("SageAttention" article, section 技术方案; "SageAttention2" article, 技术方案
+// (3)-(4)): S = Q_i8 K_i8^T with INT32 accumulation, dequantized by
+// q_scale * k_scale * sm_scale, FlashAttention online softmax over 128-key tiles, and
+// P.V with P, V in FP16 (FP16 mode) or both in E4M3 (FP8 mode), each tile's P.V
+// product accumulated across tiles in fp32 registers (the two-level accumulation of
+// the SageAttention2 article, item (3)).
+//
+// B200 design. One CTA owns NQT = 2 query tiles of 128 rows of one (sequence, head)
+// and walks the KV tiles once for both, so each K/V tile read from L2 feeds 256 rows:
+//   warps 0-3 / 4-7   softmax warpgroups, one per query tile: thread t owns row t
+//                     (TMEM lane t); O (d fp32) lives in its registers
+//   warp 8            TMA producer: Q tiles once, then K/V tiles into a STAGES-deep
+//                     shared-memory ring (mbarrier full/empty pairs)
+//   warp 9            MMA issuer (one thread) + TMEM owner:
+//                       S_i = Q_i K^T       tcgen05.mma kind::i8 -> TMEM (s32, 128 cols)
+//                       PV_i = P_i V        tcgen05.mma kind::f16 | kind::f8f6f4 with P
+//                                           read from TMEM (aliasing S_i) and V from
+//                                           shared memory (MN-major) -> TMEM (f32)
+//   warps 10-11       idle (complete the warpgroup for the register split)
+// TMEM columns: [S_0 | S_1 | PV_0 | PV_1] = 2*128 + 2*d <= 512.
+//
+// Softmax per tile (thread = row): pass 1 reads S (int32) and takes the integer max of
+// each 64-key half (the two K blocks carry different scales); pass 2 re-reads S,
+// p = 2^(S*sc - m) with one FFMA + ex2, sums p, packs P to f16 (or E4M3 of 448 p) and
+// stores it over S in TMEM. The O update for tile j-1 (O = alpha O + PV) is done after
+// P of tile j is handed to the tensor core, so the softmax never waits on its own PV.
+//
+// Every wait is bounded (global timer); a timeout sets the device status word, all
+// roles drain and the CTA releases TMEM and exits. Nothing traps.
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <climits>
+#include <cstdio>
+#include <mutex>
+
+#include "sage_common.cuh"
+#include "sm100_ptx.cuh"
+
+namespace sage {
+
+namespace {
+
+constexpr uint64_t kTimeoutNs = 2000000000ull;   // 2 s: far above any legitimate wait
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLog2_448 = 8.807354922057604f;  // log2(448): E4M3 P = e4m3(448 p)
+
+template <int D, bool FP8, int NQT>
+struct Cfg {
+    static constexpr int BM = 128, BN = 128;
+    static constexpr int kQBytes = BM * D;                   // int8 Q tile
+    static constexpr int kKBytes = BN * D;                   // int8 K tile
+    static constexpr int kVBytes = BN * D * (FP8 ? 1 : 2);   // V tile
+    static constexpr int kStageBytes = kKBytes + kVBytes;
+    static constexpr int kBudget = 200 * 1024;
+    static constexpr int kStagesFit = (kBudget - NQT * kQBytes) / kStageBytes;
+    static constexpr int STAGES = kStagesFit > 4 ? 4 : kStagesFit;
+    static_assert(STAGES >= 2, "shared-memory ring too shallow");
+    static constexpr int kSoftmaxWarps = 4 * NQT;
+    static constexpr int kProducerWarp = kSoftmaxWarps;
+    static constexpr int kMmaWarp = kSoftmaxWarps + 1;
+    static constexpr int kThreads = (kSoftmaxWarps + 4) * 32;
+    static constexpr int kTmemNeed = NQT * (BN + D);
+    static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128 : kTmemNeed <= 256 ? 256 : 512;
+    static_assert(kTmemNeed <= 512, "TMEM budget exceeded");
+    // shared memory map (offsets from a 1024-byte aligned base)
+    static constexpr int kOffQ = 0;
+    static constexpr int kOffK = kOffQ + NQT * kQBytes;
+    static constexpr int kOffV = kOffK + STAGES * kKBytes;
+    static constexpr int kOffBar = kOffV + STAGES * kVBytes;
+    // barriers: q, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[NQT],
+    //           p_full[NQT], pv_full[NQT], pv_free[NQT], drain
+    static constexpr int kNumBars = 1 + 4 * STAGES + 4 * NQT + 1;
+    static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+    static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
+    // V operand geometry (MN-major): bytes per token row inside one swizzle chunk
+    static constexpr int kVElem = FP8 ? 1 : 2;
+    static constexpr int kVRowBytes = (D * kVElem) >= 128 ? 128 : D * kVElem;
+    static constexpr int kVChunks = (D * kVElem) / kVRowBytes;          // boxes per V tile
+    static constexpr int kVBoxBytes = BN * kVRowBytes;
+    static constexpr int kPvK = FP8 ? 32 : 16;                          // K per PV MMA
+    // Q/K operand geometry (K-major, one swizzle atom wide)
+    static constexpr int kQkSwizzle = D == 128 ? 2 : 4;                 // 128B / 64B
+    static constexpr int kQkSbo = 8 * D;                                 // 8 rows
+    static constexpr int kVSwizzle = kVRowBytes == 128 ? 2 : 4;
+    static constexpr int kVSbo = 8 * kVRowBytes;
+};
+
+struct KParams {
+    const float *q_scale;
+    const float *k_scale;
+    const float *v_scale;
+    __half *out;
+    int32_t *s_dump;
+    SeqLayout L;
+    int nqb, nkb;        // scale blocks per (sequence, head) row of the scale arrays
+    int causal;
+    float sc_log2;       // sm_scale * log2(e)
+    int *status;
+};
+
+__device__ __forceinline__ void tma_coords(const SeqLayout &L, int s, int start, int h, int row,
+                                           int &c1, int &c2)
+{
+    if (L.cu == nullptr) {
+        c1 = row;
+        c2 = s * L.H + h;
+    } else {
+        c1 = h;
+        c2 = start + row;
+    }
+}
+
+// Bit e set iff key e of a 32-key chunk is visible, given `n` visible keys from the
+// chunk start.
+__device__ __forceinline__ uint32_t chunk_mask(int n)
+{
+    return n >= 32 ? ~0u : (n <= 0 ? 0u : (1u << n) - 1u);
+}
+
+// Lane 0 waits, the result is broadcast so the warp stays converged for .sync.aligned ops.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                          int *status)
+{
+    bool ok = true;
+    if ((threadIdx.x & 31) == 0)
+        ok = mbar_wait(bar, parity, abort, status, status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs);
+    ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    __syncwarp();
+    return ok;
+}
+
+template <int D, bool FP8, int NQT, bool DUMP>
+__global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
+    attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                const __grid_constant__ CUtensorMap tmV, const KParams p)
+{
+    using C = Cfg<D, FP8, NQT>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_addr = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
+
+    const SeqLayout &L = p.L;
+    const int s = blockIdx.z, h = blockIdx.y;
+    int start, len;
+    if (!L.range(s, start, len, p.status))
+        return;
+    const int cta_x = p.causal ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
+    const int qt0 = cta_x * NQT;
+    if (qt0 * C::BM >= len)
+        return;                                    // whole CTA beyond this sequence
+    const int last_row = min(len, (qt0 + NQT) * C::BM) - 1;
+    const int nkv = p.causal ? last_row / C::BN + 1 : (len + C::BN - 1) / C::BN;
+
+    uint8_t *sQ = smem + C::kOffQ;
+    uint8_t *sK = smem + C::kOffK;
+    uint8_t *sV = smem + C::kOffV;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
+    uint64_t *bar_q = bars;
+    uint64_t *k_full = bars + 1;
+    uint64_t *k_empty = k_full + C::STAGES;
+    uint64_t *v_full = k_empty + C::STAGES;
+    uint64_t *v_empty = v_full + C::STAGES;
+    uint64_t *s_full = v_empty + C::STAGES;
+    uint64_t *p_full = s_full + NQT;
+    uint64_t *pv_full = p_full + NQT;
+    uint64_t *pv_free = pv_full + NQT;
+    uint64_t *bar_drain = pv_free + NQT;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffMisc);
+    volatile int *abort = reinterpret_cast<volatile int *>(smem + C::kOffMisc + 4);
+
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (threadIdx.x == 0) {
+        mbar_init(bar_q, 1);
+        for (int i = 0; i < C::STAGES; i++) {
+            mbar_init(&k_full[i], 1);
+            mbar_init(&k_empty[i], 1);
+            mbar_init(&v_full[i], 1);
+            mbar_init(&v_empty[i], 1);
+        }
+        for (int i = 0; i < NQT; i++) {
+            mbar_init(&s_full[i], 1);
+            mbar_init(&p_full[i], 4);
+            mbar_init(&pv_full[i], 1);
+            mbar_init(&pv_free[i], 4);
+        }
+        mbar_init(bar_drain, 1);
+        *abort = 0;
+        fence_barrier_init();
+    }
+    if (warp == C::kMmaWarp)
+        tmem_alloc(tmem_slot, C::kTmemCols);
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    if (warp < C::kSoftmaxWarps) {
+        // ------------------------------------------------------------ softmax warps
+        if constexpr (NQT == 2)
+            asm volatile("setmaxnreg.inc.sync.aligned.u32 224;\n" ::: "memory");
+        const int i = warp / 4;                    // query tile within the CTA
+        const int quarter = warp % 4;              // TMEM lane quarter of this warp
+        const int qt = qt0 + i;
+        const int row_in_tile = quarter * 32 + lane;
+        const int qrow = qt * C::BM + row_in_tile;
+        const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+        const uint32_t tS = tmem_base + lane_off + i * C::BN;
+        const uint32_t tPV = tmem_base + lane_off + NQT * C::BN + i * D;
+        const int64_t sh = (int64_t)s * L.H + h;
+        const bool tile_valid = qt * C::BM < len;
+        const float qsc = (tile_valid ? __ldg(p.q_scale + sh * p.nqb + qt) : 0.0f) * p.sc_log2;
+        const int kb_valid = (len + kKBlock - 1) / kKBlock;
+
+        float o[D];
+#pragma unroll
+        for (int c = 0; c < D; c++)
+            o[c] = 0.0f;
+        float m = -INFINITY, l = 0.0f, alpha_prev = 0.0f;
+        bool ok = true;
+
+        for (int j = 0; j < nkv && ok; j++) {
+            if (!(ok = warp_wait(&s_full[i], j & 1, abort, p.status)))
+                break;
+            tc_fence_after();
+            const int kb0 = 2 * j, kb1 = 2 * j + 1;
+            const float sc0 = qsc * (kb0 < kb_valid ? __ldg(p.k_scale + sh * p.nkb + kb0) : 0.0f);
+            const float sc1 = qsc * (kb1 < kb_valid ? __ldg(p.k_scale + sh * p.nkb + kb1) : 0.0f);
+            const int kcol0 = j * C::BN;
+            const bool need_mask =
+                (kcol0 + C::BN > len) || (p.causal && kcol0 + C::BN - 1 > qt * C::BM);
+            const int col_lim = p.causal ? min(len, qrow + 1) : len;   // keys < col_lim visible
+
+            // pass 1: integer maxima of the two 64-key halves
+            int im0 = INT_MIN, im1 = INT_MIN;
+#pragma unroll
+            for (int ch = 0; ch < 4; ch++) {
+                uint32_t r[32];
+                tmem_ld32(tS + ch * 32, r);
+                if constexpr (DUMP) {
+                    if (qrow < len) {
+                        int32_t *drow = p.s_dump + (sh * L.maxlen + qrow) * L.maxlen;
+                        for (int e = 0; e < 32; e++)
+                            if (kcol0 + ch * 32 + e < len)
+                                drow[kcol0 + ch * 32 + e] = static_cast<int>(r[e]);
+                    }
+                }
+                const uint32_t keep = need_mask ? chunk_mask(col_lim - kcol0 - ch * 32) : ~0u;
+                int mx = INT_MIN;
+#pragma unroll
+                for (int e = 0; e < 32; e++) {
+                    const int v = static_cast<int>(r[e]);
+                    mx = ((keep >> e) & 1u) ? max(mx, v) : mx;
+                }
+                if (ch < 2)
+                    im0 = max(im0, mx);
+                else
+                    im1 = max(im1, mx);
+            }
+            float tmax = -INFINITY;
+            if (im0 != INT_MIN)
+                tmax = static_cast<float>(im0) * sc0;
+            if (im1 != INT_MIN)
+                tmax = fmaxf(tmax, static_cast<float>(im1) * sc1);
+            const float m_new = fmaxf(m, tmax);
+            const float alpha = ex2_approx(m - m_new);
+            const float bias = FP8 ? m_new - kLog2_448 : m_new;
+
+            // pass 2: p = 2^(S sc - m), row sum, P packed over S in TMEM (16 keys at a
+            // time keeps the working set small next to the d registers of O)
+            float lsum = 0.0f;
+#pragma unroll
+            for (int ch = 0; ch < 8; ch++) {
+                uint32_t r[16];
+                tmem_ld16(tS + ch * 16, r);
+                const float sc = ch < 4 ? sc0 : sc1;
+                const uint32_t keep =
+                    need_mask ? chunk_mask(col_lim - kcol0 - ch * 16) & 0xffffu : 0xffffu;
+                float pe[16];
+#pragma unroll
+                for (int e = 0; e < 16; e++) {
+                    const float sf = static_cast<float>(static_cast<int>(r[e]));
+                    const float pv = ex2_approx(fmaf(sf, sc, -bias));
+                    pe[e] = ((keep >> e) & 1u) ? pv : 0.0f;
+                    lsum += pe[e];
+                }
+                if constexpr (!FP8) {
+                    uint32_t w[8];
+#pragma unroll
+                    for (int e = 0; e < 8; e++)
+                        w[e] = pack_half2(pe[2 * e], pe[2 * e + 1]);
+                    tmem_st8(tS + ch * 8, w);
+                } else {
+                    uint32_t w[4];
+#pragma unroll
+                    for (int e = 0; e < 4; e++)
+                        w[e] = static_cast<uint32_t>(pack_e4m3x2(pe[4 * e], pe[4 * e + 1])) |
+                               (static_cast<uint32_t>(pack_e4m3x2(pe[4 * e + 2], pe[4 * e + 3]))
+                                << 16);
+                    tmem_st4(tS + ch * 4, w);
+                }
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&p_full[i]);
+            l = alpha * l + lsum;
+            m = m_new;
+
+            // O update for the previous tile (its PV has had a whole softmax to finish)
+            if (j > 0) {
+                if (!(ok = warp_wait(&pv_full[i], (j - 1) & 1, abort, p.status)))
+                    break;
+                tc_fence_after();
+#pragma unroll
+                for (int ch = 0; ch < D / 32; ch++) {
+                    uint32_t r[32];
+                    tmem_ld32(tPV + ch * 32, r);
+#pragma unroll
+                    for (int e = 0; e < 32; e++)
+                        o[ch * 32 + e] = fmaf(alpha_prev, o[ch * 32 + e], __uint_as_float(r[e]));
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    mbar_arrive(&pv_free[i]);
+            }
+            alpha_prev = alpha;
+        }
+        if (ok && (ok = warp_wait(&pv_full[i], (nkv - 1) & 1, abort, p.status))) {
+            tc_fence_after();
+#pragma unroll
+            for (int ch = 0; ch < D / 32; ch++) {
+                uint32_t r[32];
+                tmem_ld32(tPV + ch * 32, r);
+#pragma unroll
+                for (int e = 0; e < 32; e++)
+                    o[ch * 32 + e] = fmaf(alpha_prev, o[ch * 32 + e], __uint_as_float(r[e]));
+            }
+        }
+        // epilogue: normalize, round to fp16, store the row
+        if (ok && qrow < len) {
+            const float inv_l = 1.0f / l;
+            __half *dst = p.out + L.offset(s, start, h, qrow);
+#pragma unroll
+            for (int c = 0; c < D; c += 8) {
+                float f[8];
+#pragma unroll
+                for (int e = 0; e < 8; e++) {
+                    float sc = inv_l;
+                    if constexpr (FP8)
+                        sc = __ldg(p.v_scale + sh * D + c + e) * inv_l;
+                    f[e] = o[c + e] * sc;
+                }
+                uint4 u;
+                u.x = pack_half2(f[0], f[1]);
+                u.y = pack_half2(f[2], f[3]);
+                u.z = pack_half2(f[4], f[5]);
+                u.w = pack_half2(f[6], f[7]);
+                *reinterpret_cast<uint4 *>(dst + c) = u;
+            }
+        }
+    } else if (warp == C::kProducerWarp) {
+        // ----------------------------------------------------------------- producer
+        if constexpr (NQT == 2)
+            asm volatile("setmaxnreg.dec.sync.aligned.u32 56;\n" ::: "memory");
+        if (lane == 0) {
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmV);
+            int c1, c2;
+            mbar_arrive_expect_tx(bar_q, NQT * C::kQBytes);
+            for (int i = 0; i < NQT; i++) {
+                tma_coords(L, s, start, h, (qt0 + i) * C::BM, c1, c2);
+                tma_load_3d(sQ + i * C::kQBytes, &tmQ, bar_q, 0, c1, c2);
+            }
+            int issued = 0;
+            for (int j = 0; j < nkv; j++) {
+                const int stg = j % C::STAGES;
+                const uint32_t ph = (j / C::STAGES) & 1;
+                tma_coords(L, s, start, h, j * C::BN, c1, c2);
+                if (!mbar_wait(&k_empty[stg], ph ^ 1, abort, p.status,
+                               status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs))
+                    break;
+                mbar_arrive_expect_tx(&k_full[stg], C::kKBytes);
+                tma_load_3d(sK + stg * C::kKBytes, &tmK, &k_full[stg], 0, c1, c2);
+                if (!mbar_wait(&v_empty[stg], ph ^ 1, abort, p.status,
+                               status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs)) {
+                    issued = j + 1;   // the K load of this tile is in flight
+                    break;
+                }
+                mbar_arrive_expect_tx(&v_full[stg], C::kVBytes);
+#pragma unroll
+                for (int cb = 0; cb < C::kVChunks; cb++)
+                    tma_load_3d(sV + stg * C::kVBytes + cb * C::kVBoxBytes, &tmV, &v_full[stg],
+                                cb * (C::kVRowBytes / C::kVElem), c1, c2);
+                issued = j + 1;
+            }
+            // drain: make sure no copy is still landing in shared memory when we leave
+            mbar_wait(bar_q, 0, nullptr, p.status, status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs);
+            for (int j = max(0, issued - C::STAGES); j < issued; j++) {
+                const int stg = j % C::STAGES;
+                const uint32_t ph = (j / C::STAGES) & 1;
+                mbar_wait(&k_full[stg], ph, nullptr, p.status, status_bit(SAGE_ERR_TIMEOUT),
+                          kTimeoutNs);
+                mbar_wait(&v_full[stg], ph, nullptr, p.status, status_bit(SAGE_ERR_TIMEOUT),
+                          kTimeoutNs);
+            }
+        }
+    } else if (warp == C::kMmaWarp) {
+        // ---------------------------------------------------------------- MMA issuer
+        if constexpr (NQT == 2)
+            asm volatile("setmaxnreg.dec.sync.aligned.u32 56;\n" ::: "memory");
+        if (lane == 0) {
+            constexpr uint32_t idesc_qk = instr_desc(2 /*s32*/, 1 /*s8*/, 1 /*s8*/, 0, 0, 128, 128);
+            constexpr uint32_t idesc_pv = instr_desc(1 /*f32*/, 0 /*f16|e4m3*/, 0, 0,
+                                                     1 /*V MN-major*/, 128, D);
+            // descriptors are built once; a tile/k-step offset is added to the start
+            // address field (bits 0-13, 16-byte units; shared addresses stay < 2^18)
+            const uint64_t dQ0 = smem_desc(smem_u32(sQ), 16, C::kQkSbo, C::kQkSwizzle);
+            const uint64_t dK0 = smem_desc(smem_u32(sK), 16, C::kQkSbo, C::kQkSwizzle);
+            const uint64_t dV0 = smem_desc(smem_u32(sV), C::kVBoxBytes, C::kVSbo, C::kVSwizzle);
+            bool ok = mbar_wait(bar_q, 0, abort, p.status, status_bit(SAGE_ERR_TIMEOUT),
+                                kTimeoutNs);
+            for (int j = 0; j < nkv && ok; j++) {
+                const int stg = j % C::STAGES;
+                const uint32_t ph = (j / C::STAGES) & 1;
+                if (!(ok = mbar_wait(&k_full[stg], ph, abort, p.status,
+                                     status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs)))
+                    break;
+                for (int i = 0; i < NQT && ok; i++) {
+                    // S_i is overwritten: P_i of the previous tile must have been consumed
+                    if (j > 0 && !(ok = mbar_wait(&pv_full[i], (j - 1) & 1, abort, p.status,
+                                                  status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs)))
+                        break;
+                    tc_fence_after();
+                    const uint32_t dS = tmem_base + i * C::BN;
+#pragma unroll
+                    for (int kk = 0; kk < D / 32; kk++) {
+                        const uint64_t a = dQ0 + ((i * C::kQBytes + kk * 32) >> 4);
+                        const uint64_t b = dK0 + ((stg * C::kKBytes + kk * 32) >> 4);
+                        mma_i8_ss(dS, a, b, idesc_qk, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&s_full[i]);
+                }
+                if (!ok)
+                    break;
+                mma_commit(&k_empty[stg]);
+                if (!(ok = mbar_wait(&v_full[stg], ph, abort, p.status,
+                                     status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs)))
+                    break;
+                for (int i = 0; i < NQT && ok; i++) {
+                    if (!(ok = mbar_wait(&p_full[i], j & 1, abort, p.status,
+                                         status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs)))
+                        break;
+                    if (j > 0 && !(ok = mbar_wait(&pv_free[i], (j - 1) & 1, abort, p.status,
+                                                  status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs)))
+                        break;
+                    tc_fence_after();
+                    const uint32_t dPV = tmem_base + NQT * C::BN + i * D;
+                    const uint32_t aP = tmem_base + i * C::BN;
+#pragma unroll
+                    for (int kk = 0; kk < C::BN / C::kPvK; kk++) {
+                        const uint64_t b =
+                            dV0 + ((stg * C::kVBytes + kk * C::kPvK * C::kVRowBytes) >> 4);
+                        if constexpr (FP8)
+                            mma_f8_ts(dPV, aP + kk * 8, b, idesc_pv, kk > 0 ? 1u : 0u);
+                        else
+                            mma_f16_ts(dPV, aP + kk * 8, b, idesc_pv, kk > 0 ? 1u : 0u);
+                    }
+                    mma_commit(&pv_full[i]);
+                }
+                if (!ok)
+                    break;
+                mma_commit(&v_empty[stg]);
+            }
+            // drain: every MMA issued above has completed before TMEM is released
+            mma_commit(bar_drain);
+            mbar_wait(bar_drain, 0, nullptr, p.status, status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs);
+        }
+    } else {
+        if constexpr (NQT == 2)
+            asm volatile("setmaxnreg.dec.sync.aligned.u32 56;\n" ::: "memory");
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == C::kMmaWarp) {
+        __syncwarp();
+        tmem_dealloc(tmem_base, C::kTmemCols);
+    }
+}
+
+// ----------------------------------------------------------------- host side
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000,
+                                             cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    });
+    return fn;
+}
+
+// 3-D map over the tensor [.., .., d] seen as (d, rows, heads) for the dense layout or
+// (d, H, T) for the packed layout; a box is one tile of `box_rows` tokens of one head.
+bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int elem_bytes,
+              const SeqLayout &L, int box_inner, int box_rows, CUtensorMapSwizzle swz)
+{
+    auto enc = get_encode();
+    if (!enc)
+        return false;
+    cuuint64_t dims[3];
+    cuuint64_t strides[2];
+    cuuint32_t box[3];
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (L.cu == nullptr) {
+        dims[0] = L.d;
+        dims[1] = L.maxlen;
+        dims[2] = (cuuint64_t)L.nseq * L.H;
+        strides[0] = (cuuint64_t)L.d * elem_bytes;
+        strides[1] = (cuuint64_t)L.maxlen * L.d * elem_bytes;
+        box[0] = box_inner;
+        box[1] = box_rows;
+        box[2] = 1;
+    } else {
+        dims[0] = L.d;
+        dims[1] = L.H;
+        dims[2] = L.total;
+        strides[0] = (cuuint64_t)L.d * elem_bytes;
+        strides[1] = (cuuint64_t)L.H * L.d * elem_bytes;
+        box[0] = box_inner;
+        box[1] = 1;
+        box[2] = box_rows;
+    }
+    CUresult r = enc(m, dt, 3, const_cast<void *>(base), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int D, bool FP8, int NQT, bool DUMP>
+cudaError_t run(const AttnArgs &a, const SeqLayout &L, int *status, cudaStream_t st,
+                sage_status_t *host_err)
+{
+    using C = Cfg<D, FP8, NQT>;
+    CUtensorMap mq, mk, mv;
+    const CUtensorMapSwizzle qk_swz =
+        D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    const CUtensorMapSwizzle v_swz =
+        C::kVRowBytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    bool ok = make_map(&mq, a.q_i8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L, D, C::BM, qk_swz) &&
+              make_map(&mk, a.k_i8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L, D, C::BN, qk_swz) &&
+              make_map(&mv, a.v,
+                       FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
+                       C::kVElem, L, C::kVRowBytes / C::kVElem, C::BN, v_swz);
+    if (!ok) {
+        *host_err = SAGE_ERR_CUDA;
+        return cudaErrorInvalidValue;
+    }
+    KParams p;
+    p.q_scale = a.q_scale;
+    p.k_scale = a.k_scale;
+    p.v_scale = a.v_scale;
+    p.out = a.out;
+    p.s_dump = a.s_dump;
+    p.L = L;
+    p.nqb = (L.maxlen + kQBlock - 1) / kQBlock;
+    p.nkb = (L.maxlen + kKBlock - 1) / kKBlock;
+    p.causal = a.causal;
+    p.sc_log2 = a.sm_scale * kLog2e;
+    p.status = status;
+
+    auto kern = attn_kernel<D, FP8, NQT, DUMP>;
+    cudaError_t e =
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+    if (e != cudaSuccess)
+        return e;
+    const int nqt = (L.maxlen + C::BM - 1) / C::BM;
+    dim3 grid((nqt + NQT - 1) / NQT, L.H, L.nseq);
+    kern<<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_attention(const AttnArgs &a, const SeqLayout &L, int *status, cudaStream_t st,
+                             sage_status_t *host_err)
+{
+    *host_err = SAGE_OK;
+    const bool fp8 = a.pv_mode == SAGE_PV_FP8;
+    if (a.s_dump != nullptr) {
+        if (L.d == 128)
+            return run<128, false, 2, true>(a, L, status, st, host_err);
+        return run<64, false, 2, true>(a, L, status, st, host_err);
+    }
+    if (L.d == 128)
+        return fp8 ? run<128, true, 2, false>(a, L, status, st, host_err)
+                   : run<128, false, 2, false>(a, L, status, st, host_err);
+    return fp8 ? run<64, true, 2, false>(a, L, status, st, host_err)
+               : run<64, false, 2, false>(a, L, status, st, host_err);
+}
+
+}  // namespace sage

@@ -1,0 +1,314 @@
+// K-QUANT: smooth K and per-block INT8 quantization of Q and K; E4M3 quantization of V.
+//
+// "SageAttention" article, section 技术方案: K <- K - mean(K) with the mean per channel
+// over tokens; Q and K quantized to INT8 per block of FlashAttention size (Q: 128
+// tokens, K: 64 tokens) with one fp32 scale amax/127 per block. "SageAttention2"
+// article, 技术方案 (4): V in E4M3, here with one fp32 scale (amax/448) per channel.
+//
+// Two HBM-bound passes:
+//   colstats: per-(sequence, head, channel) reductions over tokens: fp64 sums of K
+//             (exact for |K| N < 2^29, so the mean does not depend on summation order)
+//             and the fp32 amax of |V|. Row chunks of 512 tokens, fp64 atomics.
+//   quant:    one CTA per 128-token chunk of Q (one Q block), K (two K blocks) or V;
+//             16-byte vector loads/stores, warp-shuffle amax, IEEE-exact fp32 divisions
+//             (__fdiv_rn) and round-half-even so codes match the definition bit for bit.
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "sage_common.cuh"
+#include "sm100_ptx.cuh"
+
+namespace sage {
+
+namespace {
+
+constexpr int kColChunk = 512;   // tokens per colstats CTA
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8])
+{
+    const __half2 *h = reinterpret_cast<const __half2 *>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const float2 t = __half22float2(h[i]);
+        f[2 * i] = t.x;
+        f[2 * i + 1] = t.y;
+    }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) colstats_kernel(const __half *__restrict__ k,
+                                                            const __half *__restrict__ v,
+                                                            double *__restrict__ ksum,
+                                                            uint32_t *__restrict__ vamax,
+                                                            SeqLayout L, int *status)
+{
+    constexpr int kGroups = D / 8;              // 16-byte column groups per row
+    constexpr int kRowsPerPass = kThreads / kGroups;
+    const int s = blockIdx.z, h = blockIdx.y;
+    int start, len;
+    if (!L.range(s, start, len, status))
+        return;
+    const int r_begin = blockIdx.x * kColChunk;
+    if (r_begin >= len)
+        return;
+    const int r_end = min(len, r_begin + kColChunk);
+    const int g = threadIdx.x % kGroups, r0 = threadIdx.x / kGroups;
+
+    double acc[8];
+    float amx[8];
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        acc[i] = 0.0;
+        amx[i] = 0.0f;
+    }
+    for (int r = r_begin + r0; r < r_end; r += kRowsPerPass) {
+        const int64_t off = L.offset(s, start, h, r) + g * 8;
+        float f[8];
+        if (ksum != nullptr) {
+            unpack8(__ldg(reinterpret_cast<const uint4 *>(k + off)), f);
+#pragma unroll
+            for (int i = 0; i < 8; i++)
+                acc[i] += (double)f[i];
+        }
+        if (vamax != nullptr) {
+            unpack8(__ldg(reinterpret_cast<const uint4 *>(v + off)), f);
+#pragma unroll
+            for (int i = 0; i < 8; i++)
+                amx[i] = fmaxf(amx[i], fabsf(f[i]));
+        }
+    }
+
+    __shared__ double s_sum[kRowsPerPass][D];
+    __shared__ float s_max[kRowsPerPass][D];
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        s_sum[r0][g * 8 + i] = acc[i];
+        s_max[r0][g * 8 + i] = amx[i];
+    }
+    __syncthreads();
+    if (threadIdx.x < D) {
+        const int c = threadIdx.x;
+        double t = 0.0;
+        float m = 0.0f;
+        for (int r = 0; r < kRowsPerPass; r++) {
+            t += s_sum[r][c];
+            m = fmaxf(m, s_max[r][c]);
+        }
+        const int64_t o = ((int64_t)s * L.H + h) * D + c;
+        if (ksum != nullptr)
+            atomicAdd(ksum + o, t);
+        if (vamax != nullptr)
+            atomicMax(vamax + o, __float_as_uint(m));   // non-negative floats order as ints
+    }
+}
+
+// Block-wide max over `nthreads` consecutive threads starting at warp `w0`.
+template <int NWARPS>
+__device__ __forceinline__ float group_max(float x, float *s_red, int w0)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+        x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (lane == 0)
+        s_red[warp] = x;
+    __syncthreads();
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < NWARPS; i++)
+        m = fmaxf(m, s_red[w0 + i]);
+    return m;
+}
+
+__device__ __forceinline__ int8_t int8_code(float x, float s)
+{
+    if (s == 0.0f)
+        return 0;
+    int c = __float2int_rn(__fdiv_rn(x, s));   // round half to even of the fp32 quotient
+    c = max(-127, min(127, c));
+    return (int8_t)c;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads) quant_kernel(
+    const __half *__restrict__ q, const __half *__restrict__ k, const __half *__restrict__ v,
+    const double *__restrict__ ksum, const uint32_t *__restrict__ vamax, int8_t *__restrict__ q_i8,
+    float *__restrict__ q_scale, int8_t *__restrict__ k_i8, float *__restrict__ k_scale,
+    float *__restrict__ k_mean, uint8_t *__restrict__ v_e4m3, float *__restrict__ v_scale,
+    SeqLayout L, int nqb, int nkb, int part0, int *status)
+{
+    constexpr int kHalf = D / 2;          // elements per thread (two threads per token)
+    constexpr int kVec = kHalf / 8;       // 16-byte loads per thread
+    __shared__ float s_red[8];
+    __shared__ float s_aux[D];            // K mean or V scale per channel
+
+    const int s = blockIdx.z, h = blockIdx.y;
+    int start, len;
+    if (!L.range(s, start, len, status))
+        return;
+    const int64_t sh = (int64_t)s * L.H + h;
+    // 0: Q block, 1: K pair of blocks, 2: V chunk; grid.x spans consecutive parts
+    const int kind = part0 + (int)blockIdx.x / nqb;
+    const int chunk = (int)blockIdx.x % nqb;
+    const int row0 = chunk * kQBlock;
+    const int row = row0 + threadIdx.x / 2;
+    const int col0 = (threadIdx.x & 1) * kHalf;
+    const bool valid = row < len;
+
+    if (row0 >= len) {                    // padding block of a short sequence
+        if (kind == 1 && chunk == 0 && threadIdx.x < D)
+            k_mean[sh * D + threadIdx.x] = 0.0f;
+        if (threadIdx.x == 0) {
+            if (kind == 0)
+                q_scale[sh * nqb + chunk] = 0.0f;
+            if (kind == 1) {
+                if (2 * chunk < nkb)
+                    k_scale[sh * nkb + 2 * chunk] = 0.0f;
+                if (2 * chunk + 1 < nkb)
+                    k_scale[sh * nkb + 2 * chunk + 1] = 0.0f;
+            }
+        }
+        return;
+    }
+
+    if (kind == 1 && threadIdx.x < D) {
+        const int c = threadIdx.x;
+        const float mu = ksum ? (float)(ksum[sh * D + c] / (double)len) : 0.0f;
+        s_aux[c] = mu;
+        if (chunk == 0)
+            k_mean[sh * D + c] = mu;
+    }
+    if (kind == 2 && threadIdx.x < D) {
+        const int c = threadIdx.x;
+        const float sv = __fdiv_rn(__uint_as_float(vamax[sh * D + c]), 448.0f);
+        s_aux[c] = sv;
+        if (chunk == 0)
+            v_scale[sh * D + c] = sv;
+    }
+    __syncthreads();
+
+    const int64_t off = L.offset(s, start, h, row) + col0;
+    const __half *src = kind == 0 ? q : (kind == 1 ? k : v);
+    float x[kHalf];
+#pragma unroll
+    for (int i = 0; i < kVec; i++) {
+        float f[8];
+        if (valid)
+            unpack8(__ldg(reinterpret_cast<const uint4 *>(src + off) + i), f);
+        else
+#pragma unroll
+            for (int e = 0; e < 8; e++)
+                f[e] = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 8; e++)
+            x[i * 8 + e] = f[e];
+    }
+
+    if (kind == 2) {
+        // E4M3 codes with the per-channel scale
+        if (!valid)
+            return;
+        uint32_t w[kHalf / 4];
+#pragma unroll
+        for (int i = 0; i < kHalf; i += 4) {
+            float qv[4];
+#pragma unroll
+            for (int e = 0; e < 4; e++) {
+                const float sv = s_aux[col0 + i + e];
+                qv[e] = sv != 0.0f ? __fdiv_rn(x[i + e], sv) : 0.0f;
+            }
+            const uint32_t lo = pack_e4m3x2(qv[0], qv[1]);
+            const uint32_t hi = pack_e4m3x2(qv[2], qv[3]);
+            w[i / 4] = lo | (hi << 16);
+        }
+        uint4 *dst = reinterpret_cast<uint4 *>(v_e4m3 + off);
+#pragma unroll
+        for (int i = 0; i < kHalf / 16; i++)
+            dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        return;
+    }
+
+    float amax = 0.0f;
+    if (kind == 1) {
+#pragma unroll
+        for (int i = 0; i < kHalf; i++)
+            x[i] = __fsub_rn(x[i], s_aux[col0 + i]);
+    }
+    if (valid) {
+#pragma unroll
+        for (int i = 0; i < kHalf; i++)
+            amax = fmaxf(amax, fabsf(x[i]));
+    }
+
+    float scale;
+    if (kind == 0) {
+        scale = __fdiv_rn(group_max<8>(amax, s_red, 0), 127.0f);
+        if (threadIdx.x == 0)
+            q_scale[sh * nqb + chunk] = scale;
+    } else {
+        const int half_blk = threadIdx.x / 128;    // 64-token K block within the chunk
+        scale = __fdiv_rn(group_max<4>(amax, s_red, half_blk * 4), 127.0f);
+        const int kb = 2 * chunk + half_blk;
+        if ((threadIdx.x & 127) == 0 && kb < nkb)
+            k_scale[sh * nkb + kb] = scale;
+    }
+    if (!valid)
+        return;
+
+    uint32_t w[kHalf / 4];
+#pragma unroll
+    for (int i = 0; i < kHalf; i += 4) {
+        const uint32_t b0 = (uint8_t)int8_code(x[i], scale);
+        const uint32_t b1 = (uint8_t)int8_code(x[i + 1], scale);
+        const uint32_t b2 = (uint8_t)int8_code(x[i + 2], scale);
+        const uint32_t b3 = (uint8_t)int8_code(x[i + 3], scale);
+        w[i / 4] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+    }
+    int8_t *dst8 = (kind == 0 ? q_i8 : k_i8) + off;
+    uint4 *dst = reinterpret_cast<uint4 *>(dst8);
+#pragma unroll
+    for (int i = 0; i < kHalf / 16; i++)
+        dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+}
+
+}  // namespace
+
+cudaError_t launch_colstats(const __half *k, const __half *v, double *ksum, uint32_t *vamax,
+                            const SeqLayout &L, int *status, cudaStream_t st)
+{
+    if (ksum == nullptr && vamax == nullptr)
+        return cudaSuccess;
+    dim3 grid((L.maxlen + kColChunk - 1) / kColChunk, L.H, L.nseq);
+    if (L.d == 128)
+        colstats_kernel<128><<<grid, kThreads, 0, st>>>(k, v, ksum, vamax, L, status);
+    else
+        colstats_kernel<64><<<grid, kThreads, 0, st>>>(k, v, ksum, vamax, L, status);
+    return cudaGetLastError();
+}
+
+// Quantizes Q and K (q_i8 != nullptr) and/or V (v_e4m3 != nullptr) in one launch.
+cudaError_t launch_quant(const __half *q, const __half *k, const __half *v, const double *ksum,
+                         const uint32_t *vamax, int8_t *q_i8, float *q_scale, int8_t *k_i8,
+                         float *k_scale, float *k_mean, uint8_t *v_e4m3, float *v_scale,
+                         const SeqLayout &L, int *status, cudaStream_t st)
+{
+    const int nqb = (L.maxlen + kQBlock - 1) / kQBlock;
+    const int nkb = (L.maxlen + kKBlock - 1) / kKBlock;
+    const int part0 = q_i8 != nullptr ? 0 : 2;
+    const int part1 = v_e4m3 != nullptr ? 3 : 2;
+    if (part1 <= part0)
+        return cudaSuccess;
+    dim3 grid(nqb * (part1 - part0), L.H, L.nseq);
+    if (L.d == 128)
+        quant_kernel<128><<<grid, kThreads, 0, st>>>(q, k, v, ksum, vamax, q_i8, q_scale, k_i8,
+                                                     k_scale, k_mean, v_e4m3, v_scale, L, nqb,
+                                                     nkb, part0, status);
+    else
+        quant_kernel<64><<<grid, kThreads, 0, st>>>(q, k, v, ksum, vamax, q_i8, q_scale, k_i8,
+                                                    k_scale, k_mean, v_e4m3, v_scale, L, nqb,
+                                                    nkb, part0, status);
+    return cudaGetLastError();
+}
+
+}  // namespace sage

@@ -1,0 +1,91 @@
+// Shared definitions of the CUDA library: sequence layouts, status codes, launch helpers.
+#pragma once
+#include <cstdint>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+
+#include "../../include/sage.h"
+
+namespace sage {
+
+constexpr int kQBlock = 128;   // Q tokens per INT8 scale block (= the attention Q tile)
+constexpr int kKBlock = 64;    // K tokens per INT8 scale block
+constexpr int kKvTile = 128;   // keys per attention KV tile (two K blocks)
+
+// Where the tokens of one (sequence, head) live. Dense [B,H,N,d]: cu == nullptr,
+// nseq = B, maxlen = N. Packed [T,H,d]: cu = device cu_seqlens, maxlen bounds lengths.
+struct SeqLayout {
+    const int32_t *cu;
+    int nseq, H, d;
+    int maxlen;
+    int total;          // total tokens (dense: B*N)
+    int64_t tok_stride; // elements between consecutive tokens of one head
+    int64_t head_stride;
+
+    __host__ static SeqLayout dense(int B, int H, int N, int d)
+    {
+        return SeqLayout{nullptr, B, H, d, N, B * N, (int64_t)d, (int64_t)N * d};
+    }
+    __host__ static SeqLayout packed(const int32_t *cu, int nseq, int total, int maxlen, int H,
+                                     int d)
+    {
+        return SeqLayout{cu, nseq, H, d, maxlen, total, (int64_t)H * d, (int64_t)d};
+    }
+
+    // Token range of sequence s; false (and a status bit) if cu_seqlens is malformed.
+    __device__ bool range(int s, int &start, int &len, int *status) const
+    {
+        if (cu == nullptr) {
+            start = s * maxlen;
+            len = maxlen;
+            return true;
+        }
+        const int a = __ldg(cu + s), b = __ldg(cu + s + 1);
+        if (a < 0 || b < a || b > total || b - a > maxlen || (s == 0 && a != 0)) {
+            atomicOr(status, 1 << SAGE_ERR_BAD_SEQLENS);
+            start = 0;
+            len = 0;
+            return false;
+        }
+        start = a;
+        len = b - a;
+        return true;
+    }
+
+    // Element offset of token `row` of head h of the sequence starting at token `start`.
+    __device__ __host__ int64_t offset(int s, int start, int h, int64_t row) const
+    {
+        if (cu == nullptr)
+            return ((int64_t)s * H + h) * maxlen * d + row * d;
+        return ((int64_t)start + row) * H * d + (int64_t)h * d;
+    }
+};
+
+// Device status bits are 1 << sage_status_t; the host reports the lowest set.
+__host__ __device__ constexpr int status_bit(sage_status_t s) { return 1 << (int)s; }
+
+// Launchers (quant.cu, attn_sm100.cu). All return cudaSuccess or the launch error.
+cudaError_t launch_colstats(const __half *k, const __half *v, double *ksum, uint32_t *vamax,
+                            const SeqLayout &L, int *status, cudaStream_t st);
+cudaError_t launch_quant(const __half *q, const __half *k, const __half *v, const double *ksum,
+                         const uint32_t *vamax, int8_t *q_i8, float *q_scale, int8_t *k_i8,
+                         float *k_scale, float *k_mean, uint8_t *v_e4m3, float *v_scale,
+                         const SeqLayout &L, int *status, cudaStream_t st);
+
+struct AttnArgs {
+    const int8_t *q_i8;
+    const float *q_scale;
+    const int8_t *k_i8;
+    const float *k_scale;
+    const void *v;        // fp16 V or E4M3 codes
+    const float *v_scale; // FP8 mode
+    __half *out;
+    int32_t *s_dump;      // debug: int32 scores [nseq,H,maxlen,maxlen] or nullptr
+    int causal;
+    int pv_mode;
+    float sm_scale;
+};
+cudaError_t launch_attention(const AttnArgs &a, const SeqLayout &L, int *status, cudaStream_t st,
+                             sage_status_t *host_err);
+
+}  // namespace sage

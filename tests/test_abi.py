@@ -1,0 +1,98 @@
+"""The C-ABI library: it loads, exports every symbol include/sage.h declares, and rejects
+bad arguments on the host before anything is enqueued (no GPU needed: these calls return
+before any CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import quantized_attention_03_b200 as sage
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sage.h")
+
+
+def _declared():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"SAGE_API\s+[\w\s\*]*?\b(sage_\w+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from quantized_attention_03_b200 import build
+    build.build()
+    return sage.lib()
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("sage_quant_qk", "sage_attn_fwd", "sage_attn_varlen_fwd", "sage_get_device_status"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+        assert name in sage.SIGNATURES, f"binding lacks {name}"
+        assert callable(getattr(sage, name)), name
+
+
+def test_status_strings(lib):
+    assert sage.status_string(0) == "SAGE_OK"
+    assert sage.status_string(6) == "SAGE_ERR_TIMEOUT"
+    assert sage.sage_version() >= 100
+
+
+FAKE = 0x10000          # 16-byte aligned, never dereferenced: validation fails first
+MIS = 0x10008           # 8-byte aligned only
+
+
+def _fwd(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, B=1, H=1, N=128, d=64, pv=0):
+    return lib.sage_attn_fwd(q, k, v, o, B, H, N, d, 0, 1, pv, 0.0, None)
+
+
+def test_host_validation(lib):
+    assert _fwd(lib, d=96) == sage.SAGE_ERR_UNSUPPORTED
+    assert _fwd(lib, d=256) == sage.SAGE_ERR_UNSUPPORTED
+    assert _fwd(lib, N=-1) == sage.SAGE_ERR_INVALID_ARG
+    assert _fwd(lib, pv=2) == sage.SAGE_ERR_INVALID_ARG
+    assert _fwd(lib, q=0) == sage.SAGE_ERR_INVALID_ARG
+    assert _fwd(lib, v=MIS) == sage.SAGE_ERR_MISALIGNED
+    assert _fwd(lib, o=MIS) == sage.SAGE_ERR_MISALIGNED
+    assert _fwd(lib, H=70000) == sage.SAGE_ERR_UNSUPPORTED
+
+
+def test_empty_inputs_are_noops(lib):
+    assert _fwd(lib, B=0) == sage.SAGE_OK
+    assert _fwd(lib, N=0) == sage.SAGE_OK
+    assert _fwd(lib, q=0, B=0) == sage.SAGE_OK
+    assert lib.sage_quant_qk(0, 0, 0, 0, 0, 0, 0, 0, 4, 128, 64, 1, None) == sage.SAGE_OK
+
+
+def test_workspace_checks(lib):
+    need = lib.sage_workspace_size(2, 4, 300, 600, 128, 0)
+    need8 = lib.sage_workspace_size(2, 4, 300, 600, 128, 1)
+    # Q and K codes (one byte per element each) plus scales, means and fp64 sums
+    assert need >= 2 * 600 * 4 * 128 and need8 >= need + 600 * 4 * 128
+    rc = lib.sage_attn_fwd_ws(FAKE, FAKE, FAKE, FAKE, 2, 4, 300, 128, 0, 1, 0, 0.0, FAKE,
+                              need - 1, None)
+    assert rc == sage.SAGE_ERR_WORKSPACE
+    rc = lib.sage_attn_fwd_ws(FAKE, FAKE, FAKE, FAKE, 2, 4, 300, 128, 0, 1, 0, 0.0, 0, 0, None)
+    assert rc == sage.SAGE_ERR_WORKSPACE
+    rc = lib.sage_attn_fwd_ws(FAKE, FAKE, FAKE, FAKE, 2, 4, 300, 128, 0, 1, 0, 0.0, FAKE + 16,
+                              need, None)
+    assert rc == sage.SAGE_ERR_MISALIGNED       # scratch must be 256-byte aligned
+
+
+def test_varlen_requires_cu_seqlens(lib):
+    rc = lib.sage_attn_varlen_fwd(FAKE, FAKE, FAKE, FAKE, 0, 2, 100, 60, 4, 64, 1, 1, 0, 0.0,
+                                  0, 0, None)
+    assert rc == sage.SAGE_ERR_INVALID_ARG
+
+
+def test_missing_library_fails_loudly(monkeypatch, tmp_path):
+    monkeypatch.setattr(sage, "LIB_PATH", str(tmp_path / "absent.so"))
+    monkeypatch.setattr(sage, "_lib", None)
+    with pytest.raises(RuntimeError, match="no fallback"):
+        sage.lib()

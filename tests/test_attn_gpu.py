@@ -1,0 +1,200 @@
+"""GPU attention (K-ATTN and the fused entry points) vs the oracle, through the C ABI.
+
+* Integer score tiles S = Q_i8 K_i8^T from the tensor-core pass are compared bit for bit
+  with a library int64 matmul of the same codes.
+* Outputs are compared with the quantized oracle (cosine >= 0.9999, max |err| <= 1e-2)
+  and with exact fp64 attention (cosine >= 0.999, relative L1 <= 0.02 in FP16 mode).
+* Small shapes span several tiles and ragged tails and are compared element by element
+  everywhere; the full-size workloads, run in the benchmark's launch configuration, are
+  compared on sampled heads and row ranges the oracle computes one by one.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import quantized_attention_03_b200 as sage
+from quantized_attention_03_b200 import inputs
+from helpers import assert_vs_fp64, assert_vs_oracle, rel_l1
+
+pytestmark = pytest.mark.gpu
+
+PV = {"fp16": sage.SAGE_PV_FP16, "fp8": sage.SAGE_PV_FP8}
+
+
+def _np(t):
+    return t.detach().cpu().numpy()
+
+
+def _run_dense(q, k, v, causal, pv, smooth=True):
+    out = sage.sageattn(q.cuda(), k.cuda(), v.cuda(), causal, smooth, PV[pv])
+    status = sage.sage_get_device_status()
+    assert status == 0, sage.status_string(status)
+    return _np(out)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("N", [64, 300, 513])
+def test_qk_int32_tiles_bit_exact(N, d):
+    w = inputs.Workload("t", 100 + N, 1, 2, N, d, False, 2.0)
+    q, k, _ = inputs.make_dense(w)
+    z = sage.quant_qk(q.cuda(), k.cuda(), True)
+    s = _np(sage.qk_int32(z["q_i8"], z["k_i8"]))
+    assert sage.sage_get_device_status() == 0
+    qc = _np(z["q_i8"]).astype(np.int64)
+    kc = _np(z["k_i8"]).astype(np.int64)
+    ref = np.einsum("bhnc,bhmc->bhnm", qc, kc)
+    assert np.array_equal(s.astype(np.int64), ref)
+
+
+SMALL = [
+    # N, d, causal
+    (1, 64, False), (1, 128, True), (17, 64, True), (128, 128, False), (129, 64, False),
+    (256, 64, False), (300, 128, True), (513, 128, False), (640, 64, True), (1000, 128, True),
+]
+
+
+@pytest.mark.parametrize("pv", ["fp16", "fp8"])
+@pytest.mark.parametrize("N,d,causal", SMALL)
+def test_attention_small_full_compare(N, d, causal, pv):
+    B, H = 1, 2
+    w = inputs.Workload("t", 200 + N + d, B, H, N, d, causal, 2.0)
+    q, k, v = inputs.make_dense(w)
+    got = _run_dense(q, k, v, causal, pv)
+    lay = oracle.Layout.dense(B, H, N, d)
+    ref = oracle.sage_attention(q.numpy(), k.numpy(), v.numpy(), lay, causal, True, PV[pv])
+    assert_vs_oracle(got, ref, f"N={N} d={d} causal={causal} {pv}")
+    exact = oracle.attn_fp64(q.numpy(), k.numpy(), v.numpy(), lay, causal, 1 / math.sqrt(d))
+    assert_vs_fp64(got, exact, pv == "fp8", f"N={N} d={d} causal={causal} {pv}")
+
+
+def test_tiny_config_both_smoothing_modes():
+    w = inputs.tiny()
+    q, k, v = inputs.make_dense(w)
+    lay = oracle.Layout.dense(w.B, w.H, w.N, w.d)
+    for smooth in (True, False):
+        got = _run_dense(q, k, v, False, "fp16", smooth)
+        ref = oracle.sage_attention(q.numpy(), k.numpy(), v.numpy(), lay, False, smooth)
+        assert_vs_oracle(got, ref, f"tiny smooth={smooth}")
+
+
+def test_quantized_entry_matches_fused():
+    B, H, N, d = 2, 2, 384, 128
+    w = inputs.Workload("t", 31, B, H, N, d, True, 1.0)
+    q, k, v = inputs.make_dense(w)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    fused = sage.sageattn(qd, kd, vd, True, True, sage.SAGE_PV_FP16)
+    z = sage.quant_qk(qd, kd, True)
+    split = sage.attn_quantized(z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], vd, None, True)
+    codes, scales = sage.quant_v_fp8(vd)
+    fused8 = sage.sageattn(qd, kd, vd, True, True, sage.SAGE_PV_FP8)
+    split8 = sage.attn_quantized(z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], codes, scales,
+                                 True, sage.SAGE_PV_FP8)
+    assert sage.sage_get_device_status() == 0
+    assert torch.equal(fused, split) and torch.equal(fused8, split8)
+
+
+def test_workspace_entry_matches_fused():
+    B, H, N, d = 1, 4, 700, 64
+    w = inputs.Workload("t", 41, B, H, N, d, False, 1.0)
+    q, k, v = (t.cuda() for t in inputs.make_dense(w))
+    ref = sage.sageattn(q, k, v)
+    need = sage.sage_workspace_size(B, H, N, B * N, d, 0)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(q)
+    sage.sage_attn_fwd_ws(q, k, v, out, B, H, N, d, 0, 1, 0, 0.0, ws, need)
+    assert sage.sage_get_device_status() == 0
+    assert torch.equal(out, ref)
+
+
+@pytest.mark.parametrize("pv", ["fp16", "fp8"])
+def test_varlen_small_full_compare(pv):
+    H, d = 4, 128
+    lens = [1, 200, 128, 129, 700, 64, 0, 333]
+    w = inputs.Workload("t", 51, 0, H, 0, d, True, 2.0, nseq=len(lens))
+    q, k, v, cu = inputs.make_varlen(w, lens=lens)
+    out = sage.sageattn_varlen(q.cuda(), k.cuda(), v.cuda(), cu.cuda(), max(lens), True, True,
+                               PV[pv])
+    assert sage.sage_get_device_status() == 0
+    got = _np(out)
+    lay = oracle.Layout.packed(cu.tolist(), H, d)
+    ref = oracle.sage_attention(q.numpy(), k.numpy(), v.numpy(), lay, True, True, PV[pv])
+    assert_vs_oracle(got, ref, f"varlen {pv}")
+    exact = oracle.attn_fp64(q.numpy(), k.numpy(), v.numpy(), lay, True, 1 / math.sqrt(d))
+    assert_vs_fp64(got, exact, pv == "fp8", f"varlen {pv}")
+
+
+# --------------------------------------------------- full-size workloads, sampled rows
+
+
+def _sample_rows(N):
+    rows = [(0, min(N, 160)), (max(0, N // 2 - 70), min(N, N // 2 + 70)), (max(0, N - 200), N)]
+    return rows
+
+
+def _compare_sampled(got, q, k, v, lay, causal, pv, heads, what):
+    d = lay.d
+    for r0, r1 in _sample_rows(lay.maxlen):
+        ref = oracle.sage_attention(q, k, v, lay, causal, True, PV[pv], heads=heads, rows=(r0, r1))
+        exact = oracle.attn_fp64(q, k, v, lay, causal, 1 / math.sqrt(d), heads=heads,
+                                 rows=(r0, r1))
+        mask = ~np.isnan(ref)
+        assert mask.any()
+        assert_vs_oracle(got[mask], ref[mask], f"{what} rows {r0}:{r1}")
+        assert_vs_fp64(got[mask], exact[mask], pv == "fp8", f"{what} rows {r0}:{r1}")
+
+
+FULL = [
+    ("llm_prefill", "fp16"),
+    ("video_dit", "fp16"),
+    ("video_dit", "fp8"),
+]
+
+
+@pytest.mark.parametrize("name,pv", FULL)
+def test_full_size_configs_sampled(name, pv):
+    w = getattr(inputs, name)()
+    q, k, v = inputs.make_dense(w)
+    got = _run_dense(q, k, v, w.causal, pv)
+    lay = oracle.Layout.dense(w.B, w.H, w.N, w.d)
+    heads = [(0, 0), (w.B - 1, w.H - 1)]
+    _compare_sampled(got, q.numpy(), k.numpy(), v.numpy(), lay, w.causal, pv, heads,
+                     f"{name} {pv}")
+
+
+@pytest.mark.parametrize("N,d,causal", [(16384, 128, False), (32768, 128, True), (1024, 64, True),
+                                        (8192, 64, False)])
+def test_sweep_points_sampled(N, d, causal):
+    w = inputs.sweep(N, d, causal)
+    q, k, v = inputs.make_dense(w)
+    got = _run_dense(q, k, v, causal, "fp16")
+    lay = oracle.Layout.dense(w.B, w.H, w.N, w.d)
+    _compare_sampled(got, q.numpy(), k.numpy(), v.numpy(), lay, causal, "fp16",
+                     [(w.B - 1, 7)], w.name)
+
+
+def test_varlen_config_sampled():
+    w = inputs.varlen()
+    q, k, v, cu = inputs.make_varlen(w)
+    lens = (cu[1:] - cu[:-1]).tolist()
+    out = sage.sageattn_varlen(q.cuda(), k.cuda(), v.cuda(), cu.cuda(), max(lens), True, True,
+                               sage.SAGE_PV_FP8)
+    assert sage.sage_get_device_status() == 0
+    got = _np(out)
+    lay = oracle.Layout.packed(cu.tolist(), w.H, w.d)
+    heads = [(0, 3), (len(lens) - 1, w.H - 1)]
+    _compare_sampled(got, q.numpy(), k.numpy(), v.numpy(), lay, True, "fp8", heads, "varlen")
+
+
+def test_fp8_relative_l1_is_reported():
+    """FP8 PV mode: report the relative L1 against fp64 (the 0.02 bound is not reachable)."""
+    w = inputs.Workload("t", 61, 1, 2, 1024, 128, False, 1.0)
+    q, k, v = inputs.make_dense(w)
+    got = _run_dense(q, k, v, False, "fp8")
+    lay = oracle.Layout.dense(1, 2, 1024, 128)
+    exact = oracle.attn_fp64(q.numpy(), k.numpy(), v.numpy(), lay, False, 1 / math.sqrt(128))
+    r = rel_l1(got, exact)
+    print(f"FP8 PV relative L1 vs fp64: {r:.4f}")
+    assert r < 0.06

@@ -1,0 +1,112 @@
+"""GPU K-QUANT vs the oracle, through the C ABI: INT8 codes, block scales, K means and
+E4M3 V codes must match bit for bit (the K mean is an exact fp64 sum rounded once, so
+smoothed-K codes need no +-1 allowance on these inputs)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import quantized_attention_03_b200 as sage
+from quantized_attention_03_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+def _np(t):
+    return t.detach().cpu().numpy()
+
+
+def _check_qk(z, ref, what):
+    assert np.array_equal(_np(z["q_scale"]), ref["q_scale"]), f"{what}: q_scale"
+    assert np.array_equal(_np(z["q_i8"]), ref["q_i8"]), f"{what}: q_i8"
+    assert np.array_equal(_np(z["k_mean"]), ref["k_mean"]), f"{what}: k_mean"
+    assert np.array_equal(_np(z["k_scale"]), ref["k_scale"]), f"{what}: k_scale"
+    assert np.array_equal(_np(z["k_i8"]), ref["k_i8"]), f"{what}: k_i8"
+
+
+DENSE_CASES = [
+    (1, 2, 256, 64, True),
+    (1, 2, 256, 64, False),
+    (2, 3, 300, 128, True),      # ragged: 2 full Q blocks + 44 rows
+    (1, 1, 1, 64, True),
+    (1, 2, 17, 128, True),
+    (1, 2, 129, 64, True),
+]
+
+
+@pytest.mark.parametrize("B,H,N,d,smooth", DENSE_CASES)
+def test_quant_qk_bit_exact(B, H, N, d, smooth):
+    w = inputs.Workload("t", 7 + N + d, B, H, N, d, False, 2.0)
+    q, k, _ = inputs.make_dense(w)
+    z = sage.quant_qk(q.cuda(), k.cuda(), smooth)
+    assert sage.sage_get_device_status() == 0
+    ref = oracle.quant_qk(q.numpy(), k.numpy(), oracle.Layout.dense(B, H, N, d), smooth)
+    _check_qk(z, ref, f"{B}x{H}x{N}x{d}")
+
+
+def test_quant_qk_edge_values():
+    B, H, N, d = 1, 2, 384, 128
+    g = torch.Generator().manual_seed(5)
+    q = torch.randn((B, H, N, d), generator=g).half()
+    k = torch.randn((B, H, N, d), generator=g).half()
+    q[0, 0, 128:256] = 0                    # an all-zero Q block
+    k[0, 1, 64:128] = 3.0                   # a constant K block
+    q[0, 1, 5, 7] = 65504.0                 # extreme magnitudes
+    q[0, 1, 6, 9] = -65504.0
+    k[0, 0, 300, 3] = 60000.0
+    z = sage.quant_qk(q.cuda(), k.cuda(), True)
+    ref = oracle.quant_qk(q.numpy(), k.numpy(), oracle.Layout.dense(B, H, N, d), True)
+    _check_qk(z, ref, "edge")
+    assert float(z["q_scale"][0, 0, 1]) == 0.0
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_quant_v_fp8_bit_exact(d):
+    B, H, N = 2, 2, 300
+    w = inputs.Workload("t", 11, B, H, N, d, False, 1.0)
+    _, _, v = inputs.make_dense(w)
+    v[0, 1, :, 5] = 0                       # an all-zero channel
+    codes, scales = sage.quant_v_fp8(v.cuda())
+    rc, rs = oracle.quant_v_fp8(v.numpy(), oracle.Layout.dense(B, H, N, d))
+    assert np.array_equal(_np(scales), rs)
+    assert np.array_equal(_np(codes), rc)
+
+
+def test_quant_varlen_bit_exact():
+    H, d = 4, 128
+    lens = [1, 127, 128, 129, 700, 64]
+    w = inputs.Workload("t", 21, 0, H, 0, d, True, 2.0, nseq=len(lens))
+    q, k, v, cu = inputs.make_varlen(w, lens=lens)
+    maxlen = max(lens)
+    cu_d = cu.cuda()
+    z = sage.quant_qk_varlen(q.cuda(), k.cuda(), cu_d, maxlen, True)
+    lay = oracle.Layout.packed(cu.tolist(), H, d)
+    ref = oracle.quant_qk(q.numpy(), k.numpy(), lay, True)
+    _check_qk(z, ref, "varlen")
+    codes, scales = sage.quant_v_fp8_varlen(v.cuda(), cu_d, maxlen)
+    rc, rs = oracle.quant_v_fp8(v.numpy(), lay)
+    assert np.array_equal(_np(scales), rs)
+    assert np.array_equal(_np(codes), rc)
+    assert sage.sage_get_device_status() == 0
+
+
+@pytest.mark.parametrize("name", ["llm_prefill", "video_dit"])
+def test_quant_full_size_configs(name):
+    w = getattr(inputs, name)()
+    q, k, v = inputs.make_dense(w)
+    z = sage.quant_qk(q.cuda(), k.cuda(), True)
+    ref = oracle.quant_qk(q.numpy(), k.numpy(), oracle.Layout.dense(w.B, w.H, w.N, w.d), True)
+    _check_qk(z, ref, name)
+    if "fp8" in w.pv_modes:
+        codes, scales = sage.quant_v_fp8(v.cuda())
+        rc, rs = oracle.quant_v_fp8(v.numpy(), oracle.Layout.dense(w.B, w.H, w.N, w.d))
+        assert np.array_equal(_np(scales), rs) and np.array_equal(_np(codes), rc)
+
+
+def test_bad_cu_seqlens_sets_device_status():
+    H, d = 2, 64
+    q = torch.zeros((100, H, d), dtype=torch.float16, device="cuda")
+    cu = torch.tensor([0, 60, 40, 100], dtype=torch.int32, device="cuda")   # not monotonic
+    sage.quant_qk_varlen(q, q, cu, 60, True)
+    assert sage.sage_get_device_status() == sage.SAGE_ERR_BAD_SEQLENS
+    assert sage.sage_get_device_status() == sage.SAGE_OK                   # cleared

@@ -78,7 +78,10 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.time(), line.strip()))
+
+    def mark(self, name):
+        setattr(self, name, time.time())
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -90,9 +93,14 @@ class ClockSampler:
             self.thread.join(timeout=2)
 
     def summary(self):
+        """Samples taken between mark('t0') and mark('t1') (the timed region)."""
         sm, mx, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        t0 = getattr(self, "t0", 0.0) - 0.1
+        t1 = getattr(self, "t1", float("inf")) + 0.1
+        for ts, ln in self.lines:
+            if not (t0 <= ts <= t1):
+                continue
             parts = [x.strip() for x in ln.split(",")]
             if len(parts) < 8:
                 continue
@@ -226,6 +234,8 @@ def run_ours(args):
         sage.sage_attn_fwd_quantized(q_i8, q_scale, k_i8, k_scale, v, None, out, B, H, N, d,
                                      W["causal"], pv, sm_scale, stream)
 
+    clocks = ClockSampler(local)
+    clocks.__enter__()
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
@@ -238,7 +248,8 @@ def run_ours(args):
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
-    with ClockSampler(local) as clocks:
+    clocks.mark("t0")
+    if True:
         t_start = torch.cuda.Event(enable_timing=True)
         t_end = torch.cuda.Event(enable_timing=True)
         t_start.record(stream)
@@ -253,6 +264,8 @@ def run_ours(args):
             e2.record(stream)
         t_end.record(stream)
         torch.cuda.synchronize()
+    clocks.mark("t1")
+    clocks.__exit__(None, None, None)
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
@@ -369,7 +382,7 @@ def _kernel_hash():
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--ref-rows", type=int, default=1024)

@@ -5,7 +5,7 @@
  * Acceleration", and the follow-up article on SageAttention2) computes attention
  * O = softmax(sm_scale * Q K^T) V with:
  *   1. smooth K: K <- K - mean(K), the mean per channel over the tokens of one head
- *      ("SageAttention" article, section 技术方案, paragraph on smoothing K; softmax is
+ *      (「SageAttention：低比特量化Attention，实现推理加速」, section 技术方案, paragraph on smoothing K; softmax is
  *      unchanged because q.mean(K) is constant along a row);
  *   2. per-block INT8 quantization of Q and K with one fp32 scale per block
  *      (scale = amax/127), blocks of FlashAttention size: 128 Q tokens, 64 K tokens
@@ -97,7 +97,7 @@ SAGE_API sage_status_t sage_quant_qk_varlen(const void *q, const void *k, const 
                                    float *k_mean, int smooth_k, sage_stream_t stream);
 
 /*
- * V to FP8 E4M3 ("SageAttention2" article, 技术方案 (4)) with one fp32 scale per
+ * V to FP8 E4M3 (「4比特量化三倍加速不掉点！清华即插即用的SageAttention迎来升级」, 技术方案 (4)) with one fp32 scale per
  * channel over all tokens of a head: v_scale = amax/448, v_e4m3 = round-to-nearest-even
  * saturating E4M3 of the fp32 quotient V/v_scale (same [B,H,N,d] layout, one byte each).
  */

@@ -6,7 +6,7 @@ shares nothing with the CUDA library) and adds the per-head bookkeeping for the 
 tensor layouts:
 
 * dense  ``[B, H, N, d]`` (the layout of the ``scaled_dot_product_attention`` call the
-  method replaces: "SageAttention" article, section "即插即用举例");
+  method replaces: 「SageAttention：低比特量化Attention，实现推理加速」, section "即插即用举例");
 * packed varlen ``[T, H, d]`` with ``cu_seqlens`` (sequence s holds tokens
   ``cu[s]:cu[s+1]``); every per-head quantity (K mean, blocks, causal mask, V scale)
   is taken within one sequence.

@@ -8,7 +8,7 @@
  *
  * What it restates, with the passage each step follows:
  *   - Smooth K: K <- K - mean(K), the mean taken per channel over the tokens of one
- *     head. ("SageAttention" article, section "技术方案", paragraph "对 K 进行平滑处理".)
+ *     head. (「SageAttention：低比特量化Attention，实现推理加速」, section "技术方案", paragraph "对 K 进行平滑处理".)
  *   - Per-block INT8 quantization of Q and K, one fp32 scale per block of tokens of
  *     FlashAttention block size; INT8 products accumulate in INT32. (Same section,
  *     paragraph "对 Q, K 进行分块 INT8 量化".) The scale is amax/127 (the method's
@@ -16,7 +16,7 @@
  *   - FlashAttention tiling with online softmax over KV tiles; P and V in FP16 for
  *     P.V. (Same section, paragraph "对 P, V 采用 FP16 数据类型的矩阵乘法累加器".)
  *   - FP8 mode: P and V quantized to E4M3, each tile's P.V product summed into an
- *     FP32-or-wider accumulator across tiles. ("SageAttention2" article, section
+ *     FP32-or-wider accumulator across tiles. (「4比特量化三倍加速不掉点！清华即插即用的SageAttention迎来升级」, section
  *     "技术方案", items (3) and (4).)
  *   - The exact reference O = softmax(sm_scale Q K^T + mask) V in fp64, and the
  *     smoothing invariant softmax(QK^T) = softmax(Q(K - mean K)^T) it must satisfy.

@@ -1,11 +1,11 @@
 // K-ATTN: the fused quantized attention pass for sm_100a.
 //
-// Method ("SageAttention" article, section 技术方案; "SageAttention2" article, 技术方案
+// Method (「SageAttention：低比特量化Attention，实现推理加速」, section 技术方案; 「4比特量化三倍加速不掉点！清华即插即用的SageAttention迎来升级」, 技术方案
 // (3)-(4)): S = Q_i8 K_i8^T with INT32 accumulation, dequantized by
 // q_scale * k_scale * sm_scale, FlashAttention online softmax over 128-key tiles, and
 // P.V with P, V in FP16 (FP16 mode) or both in E4M3 (FP8 mode), each tile's P.V
 // product accumulated across tiles in fp32 registers (the two-level accumulation of
-// the SageAttention2 article, item (3)).
+// 「4比特量化三倍加速不掉点！清华即插即用的SageAttention迎来升级」, item (3)).
 //
 // B200 design. One CTA owns NQT = 2 query tiles of 128 rows of one (sequence, head)
 // and walks the KV tiles once for both, so each K/V tile read from L2 feeds 256 rows:

@@ -1,6 +1,6 @@
 // K-QUANT: smooth K and per-block INT8 quantization of Q and K; E4M3 quantization of V.
 //
-// "SageAttention" article, section 技术方案: K <- K - mean(K) with the mean per channel
+// 「SageAttention：低比特量化Attention，实现推理加速」, section 技术方案: K <- K - mean(K) with the mean per channel
 // over tokens; Q and K quantized to INT8 per block of FlashAttention size (Q: 128
 // tokens, K: 64 tokens) with one fp32 scale amax/127 per block. "SageAttention2"
 // article, 技术方案 (4): V in E4M3, here with one fp32 scale (amax/448) per channel.

@@ -129,21 +129,24 @@ def test_varlen_small_full_compare(pv):
 # --------------------------------------------------- full-size workloads, sampled rows
 
 
-def _sample_rows(N):
-    rows = [(0, min(N, 160)), (max(0, N // 2 - 70), min(N, N // 2 + 70)), (max(0, N - 200), N)]
-    return rows
+def _sample_rows(n):
+    """First rows, a middle band and the ragged tail of a head of length n."""
+    return [(0, min(n, 160)), (max(0, n // 2 - 70), min(n, n // 2 + 70)), (max(0, n - 200), n)]
 
 
 def _compare_sampled(got, q, k, v, lay, causal, pv, heads, what):
     d = lay.d
-    for r0, r1 in _sample_rows(lay.maxlen):
-        ref = oracle.sage_attention(q, k, v, lay, causal, True, PV[pv], heads=heads, rows=(r0, r1))
-        exact = oracle.attn_fp64(q, k, v, lay, causal, 1 / math.sqrt(d), heads=heads,
-                                 rows=(r0, r1))
-        mask = ~np.isnan(ref)
-        assert mask.any()
-        assert_vs_oracle(got[mask], ref[mask], f"{what} rows {r0}:{r1}")
-        assert_vs_fp64(got[mask], exact[mask], pv == "fp8", f"{what} rows {r0}:{r1}")
+    for s, h in heads:
+        for r0, r1 in _sample_rows(lay.lens[s]):
+            ref = oracle.sage_attention(q, k, v, lay, causal, True, PV[pv], heads=[(s, h)],
+                                        rows=(r0, r1))
+            exact = oracle.attn_fp64(q, k, v, lay, causal, 1 / math.sqrt(d), heads=[(s, h)],
+                                     rows=(r0, r1))
+            mask = ~np.isnan(ref)
+            assert mask.sum() == (r1 - r0) * d
+            tag = f"{what} head {(s, h)} rows {r0}:{r1}"
+            assert_vs_oracle(got[mask], ref[mask], tag)
+            assert_vs_fp64(got[mask], exact[mask], pv == "fp8", tag)
 
 
 FULL = [

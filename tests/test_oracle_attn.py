@@ -4,7 +4,7 @@
   N = 1 gives O = V; identical keys give O = mean(V).
 * The smoothing invariant softmax(QK^T) = softmax(Q(K - mean K)^T) ("SageAttention"
   article, section 技术方案, paragraph on smoothing K), to ~1e-12 in fp64.
-* The quantized method (same section; "SageAttention2" article, 技术方案 (3)-(4)):
+* The quantized method (same section; 「4比特量化三倍加速不掉点！清华即插即用的SageAttention迎来升级」, 技术方案 (3)-(4)):
   a single KV tile reduces the online softmax to a plain softmax over integer scores,
   recomputed here with a library integer matmul; many tiles agree with one tile up to
   the FP16 rounding of P; the result tracks fp64 attention on inputs built so that a
@@ -199,7 +199,7 @@ def test_fp8_single_token_is_exact():
 
 
 def test_smoothing_helps_with_channel_outliers():
-    # "SageAttention" article, 挑战: channel outliers in K ruin direct INT8 quantization;
+    # 「SageAttention：低比特量化Attention，实现推理加速」, 挑战: channel outliers in K ruin direct INT8 quantization;
     # smoothing K fixes it
     N, d = 512, 64
     q, k, v = (_rand16((1, 1, N, d), s) for s in (81, 82, 83))

@@ -1,9 +1,9 @@
 """Pins for the oracle's smooth-K and quantization steps.
 
-Smooth K ("SageAttention" article, section 技术方案, paragraph on smoothing K): the mean
+Smooth K (「SageAttention：低比特量化Attention，实现推理加速」, section 技术方案, paragraph on smoothing K): the mean
 is per channel over tokens. Per-block INT8 (same section, paragraph on per-block INT8 of
 Q, K): one fp32 scale per block, Q blocks 128 tokens, K blocks 64 tokens, scale =
-amax/127. V to E4M3 with a per-channel scale ("SageAttention2" article, 技术方案 (4)).
+amax/127. V to E4M3 with a per-channel scale (「4比特量化三倍加速不掉点！清华即插即用的SageAttention迎来升级」, 技术方案 (4)).
 The checks are closed forms, invariants and library routines; none re-types the
 oracle's own formula.
 """

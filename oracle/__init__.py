@@ -140,43 +140,47 @@ def f16_to_f64(bits: int) -> float:
 # ------------------------------------------------------------------ method steps
 
 
-def k_mean(k: np.ndarray, layout: Layout) -> np.ndarray:
-    """Per-channel token mean of K for every (sequence, head): [nseq, H, d] fp32."""
+def k_mean(k: np.ndarray, layout: Layout, heads=None) -> np.ndarray:
+    """Per-channel token mean of K for every (or each selected) (sequence, head):
+    [nseq, H, d] fp32."""
     kb = _bits16(k)
     mu = np.zeros((layout.nseq, layout.H, layout.d), np.float32)
-    for s, h, off, n in layout.heads():
+    for s, h, off, n in layout.heads(heads):
         lib().oracle_head_k_mean(_ptr(kb, off), n, layout.stride, layout.d,
                                  _ptr(mu, (s * layout.H + h) * layout.d))
     return mu
 
 
-def quant_int8(x: np.ndarray, layout: Layout, blk: int, mu: Optional[np.ndarray] = None):
+def quant_int8(x: np.ndarray, layout: Layout, blk: int, mu: Optional[np.ndarray] = None,
+               heads=None):
     """Per-block INT8 codes (same shape as x) and scales [nseq, H, nblk]."""
     xb = _bits16(x)
     codes = np.zeros(x.shape, np.int8)
     nb = layout.nblk(blk)
     scales = np.zeros((layout.nseq, layout.H, nb), np.float32)
-    for s, h, off, n in layout.heads():
+    for s, h, off, n in layout.heads(heads):
         mup = _ptr(mu, (s * layout.H + h) * layout.d) if mu is not None else None
         lib().oracle_head_quant_int8(_ptr(xb, off), mup, n, layout.stride, layout.d, blk,
                                      _ptr(codes, off), _ptr(scales, (s * layout.H + h) * nb))
     return codes, scales
 
 
-def quant_qk(q: np.ndarray, k: np.ndarray, layout: Layout, smooth_k: bool = True):
-    """Smooth K, then per-block INT8 of Q (128 tokens) and K (64 tokens)."""
-    mu = k_mean(k, layout) if smooth_k else np.zeros((layout.nseq, layout.H, layout.d), np.float32)
-    q_i8, q_scale = quant_int8(q, layout, Q_BLOCK)
-    k_i8, k_scale = quant_int8(k, layout, K_BLOCK, mu if smooth_k else None)
+def quant_qk(q: np.ndarray, k: np.ndarray, layout: Layout, smooth_k: bool = True, heads=None):
+    """Smooth K, then per-block INT8 of Q (128 tokens) and K (64 tokens), for every (or
+    each selected) head."""
+    zeros = np.zeros((layout.nseq, layout.H, layout.d), np.float32)
+    mu = k_mean(k, layout, heads) if smooth_k else zeros
+    q_i8, q_scale = quant_int8(q, layout, Q_BLOCK, None, heads)
+    k_i8, k_scale = quant_int8(k, layout, K_BLOCK, mu if smooth_k else None, heads)
     return dict(q_i8=q_i8, q_scale=q_scale, k_i8=k_i8, k_scale=k_scale, k_mean=mu)
 
 
-def quant_v_fp8(v: np.ndarray, layout: Layout):
+def quant_v_fp8(v: np.ndarray, layout: Layout, heads=None):
     """E4M3 codes of V (same shape) and per-channel scales [nseq, H, d]."""
     vb = _bits16(v)
     codes = np.zeros(v.shape, np.uint8)
     scales = np.zeros((layout.nseq, layout.H, layout.d), np.float32)
-    for s, h, off, n in layout.heads():
+    for s, h, off, n in layout.heads(heads):
         lib().oracle_head_quant_v_fp8(_ptr(vb, off), n, layout.stride, layout.d,
                                       _ptr(codes, off), _ptr(scales, (s * layout.H + h) * layout.d))
     return codes, scales
@@ -231,9 +235,9 @@ def sage_attention(q, k, v, layout: Layout, causal: bool = False, smooth_k: bool
                    tile_n: int = 128, heads=None, rows=None) -> np.ndarray:
     """The whole method from fp16 Q, K, V: smooth K, quantize, quantized attention."""
     sm = default_sm_scale(layout.d, sm_scale)
-    z = quant_qk(q, k, layout, smooth_k)
+    z = quant_qk(q, k, layout, smooth_k, heads)
     if pv_mode == PV_FP8:
-        v8, vs = quant_v_fp8(v, layout)
+        v8, vs = quant_v_fp8(v, layout, heads)
         return attn_quant(z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], v8, vs, layout,
                           causal, PV_FP8, sm, tile_n, heads, rows)
     return attn_quant(z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], v, None, layout,

@@ -73,7 +73,7 @@ struct Cfg {
     static constexpr int kOffV = kOffK + STAGES * kKBytes;
     static constexpr int kOffBar = kOffV + STAGES * kVBytes;
     // barriers: q, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[NQT],
-    //           p_full[NQT], pv_full[NQT], pv_free[NQT], drain
+    //           p_full[NQT], pv_full[NQT], turn[NQT], drain
     static constexpr int kNumBars = 1 + 4 * STAGES + 4 * NQT + 1;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
@@ -88,6 +88,10 @@ struct Cfg {
     static constexpr int kQkSbo = 8 * D;                                 // 8 rows
     static constexpr int kVSwizzle = kVRowBytes == 128 ? 2 : 4;
     static constexpr int kVSbo = 8 * kVRowBytes;
+    // The reference max of a row is refreshed only when the row max exceeds it by more
+    // than this (log2 units): FP16 P then stays <= 2^8, far inside fp16. FP8 mode keeps
+    // P <= 1 so that 448 P fits E4M3.
+    static constexpr float kRescaleSlack = FP8 ? 0.0f : 8.0f;
 };
 
 struct KParams {
@@ -134,7 +138,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     return ok;
 }
 
-template <int D, bool FP8, int NQT, bool DUMP>
+template <int D, bool FP8, int NQT, bool DUMP, bool PINGPONG>
 __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const KParams p)
@@ -168,8 +172,8 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
     uint64_t *s_full = v_empty + C::STAGES;
     uint64_t *p_full = s_full + NQT;
     uint64_t *pv_full = p_full + NQT;
-    uint64_t *pv_free = pv_full + NQT;
-    uint64_t *bar_drain = pv_free + NQT;
+    uint64_t *turn = pv_full + NQT;        // softmax warpgroups take turns on the exp phase
+    uint64_t *bar_drain = turn + NQT;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffMisc);
     volatile int *abort = reinterpret_cast<volatile int *>(smem + C::kOffMisc + 4);
 
@@ -186,7 +190,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
             mbar_init(&s_full[i], 1);
             mbar_init(&p_full[i], 4);
             mbar_init(&pv_full[i], 1);
-            mbar_init(&pv_free[i], 4);
+            mbar_init(&turn[i], 4);
         }
         mbar_init(bar_drain, 1);
         *abort = 0;
@@ -210,17 +214,15 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
         const int qrow = qt * C::BM + row_in_tile;
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
         const uint32_t tS = tmem_base + lane_off + i * C::BN;
-        const uint32_t tPV = tmem_base + lane_off + NQT * C::BN + i * D;
+        const uint32_t tO = tmem_base + lane_off + NQT * C::BN + i * D;
         const int64_t sh = (int64_t)s * L.H + h;
         const bool tile_valid = qt * C::BM < len;
         const float qsc = (tile_valid ? __ldg(p.q_scale + sh * p.nqb + qt) : 0.0f) * p.sc_log2;
         const int kb_valid = (len + kKBlock - 1) / kKBlock;
 
-        float o[D];
-#pragma unroll
-        for (int c = 0; c < D; c++)
-            o[c] = 0.0f;
-        float m = -INFINITY, l = 0.0f, alpha_prev = 0.0f;
+        // m_ref: the max that P is taken relative to; it moves only when the row max
+        // exceeds it by more than kRescaleSlack (0 in FP8 mode, so P <= 1 and 448 P fits E4M3)
+        float m_ref = -INFINITY, l = 0.0f;
         bool ok = true;
 
         for (int j = 0; j < nkv && ok; j++) {
@@ -235,58 +237,67 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
                 (kcol0 + C::BN > len) || (p.causal && kcol0 + C::BN - 1 > qt * C::BM);
             const int col_lim = p.causal ? min(len, qrow + 1) : len;   // keys < col_lim visible
 
-            // pass 1: integer maxima of the two 64-key halves
-            int im0 = INT_MIN, im1 = INT_MIN;
+            // the whole 128-key score row into registers (one TMEM pass)
+            uint32_t sreg[4][32];
+#pragma unroll
+            for (int ch = 0; ch < 4; ch++)
+                tmem_ld32_async(tS + ch * 32, sreg[ch]);
+#pragma unroll
+            for (int ch = 0; ch < 4; ch++)
+                tmem_ld_wait(sreg[ch]);
+            if constexpr (DUMP) {
+                if (qrow < len) {
+                    int32_t *drow = p.s_dump + (sh * L.maxlen + qrow) * L.maxlen;
+                    for (int e = 0; e < C::BN; e++)
+                        if (kcol0 + e < len)
+                            drow[kcol0 + e] = static_cast<int>(sreg[e / 32][e % 32]);
+                }
+            }
+            // integer maxima of the two 64-key halves (the two K blocks have own scales)
+            int im[2] = {INT_MIN, INT_MIN};
 #pragma unroll
             for (int ch = 0; ch < 4; ch++) {
-                uint32_t r[32];
-                tmem_ld32(tS + ch * 32, r);
-                if constexpr (DUMP) {
-                    if (qrow < len) {
-                        int32_t *drow = p.s_dump + (sh * L.maxlen + qrow) * L.maxlen;
-                        for (int e = 0; e < 32; e++)
-                            if (kcol0 + ch * 32 + e < len)
-                                drow[kcol0 + ch * 32 + e] = static_cast<int>(r[e]);
-                    }
-                }
                 const uint32_t keep = need_mask ? chunk_mask(col_lim - kcol0 - ch * 32) : ~0u;
                 int mx = INT_MIN;
 #pragma unroll
-                for (int e = 0; e < 32; e++) {
-                    const int v = static_cast<int>(r[e]);
-                    mx = ((keep >> e) & 1u) ? max(mx, v) : mx;
-                }
-                if (ch < 2)
-                    im0 = max(im0, mx);
-                else
-                    im1 = max(im1, mx);
+                for (int e = 0; e < 32; e++)
+                    mx = ((keep >> e) & 1u) ? max(mx, static_cast<int>(sreg[ch][e])) : mx;
+                im[ch / 2] = max(im[ch / 2], mx);
             }
             float tmax = -INFINITY;
-            if (im0 != INT_MIN)
-                tmax = static_cast<float>(im0) * sc0;
-            if (im1 != INT_MIN)
-                tmax = fmaxf(tmax, static_cast<float>(im1) * sc1);
-            const float m_new = fmaxf(m, tmax);
-            const float alpha = ex2_approx(m - m_new);
+            if (im[0] != INT_MIN)
+                tmax = static_cast<float>(im[0]) * sc0;
+            if (im[1] != INT_MIN)
+                tmax = fmaxf(tmax, static_cast<float>(im[1]) * sc1);
+            const float m_new = tmax > m_ref + C::kRescaleSlack ? tmax : m_ref;
+            const float alpha = m_new == m_ref ? 1.0f : ex2_approx(m_ref - m_new);
             const float bias = FP8 ? m_new - kLog2_448 : m_new;
 
-            // pass 2: p = 2^(S sc - m), row sum, P packed over S in TMEM (16 keys at a
-            // time keeps the working set small next to the d registers of O)
-            float lsum = 0.0f;
+            // p = 2^(S sc - m): S to fp32 exactly through the magic bias
+            // (|S| <= 127^2 d < 2^22), one packed FFMA, ex2; P packed over S in TMEM.
+            if constexpr (PINGPONG) {
+                if (!(ok = warp_wait(&turn[i], (j & 1) ^ (i == 0 ? 1 : 0), abort, p.status)))
+                    break;
+            }
+            float2 lsum2 = make_float2(0.0f, 0.0f);
 #pragma unroll
             for (int ch = 0; ch < 8; ch++) {
-                uint32_t r[16];
-                tmem_ld16(tS + ch * 16, r);
                 const float sc = ch < 4 ? sc0 : sc1;
                 const uint32_t keep =
                     need_mask ? chunk_mask(col_lim - kcol0 - ch * 16) & 0xffffu : 0xffffu;
                 float pe[16];
 #pragma unroll
-                for (int e = 0; e < 16; e++) {
-                    const float sf = static_cast<float>(static_cast<int>(r[e]));
-                    const float pv = ex2_approx(fmaf(sf, sc, -bias));
-                    pe[e] = ((keep >> e) & 1u) ? pv : 0.0f;
-                    lsum += pe[e];
+                for (int e = 0; e < 16; e += 2) {
+                    float2 x = make_float2(magic_biased(sreg[ch / 2][(ch % 2) * 16 + e]),
+                                           magic_biased(sreg[ch / 2][(ch % 2) * 16 + e + 1]));
+                    x = add2(x, make_float2(-kMagic, -kMagic));          // exact S
+                    const float2 t = fma2(x, make_float2(sc, sc), make_float2(-bias, -bias));
+                    float2 pv = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+                    pv.x = ((keep >> e) & 1u) ? pv.x : 0.0f;
+                    pv.y = ((keep >> (e + 1)) & 1u) ? pv.y : 0.0f;
+                    pe[e] = pv.x;
+                    pe[e + 1] = pv.y;
+                    lsum2 = add2(lsum2, pv);
                 }
                 if constexpr (!FP8) {
                     uint32_t w[8];
@@ -304,65 +315,75 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
                     tmem_st4(tS + ch * 4, w);
                 }
             }
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&p_full[i]);
-            l = alpha * l + lsum;
-            m = m_new;
+            l = alpha * l + (lsum2.x + lsum2.y);
+            m_ref = m_new;
 
-            // O update for the previous tile (its PV has had a whole softmax to finish)
-            if (j > 0) {
+            // O (fp32 in TMEM, accumulated across tiles by the tensor core) is rescaled
+            // before this tile's P.V lands on it; the whole warp takes part if any row
+            // of it moved its reference max
+            if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
                 if (!(ok = warp_wait(&pv_full[i], (j - 1) & 1, abort, p.status)))
                     break;
                 tc_fence_after();
+                uint32_t orow[D / 32][32];
+#pragma unroll
+                for (int ch = 0; ch < D / 32; ch++)
+                    tmem_ld32_async(tO + ch * 32, orow[ch]);
 #pragma unroll
                 for (int ch = 0; ch < D / 32; ch++) {
-                    uint32_t r[32];
-                    tmem_ld32(tPV + ch * 32, r);
+                    tmem_ld_wait(orow[ch]);
 #pragma unroll
-                    for (int e = 0; e < 32; e++)
-                        o[ch * 32 + e] = fmaf(alpha_prev, o[ch * 32 + e], __uint_as_float(r[e]));
+                    for (int e = 0; e < 32; e += 2) {
+                        const float2 ov = fma2(make_float2(__uint_as_float(orow[ch][e]),
+                                                           __uint_as_float(orow[ch][e + 1])),
+                                               make_float2(alpha, alpha), make_float2(0.0f, 0.0f));
+                        orow[ch][e] = __float_as_uint(ov.x);
+                        orow[ch][e + 1] = __float_as_uint(ov.y);
+                    }
+                    tmem_st32(tO + ch * 32, orow[ch]);
                 }
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0)
-                    mbar_arrive(&pv_free[i]);
             }
-            alpha_prev = alpha;
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&p_full[i]);
+                if constexpr (PINGPONG)
+                    mbar_arrive(&turn[i ^ 1]);   // the other warpgroup's exp phase may start
+            }
         }
+        // epilogue: the last P.V, normalize, round to fp16, store the row
         if (ok && (ok = warp_wait(&pv_full[i], (nkv - 1) & 1, abort, p.status))) {
             tc_fence_after();
-#pragma unroll
-            for (int ch = 0; ch < D / 32; ch++) {
-                uint32_t r[32];
-                tmem_ld32(tPV + ch * 32, r);
-#pragma unroll
-                for (int e = 0; e < 32; e++)
-                    o[ch * 32 + e] = fmaf(alpha_prev, o[ch * 32 + e], __uint_as_float(r[e]));
-            }
-        }
-        // epilogue: normalize, round to fp16, store the row
-        if (ok && qrow < len) {
             const float inv_l = 1.0f / l;
             __half *dst = p.out + L.offset(s, start, h, qrow);
+            uint32_t orow[D / 32][32];
 #pragma unroll
-            for (int c = 0; c < D; c += 8) {
-                float f[8];
+            for (int ch = 0; ch < D / 32; ch++)
+                tmem_ld32_async(tO + ch * 32, orow[ch]);
 #pragma unroll
-                for (int e = 0; e < 8; e++) {
-                    float sc = inv_l;
-                    if constexpr (FP8)
-                        sc = __ldg(p.v_scale + sh * D + c + e) * inv_l;
-                    f[e] = o[c + e] * sc;
+            for (int ch = 0; ch < D / 32; ch++) {
+                uint32_t(&r)[32] = orow[ch];
+                tmem_ld_wait(r);
+                if (qrow < len) {
+#pragma unroll
+                    for (int c = 0; c < 32; c += 8) {
+                        float f[8];
+#pragma unroll
+                        for (int e = 0; e < 8; e++) {
+                            float sc = inv_l;
+                            if constexpr (FP8)
+                                sc = __ldg(p.v_scale + sh * D + ch * 32 + c + e) * inv_l;
+                            f[e] = __uint_as_float(r[c + e]) * sc;
+                        }
+                        uint4 u;
+                        u.x = pack_half2(f[0], f[1]);
+                        u.y = pack_half2(f[2], f[3]);
+                        u.z = pack_half2(f[4], f[5]);
+                        u.w = pack_half2(f[6], f[7]);
+                        *reinterpret_cast<uint4 *>(dst + ch * 32 + c) = u;
+                    }
                 }
-                uint4 u;
-                u.x = pack_half2(f[0], f[1]);
-                u.y = pack_half2(f[2], f[3]);
-                u.z = pack_half2(f[4], f[5]);
-                u.w = pack_half2(f[6], f[7]);
-                *reinterpret_cast<uint4 *>(dst + c) = u;
             }
         }
     } else if (warp == C::kProducerWarp) {
@@ -425,59 +446,73 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
             const uint64_t dQ0 = smem_desc(smem_u32(sQ), 16, C::kQkSbo, C::kQkSwizzle);
             const uint64_t dK0 = smem_desc(smem_u32(sK), 16, C::kQkSbo, C::kQkSwizzle);
             const uint64_t dV0 = smem_desc(smem_u32(sV), C::kVBoxBytes, C::kVSbo, C::kVSwizzle);
-            bool ok = mbar_wait(bar_q, 0, abort, p.status, status_bit(SAGE_ERR_TIMEOUT),
-                                kTimeoutNs);
+            auto issue_s = [&](int i, int stg) {
+                const uint32_t dS = tmem_base + i * C::BN;
+#pragma unroll
+                for (int kk = 0; kk < D / 32; kk++) {
+                    const uint64_t a = dQ0 + ((i * C::kQBytes + kk * 32) >> 4);
+                    const uint64_t b = dK0 + ((stg * C::kKBytes + kk * 32) >> 4);
+                    mma_i8_ss(dS, a, b, idesc_qk, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(&s_full[i]);
+            };
+            auto issue_pv = [&](int i, int stg, int j) {
+                const uint32_t dO = tmem_base + NQT * C::BN + i * D;
+                const uint32_t aP = tmem_base + i * C::BN;
+#pragma unroll
+                for (int kk = 0; kk < C::BN / C::kPvK; kk++) {
+                    const uint64_t b =
+                        dV0 + ((stg * C::kVBytes + kk * C::kPvK * C::kVRowBytes) >> 4);
+                    const uint32_t acc = (kk > 0 || j > 0) ? 1u : 0u;
+                    if constexpr (FP8)
+                        mma_f8_ts(dO, aP + kk * 8, b, idesc_pv, acc);
+                    else
+                        mma_f16_ts(dO, aP + kk * 8, b, idesc_pv, acc);
+                }
+                mma_commit(&pv_full[i]);
+            };
+            auto wait = [&](uint64_t *bar, uint32_t parity) {
+                return mbar_wait(bar, parity, abort, p.status, status_bit(SAGE_ERR_TIMEOUT),
+                                 kTimeoutNs);
+            };
+            // Issue order S_0(0) S_1(0) | PV_0(j) S_0(j+1) PV_1(j) S_1(j+1) | ...: each
+            // query tile's next scores follow its own P.V, so one softmax warpgroup works
+            // while the tensor core serves the other. S_i(j+1) overwrites P_i(j), so it is
+            // issued only once PV_i(j) has completed.
+            bool ok = wait(bar_q, 0) && wait(&k_full[0], 0);
+            if (ok) {
+                tc_fence_after();
+                for (int i = 0; i < NQT; i++)
+                    issue_s(i, 0);
+                mma_commit(&k_empty[0]);
+            }
             for (int j = 0; j < nkv && ok; j++) {
                 const int stg = j % C::STAGES;
                 const uint32_t ph = (j / C::STAGES) & 1;
-                if (!(ok = mbar_wait(&k_full[stg], ph, abort, p.status,
-                                     status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs)))
+                const int stg1 = (j + 1) % C::STAGES;
+                const uint32_t ph1 = ((j + 1) / C::STAGES) & 1;
+                const bool more = j + 1 < nkv;
+                if (!(ok = wait(&v_full[stg], ph)))
+                    break;
+                if (more && !(ok = wait(&k_full[stg1], ph1)))
                     break;
                 for (int i = 0; i < NQT && ok; i++) {
-                    // S_i is overwritten: P_i of the previous tile must have been consumed
-                    if (j > 0 && !(ok = mbar_wait(&pv_full[i], (j - 1) & 1, abort, p.status,
-                                                  status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs)))
+                    if (!(ok = wait(&p_full[i], j & 1)))
                         break;
                     tc_fence_after();
-                    const uint32_t dS = tmem_base + i * C::BN;
-#pragma unroll
-                    for (int kk = 0; kk < D / 32; kk++) {
-                        const uint64_t a = dQ0 + ((i * C::kQBytes + kk * 32) >> 4);
-                        const uint64_t b = dK0 + ((stg * C::kKBytes + kk * 32) >> 4);
-                        mma_i8_ss(dS, a, b, idesc_qk, kk > 0 ? 1u : 0u);
+                    issue_pv(i, stg, j);
+                    if (more) {
+                        if (!(ok = wait(&pv_full[i], j & 1)))
+                            break;
+                        tc_fence_after();
+                        issue_s(i, stg1);
                     }
-                    mma_commit(&s_full[i]);
-                }
-                if (!ok)
-                    break;
-                mma_commit(&k_empty[stg]);
-                if (!(ok = mbar_wait(&v_full[stg], ph, abort, p.status,
-                                     status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs)))
-                    break;
-                for (int i = 0; i < NQT && ok; i++) {
-                    if (!(ok = mbar_wait(&p_full[i], j & 1, abort, p.status,
-                                         status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs)))
-                        break;
-                    if (j > 0 && !(ok = mbar_wait(&pv_free[i], (j - 1) & 1, abort, p.status,
-                                                  status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs)))
-                        break;
-                    tc_fence_after();
-                    const uint32_t dPV = tmem_base + NQT * C::BN + i * D;
-                    const uint32_t aP = tmem_base + i * C::BN;
-#pragma unroll
-                    for (int kk = 0; kk < C::BN / C::kPvK; kk++) {
-                        const uint64_t b =
-                            dV0 + ((stg * C::kVBytes + kk * C::kPvK * C::kVRowBytes) >> 4);
-                        if constexpr (FP8)
-                            mma_f8_ts(dPV, aP + kk * 8, b, idesc_pv, kk > 0 ? 1u : 0u);
-                        else
-                            mma_f16_ts(dPV, aP + kk * 8, b, idesc_pv, kk > 0 ? 1u : 0u);
-                    }
-                    mma_commit(&pv_full[i]);
                 }
                 if (!ok)
                     break;
                 mma_commit(&v_empty[stg]);
+                if (more)
+                    mma_commit(&k_empty[stg1]);
             }
             // drain: every MMA issued above has completed before TMEM is released
             mma_commit(bar_drain);
@@ -551,6 +586,10 @@ bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int elem
     return r == CUDA_SUCCESS;
 }
 
+#ifndef SAGE_PINGPONG
+#define SAGE_PINGPONG 0
+#endif
+
 template <int D, bool FP8, int NQT, bool DUMP>
 cudaError_t run(const AttnArgs &a, const SeqLayout &L, int *status, cudaStream_t st,
                 sage_status_t *host_err)
@@ -583,7 +622,7 @@ cudaError_t run(const AttnArgs &a, const SeqLayout &L, int *status, cudaStream_t
     p.sc_log2 = a.sm_scale * kLog2e;
     p.status = status;
 
-    auto kern = attn_kernel<D, FP8, NQT, DUMP>;
+    auto kern = attn_kernel<D, FP8, NQT, DUMP, SAGE_PINGPONG != 0>;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess)

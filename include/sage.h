@@ -156,6 +156,32 @@ SAGE_API sage_status_t sage_attn_fwd_quantized(const int8_t *q_i8, const float *
 SAGE_API sage_status_t sage_debug_qk_int32(const int8_t *q_i8, const int8_t *k_i8, int32_t *s_out,
                                   int B, int H, int N, int d, sage_stream_t stream);
 
+/*
+ * sage_attn_fwd without any allocation, for callers that cannot allocate device memory
+ * while they run (for instance a serving process whose own allocator owns all GPU
+ * memory after start-up, or a latency-critical loop that must not risk an allocation
+ * stalling or failing) and have no scratch buffer to pass to sage_attn_fwd_ws. The
+ * paper has no counterpart; this is an interface convenience of this library.
+ *
+ * Scratch comes from a static device array of SAGE_NOALLOC_SCRATCH_BYTES (64 MiB) that
+ * every GPU which loads this library holds until the process exits. A call whose
+ * sage_workspace_size(B, H, N, B*N, d, pv_mode) exceeds that returns SAGE_ERR_WORKSPACE
+ * before anything is enqueued (set SAGE_LOG=1 for the byte counts). Arguments, layout
+ * and results are those of sage_attn_fwd.
+ *
+ * The first call on each device looks up the array's device address (cudaGetSymbolAddress,
+ * with that device current) and caches it; make that first call before any stream
+ * capture. All calls share the one array and it keeps the previous call's contents (the
+ * parts that must start at zero are cleared on every call): calls that can overlap on
+ * the GPU, on different streams of one device, race and must be serialized by the caller.
+ * Calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+#define SAGE_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+SAGE_API sage_status_t sage_attn_fwd_noalloc(const void *q, const void *k, const void *v,
+                                             void *out, int B, int H, int N, int d, int causal,
+                                             int smooth_k, int pv_mode, float sm_scale,
+                                             sage_stream_t stream);
+
 /* Synchronizes `stream`, returns the device status word (SAGE_OK if clean) and clears
  * it. SAGE_ERR_CUDA if the synchronization itself failed. */
 SAGE_API sage_status_t sage_get_device_status(sage_stream_t stream);

@@ -54,6 +54,7 @@ SIGNATURES = {
     "sage_attn_fwd_quantized": (_S, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F,
                                      _P]),
     "sage_debug_qk_int32": (_S, [_P, _P, _P, _I, _I, _I, _I, _P]),
+    "sage_attn_fwd_noalloc": (_S, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
     "sage_get_device_status": (_S, [_P]),
     "sage_status_string": (ctypes.c_char_p, [_I]),
     "sage_last_cuda_error": (_I, []),
@@ -174,6 +175,13 @@ def sage_attn_fwd_quantized(q_i8, q_scale, k_i8, k_scale, v, v_scale, out, B, H,
 def sage_debug_qk_int32(q_i8, k_i8, s_out, B, H, N, d, stream=None):
     return _call("sage_debug_qk_int32", _ptr(q_i8), _ptr(k_i8), _ptr(s_out), B, H, N, d,
                  _stream(stream))
+
+
+def sage_attn_fwd_noalloc(q, k, v, out, B, H, N, d, causal, smooth_k, pv_mode, sm_scale,
+                          stream=None):
+    """sage_attn_fwd with the library's static scratch (no allocation; see sage.h)."""
+    return _call("sage_attn_fwd_noalloc", _ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d,
+                 int(causal), int(smooth_k), int(pv_mode), float(sm_scale), _stream(stream))
 
 
 def sage_get_device_status(stream=None) -> int:

@@ -460,3 +460,79 @@ int sage_last_cuda_error(void) { return g_last_cuda_error; }
 int sage_version(void) { return 100; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------------
+// Allocation-free variant of sage_attn_fwd.
+//
+// Some callers cannot allocate device memory once they are running: a serving process
+// that hands all GPU memory to its own allocator at start-up and forbids further driver
+// allocations, or a latency-critical loop that must not risk an allocation stalling or
+// failing. If such a caller also has no scratch buffer of its own to pass to
+// sage_attn_fwd_ws, it uses this entry point: its scratch is a fixed array in device
+// memory that belongs to this library (every GPU that loads the library holds it until
+// the process exits).
+namespace sage {
+namespace {
+
+// Host code may not use the array's name as a device address: on the host it is only a
+// stand-in symbol. Its device address is looked up once per device with
+// cudaGetSymbolAddress and cached here.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SAGE_NOALLOC_SCRATCH_BYTES];
+char *g_noalloc_ptr[64] = {};
+
+sage_status_t noalloc_scratch(char **out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess || dev < 0 || dev >= 64)
+        return cuda_fail(e == cudaSuccess ? cudaErrorInvalidDevice : e);
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_scratch);   // with `dev` current
+        if (e != cudaSuccess)
+            return cuda_fail(e);
+        g_noalloc_ptr[dev] = static_cast<char *>(p);
+    }
+    *out = g_noalloc_ptr[dev];
+    return SAGE_OK;
+}
+
+}  // namespace
+}  // namespace sage
+
+extern "C" sage_status_t sage_attn_fwd_noalloc(const void *q, const void *k, const void *v,
+                                               void *out, int B, int H, int N, int d, int causal,
+                                               int smooth_k, int pv_mode, float sm_scale,
+                                               sage_stream_t stream)
+{
+    sage_status_t r = check_shape(B, H, N, d);
+    if (r != SAGE_OK)
+        return r;
+    if (pv_mode != SAGE_PV_FP16 && pv_mode != SAGE_PV_FP8)
+        return SAGE_ERR_INVALID_ARG;
+    if (B == 0 || H == 0 || N == 0)
+        return SAGE_OK;
+    if ((int64_t)B * N > INT32_MAX)
+        return SAGE_ERR_UNSUPPORTED;
+    if (!q || !k || !v || !out)
+        return SAGE_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+        return SAGE_ERR_MISALIGNED;
+    const size_t need = sage_workspace_size(B, H, N, B * N, d, pv_mode);
+    if (need > (size_t)SAGE_NOALLOC_SCRATCH_BYTES) {
+        if (std::getenv("SAGE_LOG"))
+            std::fprintf(stderr,
+                         "sage_attn_fwd_noalloc: this call needs %zu bytes of scratch, more than "
+                         "the %zu-byte static buffer; use sage_attn_fwd or sage_attn_fwd_ws\n",
+                         need, (size_t)SAGE_NOALLOC_SCRATCH_BYTES);
+        return SAGE_ERR_WORKSPACE;
+    }
+    char *ws = nullptr;
+    if ((r = noalloc_scratch(&ws)) != SAGE_OK)
+        return r;
+    // forward() zeroes the only scratch that must start at zero (the K column sums and
+    // V maxima) before its kernels run; everything else is written before it is read.
+    return forward(q, k, v, out, SeqLayout::dense(B, H, N, d), causal, smooth_k, pv_mode,
+                   sm_scale, ws, reinterpret_cast<cudaStream_t>(stream));
+}

@@ -198,6 +198,24 @@ def cpu_baseline(seconds_target: float = 15.0):
                       f"({t_total:.1f} s of CPU work)"}
 
 
+def _workload(args):
+    """The headline workload, optionally overridden (smaller cases for profiling)."""
+    W = dict(WORKLOAD)
+    for key in ("B", "N", "d"):
+        if getattr(args, key) is not None:
+            W[key] = getattr(args, key)
+    if args.causal:
+        W["causal"] = True
+    if args.pv is not None:
+        W["pv_mode"] = args.pv
+    return W
+
+
+def _workload_name(W):
+    return (f"B={W['B']} H={W['H']} N={W['N']} d={W['d']} "
+            f"{'causal' if W['causal'] else 'non-causal'} PV={W['pv_mode']} smooth_k")
+
+
 def run_ours(args):
     import torch
     import quantized_attention_03_b200 as sage
@@ -211,12 +229,16 @@ def run_ours(args):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
 
-    W = WORKLOAD
+    W = _workload(args)
     B, H, N, d = W["B"], W["H"], W["N"], W["d"]
     w = inputs.sweep(N, d, W["causal"])
     qc, kc, vc = inputs.make_dense(w, B=B)
     q, k, v = qc.cuda(), kc.cuda(), vc.cuda()
     pv = sage.SAGE_PV_FP16 if W["pv_mode"] == "fp16" else sage.SAGE_PV_FP8
+    vq, vscale = v, None
+    if pv == sage.SAGE_PV_FP8:
+        vq = torch.empty(v.shape, dtype=torch.uint8, device=v.device)
+        vscale = torch.empty((B, H, d), dtype=torch.float32, device=v.device)
     sm_scale = 1.0 / math.sqrt(d)
     dev = q.device
     nqb, nkb = math.ceil(N / 128), math.ceil(N / 64)
@@ -228,11 +250,19 @@ def run_ours(args):
     out = torch.empty_like(q)
     stream = torch.cuda.current_stream()
 
-    def step():
+    def quant():
         sage.sage_quant_qk(q, k, q_i8, q_scale, k_i8, k_scale, k_mean, B, H, N, d,
                            W["smooth_k"], stream)
-        sage.sage_attn_fwd_quantized(q_i8, q_scale, k_i8, k_scale, v, None, out, B, H, N, d,
+        if pv == sage.SAGE_PV_FP8:
+            sage.sage_quant_v_fp8(v, vq, vscale, B, H, N, d, stream)
+
+    def attend():
+        sage.sage_attn_fwd_quantized(q_i8, q_scale, k_i8, k_scale, vq, vscale, out, B, H, N, d,
                                      W["causal"], pv, sm_scale, stream)
+
+    def step():
+        quant()
+        attend()
 
     clocks = ClockSampler(local)
     clocks.__enter__()
@@ -256,11 +286,9 @@ def run_ours(args):
         for i in range(args.steps):
             e0, e1, e2 = ev[i]
             e0.record(stream)
-            sage.sage_quant_qk(q, k, q_i8, q_scale, k_i8, k_scale, k_mean, B, H, N, d,
-                               W["smooth_k"], stream)
+            quant()
             e1.record(stream)
-            sage.sage_attn_fwd_quantized(q_i8, q_scale, k_i8, k_scale, v, None, out, B, H, N,
-                                         d, W["causal"], pv, sm_scale, stream)
+            attend()
             e2.record(stream)
         t_end.record(stream)
         torch.cuda.synchronize()
@@ -287,7 +315,7 @@ def run_ours(args):
     attn_tops = ops / (attn_avg_ms * 1e-3) / 1e12
 
     # end to end through the public API: pinned host inputs -> device -> result -> host
-    e2e_steps = max(3, args.steps // 4)
+    e2e_steps = 0 if args.no_e2e else max(3, args.steps // 4)
     qh, kh, vh = (t.pin_memory() for t in (qc, kc, vc))
     oh = torch.empty_like(qc).pin_memory()
     qd, kd, vd, od = (torch.empty_like(q) for _ in range(4))
@@ -300,7 +328,8 @@ def run_ours(args):
                            stream)
         oh.copy_(od, non_blocking=True)
 
-    e2e_step()
+    if e2e_steps:
+        e2e_step()
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
@@ -311,7 +340,7 @@ def run_ours(args):
         e2e_step()
     s1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = s0.elapsed_time(s1)
+    e2e_ms = max(s0.elapsed_time(s1), 1e-9)
     if dist is not None:
         t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
@@ -319,20 +348,21 @@ def run_ours(args):
     status = sage.sage_get_device_status()
     if status != 0:
         raise RuntimeError(f"device status after e2e: {sage.status_string(status)}")
-    e2e_value = world * ops * e2e_steps / (e2e_ms * 1e-3) / 1e12
+    e2e_value = world * ops * e2e_steps / (e2e_ms * 1e-3) / 1e12 if e2e_steps else None
     elem_bytes = B * H * N * d * 2
 
     peaks, src = _peaks()
     bf16 = peaks["bf16_tflops_sustained"]
     int8_peak = 2.0 * bf16            # nominal dense ratio int8 : bf16 = 4.5 : 2.25
-    f16_peak = bf16                   # fp16 dense = bf16 dense
-    mixed = 1.0 / (0.5 / int8_peak + 0.5 / f16_peak)
+    pv_peak = bf16 if pv == sage.SAGE_PV_FP16 else 2.0 * bf16   # fp16 = bf16; fp8 = int8
+    mixed = 1.0 / (0.5 / int8_peak + 0.5 / pv_peak)
     roofline = {
         "bound": "tensor", "achieved": attn_tops, "peak": mixed, "unit": "TOPS",
         "frac": attn_tops / mixed, "traffic": None,
-        "kernel": "attn_kernel<128,fp16-PV,2 q-tiles>",
-        "peak_note": (f"mixed INT8-QK/FP16-PV peak from the {src} sustained bf16 GEMM "
-                      f"({bf16:.1f} TF/s): int8 = 2x, fp16 = 1x, half the ops each"),
+        "kernel": f"attn_kernel<d={d}, PV={W['pv_mode']}, 2 query tiles per CTA>",
+        "peak_note": (f"mixed INT8-QK/{W['pv_mode'].upper()}-PV dense peak from the {src} "
+                      f"sustained bf16 GEMM ({bf16:.1f} TF/s): int8 and fp8 = 2x, fp16 = 1x, "
+                      f"half the operations each (of measured)"),
         "frac_of_int8_peak": attn_tops / int8_peak,
         "attn_ms": attn_avg_ms, "quant_ms": sum(quant_ms) / len(quant_ms),
     }
@@ -349,8 +379,8 @@ def run_ours(args):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "s8+f16", "data": "synthetic",
-            "config": {"workload": "sweep point B=2 H=32 N=16384 d=128 non-causal PV=fp16 "
-                                   "smooth_k (per GPU)",
+            "config": {"workload": "sequence-length sweep point " + _workload_name(W) +
+                                   " (per GPU)",
                        "B": B, "H": H, "N": N, "d": d, "causal": W["causal"],
                        "pv_mode": W["pv_mode"], "smooth_k": W["smooth_k"],
                        "parallelism": f"replicas x{world}",
@@ -359,7 +389,7 @@ def run_ours(args):
             "e2e": {"value": e2e_value, "unit": "TOPS",
                     "h2d_bytes_per_step": 3 * elem_bytes, "d2h_bytes_per_step": elem_bytes,
                     "steps": e2e_steps},
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": (3 if pv == sage.SAGE_PV_FP16 else 5) * args.steps,
             "clocks": clocks.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -371,11 +401,17 @@ def run_ours(args):
 
 
 def _kernel_hash():
+    """Hash of the attention kernel's code (comments and blank lines ignored): a stored
+    DRAM-traffic figure is used only for the kernel it was measured on."""
     import hashlib
+    import re
     h = hashlib.sha256()
     for f in ("attn_sm100.cu", "sm100_ptx.cuh", "sage_common.cuh"):
-        with open(os.path.join(ROOT, "quantized_attention_03_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "quantized_attention_03_b200", "csrc", f)) as fh:
+            for line in fh:
+                code = re.sub(r"//.*", "", line).strip()
+                if code:
+                    h.update(code.encode())
     return h.hexdigest()[:16]
 
 
@@ -388,6 +424,12 @@ def main():
     ap.add_argument("--ref-rows", type=int, default=64)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--B", type=int, default=None, help="override the batch (profiling)")
+    ap.add_argument("--N", type=int, default=None, help="override the sequence length")
+    ap.add_argument("--d", type=int, default=None, choices=[64, 128])
+    ap.add_argument("--causal", action="store_true")
+    ap.add_argument("--pv", choices=["fp16", "fp8"], default=None)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

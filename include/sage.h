@@ -182,6 +182,15 @@ SAGE_API sage_status_t sage_attn_fwd_noalloc(const void *q, const void *k, const
                                              int smooth_k, int pv_mode, float sm_scale,
                                              sage_stream_t stream);
 
+/*
+ * Debug: exercises the bounded-wait path every kernel uses. One thread waits on a
+ * barrier that nothing arrives on; after timeout_ns (1 us .. 1 s) the wait gives up,
+ * SAGE_ERR_TIMEOUT is recorded in the device status word and the kernel returns, so the
+ * context stays usable. Read the result with sage_get_device_status().
+ */
+SAGE_API sage_status_t sage_debug_wait_timeout(unsigned long long timeout_ns,
+                                               sage_stream_t stream);
+
 /* Synchronizes `stream`, returns the device status word (SAGE_OK if clean) and clears
  * it. SAGE_ERR_CUDA if the synchronization itself failed. */
 SAGE_API sage_status_t sage_get_device_status(sage_stream_t stream);

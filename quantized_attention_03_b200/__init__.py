@@ -55,6 +55,7 @@ SIGNATURES = {
                                      _P]),
     "sage_debug_qk_int32": (_S, [_P, _P, _P, _I, _I, _I, _I, _P]),
     "sage_attn_fwd_noalloc": (_S, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
+    "sage_debug_wait_timeout": (_S, [ctypes.c_ulonglong, _P]),
     "sage_get_device_status": (_S, [_P]),
     "sage_status_string": (ctypes.c_char_p, [_I]),
     "sage_last_cuda_error": (_I, []),
@@ -182,6 +183,10 @@ def sage_attn_fwd_noalloc(q, k, v, out, B, H, N, d, causal, smooth_k, pv_mode, s
     """sage_attn_fwd with the library's static scratch (no allocation; see sage.h)."""
     return _call("sage_attn_fwd_noalloc", _ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d,
                  int(causal), int(smooth_k), int(pv_mode), float(sm_scale), _stream(stream))
+
+
+def sage_debug_wait_timeout(timeout_ns, stream=None):
+    return _call("sage_debug_wait_timeout", int(timeout_ns), _stream(stream))
 
 
 def sage_get_device_status(stream=None) -> int:

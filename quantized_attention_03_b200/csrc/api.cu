@@ -421,6 +421,19 @@ sage_status_t sage_debug_qk_int32(const int8_t *q_i8, const int8_t *k_i8, int32_
     return e == cudaSuccess ? SAGE_OK : cuda_fail(e);
 }
 
+sage_status_t sage_debug_wait_timeout(unsigned long long timeout_ns, sage_stream_t stream)
+{
+    if (timeout_ns < 1000ull || timeout_ns > 1000000000ull)
+        return SAGE_ERR_INVALID_ARG;
+    sage_status_t r;
+    int *status = status_ptr(&r);
+    if (!status)
+        return r;
+    cudaError_t e =
+        launch_wait_selftest(status, timeout_ns, reinterpret_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SAGE_OK : cuda_fail(e);
+}
+
 sage_status_t sage_get_device_status(sage_stream_t stream)
 {
     cudaError_t e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));

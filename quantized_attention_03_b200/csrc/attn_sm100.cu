@@ -1,31 +1,34 @@
 // K-ATTN: the fused quantized attention pass for sm_100a.
 //
-// Method (「SageAttention：低比特量化Attention，实现推理加速」, section 技术方案; 「4比特量化三倍加速不掉点！清华即插即用的SageAttention迎来升级」, 技术方案
-// (3)-(4)): S = Q_i8 K_i8^T with INT32 accumulation, dequantized by
-// q_scale * k_scale * sm_scale, FlashAttention online softmax over 128-key tiles, and
-// P.V with P, V in FP16 (FP16 mode) or both in E4M3 (FP8 mode), each tile's P.V
-// product accumulated across tiles in fp32 registers (the two-level accumulation of
-// 「4比特量化三倍加速不掉点！清华即插即用的SageAttention迎来升级」, item (3)).
+// Method (「SageAttention：低比特量化Attention，实现推理加速」, section 技术方案;
+// 「4比特量化三倍加速不掉点！清华即插即用的SageAttention迎来升级」, 技术方案 (3)-(4)):
+// S = Q_i8 K_i8^T with INT32 accumulation, dequantized by q_scale * k_scale * sm_scale,
+// FlashAttention online softmax over 128-key tiles, and P.V with P, V in FP16 (FP16
+// mode) or both in E4M3 (FP8 mode); each tile's P.V is a fresh tensor-core product
+// added into an fp32 accumulator across tiles.
 //
-// B200 design. One CTA owns NQT = 2 query tiles of 128 rows of one (sequence, head)
-// and walks the KV tiles once for both, so each K/V tile read from L2 feeds 256 rows:
-//   warps 0-3 / 4-7   softmax warpgroups, one per query tile: thread t owns row t
-//                     (TMEM lane t); O (d fp32) lives in its registers
+// B200 design. One CTA owns NQT = 2 query tiles of 128 rows of one (sequence, head) and
+// walks the KV tiles once for both, so each K/V tile read from L2 feeds 256 rows:
+//   warps 0-3 / 4-7   softmax warpgroups, one per query tile; thread t owns row t
+//                     (TMEM lane t)
 //   warp 8            TMA producer: Q tiles once, then K/V tiles into a STAGES-deep
 //                     shared-memory ring (mbarrier full/empty pairs)
-//   warp 9            MMA issuer (one thread) + TMEM owner:
-//                       S_i = Q_i K^T       tcgen05.mma kind::i8 -> TMEM (s32, 128 cols)
-//                       PV_i = P_i V        tcgen05.mma kind::f16 | kind::f8f6f4 with P
-//                                           read from TMEM (aliasing S_i) and V from
-//                                           shared memory (MN-major) -> TMEM (f32)
+//   warp 9            MMA issuer (one thread) and TMEM owner:
+//                       S_i  = Q_i K^T    tcgen05.mma kind::i8, smem x smem -> TMEM s32
+//                       O_i += P_i V      tcgen05.mma kind::f16 | kind::f8f6f4, P and V
+//                                         from shared memory (V MN-major) -> TMEM f32
 //   warps 10-11       idle (complete the warpgroup for the register split)
-// TMEM columns: [S_0 | S_1 | PV_0 | PV_1] = 2*128 + 2*d <= 512.
+// TMEM columns: [S_0 | S_1 | O_0 | O_1] = 2*128 + 2*d <= 512.
 //
-// Softmax per tile (thread = row): pass 1 reads S (int32) and takes the integer max of
-// each 64-key half (the two K blocks carry different scales); pass 2 re-reads S,
-// p = 2^(S*sc - m) with one FFMA + ex2, sums p, packs P to f16 (or E4M3 of 448 p) and
-// stores it over S in TMEM. The O update for tile j-1 (O = alpha O + PV) is done after
-// P of tile j is handed to the tensor core, so the softmax never waits on its own PV.
+// Per tile, a softmax thread reads its 128 scores from TMEM into registers once and
+// releases S_i at once, so the tensor core computes S_i(j+1) while the exponentials of
+// tile j run. It takes the integer max of each 64-key half (the two K blocks carry
+// their own scales), converts S to fp32 exactly with a magic-number bias, forms
+// p = 2^(S*sc - m) with one packed FFMA + ex2, and writes P (f16, or E4M3 of 448 p)
+// into shared memory in the 128-byte-swizzled K-major layout the MMA reads. O lives in
+// TMEM; a row's O is rescaled in place only when its reference max m moves (in FP16
+// mode only when the max grows by more than 2^8, so P <= 256; in FP8 mode on every
+// increase, so 448 P fits E4M3).
 //
 // Every wait is bounded (global timer); a timeout sets the device status word, all
 // roles drain and the CTA releases TMEM and exits. Nothing traps.
@@ -55,9 +58,10 @@ struct Cfg {
     static constexpr int kQBytes = BM * D;                   // int8 Q tile
     static constexpr int kKBytes = BN * D;                   // int8 K tile
     static constexpr int kVBytes = BN * D * (FP8 ? 1 : 2);   // V tile
+    static constexpr int kPBytes = BM * BN * (FP8 ? 1 : 2);      // P tile (A operand of P.V)
     static constexpr int kStageBytes = kKBytes + kVBytes;
-    static constexpr int kBudget = 200 * 1024;
-    static constexpr int kStagesFit = (kBudget - NQT * kQBytes) / kStageBytes;
+    static constexpr int kBudget = 220 * 1024;
+    static constexpr int kStagesFit = (kBudget - NQT * (kQBytes + kPBytes)) / kStageBytes;
     static constexpr int STAGES = kStagesFit > 4 ? 4 : kStagesFit;
     static_assert(STAGES >= 2, "shared-memory ring too shallow");
     static constexpr int kSoftmaxWarps = 4 * NQT;
@@ -71,9 +75,10 @@ struct Cfg {
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + NQT * kQBytes;
     static constexpr int kOffV = kOffK + STAGES * kKBytes;
-    static constexpr int kOffBar = kOffV + STAGES * kVBytes;
+    static constexpr int kOffP = kOffV + STAGES * kVBytes;
+    static constexpr int kOffBar = kOffP + NQT * kPBytes;
     // barriers: q, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[NQT],
-    //           p_full[NQT], pv_full[NQT], turn[NQT], drain
+    //           p_full[NQT], pv_full[NQT], s_free[NQT], drain
     static constexpr int kNumBars = 1 + 4 * STAGES + 4 * NQT + 1;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
@@ -86,6 +91,10 @@ struct Cfg {
     // Q/K operand geometry (K-major, one swizzle atom wide)
     static constexpr int kQkSwizzle = D == 128 ? 2 : 4;                 // 128B / 64B
     static constexpr int kQkSbo = 8 * D;                                 // 8 rows
+    // P in shared memory, K-major 128-byte swizzle: 64-key (FP16) or 128-key (FP8)
+    // sub-tiles of 128 rows x 128 bytes
+    static constexpr int kPSubBytes = BM * 128;
+    static constexpr int kPSubKeys = FP8 ? 128 : 64;
     static constexpr int kVSwizzle = kVRowBytes == 128 ? 2 : 4;
     static constexpr int kVSbo = 8 * kVRowBytes;
     // The reference max of a row is refreshed only when the row max exceeds it by more
@@ -138,7 +147,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     return ok;
 }
 
-template <int D, bool FP8, int NQT, bool DUMP, bool PINGPONG>
+template <int D, bool FP8, int NQT, bool DUMP>
 __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const KParams p)
@@ -163,6 +172,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
     uint8_t *sQ = smem + C::kOffQ;
     uint8_t *sK = smem + C::kOffK;
     uint8_t *sV = smem + C::kOffV;
+    uint8_t *sP = smem + C::kOffP;
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
     uint64_t *bar_q = bars;
     uint64_t *k_full = bars + 1;
@@ -172,8 +182,8 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
     uint64_t *s_full = v_empty + C::STAGES;
     uint64_t *p_full = s_full + NQT;
     uint64_t *pv_full = p_full + NQT;
-    uint64_t *turn = pv_full + NQT;        // softmax warpgroups take turns on the exp phase
-    uint64_t *bar_drain = turn + NQT;
+    uint64_t *s_free = pv_full + NQT;      // S_i read into registers: TMEM free for S_i(j+1)
+    uint64_t *bar_drain = s_free + NQT;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffMisc);
     volatile int *abort = reinterpret_cast<volatile int *>(smem + C::kOffMisc + 4);
 
@@ -190,7 +200,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
             mbar_init(&s_full[i], 1);
             mbar_init(&p_full[i], 4);
             mbar_init(&pv_full[i], 1);
-            mbar_init(&turn[i], 4);
+            mbar_init(&s_free[i], 4);
         }
         mbar_init(bar_drain, 1);
         *abort = 0;
@@ -253,16 +263,25 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
                             drow[kcol0 + e] = static_cast<int>(sreg[e / 32][e % 32]);
                 }
             }
+            // S_i is in registers: the tensor core may write S_i(j+1) now
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(&s_free[i]);
+
             // integer maxima of the two 64-key halves (the two K blocks have own scales)
             int im[2] = {INT_MIN, INT_MIN};
 #pragma unroll
             for (int ch = 0; ch < 4; ch++) {
                 const uint32_t keep = need_mask ? chunk_mask(col_lim - kcol0 - ch * 32) : ~0u;
-                int mx = INT_MIN;
+                int mx0 = INT_MIN, mx1 = INT_MIN;
 #pragma unroll
-                for (int e = 0; e < 32; e++)
-                    mx = ((keep >> e) & 1u) ? max(mx, static_cast<int>(sreg[ch][e])) : mx;
-                im[ch / 2] = max(im[ch / 2], mx);
+                for (int e = 0; e < 32; e += 2) {
+                    mx0 = ((keep >> e) & 1u) ? max(mx0, static_cast<int>(sreg[ch][e])) : mx0;
+                    mx1 = ((keep >> (e + 1)) & 1u) ? max(mx1, static_cast<int>(sreg[ch][e + 1]))
+                                                   : mx1;
+                }
+                im[ch / 2] = max(im[ch / 2], max(mx0, mx1));
             }
             float tmax = -INFINITY;
             if (im[0] != INT_MIN)
@@ -274,12 +293,10 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
             const float bias = FP8 ? m_new - kLog2_448 : m_new;
 
             // p = 2^(S sc - m): S to fp32 exactly through the magic bias
-            // (|S| <= 127^2 d < 2^22), one packed FFMA, ex2; P packed over S in TMEM.
-            if constexpr (PINGPONG) {
-                if (!(ok = warp_wait(&turn[i], (j & 1) ^ (i == 0 ? 1 : 0), abort, p.status)))
-                    break;
-            }
-            float2 lsum2 = make_float2(0.0f, 0.0f);
+            // (|S| <= 127^2 d < 2^22), one packed FFMA, ex2; packed to f16 / E4M3 words
+            constexpr int kWords = FP8 ? C::BN / 4 : C::BN / 2;
+            uint32_t pw[kWords];
+            float2 lsum2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
             for (int ch = 0; ch < 8; ch++) {
                 const float sc = ch < 4 ? sc0 : sc1;
@@ -297,60 +314,69 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
                     pv.y = ((keep >> (e + 1)) & 1u) ? pv.y : 0.0f;
                     pe[e] = pv.x;
                     pe[e + 1] = pv.y;
-                    lsum2 = add2(lsum2, pv);
+                    lsum2[(e >> 1) & 1] = add2(lsum2[(e >> 1) & 1], pv);
                 }
                 if constexpr (!FP8) {
-                    uint32_t w[8];
 #pragma unroll
                     for (int e = 0; e < 8; e++)
-                        w[e] = pack_half2(pe[2 * e], pe[2 * e + 1]);
-                    tmem_st8(tS + ch * 8, w);
+                        pw[ch * 8 + e] = pack_half2(pe[2 * e], pe[2 * e + 1]);
                 } else {
-                    uint32_t w[4];
 #pragma unroll
                     for (int e = 0; e < 4; e++)
-                        w[e] = static_cast<uint32_t>(pack_e4m3x2(pe[4 * e], pe[4 * e + 1])) |
-                               (static_cast<uint32_t>(pack_e4m3x2(pe[4 * e + 2], pe[4 * e + 3]))
-                                << 16);
-                    tmem_st4(tS + ch * 4, w);
+                        pw[ch * 4 + e] =
+                            static_cast<uint32_t>(pack_e4m3x2(pe[4 * e], pe[4 * e + 1])) |
+                            (static_cast<uint32_t>(pack_e4m3x2(pe[4 * e + 2], pe[4 * e + 3])) << 16);
                 }
             }
-            l = alpha * l + (lsum2.x + lsum2.y);
+            l = alpha * l + (lsum2[0].x + lsum2[0].y + lsum2[1].x + lsum2[1].y);
             m_ref = m_new;
 
-            // O (fp32 in TMEM, accumulated across tiles by the tensor core) is rescaled
-            // before this tile's P.V lands on it; the whole warp takes part if any row
-            // of it moved its reference max
-            if (j > 0 && __any_sync(0xffffffffu, alpha != 1.0f)) {
+            // PV_i(j-1) must be complete: it reads the P buffer rewritten below, and O is
+            // rescaled in TMEM before this tile's P.V lands on it (the whole warp takes
+            // part if any of its rows moved its reference max)
+            if (j > 0) {
                 if (!(ok = warp_wait(&pv_full[i], (j - 1) & 1, abort, p.status)))
                     break;
                 tc_fence_after();
-                uint32_t orow[D / 32][32];
+                if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+                    uint32_t orow[D / 32][32];
 #pragma unroll
-                for (int ch = 0; ch < D / 32; ch++)
-                    tmem_ld32_async(tO + ch * 32, orow[ch]);
+                    for (int ch = 0; ch < D / 32; ch++)
+                        tmem_ld32_async(tO + ch * 32, orow[ch]);
 #pragma unroll
-                for (int ch = 0; ch < D / 32; ch++) {
-                    tmem_ld_wait(orow[ch]);
+                    for (int ch = 0; ch < D / 32; ch++) {
+                        tmem_ld_wait(orow[ch]);
 #pragma unroll
-                    for (int e = 0; e < 32; e += 2) {
-                        const float2 ov = fma2(make_float2(__uint_as_float(orow[ch][e]),
-                                                           __uint_as_float(orow[ch][e + 1])),
-                                               make_float2(alpha, alpha), make_float2(0.0f, 0.0f));
-                        orow[ch][e] = __float_as_uint(ov.x);
-                        orow[ch][e + 1] = __float_as_uint(ov.y);
+                        for (int e = 0; e < 32; e += 2) {
+                            const float2 ov = fma2(make_float2(__uint_as_float(orow[ch][e]),
+                                                               __uint_as_float(orow[ch][e + 1])),
+                                                   make_float2(alpha, alpha),
+                                                   make_float2(0.0f, 0.0f));
+                            orow[ch][e] = __float_as_uint(ov.x);
+                            orow[ch][e + 1] = __float_as_uint(ov.y);
+                        }
+                        tmem_st32(tO + ch * 32, orow[ch]);
                     }
-                    tmem_st32(tO + ch * 32, orow[ch]);
+                    tmem_st_wait();
                 }
             }
-            tmem_st_wait();
+            // P row into shared memory in the K-major 128-byte-swizzle layout: 16-byte
+            // chunk c of row r sits at chunk c ^ (r % 8) of the row's 128-byte line
+            {
+                const uint32_t prow = smem_u32(sP) + i * C::kPBytes + row_in_tile * 128;
+                const uint32_t sw = row_in_tile & 7;
+#pragma unroll
+                for (int c = 0; c < kWords / 4; c++) {
+                    const int sub = c / 8, c8 = c % 8;
+                    st_shared_v4(prow + sub * C::kPSubBytes + ((c8 ^ sw) << 4), pw[4 * c],
+                                 pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+                }
+            }
+            fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
+            if (lane == 0)
                 mbar_arrive(&p_full[i]);
-                if constexpr (PINGPONG)
-                    mbar_arrive(&turn[i ^ 1]);   // the other warpgroup's exp phase may start
-            }
         }
         // epilogue: the last P.V, normalize, round to fp16, store the row
         if (ok && (ok = warp_wait(&pv_full[i], (nkv - 1) & 1, abort, p.status))) {
@@ -456,18 +482,21 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
                 }
                 mma_commit(&s_full[i]);
             };
+            const uint64_t dP0 = smem_desc(smem_u32(sP), 16, 1024, 2 /*128B*/);
             auto issue_pv = [&](int i, int stg, int j) {
                 const uint32_t dO = tmem_base + NQT * C::BN + i * D;
-                const uint32_t aP = tmem_base + i * C::BN;
 #pragma unroll
                 for (int kk = 0; kk < C::BN / C::kPvK; kk++) {
+                    const int key0 = kk * C::kPvK;            // first key of this k-step
+                    const uint64_t a = dP0 + ((i * C::kPBytes + (key0 / C::kPSubKeys) * C::kPSubBytes +
+                                               (key0 % C::kPSubKeys) * (FP8 ? 1 : 2)) >> 4);
                     const uint64_t b =
-                        dV0 + ((stg * C::kVBytes + kk * C::kPvK * C::kVRowBytes) >> 4);
+                        dV0 + ((stg * C::kVBytes + key0 * C::kVRowBytes) >> 4);
                     const uint32_t acc = (kk > 0 || j > 0) ? 1u : 0u;
                     if constexpr (FP8)
-                        mma_f8_ts(dO, aP + kk * 8, b, idesc_pv, acc);
+                        mma_f8_ss(dO, a, b, idesc_pv, acc);
                     else
-                        mma_f16_ts(dO, aP + kk * 8, b, idesc_pv, acc);
+                        mma_f16_ss(dO, a, b, idesc_pv, acc);
                 }
                 mma_commit(&pv_full[i]);
             };
@@ -475,10 +504,9 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
                 return mbar_wait(bar, parity, abort, p.status, status_bit(SAGE_ERR_TIMEOUT),
                                  kTimeoutNs);
             };
-            // Issue order S_0(0) S_1(0) | PV_0(j) S_0(j+1) PV_1(j) S_1(j+1) | ...: each
-            // query tile's next scores follow its own P.V, so one softmax warpgroup works
-            // while the tensor core serves the other. S_i(j+1) overwrites P_i(j), so it is
-            // issued only once PV_i(j) has completed.
+            // S_i(j+1) is issued as soon as the softmax warps have read S_i(j) into
+            // registers, so the next scores are computed while the current tile's
+            // exponentials run; PV_i(j) follows once P_i(j) is in shared memory.
             bool ok = wait(bar_q, 0) && wait(&k_full[0], 0);
             if (ok) {
                 tc_fence_after();
@@ -489,30 +517,32 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
             for (int j = 0; j < nkv && ok; j++) {
                 const int stg = j % C::STAGES;
                 const uint32_t ph = (j / C::STAGES) & 1;
-                const int stg1 = (j + 1) % C::STAGES;
-                const uint32_t ph1 = ((j + 1) / C::STAGES) & 1;
-                const bool more = j + 1 < nkv;
+                if (j + 1 < nkv) {
+                    const int stg1 = (j + 1) % C::STAGES;
+                    const uint32_t ph1 = ((j + 1) / C::STAGES) & 1;
+                    if (!(ok = wait(&k_full[stg1], ph1)))
+                        break;
+                    for (int i = 0; i < NQT && ok; i++) {
+                        if (!(ok = wait(&s_free[i], j & 1)))
+                            break;
+                        tc_fence_after();
+                        issue_s(i, stg1);
+                    }
+                    if (!ok)
+                        break;
+                    mma_commit(&k_empty[stg1]);
+                }
                 if (!(ok = wait(&v_full[stg], ph)))
-                    break;
-                if (more && !(ok = wait(&k_full[stg1], ph1)))
                     break;
                 for (int i = 0; i < NQT && ok; i++) {
                     if (!(ok = wait(&p_full[i], j & 1)))
                         break;
                     tc_fence_after();
                     issue_pv(i, stg, j);
-                    if (more) {
-                        if (!(ok = wait(&pv_full[i], j & 1)))
-                            break;
-                        tc_fence_after();
-                        issue_s(i, stg1);
-                    }
                 }
                 if (!ok)
                     break;
                 mma_commit(&v_empty[stg]);
-                if (more)
-                    mma_commit(&k_empty[stg1]);
             }
             // drain: every MMA issued above has completed before TMEM is released
             mma_commit(bar_drain);
@@ -586,10 +616,6 @@ bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int elem
     return r == CUDA_SUCCESS;
 }
 
-#ifndef SAGE_PINGPONG
-#define SAGE_PINGPONG 0
-#endif
-
 template <int D, bool FP8, int NQT, bool DUMP>
 cudaError_t run(const AttnArgs &a, const SeqLayout &L, int *status, cudaStream_t st,
                 sage_status_t *host_err)
@@ -622,7 +648,7 @@ cudaError_t run(const AttnArgs &a, const SeqLayout &L, int *status, cudaStream_t
     p.sc_log2 = a.sm_scale * kLog2e;
     p.status = status;
 
-    auto kern = attn_kernel<D, FP8, NQT, DUMP, SAGE_PINGPONG != 0>;
+    auto kern = attn_kernel<D, FP8, NQT, DUMP>;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess)

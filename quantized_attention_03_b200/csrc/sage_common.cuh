@@ -87,5 +87,6 @@ struct AttnArgs {
 };
 cudaError_t launch_attention(const AttnArgs &a, const SeqLayout &L, int *status, cudaStream_t st,
                              sage_status_t *host_err);
+cudaError_t launch_wait_selftest(int *status, uint64_t timeout_ns, cudaStream_t st);
 
 }  // namespace sage

@@ -216,6 +216,20 @@ def _workload_name(W):
             f"{'causal' if W['causal'] else 'non-causal'} PV={W['pv_mode']} smooth_k")
 
 
+def _keep_pool_cached(device: int):
+    """Let the device's stream-ordered memory pool keep freed blocks (plumbing): the
+    library's own small scratch allocations then never go back to the driver between
+    steps."""
+    try:
+        from cuda.bindings import runtime as rt
+        err, pool = rt.cudaDeviceGetDefaultMemPool(device)
+        if err == rt.cudaError_t.cudaSuccess:
+            rt.cudaMemPoolSetAttribute(pool, rt.cudaMemPoolAttr.cudaMemPoolAttrReleaseThreshold,
+                                       rt.cuuint64_t(2 ** 64 - 1))
+    except Exception:
+        pass
+
+
 def run_ours(args):
     import torch
     import quantized_attention_03_b200 as sage
@@ -223,6 +237,7 @@ def run_ours(args):
 
     world, rank, local = _dist()
     torch.cuda.set_device(local)
+    _keep_pool_cached(local)
     dist = None
     if world > 1:
         import torch.distributed as dist

@@ -38,6 +38,7 @@
 #include <cudaTypedefs.h>
 
 #include <climits>
+#include <type_traits>
 #include <cstdio>
 #include <mutex>
 
@@ -269,67 +270,83 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
             if (lane == 0)
                 mbar_arrive(&s_free[i]);
 
-            // integer maxima of the two 64-key halves (the two K blocks have own scales)
-            int im[2] = {INT_MIN, INT_MIN};
-#pragma unroll
-            for (int ch = 0; ch < 4; ch++) {
-                const uint32_t keep = need_mask ? chunk_mask(col_lim - kcol0 - ch * 32) : ~0u;
-                int mx0 = INT_MIN, mx1 = INT_MIN;
-#pragma unroll
-                for (int e = 0; e < 32; e += 2) {
-                    mx0 = ((keep >> e) & 1u) ? max(mx0, static_cast<int>(sreg[ch][e])) : mx0;
-                    mx1 = ((keep >> (e + 1)) & 1u) ? max(mx1, static_cast<int>(sreg[ch][e + 1]))
-                                                   : mx1;
-                }
-                im[ch / 2] = max(im[ch / 2], max(mx0, mx1));
-            }
-            float tmax = -INFINITY;
-            if (im[0] != INT_MIN)
-                tmax = static_cast<float>(im[0]) * sc0;
-            if (im[1] != INT_MIN)
-                tmax = fmaxf(tmax, static_cast<float>(im[1]) * sc1);
-            const float m_new = tmax > m_ref + C::kRescaleSlack ? tmax : m_ref;
-            const float alpha = m_new == m_ref ? 1.0f : ex2_approx(m_ref - m_new);
-            const float bias = FP8 ? m_new - kLog2_448 : m_new;
-
-            // p = 2^(S sc - m): S to fp32 exactly through the magic bias
-            // (|S| <= 127^2 d < 2^22), one packed FFMA, ex2; packed to f16 / E4M3 words
+            // Score math of one tile. Only the diagonal (causal) and the ragged last tile
+            // need the per-key visibility mask; every other tile takes the MASKED = false
+            // instantiation with no per-key tests.
             constexpr int kWords = FP8 ? C::BN / 4 : C::BN / 2;
             uint32_t pw[kWords];
-            float2 lsum2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+            float alpha = 1.0f;
+            auto tile_math = [&](auto masked) {
+                constexpr bool MASKED = decltype(masked)::value;
+                // integer maxima of the two 64-key halves (each K block has its own scale)
+                int im[2] = {INT_MIN, INT_MIN};
 #pragma unroll
-            for (int ch = 0; ch < 8; ch++) {
-                const float sc = ch < 4 ? sc0 : sc1;
-                const uint32_t keep =
-                    need_mask ? chunk_mask(col_lim - kcol0 - ch * 16) & 0xffffu : 0xffffu;
-                float pe[16];
+                for (int ch = 0; ch < 4; ch++) {
+                    const uint32_t keep = MASKED ? chunk_mask(col_lim - kcol0 - ch * 32) : ~0u;
+                    int mx[4] = {INT_MIN, INT_MIN, INT_MIN, INT_MIN};
 #pragma unroll
-                for (int e = 0; e < 16; e += 2) {
-                    float2 x = make_float2(magic_biased(sreg[ch / 2][(ch % 2) * 16 + e]),
-                                           magic_biased(sreg[ch / 2][(ch % 2) * 16 + e + 1]));
-                    x = add2(x, make_float2(-kMagic, -kMagic));          // exact S
-                    const float2 t = fma2(x, make_float2(sc, sc), make_float2(-bias, -bias));
-                    float2 pv = make_float2(ex2_approx(t.x), ex2_approx(t.y));
-                    pv.x = ((keep >> e) & 1u) ? pv.x : 0.0f;
-                    pv.y = ((keep >> (e + 1)) & 1u) ? pv.y : 0.0f;
-                    pe[e] = pv.x;
-                    pe[e + 1] = pv.y;
-                    lsum2[(e >> 1) & 1] = add2(lsum2[(e >> 1) & 1], pv);
+                    for (int e = 0; e < 32; e++) {
+                        const int v = static_cast<int>(sreg[ch][e]);
+                        if constexpr (MASKED)
+                            mx[e & 3] = ((keep >> e) & 1u) ? max(mx[e & 3], v) : mx[e & 3];
+                        else
+                            mx[e & 3] = max(mx[e & 3], v);
+                    }
+                    im[ch / 2] = max(im[ch / 2], max(max(mx[0], mx[1]), max(mx[2], mx[3])));
                 }
-                if constexpr (!FP8) {
+                float tmax = -INFINITY;
+                if (im[0] != INT_MIN)
+                    tmax = static_cast<float>(im[0]) * sc0;
+                if (im[1] != INT_MIN)
+                    tmax = fmaxf(tmax, static_cast<float>(im[1]) * sc1);
+                const float m_new = tmax > m_ref + C::kRescaleSlack ? tmax : m_ref;
+                alpha = m_new == m_ref ? 1.0f : ex2_approx(m_ref - m_new);
+                const float bias = FP8 ? m_new - kLog2_448 : m_new;
+
+                // p = 2^(S sc - m): S to fp32 exactly through the magic bias
+                // (|S| <= 127^2 d < 2^22), one packed FFMA, ex2; packed to f16 / E4M3
+                float2 lsum2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
-                    for (int e = 0; e < 8; e++)
-                        pw[ch * 8 + e] = pack_half2(pe[2 * e], pe[2 * e + 1]);
-                } else {
+                for (int ch = 0; ch < 8; ch++) {
+                    const float sc = ch < 4 ? sc0 : sc1;
+                    const uint32_t keep =
+                        MASKED ? chunk_mask(col_lim - kcol0 - ch * 16) & 0xffffu : 0xffffu;
+                    float pe[16];
 #pragma unroll
-                    for (int e = 0; e < 4; e++)
-                        pw[ch * 4 + e] =
-                            static_cast<uint32_t>(pack_e4m3x2(pe[4 * e], pe[4 * e + 1])) |
-                            (static_cast<uint32_t>(pack_e4m3x2(pe[4 * e + 2], pe[4 * e + 3])) << 16);
+                    for (int e = 0; e < 16; e += 2) {
+                        float2 x = make_float2(magic_biased(sreg[ch / 2][(ch % 2) * 16 + e]),
+                                               magic_biased(sreg[ch / 2][(ch % 2) * 16 + e + 1]));
+                        x = add2(x, make_float2(-kMagic, -kMagic));          // exact S
+                        const float2 t = fma2(x, make_float2(sc, sc), make_float2(-bias, -bias));
+                        float2 pv = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+                        if constexpr (MASKED) {
+                            pv.x = ((keep >> e) & 1u) ? pv.x : 0.0f;
+                            pv.y = ((keep >> (e + 1)) & 1u) ? pv.y : 0.0f;
+                        }
+                        pe[e] = pv.x;
+                        pe[e + 1] = pv.y;
+                        lsum2[(e >> 1) & 1] = add2(lsum2[(e >> 1) & 1], pv);
+                    }
+                    if constexpr (!FP8) {
+#pragma unroll
+                        for (int e = 0; e < 8; e++)
+                            pw[ch * 8 + e] = pack_half2(pe[2 * e], pe[2 * e + 1]);
+                    } else {
+#pragma unroll
+                        for (int e = 0; e < 4; e++)
+                            pw[ch * 4 + e] =
+                                static_cast<uint32_t>(pack_e4m3x2(pe[4 * e], pe[4 * e + 1])) |
+                                (static_cast<uint32_t>(pack_e4m3x2(pe[4 * e + 2], pe[4 * e + 3]))
+                                 << 16);
+                    }
                 }
-            }
-            l = alpha * l + (lsum2[0].x + lsum2[0].y + lsum2[1].x + lsum2[1].y);
-            m_ref = m_new;
+                l = alpha * l + (lsum2[0].x + lsum2[0].y + lsum2[1].x + lsum2[1].y);
+                m_ref = m_new;
+            };
+            if (need_mask)
+                tile_math(std::true_type{});
+            else
+                tile_math(std::false_type{});
 
             // PV_i(j-1) must be complete: it reads the P buffer rewritten below, and O is
             // rescaled in TMEM before this tile's P.V lands on it (the whole warp takes

@@ -52,6 +52,14 @@ namespace {
 constexpr uint64_t kTimeoutNs = 2000000000ull;   // 2 s: far above any legitimate wait
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLog2_448 = 8.807354922057604f;  // log2(448): E4M3 P = e4m3(448 p)
+#ifndef SAGE_EXP_EMU_EVERY
+#define SAGE_EXP_EMU_EVERY 0
+#endif
+// FP16 mode: one exponential pair in this many is evaluated by exp2_poly2 on the FMA
+// pipe instead of MUFU ex2 (0: none), so the two units share the work. Its 1e-4 relative
+// error is a fraction of an f16 ulp of P; E4M3 P (FP8 mode) always uses MUFU ex2, whose
+// error is far from the E4M3 rounding boundaries.
+constexpr int kEmuEveryF16 = SAGE_EXP_EMU_EVERY;
 
 template <int D, bool FP8, int NQT>
 struct Cfg {
@@ -318,7 +326,13 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
                                                magic_biased(sreg[ch / 2][(ch % 2) * 16 + e + 1]));
                         x = add2(x, make_float2(-kMagic, -kMagic));          // exact S
                         const float2 t = fma2(x, make_float2(sc, sc), make_float2(-bias, -bias));
-                        float2 pv = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+                        // one pair in kEmuEvery on the FMA pipe, the rest on MUFU
+                        float2 pv;
+                        constexpr int kEmuEvery = FP8 ? 0 : kEmuEveryF16;
+                        if (kEmuEvery > 0 && (e / 2) % kEmuEvery == kEmuEvery - 1)
+                            pv = exp2_poly2(t);
+                        else
+                            pv = make_float2(ex2_approx(t.x), ex2_approx(t.y));
                         if constexpr (MASKED) {
                             pv.x = ((keep >> e) & 1u) ? pv.x : 0.0f;
                             pv.y = ((keep >> (e + 1)) & 1u) ? pv.y : 0.0f;

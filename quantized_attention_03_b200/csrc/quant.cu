@@ -10,8 +10,10 @@
 //             (exact for |K| N < 2^29, so the mean does not depend on summation order)
 //             and the fp32 amax of |V|. Row chunks of 512 tokens, fp64 atomics.
 //   quant:    one CTA per 128-token chunk of Q (one Q block), K (two K blocks) or V;
-//             16-byte vector loads/stores, warp-shuffle amax, IEEE-exact fp32 divisions
-//             (__fdiv_rn) and round-half-even so codes match the definition bit for bit.
+//             16-byte vector loads/stores, warp-shuffle amax. Codes are the rounding of
+//             the IEEE fp32 quotient x / scale, computed as x * (1 / scale) with an exact
+//             division only where the two could round differently, so they match the
+//             definition bit for bit without a division per element.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -121,13 +123,39 @@ __device__ __forceinline__ float group_max(float x, float *s_red, int w0)
     return m;
 }
 
-__device__ __forceinline__ int8_t int8_code(float x, float s)
+constexpr float kRound = 12582912.0f;            // 1.5 * 2^23: adding it rounds to an integer
+constexpr int kRoundBits = 0x4B400000;
+
+// round-half-even(fl(x / s)) clamped to [-127, 127], where fl(x / s) is the IEEE fp32
+// quotient and r = fl(1 / s). The product x * r is within 2^-15 of fl(x / s) (|x / s| <=
+// 127.5 keeps every ulp <= 2^-17), so both round to the same integer unless the product
+// lies within 2^-15 of a half-integer; those rare elements take the exact division.
+__device__ __forceinline__ int8_t int8_code(float x, float s, float r)
 {
     if (s == 0.0f)
         return 0;
-    int c = __float2int_rn(__fdiv_rn(x, s));   // round half to even of the fp32 quotient
+    const float q = x * r;
+    const float b = q + kRound;                    // RNE integer in the low mantissa bits
+    const float d = fabsf(q - (b - kRound));       // distance to that integer, <= 1/2
+    int c = __float_as_int(b) - kRoundBits;
+    if (d > 0.5f - 3.0517578125e-05f)              // near a tie: exact IEEE quotient
+        c = __float2int_rn(__fdiv_rn(x, s));
     c = max(-127, min(127, c));
     return (int8_t)c;
+}
+
+// fl(x / s) for the E4M3 encoder, with r = fl(1 / s): the product x * r differs from the
+// IEEE quotient by at most a few ulps, which changes the E4M3 rounding only next to a
+// rounding midpoint of a normal E4M3 binade (low 20 mantissa bits near 1 << 19) or in the
+// E4M3 subnormal range; there the exact division is used.
+__device__ __forceinline__ float e4m3_quotient(float x, float s, float r)
+{
+    const float q = x * r;
+    const uint32_t m = __float_as_uint(q) & 0xFFFFFu;
+    const bool near_mid = (m > 0x80000u - 16u) && (m < 0x80000u + 16u);
+    if (near_mid || fabsf(q) < 0.015625f)          // 2^-6: E4M3 subnormals below this
+        return __fdiv_rn(x, s);
+    return q;
 }
 
 template <int D>
@@ -142,6 +170,7 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(
     constexpr int kVec = kHalf / 8;       // 16-byte loads per thread
     __shared__ float s_red[8];
     __shared__ float s_aux[D];            // K mean or V scale per channel
+    __shared__ float s_rcp[D];            // fl(1 / V scale) per channel
 
     const int s = blockIdx.z, h = blockIdx.y;
     int start, len;
@@ -183,6 +212,7 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(
         const int c = threadIdx.x;
         const float sv = __fdiv_rn(__uint_as_float(vamax[sh * D + c]), 448.0f);
         s_aux[c] = sv;
+        s_rcp[c] = sv != 0.0f ? __fdiv_rn(1.0f, sv) : 0.0f;
         if (chunk == 0)
             v_scale[sh * D + c] = sv;
     }
@@ -216,7 +246,7 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(
 #pragma unroll
             for (int e = 0; e < 4; e++) {
                 const float sv = s_aux[col0 + i + e];
-                qv[e] = sv != 0.0f ? __fdiv_rn(x[i + e], sv) : 0.0f;
+                qv[e] = sv != 0.0f ? e4m3_quotient(x[i + e], sv, s_rcp[col0 + i + e]) : 0.0f;
             }
             const uint32_t lo = pack_e4m3x2(qv[0], qv[1]);
             const uint32_t hi = pack_e4m3x2(qv[2], qv[3]);
@@ -256,13 +286,14 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(
     if (!valid)
         return;
 
+    const float rcp = scale != 0.0f ? __fdiv_rn(1.0f, scale) : 0.0f;
     uint32_t w[kHalf / 4];
 #pragma unroll
     for (int i = 0; i < kHalf; i += 4) {
-        const uint32_t b0 = (uint8_t)int8_code(x[i], scale);
-        const uint32_t b1 = (uint8_t)int8_code(x[i + 1], scale);
-        const uint32_t b2 = (uint8_t)int8_code(x[i + 2], scale);
-        const uint32_t b3 = (uint8_t)int8_code(x[i + 3], scale);
+        const uint32_t b0 = (uint8_t)int8_code(x[i], scale, rcp);
+        const uint32_t b1 = (uint8_t)int8_code(x[i + 1], scale, rcp);
+        const uint32_t b2 = (uint8_t)int8_code(x[i + 2], scale, rcp);
+        const uint32_t b3 = (uint8_t)int8_code(x[i + 3], scale, rcp);
         w[i / 4] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
     }
     int8_t *dst8 = (kind == 0 ? q_i8 : k_i8) + off;

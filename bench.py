@@ -119,6 +119,21 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+def max_over_ranks(ms: float, dist=None, device=None) -> float:
+    """Largest elapsed time over all ranks (the job finishes with its slowest rank)."""
+    if dist is None:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_tops(ops_per_step: float, steps: int, world: int, ms: float) -> float:
+    """Whole-job throughput: every rank processes the same workload in ms (max over ranks)."""
+    return world * ops_per_step * steps / (ms * 1e-3) / 1e12
+
+
 def _dist():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -318,14 +333,11 @@ def run_ours(args):
     total_ms = t_start.elapsed_time(t_end)
     attn_ms = [e1.elapsed_time(e2) for (_, e1, e2) in ev]
     quant_ms = [e0.elapsed_time(e1) for (e0, e1, _) in ev]
-    if dist is not None:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dist, dev)
 
     ops = _ops(B, H, N, d, W["causal"])
     ms_per_step = total_ms / args.steps
-    value = world * ops * args.steps / (total_ms * 1e-3) / 1e12
+    value = weak_scaling_tops(ops, args.steps, world, total_ms)
     attn_avg_ms = sum(attn_ms) / len(attn_ms)
     attn_tops = ops / (attn_avg_ms * 1e-3) / 1e12
 
@@ -356,14 +368,11 @@ def run_ours(args):
     s1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max(s0.elapsed_time(s1), 1e-9)
-    if dist is not None:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
     status = sage.sage_get_device_status()
     if status != 0:
         raise RuntimeError(f"device status after e2e: {sage.status_string(status)}")
-    e2e_value = world * ops * e2e_steps / (e2e_ms * 1e-3) / 1e12 if e2e_steps else None
+    e2e_value = weak_scaling_tops(ops, e2e_steps, world, e2e_ms) if e2e_steps else None
     elem_bytes = B * H * N * d * 2
 
     peaks, src = _peaks()

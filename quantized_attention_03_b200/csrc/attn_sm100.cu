@@ -61,6 +61,7 @@ constexpr float kLog2_448 = 8.807354922057604f;  // log2(448): E4M3 P = e4m3(448
 // error is far from the E4M3 rounding boundaries.
 constexpr int kEmuEveryF16 = SAGE_EXP_EMU_EVERY;
 
+
 template <int D, bool FP8, int NQT>
 struct Cfg {
     static constexpr int BM = 128, BN = 128;
@@ -225,7 +226,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
     if (warp < C::kSoftmaxWarps) {
         // ------------------------------------------------------------ softmax warps
         if constexpr (NQT == 2)
-            asm volatile("setmaxnreg.inc.sync.aligned.u32 224;\n" ::: "memory");
+            asm volatile("setmaxnreg.inc.sync.aligned.u32 216;\n" ::: "memory");
         const int i = warp / 4;                    // query tile within the CTA
         const int quarter = warp % 4;              // TMEM lane quarter of this warp
         const int qt = qt0 + i;
@@ -278,13 +279,11 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
             if (lane == 0)
                 mbar_arrive(&s_free[i]);
 
-            // Score math of one tile. Only the diagonal (causal) and the ragged last tile
-            // need the per-key visibility mask; every other tile takes the MASKED = false
-            // instantiation with no per-key tests.
-            constexpr int kWords = FP8 ? C::BN / 4 : C::BN / 2;
-            uint32_t pw[kWords];
-            float alpha = 1.0f;
-            auto tile_math = [&](auto masked) {
+            // Score math of one tile, in two steps around the wait for the previous P.V.
+            // Only the diagonal (causal) and the ragged last tile need the per-key
+            // visibility mask; every other tile takes the MASKED = false instantiation.
+            float alpha = 1.0f, bias = 0.0f;
+            auto tile_max = [&](auto masked) {
                 constexpr bool MASKED = decltype(masked)::value;
                 // integer maxima of the two 64-key halves (each K block has its own scale)
                 int im[2] = {INT_MIN, INT_MIN};
@@ -309,10 +308,64 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
                     tmax = fmaxf(tmax, static_cast<float>(im[1]) * sc1);
                 const float m_new = tmax > m_ref + C::kRescaleSlack ? tmax : m_ref;
                 alpha = m_new == m_ref ? 1.0f : ex2_approx(m_ref - m_new);
-                const float bias = FP8 ? m_new - kLog2_448 : m_new;
+                bias = FP8 ? m_new - kLog2_448 : m_new;
+                m_ref = m_new;
+            };
+            if (need_mask)
+                tile_max(std::true_type{});
+            else
+                tile_max(std::false_type{});
 
-                // p = 2^(S sc - m): S to fp32 exactly through the magic bias
-                // (|S| <= 127^2 d < 2^22), one packed FFMA, ex2; packed to f16 / E4M3
+            // PV_i(j-1) must be complete before the P buffer is rewritten, and O is
+            // rescaled in TMEM before this tile's P.V lands on it (the whole warp takes
+            // part if any of its rows moved its reference max)
+            auto await_pv_and_rescale = [&]() -> bool {
+                if (j == 0)
+                    return true;
+                if (!warp_wait(&pv_full[i], (j - 1) & 1, abort, p.status))
+                    return false;
+                tc_fence_after();
+                if (__any_sync(0xffffffffu, alpha != 1.0f)) {
+#pragma unroll
+                    for (int ch = 0; ch < D / 32; ch++) {
+                        uint32_t orow[32];
+                        tmem_ld32_async(tO + ch * 32, orow);
+                        tmem_ld_wait(orow);
+#pragma unroll
+                        for (int e = 0; e < 32; e += 2) {
+                            const float2 ov = fma2(make_float2(__uint_as_float(orow[e]),
+                                                               __uint_as_float(orow[e + 1])),
+                                                   make_float2(alpha, alpha),
+                                                   make_float2(0.0f, 0.0f));
+                            orow[e] = __float_as_uint(ov.x);
+                            orow[e + 1] = __float_as_uint(ov.y);
+                        }
+                        tmem_st32(tO + ch * 32, orow);
+                    }
+                    tmem_st_wait();
+                }
+                return true;
+            };
+            // FP16 mode streams each chunk of P to shared memory as it is produced (the
+            // P.V wait comes first); FP8 mode, whose P tile is half the size, packs the
+            // whole row in registers and stores it after the wait.
+            constexpr bool kStreamP = !FP8;
+            if constexpr (kStreamP) {
+                if (!(ok = await_pv_and_rescale()))
+                    break;
+            }
+            constexpr int kWords = FP8 ? C::BN / 4 : C::BN / 2;
+            uint32_t pw[kStreamP ? 1 : kWords];
+
+            // p = 2^(S sc - m): S to fp32 exactly through the magic bias
+            // (|S| <= 127^2 d < 2^22), one packed FFMA, ex2; each 16-key chunk is packed to
+            // f16 / E4M3. The P tile in shared memory is K-major with the 128-byte swizzle:
+            // 16-byte chunk c of row r sits at chunk c ^ (r % 8) of the row's 128-byte line.
+            auto tile_exp = [&](auto masked) {
+                constexpr bool MASKED = decltype(masked)::value;
+                [[maybe_unused]] const uint32_t prow =
+                    smem_u32(sP) + i * C::kPBytes + row_in_tile * 128;
+                [[maybe_unused]] const uint32_t sw = row_in_tile & 7;
                 float2 lsum2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
                 for (int ch = 0; ch < 8; ch++) {
@@ -327,12 +380,16 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
                         x = add2(x, make_float2(-kMagic, -kMagic));          // exact S
                         const float2 t = fma2(x, make_float2(sc, sc), make_float2(-bias, -bias));
                         // one pair in kEmuEvery on the FMA pipe, the rest on MUFU
-                        float2 pv;
                         constexpr int kEmuEvery = FP8 ? 0 : kEmuEveryF16;
-                        if (kEmuEvery > 0 && (e / 2) % kEmuEvery == kEmuEvery - 1)
-                            pv = exp2_poly2(t);
-                        else
+                        float2 pv;
+                        if constexpr (kEmuEvery > 0) {
+                            if ((e / 2) % kEmuEvery == kEmuEvery - 1)
+                                pv = exp2_poly2(t);
+                            else
+                                pv = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+                        } else {
                             pv = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+                        }
                         if constexpr (MASKED) {
                             pv.x = ((keep >> e) & 1u) ? pv.x : 0.0f;
                             pv.y = ((keep >> (e + 1)) & 1u) ? pv.y : 0.0f;
@@ -342,10 +399,17 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
                         lsum2[(e >> 1) & 1] = add2(lsum2[(e >> 1) & 1], pv);
                     }
                     if constexpr (!FP8) {
+                        // 16 keys = two 16-byte chunks of the 64-key sub-tile ch / 4
+                        uint32_t w[8];
 #pragma unroll
                         for (int e = 0; e < 8; e++)
-                            pw[ch * 8 + e] = pack_half2(pe[2 * e], pe[2 * e + 1]);
+                            w[e] = pack_half2(pe[2 * e], pe[2 * e + 1]);
+                        const uint32_t line = prow + (ch / 4) * C::kPSubBytes;
+                        const uint32_t c0 = (ch % 4) * 2;
+                        st_shared_v4(line + ((c0 ^ sw) << 4), w[0], w[1], w[2], w[3]);
+                        st_shared_v4(line + (((c0 + 1) ^ sw) << 4), w[4], w[5], w[6], w[7]);
                     } else {
+                        // 16 keys = one 16-byte chunk of the 128-key line, kept for later
 #pragma unroll
                         for (int e = 0; e < 4; e++)
                             pw[ch * 4 + e] =
@@ -355,53 +419,20 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
                     }
                 }
                 l = alpha * l + (lsum2[0].x + lsum2[0].y + lsum2[1].x + lsum2[1].y);
-                m_ref = m_new;
             };
             if (need_mask)
-                tile_math(std::true_type{});
+                tile_exp(std::true_type{});
             else
-                tile_math(std::false_type{});
-
-            // PV_i(j-1) must be complete: it reads the P buffer rewritten below, and O is
-            // rescaled in TMEM before this tile's P.V lands on it (the whole warp takes
-            // part if any of its rows moved its reference max)
-            if (j > 0) {
-                if (!(ok = warp_wait(&pv_full[i], (j - 1) & 1, abort, p.status)))
+                tile_exp(std::false_type{});
+            if constexpr (!kStreamP) {
+                if (!(ok = await_pv_and_rescale()))
                     break;
-                tc_fence_after();
-                if (__any_sync(0xffffffffu, alpha != 1.0f)) {
-                    uint32_t orow[D / 32][32];
-#pragma unroll
-                    for (int ch = 0; ch < D / 32; ch++)
-                        tmem_ld32_async(tO + ch * 32, orow[ch]);
-#pragma unroll
-                    for (int ch = 0; ch < D / 32; ch++) {
-                        tmem_ld_wait(orow[ch]);
-#pragma unroll
-                        for (int e = 0; e < 32; e += 2) {
-                            const float2 ov = fma2(make_float2(__uint_as_float(orow[ch][e]),
-                                                               __uint_as_float(orow[ch][e + 1])),
-                                                   make_float2(alpha, alpha),
-                                                   make_float2(0.0f, 0.0f));
-                            orow[ch][e] = __float_as_uint(ov.x);
-                            orow[ch][e + 1] = __float_as_uint(ov.y);
-                        }
-                        tmem_st32(tO + ch * 32, orow[ch]);
-                    }
-                    tmem_st_wait();
-                }
-            }
-            // P row into shared memory in the K-major 128-byte-swizzle layout: 16-byte
-            // chunk c of row r sits at chunk c ^ (r % 8) of the row's 128-byte line
-            {
                 const uint32_t prow = smem_u32(sP) + i * C::kPBytes + row_in_tile * 128;
                 const uint32_t sw = row_in_tile & 7;
 #pragma unroll
-                for (int c = 0; c < kWords / 4; c++) {
-                    const int sub = c / 8, c8 = c % 8;
-                    st_shared_v4(prow + sub * C::kPSubBytes + ((c8 ^ sw) << 4), pw[4 * c],
-                                 pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
-                }
+                for (int c = 0; c < kWords / 4; c++)
+                    st_shared_v4(prow + ((c ^ sw) << 4), pw[4 * c], pw[4 * c + 1], pw[4 * c + 2],
+                                 pw[4 * c + 3]);
             }
             fence_proxy_async_smem();
             tc_fence_before();
@@ -446,7 +477,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
     } else if (warp == C::kProducerWarp) {
         // ----------------------------------------------------------------- producer
         if constexpr (NQT == 2)
-            asm volatile("setmaxnreg.dec.sync.aligned.u32 56;\n" ::: "memory");
+            asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
         if (lane == 0) {
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
@@ -493,7 +524,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
     } else if (warp == C::kMmaWarp) {
         // ---------------------------------------------------------------- MMA issuer
         if constexpr (NQT == 2)
-            asm volatile("setmaxnreg.dec.sync.aligned.u32 56;\n" ::: "memory");
+            asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
         if (lane == 0) {
             constexpr uint32_t idesc_qk = instr_desc(2 /*s32*/, 1 /*s8*/, 1 /*s8*/, 0, 0, 128, 128);
             constexpr uint32_t idesc_pv = instr_desc(1 /*f32*/, 0 /*f16|e4m3*/, 0, 0,
@@ -581,7 +612,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
         }
     } else {
         if constexpr (NQT == 2)
-            asm volatile("setmaxnreg.dec.sync.aligned.u32 56;\n" ::: "memory");
+            asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
     }
 
     tc_fence_before();

@@ -280,9 +280,11 @@ def run_ours(args):
     out = torch.empty_like(q)
     stream = torch.cuda.current_stream()
 
+    ksum_ws = torch.empty(B * H * d * 8, dtype=torch.uint8, device=dev)   # fp64 K sums
+
     def quant():
-        sage.sage_quant_qk(q, k, q_i8, q_scale, k_i8, k_scale, k_mean, B, H, N, d,
-                           W["smooth_k"], stream)
+        sage.sage_quant_qk_ws(q, k, q_i8, q_scale, k_i8, k_scale, k_mean, B, H, N, d,
+                              W["smooth_k"], ksum_ws, ksum_ws.numel(), stream)
         if pv == sage.SAGE_PV_FP8:
             sage.sage_quant_v_fp8(v, vq, vscale, B, H, N, d, stream)
 

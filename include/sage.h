@@ -89,6 +89,13 @@ SAGE_API sage_status_t sage_quant_qk(const void *q, const void *k, int8_t *q_i8,
                             int8_t *k_i8, float *k_scale, float *k_mean, int B, int H, int N,
                             int d, int smooth_k, sage_stream_t stream);
 
+/* sage_quant_qk with caller-owned scratch for the fp64 K column sums: at least
+ * B*H*d*8 bytes, 16-byte aligned (unused when smooth_k == 0). Allocates nothing. */
+SAGE_API sage_status_t sage_quant_qk_ws(const void *q, const void *k, int8_t *q_i8,
+                                        float *q_scale, int8_t *k_i8, float *k_scale,
+                                        float *k_mean, int B, int H, int N, int d, int smooth_k,
+                                        void *workspace, size_t ws_bytes, sage_stream_t stream);
+
 /* sage_quant_qk for the packed varlen layout (cu_seqlens on the device; NULL reads the
  * buffers as dense [nseq, H, max_seqlen, d]). */
 SAGE_API sage_status_t sage_quant_qk_varlen(const void *q, const void *k, const int32_t *cu_seqlens,

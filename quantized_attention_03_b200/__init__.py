@@ -44,6 +44,7 @@ _S = ctypes.c_int  # sage_status_t
 SIGNATURES = {
     "sage_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
     "sage_quant_qk": (_S, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
+    "sage_quant_qk_ws": (_S, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]),
     "sage_quant_qk_varlen": (_S, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _I, _P]),
     "sage_quant_v_fp8": (_S, [_P, _P, _P, _I, _I, _I, _I, _P]),
     "sage_quant_v_fp8_varlen": (_S, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
@@ -127,6 +128,13 @@ def sage_workspace_size(nseq, H, max_seqlen, total_tokens, d, pv_mode) -> int:
 def sage_quant_qk(q, k, q_i8, q_scale, k_i8, k_scale, k_mean, B, H, N, d, smooth_k, stream=None):
     return _call("sage_quant_qk", _ptr(q), _ptr(k), _ptr(q_i8), _ptr(q_scale), _ptr(k_i8),
                  _ptr(k_scale), _ptr(k_mean), B, H, N, d, int(smooth_k), _stream(stream))
+
+
+def sage_quant_qk_ws(q, k, q_i8, q_scale, k_i8, k_scale, k_mean, B, H, N, d, smooth_k, workspace,
+                     ws_bytes, stream=None):
+    return _call("sage_quant_qk_ws", _ptr(q), _ptr(k), _ptr(q_i8), _ptr(q_scale), _ptr(k_i8),
+                 _ptr(k_scale), _ptr(k_mean), B, H, N, d, int(smooth_k), _ptr(workspace),
+                 int(ws_bytes), _stream(stream))
 
 
 def sage_quant_qk_varlen(q, k, cu_seqlens, nseq, total_tokens, max_seqlen, H, d, q_i8, q_scale,

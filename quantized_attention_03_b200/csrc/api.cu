@@ -156,6 +156,11 @@ sage_status_t alloc_ws(size_t bytes, cudaStream_t st, char **p)
     return SAGE_OK;
 }
 
+sage_status_t quant_qk_entry(const void *q, const void *k, const int32_t *cu_seqlens, int nseq,
+                             int total_tokens, int max_seqlen, int H, int d, int8_t *q_i8,
+                             float *q_scale, int8_t *k_i8, float *k_scale, float *k_mean,
+                             int smooth_k, void *workspace, size_t ws_bytes, cudaStream_t st);
+
 }  // namespace
 }  // namespace sage
 
@@ -174,23 +179,22 @@ sage_status_t sage_quant_qk(const void *q, const void *k, int8_t *q_i8, float *q
                             int8_t *k_i8, float *k_scale, float *k_mean, int B, int H, int N,
                             int d, int smooth_k, sage_stream_t stream)
 {
-    sage_status_t r = check_shape(B, H, N, d);
-    if (r != SAGE_OK)
-        return r;
-    if (B == 0 || H == 0 || N == 0)
-        return SAGE_OK;
-    if (!q || !k || !q_i8 || !q_scale || !k_i8 || !k_scale || !k_mean)
-        return SAGE_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(q_i8) || !aligned16(k_i8))
-        return SAGE_ERR_MISALIGNED;
-    return sage_quant_qk_varlen(q, k, nullptr, B, B * N, N, H, d, q_i8, q_scale, k_i8, k_scale,
-                                k_mean, smooth_k, stream);
+    if (B > 0 && N > 0 && (int64_t)B * N > INT32_MAX)
+        return SAGE_ERR_UNSUPPORTED;
+    return quant_qk_entry(q, k, nullptr, B, B * N, N, H, d, q_i8, q_scale, k_i8, k_scale, k_mean,
+                          smooth_k, nullptr, 0, reinterpret_cast<cudaStream_t>(stream));
 }
 
-sage_status_t sage_quant_qk_varlen(const void *q, const void *k, const int32_t *cu_seqlens,
-                                   int nseq, int total_tokens, int max_seqlen, int H, int d,
-                                   int8_t *q_i8, float *q_scale, int8_t *k_i8, float *k_scale,
-                                   float *k_mean, int smooth_k, sage_stream_t stream)
+}  // extern "C"
+
+namespace sage {
+namespace {
+// Steps 1-2 with optional caller scratch for the fp64 K column sums (nullptr: a
+// stream-ordered allocation is made and released).
+sage_status_t quant_qk_entry(const void *q, const void *k, const int32_t *cu_seqlens, int nseq,
+                             int total_tokens, int max_seqlen, int H, int d, int8_t *q_i8,
+                             float *q_scale, int8_t *k_i8, float *k_scale, float *k_mean,
+                             int smooth_k, void *workspace, size_t ws_bytes, cudaStream_t st)
 {
     sage_status_t r = check_shape(nseq, H, max_seqlen, d);
     if (r != SAGE_OK)
@@ -201,30 +205,71 @@ sage_status_t sage_quant_qk_varlen(const void *q, const void *k, const int32_t *
         return SAGE_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(q_i8) || !aligned16(k_i8))
         return SAGE_ERR_MISALIGNED;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const size_t sum_bytes = (size_t)nseq * H * d * 8;
+    if (workspace != nullptr && smooth_k) {
+        if (ws_bytes < sum_bytes)
+            return SAGE_ERR_WORKSPACE;
+        if ((reinterpret_cast<uintptr_t>(workspace) & 15u) != 0)
+            return SAGE_ERR_MISALIGNED;
+    }
     int *status = status_ptr(&r);
     if (!status)
         return r;
     const SeqLayout L = cu_seqlens ? SeqLayout::packed(cu_seqlens, nseq, total_tokens, max_seqlen, H, d)
                                    : SeqLayout::dense(nseq, H, max_seqlen, d);
     double *ksum = nullptr;
+    bool owned = false;
     cudaError_t e;
     if (smooth_k) {
-        void *p = nullptr;
-        if ((e = cudaMallocAsync(&p, (size_t)nseq * H * d * 8, st)) != cudaSuccess)
+        if (workspace != nullptr) {
+            ksum = static_cast<double *>(workspace);
+        } else {
+            void *p = nullptr;
+            if ((e = cudaMallocAsync(&p, sum_bytes, st)) != cudaSuccess)
+                return cuda_fail(e);
+            ksum = static_cast<double *>(p);
+            owned = true;
+        }
+        if ((e = cudaMemsetAsync(ksum, 0, sum_bytes, st)) != cudaSuccess ||
+            (e = launch_colstats(static_cast<const __half *>(k), nullptr, ksum, nullptr, L, status,
+                                 st)) != cudaSuccess) {
+            if (owned)
+                cudaFreeAsync(ksum, st);
             return cuda_fail(e);
-        ksum = static_cast<double *>(p);
-        if ((e = cudaMemsetAsync(ksum, 0, (size_t)nseq * H * d * 8, st)) != cudaSuccess)
-            return cuda_fail(e);
-        if ((e = launch_colstats(static_cast<const __half *>(k), nullptr, ksum, nullptr, L, status,
-                                 st)) != cudaSuccess)
-            return cuda_fail(e);
+        }
     }
     e = launch_quant(static_cast<const __half *>(q), static_cast<const __half *>(k), nullptr, ksum,
                      nullptr, q_i8, q_scale, k_i8, k_scale, k_mean, nullptr, nullptr, L, status, st);
-    if (ksum)
+    if (owned)
         cudaFreeAsync(ksum, st);
     return e == cudaSuccess ? SAGE_OK : cuda_fail(e);
+}
+}  // namespace
+}  // namespace sage
+
+extern "C" {
+
+sage_status_t sage_quant_qk_varlen(const void *q, const void *k, const int32_t *cu_seqlens,
+                                   int nseq, int total_tokens, int max_seqlen, int H, int d,
+                                   int8_t *q_i8, float *q_scale, int8_t *k_i8, float *k_scale,
+                                   float *k_mean, int smooth_k, sage_stream_t stream)
+{
+    return quant_qk_entry(q, k, cu_seqlens, nseq, total_tokens, max_seqlen, H, d, q_i8, q_scale,
+                          k_i8, k_scale, k_mean, smooth_k, nullptr, 0,
+                          reinterpret_cast<cudaStream_t>(stream));
+}
+
+sage_status_t sage_quant_qk_ws(const void *q, const void *k, int8_t *q_i8, float *q_scale,
+                               int8_t *k_i8, float *k_scale, float *k_mean, int B, int H, int N,
+                               int d, int smooth_k, void *workspace, size_t ws_bytes,
+                               sage_stream_t stream)
+{
+    if (workspace == nullptr && smooth_k && !(B == 0 || H == 0 || N == 0))
+        return SAGE_ERR_WORKSPACE;
+    if (B > 0 && N > 0 && (int64_t)B * N > INT32_MAX)
+        return SAGE_ERR_UNSUPPORTED;
+    return quant_qk_entry(q, k, nullptr, B, B * N, N, H, d, q_i8, q_scale, k_i8, k_scale, k_mean,
+                          smooth_k, workspace, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
 sage_status_t sage_quant_v_fp8_varlen(const void *v, const int32_t *cu_seqlens, int nseq,

@@ -110,3 +110,20 @@ def test_bad_cu_seqlens_sets_device_status():
     sage.quant_qk_varlen(q, q, cu, 60, True)
     assert sage.sage_get_device_status() == sage.SAGE_ERR_BAD_SEQLENS
     assert sage.sage_get_device_status() == sage.SAGE_OK                   # cleared
+
+
+def test_quant_qk_ws_matches_allocating_entry():
+    B, H, N, d = 2, 4, 700, 128
+    w = inputs.Workload("t", 77, B, H, N, d, False, 2.0)
+    q, k, _ = (t.cuda() for t in inputs.make_dense(w))
+    ref = sage.quant_qk(q, k, True)
+    got = {name: torch.empty_like(t) for name, t in ref.items()}
+    ws = torch.empty(B * H * d * 8, dtype=torch.uint8, device="cuda")
+    sage.sage_quant_qk_ws(q, k, got["q_i8"], got["q_scale"], got["k_i8"], got["k_scale"],
+                          got["k_mean"], B, H, N, d, True, ws, ws.numel())
+    assert sage.sage_get_device_status() == 0
+    for name in ref:
+        assert torch.equal(got[name], ref[name]), name
+    with pytest.raises(sage.SageError):
+        sage.sage_quant_qk_ws(q, k, got["q_i8"], got["q_scale"], got["k_i8"], got["k_scale"],
+                              got["k_mean"], B, H, N, d, True, ws, ws.numel() - 8)

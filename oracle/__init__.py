@@ -44,10 +44,10 @@ def lib():
         i64 = ctypes.c_int64
         i32 = ctypes.c_int
         f64 = ctypes.c_double
-        L.oracle_head_k_mean.argtypes = [P, i64, i64, i32, P]
+        L.oracle_head_channel_mean.argtypes = [P, i64, i64, i32, P]
         L.oracle_head_quant_int8.argtypes = [P, P, i64, i64, i32, i32, P, P]
-        L.oracle_head_quant_v_fp8.argtypes = [P, i64, i64, i32, P, P]
-        L.oracle_head_attn_quant.argtypes = [P, P, P, P, P, P, i64, i64, i32, i32, i32, f64,
+        L.oracle_head_quant_v_fp8.argtypes = [P, P, i64, i64, i32, P, P]
+        L.oracle_head_attn_quant.argtypes = [P, P, P, P, P, P, P, i64, i64, i32, i32, i32, f64,
                                              i32, i64, i64, P]
         L.oracle_head_attn_fp64.argtypes = [P, P, P, i64, i64, i32, i32, f64, i64, i64, P]
         L.oracle_f16_to_f64.argtypes = [ctypes.c_uint16]
@@ -140,15 +140,19 @@ def f16_to_f64(bits: int) -> float:
 # ------------------------------------------------------------------ method steps
 
 
-def k_mean(k: np.ndarray, layout: Layout, heads=None) -> np.ndarray:
-    """Per-channel token mean of K for every (or each selected) (sequence, head):
-    [nseq, H, d] fp32."""
-    kb = _bits16(k)
+def channel_mean(x: np.ndarray, layout: Layout, heads=None) -> np.ndarray:
+    """Per-channel token mean of K (smooth K) or V (smooth V) for every (or each
+    selected) (sequence, head): [nseq, H, d] fp32."""
+    xb = _bits16(x)
     mu = np.zeros((layout.nseq, layout.H, layout.d), np.float32)
     for s, h, off, n in layout.heads(heads):
-        lib().oracle_head_k_mean(_ptr(kb, off), n, layout.stride, layout.d,
-                                 _ptr(mu, (s * layout.H + h) * layout.d))
+        lib().oracle_head_channel_mean(_ptr(xb, off), n, layout.stride, layout.d,
+                                       _ptr(mu, (s * layout.H + h) * layout.d))
     return mu
+
+
+k_mean = channel_mean
+v_mean = channel_mean
 
 
 def quant_int8(x: np.ndarray, layout: Layout, blk: int, mu: Optional[np.ndarray] = None,
@@ -175,23 +179,28 @@ def quant_qk(q: np.ndarray, k: np.ndarray, layout: Layout, smooth_k: bool = True
     return dict(q_i8=q_i8, q_scale=q_scale, k_i8=k_i8, k_scale=k_scale, k_mean=mu)
 
 
-def quant_v_fp8(v: np.ndarray, layout: Layout, heads=None):
-    """E4M3 codes of V (same shape) and per-channel scales [nseq, H, d]."""
+def quant_v_fp8(v: np.ndarray, layout: Layout, heads=None, mu: Optional[np.ndarray] = None):
+    """E4M3 codes of V - mu (same shape) and per-channel scales [nseq, H, d]; mu is the
+    channel mean of V [nseq, H, d] for smooth V, None for none."""
     vb = _bits16(v)
     codes = np.zeros(v.shape, np.uint8)
     scales = np.zeros((layout.nseq, layout.H, layout.d), np.float32)
     for s, h, off, n in layout.heads(heads):
-        lib().oracle_head_quant_v_fp8(_ptr(vb, off), n, layout.stride, layout.d,
-                                      _ptr(codes, off), _ptr(scales, (s * layout.H + h) * layout.d))
+        sh = (s * layout.H + h) * layout.d
+        mup = _ptr(mu, sh) if mu is not None else None
+        lib().oracle_head_quant_v_fp8(_ptr(vb, off), mup, n, layout.stride, layout.d,
+                                      _ptr(codes, off), _ptr(scales, sh))
     return codes, scales
 
 
 def attn_quant(q_i8, q_scale, k_i8, k_scale, v, v_scale, layout: Layout, causal: bool,
                pv_mode: int, sm_scale: float, tile_n: int = 128, heads=None,
-               rows: Optional[Tuple[int, int]] = None) -> np.ndarray:
+               rows: Optional[Tuple[int, int]] = None,
+               v_mean: Optional[np.ndarray] = None) -> np.ndarray:
     """Quantized attention from codes and scales; fp16 output, NaN where not computed.
 
-    ``v`` is fp16 V (FP16 mode) or its E4M3 codes as uint8 (FP8 mode)."""
+    ``v`` is fp16 V (FP16 mode) or its E4M3 codes as uint8 (FP8 mode); ``v_mean``
+    [nseq, H, d] (FP8 mode, smooth V) is added to every output row."""
     out = np.full(q_i8.shape, np.nan, np.float16)
     ob = out.view(np.uint16)
     if pv_mode == PV_FP16:
@@ -204,8 +213,9 @@ def attn_quant(q_i8, q_scale, k_i8, k_scale, v, v_scale, layout: Layout, causal:
     for s, h, off, n in layout.heads(heads):
         sh = s * layout.H + h
         vsp = _ptr(v_scale, sh * layout.d) if v_scale is not None else None
+        vmp = _ptr(v_mean, sh * layout.d) if v_mean is not None else None
         lib().oracle_head_attn_quant(_ptr(q_i8, off), _ptr(q_scale, sh * nqb), _ptr(k_i8, off),
-                                     _ptr(k_scale, sh * nkb), _ptr(vv, off), vsp, n,
+                                     _ptr(k_scale, sh * nkb), _ptr(vv, off), vsp, vmp, n,
                                      layout.stride, layout.d, int(causal), int(pv_mode),
                                      float(sm_scale), int(tile_n), r0, r1, _ptr(ob, off))
     return out
@@ -232,13 +242,18 @@ def default_sm_scale(d: int, sm_scale: Optional[float] = None) -> float:
 
 def sage_attention(q, k, v, layout: Layout, causal: bool = False, smooth_k: bool = True,
                    pv_mode: int = PV_FP16, sm_scale: Optional[float] = None,
-                   tile_n: int = 128, heads=None, rows=None) -> np.ndarray:
-    """The whole method from fp16 Q, K, V: smooth K, quantize, quantized attention."""
+                   tile_n: int = 128, heads=None, rows=None,
+                   smooth_v: bool = False) -> np.ndarray:
+    """The whole method from fp16 Q, K, V: smooth K (and, in FP8 mode, optionally V),
+    quantize, quantized attention."""
+    if smooth_v and pv_mode != PV_FP8:
+        raise ValueError("smooth V applies to the FP8 P.V mode")
     sm = default_sm_scale(layout.d, sm_scale)
     z = quant_qk(q, k, layout, smooth_k, heads)
     if pv_mode == PV_FP8:
-        v8, vs = quant_v_fp8(v, layout, heads)
+        vm = channel_mean(v, layout, heads) if smooth_v else None
+        v8, vs = quant_v_fp8(v, layout, heads, vm)
         return attn_quant(z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], v8, vs, layout,
-                          causal, PV_FP8, sm, tile_n, heads, rows)
+                          causal, PV_FP8, sm, tile_n, heads, rows, vm)
     return attn_quant(z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], v, None, layout,
                       causal, PV_FP16, sm, tile_n, heads, rows)

@@ -18,6 +18,9 @@
  *   - FP8 mode: P and V quantized to E4M3, each tile's P.V product summed into an
  *     FP32-or-wider accumulator across tiles. (「4比特量化三倍加速不掉点！清华即插即用的SageAttention迎来升级」, section
  *     "技术方案", items (3) and (4).)
+ *   - Smooth V (FP8 mode): V <- V - mean(V) with the mean per channel over the tokens
+ *     of one head, the attention run on the smoothed V, and mean(V) added to the
+ *     output. (Same section, the paragraph after item (4).)
  *   - The exact reference O = softmax(sm_scale Q K^T + mask) V in fp64, and the
  *     smoothing invariant softmax(QK^T) = softmax(Q(K - mean K)^T) it must satisfy.
  *
@@ -143,19 +146,19 @@ uint8_t oracle_e4m3_encode(double x)
     return sign | (uint8_t)(e << 3) | m;
 }
 
-/* ------------------------------------------------------ smooth K: per-channel mean */
+/* ------------------------------------------- smooth K and V: per-channel token mean */
 
 /*
- * mu[c] = (sum over the n tokens of K[t, c]) / n, summed in fp64 in token order, the
+ * mu[c] = (sum over the n tokens of X[t, c]) / n, summed in fp64 in token order, the
  * quotient taken in fp64 and rounded once to fp32. One head; row t of channel c is at
- * K[t*stride + c].
+ * X[t*stride + c]. X is K for smooth K and V for smooth V.
  */
-void oracle_head_k_mean(const uint16_t *K, int64_t n, int64_t stride, int d, float *mu)
+void oracle_head_channel_mean(const uint16_t *X, int64_t n, int64_t stride, int d, float *mu)
 {
     for (int c = 0; c < d; c++) {
         double s = 0.0;
         for (int64_t t = 0; t < n; t++)
-            s += oracle_f16_to_f64(K[t * stride + c]);
+            s += oracle_f16_to_f64(X[t * stride + c]);
         mu[c] = n > 0 ? (float)(s / (double)n) : 0.0f;
     }
 }
@@ -208,17 +211,21 @@ void oracle_head_quant_int8(const uint16_t *X, const float *mu, int64_t n, int64
 }
 
 /*
- * V to E4M3 with one fp32 scale per channel over all tokens of the head:
- * s[c] = amax_t |V[t,c]| / 448; code = e4m3_rne_satfinite(fp32(V[t,c]) / s[c]) with
- * the quotient in fp32. A channel of zeros gets scale 0 and codes 0.
+ * V to E4M3 with one fp32 scale per channel over all tokens of the head. Element
+ * x = fp32(V[t,c]) - mu[c] (one fp32 subtraction; mu is the channel mean of V for
+ * smooth V, NULL for none); s[c] = amax_t |x| / 448; code = e4m3_rne_satfinite(x / s[c])
+ * with the quotient in fp32. A channel whose x are all zero gets scale 0 and codes 0.
  */
-void oracle_head_quant_v_fp8(const uint16_t *V, int64_t n, int64_t stride, int d,
-                             uint8_t *codes, float *scales)
+void oracle_head_quant_v_fp8(const uint16_t *V, const float *mu, int64_t n, int64_t stride,
+                             int d, uint8_t *codes, float *scales)
 {
     for (int c = 0; c < d; c++) {
         float amax = 0.0f;
         for (int64_t t = 0; t < n; t++) {
-            float a = fabsf((float)oracle_f16_to_f64(V[t * stride + c]));
+            float x = (float)oracle_f16_to_f64(V[t * stride + c]);
+            if (mu)
+                x = x - mu[c];
+            float a = fabsf(x);
             if (a > amax)
                 amax = a;
         }
@@ -226,6 +233,8 @@ void oracle_head_quant_v_fp8(const uint16_t *V, int64_t n, int64_t stride, int d
         scales[c] = s;
         for (int64_t t = 0; t < n; t++) {
             float x = (float)oracle_f16_to_f64(V[t * stride + c]);
+            if (mu)
+                x = x - mu[c];
             codes[t * stride + c] = (s != 0.0f) ? oracle_e4m3_encode((double)(x / s)) : 0;
         }
     }
@@ -246,14 +255,15 @@ enum { ORACLE_PV_FP16 = 0, ORACLE_PV_FP8 = 1 };
  *     p_j = 2^(t_j - m'),  l = alpha l + sum p_j,
  *     FP16 mode: P_j = f16(p_j),          O = alpha O + sum_j P_j V[j]
  *     FP8 mode:  P_j = e4m3(448 p_j),     O = alpha O + sum_j P_j e4m3val(vc[j]);
- *   output row: FP16 mode O / l; FP8 mode O vs[c] / (448 l); rounded to fp16.
+ *   output row: FP16 mode O / l; FP8 mode O vs[c] / (448 l) + vm[c] (vm = the channel
+ *   mean of V under smooth V, NULL for none); rounded to fp16.
  * `v` is fp16 bits (FP16 mode) or E4M3 codes (FP8 mode), row stride `stride`;
  * outputs are fp16 bits written at out[i*stride + c].
  */
 void oracle_head_attn_quant(const int8_t *qc, const float *qs, const int8_t *kc,
-                            const float *ks, const void *v, const float *vs, int64_t n,
-                            int64_t stride, int d, int causal, int pv_mode, double sm_scale,
-                            int tile_n, int64_t r0, int64_t r1, uint16_t *out)
+                            const float *ks, const void *v, const float *vs, const float *vm,
+                            int64_t n, int64_t stride, int d, int causal, int pv_mode,
+                            double sm_scale, int tile_n, int64_t r0, int64_t r1, uint16_t *out)
 {
     const double log2e = 1.4426950408889634073599246810019;   /* 1/ln 2 */
     if (r1 > n)
@@ -299,6 +309,8 @@ void oracle_head_attn_quant(const int8_t *qc, const float *qs, const int8_t *kc,
         }
         for (int c = 0; c < d; c++) {
             double o = (pv_mode == ORACLE_PV_FP16) ? O[c] / l : O[c] * (double)vs[c] / (448.0 * l);
+            if (pv_mode == ORACLE_PV_FP8 && vm)
+                o += (double)vm[c];
             out[i * stride + c] = oracle_f16_bits(oracle_round_f16(o));
         }
         free(O);

@@ -237,3 +237,73 @@ def test_sampled_rows_match_full():
     part = oracle.sage_attention(q, k, v, lay, True, True, PV_FP16, 0.2, heads=[(0, 1)], rows=(100, 180))
     assert np.array_equal(part[0, 1, 100:180], full[0, 1, 100:180])
     assert np.isnan(part[0, 0]).all() and np.isnan(part[0, 1, :100]).all()
+
+
+# Smooth V (「4比特量化三倍加速不掉点！清华即插即用的SageAttention迎来升级」, 技术方案, the paragraph after (4)): the FP8 P.V runs on
+# V - mean(V) and mean(V) is added to the output; softmax rows sum to 1, so in exact
+# arithmetic the result is unchanged.
+
+def test_smooth_v_single_token_and_constant_channels():
+    d = 16
+    v = _rand16((1, 1, 1, d), 111, 8.0)
+    q = _rand16((1, 1, 1, d), 112)
+    o = oracle.sage_attention(q, q, v, Layout.dense(1, 1, 1, d), False, True, PV_FP8, 0.25,
+                              smooth_v=True)
+    assert np.array_equal(o, v)                              # N = 1: V - mean = 0, O = mean
+    N = 300
+    q, k = _rand16((1, 1, N, d), 113), _rand16((1, 1, N, d), 114)
+    row = _rand16((d,), 115, 10.0)
+    v = np.broadcast_to(row, (1, 1, N, d)).astype(np.float16)  # every token the same V
+    for causal in (False, True):
+        o = oracle.sage_attention(q, k, v, Layout.dense(1, 1, N, d), causal, True, PV_FP8,
+                                  0.25, smooth_v=True)
+        assert np.array_equal(o, v)
+
+
+def test_smooth_v_single_tile_closed_form():
+    N, d = 200, 32
+    q, k, v = (_rand16((1, 1, N, d), s) for s in (121, 122, 123))
+    v = (v.astype(np.float64) + np.linspace(-20, 20, d)).astype(np.float16)
+    lay = Layout.dense(1, 1, N, d)
+    sm = 1 / math.sqrt(d)
+    z = oracle.quant_qk(q, k, lay, True)
+    vm = oracle.v_mean(v, lay)
+    vq, vs = oracle.quant_v_fp8(v, lay, mu=vm)
+    got = oracle.attn_quant(z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], vq, vs, lay,
+                            False, PV_FP8, sm, tile_n=256, v_mean=vm)
+    ref = _single_tile_reference(z, vq, False, PV_FP8, sm, vs).astype(np.float64)
+    # the unsmoothed closed form plus the channel mean, rounded once to fp16
+    ref = ref + vm[0, 0][None, :]
+    diff = np.abs(got[0, 0].astype(np.float64) - ref)
+    assert diff.max() <= 3 * np.spacing(np.abs(ref).astype(np.float16)).astype(np.float64).max()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_smooth_v_helps_with_channel_offsets(causal):
+    # V channels with large offsets: without smoothing the E4M3 codes spend their range on
+    # the offset; smoothing keeps the error at the level of offset-free V
+    N, d = 512, 64
+    q, k, v = (_rand16((1, 1, N, d), s) for s in (131, 132, 133))
+    off = _rand16((d,), 134, 16.0).astype(np.float64)
+    vo = (v.astype(np.float64) + off).astype(np.float16)
+    lay = Layout.dense(1, 1, N, d)
+    sm = 1 / math.sqrt(d)
+    exact = oracle.attn_fp64(q, k, vo, lay, causal, sm)
+    smooth = oracle.sage_attention(q, k, vo, lay, causal, True, PV_FP8, sm, smooth_v=True)
+    raw = oracle.sage_attention(q, k, vo, lay, causal, True, PV_FP8, sm)
+    err_s = np.abs(smooth.astype(np.float64) - exact).mean()
+    err_r = np.abs(raw.astype(np.float64) - exact).mean()
+    assert err_s < 0.25 * err_r
+    # translation: O(V + off) - off tracks O(V) to the E4M3 error of offset-free V
+    base = oracle.sage_attention(q, k, v, lay, causal, True, PV_FP8, sm, smooth_v=True)
+    exact0 = oracle.attn_fp64(q, k, v, lay, causal, sm)
+    err_0 = np.abs(base.astype(np.float64) - exact0).mean()
+    assert err_s < 3 * err_0 + 1e-3
+
+
+def test_smooth_v_rejected_in_fp16_mode():
+    d = 16
+    x = _rand16((1, 1, 4, d), 141)
+    with pytest.raises(ValueError):
+        oracle.sage_attention(x, x, x, Layout.dense(1, 1, 4, d), False, True, PV_FP16, 0.25,
+                              smooth_v=True)

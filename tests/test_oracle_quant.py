@@ -146,3 +146,28 @@ def test_v_fp8_per_channel():
         # E4M3 keeps 3 mantissa bits: relative error <= 2^-4 above the subnormal range
         tol = np.maximum(np.abs(ref) * 2.0 ** -4, scales[0, 0, c] * 2.0 ** -10)
         assert np.all(np.abs(rec - ref) <= tol * 1.0001)
+
+
+def test_v_fp8_smoothed_per_channel():
+    # Smooth V (「4比特量化三倍加速不掉点！清华即插即用的SageAttention迎来升级」, 技术方案, the paragraph after (4)): codes encode
+    # V - mean(V) per channel; the mean is the numpy token mean rounded to fp32
+    lay = Layout.dense(1, 2, 70, 8)
+    v = _rand16((1, 2, 70, 8), 19).astype(np.float64)
+    v += np.array([50.0, -20.0, 0.0, 5.0, 100.0, -3.0, 7.0, 0.0])
+    v[..., 7] = 2.5                                             # constant channel
+    v = v.astype(np.float16)
+    mu = oracle.v_mean(v, lay)
+    assert np.array_equal(mu, v.astype(np.float64).mean(axis=2).astype(np.float32))
+    codes, scales = oracle.quant_v_fp8(v, lay, mu=mu)
+    vals = np.vectorize(oracle.e4m3_decode)(codes).astype(np.float64)
+    assert np.all(scales[..., 7] == 0) and not codes[..., 7].any()   # V - mean = 0 exactly
+    for h in range(2):
+        for c in range(7):
+            x = (v[0, h, :, c].astype(np.float32) - mu[0, h, c]).astype(np.float64)
+            assert np.abs(vals[0, h, :, c]).max() == 448.0      # amax of |V - mean| maps to 448
+            rec = vals[0, h, :, c] * scales[0, h, c]
+            tol = np.maximum(np.abs(x) * 2.0 ** -4, scales[0, h, c] * 2.0 ** -10)
+            assert np.all(np.abs(rec - x) <= tol * 1.0001)
+    # the offsets are gone: smoothed scales are far below the raw ones on offset channels
+    _, raw = oracle.quant_v_fp8(v, lay)
+    assert np.all(scales[0, :, [0, 1, 4]] < 0.2 * raw[0, :, [0, 1, 4]])

@@ -141,44 +141,78 @@ def _dist():
     return world, rank, local
 
 
+def _oracle_case(args):
+    """Host inputs and oracle layout of the workload the GPU arm times (one batch entry for
+    dense workloads, every packed sequence for varlen)."""
+    import oracle
+    from quantized_attention_03_b200 import inputs
+
+    W = _workload(args)
+    w = W.get("gen") or inputs.sweep(W["N"], W["d"], W["causal"])
+    if args.workload == "varlen":
+        q, k, v, cu = inputs.make_varlen(w)
+        lay = oracle.Layout.packed(cu.tolist(), w.H, w.d)
+        W.update(varlen=True, lens=lay.lens)
+    else:
+        q, k, v = inputs.make_dense(w, B=1, N=W["N"])
+        lay = oracle.Layout.dense(1, w.H, W["N"], W["d"])
+    pv = oracle.PV_FP8 if W["pv_mode"] == "fp8" else oracle.PV_FP16
+    return W, q.numpy(), k.numpy(), v.numpy(), lay, pv
+
+
+def _sample_ops(r0: int, r1: int, n: int, d: int, causal: bool) -> float:
+    """Operations of query rows [r0, r1) of one head of length n (4 d per visible key)."""
+    if not causal:
+        return 4.0 * (r1 - r0) * n * d
+    return 4.0 * d * sum(min(r + 1, n) for r in range(r0, r1))
+
+
+def _oracle_sample(case, it: int, rows: int):
+    """Run the oracle on `rows` query rows of one head; returns (seconds, ops, head)."""
+    import oracle
+    W, q, k, v, lay, pv = case
+    s = it % lay.nseq
+    h = (it // lay.nseq) % lay.H
+    n = lay.lens[s]
+    # row offsets spread over the sequence (golden-ratio steps), so that a causal sample
+    # sees on average the workload's mean number of visible keys per row
+    r0 = int(((it * 0.6180339887498949) % 1.0) * max(n - rows + 1, 1))
+    r1 = min(r0 + rows, n)
+    t0 = time.perf_counter()
+    oracle.sage_attention(q, k, v, lay, W["causal"], W["smooth_k"], pv,
+                          1.0 / math.sqrt(lay.d), heads=[(s, h)], rows=(r0, r1))
+    return time.perf_counter() - t0, _sample_ops(r0, r1, n, lay.d, W["causal"]), (s, h)
+
+
 def run_reference(args):
     """The CPU oracle, as it stands, on rank 0: each step is a bounded sample of rows."""
     world, rank, _ = _dist()
     if rank != 0:
         return
-    import numpy as np
     import oracle
-    from quantized_attention_03_b200 import inputs
 
-    W = WORKLOAD
-    w = inputs.sweep(W["N"], W["d"], W["causal"])
-    q, k, v = inputs.make_dense(w, B=1)          # the sample uses one (b, h) head
-    lay = oracle.Layout.dense(1, w.H, w.N, w.d)
+    case = _oracle_case(args)
+    W, lay = case[0], case[4]
     rows = args.ref_rows
-    q, k, v = q.numpy(), k.numpy(), v.numpy()
-    sm = 1.0 / math.sqrt(w.d)
-    times = []
+    t, ops = 0.0, 0.0
     for it in range(args.warmup + args.steps):
-        r0 = (it * rows) % w.N
-        t0 = time.perf_counter()
-        oracle.sage_attention(q, k, v, lay, W["causal"], W["smooth_k"], oracle.PV_FP16, sm,
-                              heads=[(0, it % w.H)], rows=(r0, r0 + rows))
-        t1 = time.perf_counter()
+        dt, n_ops, _ = _oracle_sample(case, it, rows)
         if it >= args.warmup:
-            times.append(t1 - t0)
-    ops_per_step = 4.0 * rows * w.N * w.d            # the sampled rows of one head
-    t = sum(times)
-    value = ops_per_step * len(times) / t / 1e12
+            t += dt
+            ops += n_ops
+    value = ops / t / 1e12
     cores = oracle.num_threads()
-    sample = (f"{rows} query rows x {w.N} keys of one head per step (d={w.d}, non-causal, "
-              f"FP16 PV, quantization of that head included)")
+    sample = (f"{rows} query rows of one head per step (heads and row offsets rotate), all "
+              f"their keys, {_workload_name(W)}, quantization of that head included")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TOPS",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1e3 * t / len(times), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "s8+f16 (oracle: fp64 accumulation)", "data": "synthetic",
-        "config": {"workload": "sweep point B=2 H=32 N=16384 d=128 non-causal PV=fp16 smooth_k",
-                   **W},
+        "ms_per_step": 1e3 * t / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "s8+f16 (oracle: fp64 accumulation)"
+        if W["pv_mode"] == "fp16" else "s8+f8 (oracle: fp64 accumulation)",
+        "data": "synthetic",
+        "config": {"workload": _workload_name(W),
+                   **{k: v for k, v in W.items() if k not in ("gen",)}},
         "cpu_baseline": {"value": value, "unit": "TOPS", "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -186,38 +220,47 @@ def run_reference(args):
     print(json.dumps(line))
 
 
-def cpu_baseline(seconds_target: float = 15.0):
-    """Time the oracle on a bounded sample (rows of one head) on the host cores."""
+def cpu_baseline(args, seconds_target: float = 15.0):
+    """Time the oracle on a bounded sample (256-row slices of heads) on the host cores."""
     import oracle
-    from quantized_attention_03_b200 import inputs
 
-    W = WORKLOAD
-    w = inputs.sweep(W["N"], W["d"], W["causal"])
-    q, k, v = inputs.make_dense(w, B=1)
-    lay = oracle.Layout.dense(1, w.H, w.N, w.d)
-    q, k, v = q.numpy(), k.numpy(), v.numpy()
-    sm = 1.0 / math.sqrt(w.d)
-    rows, total_rows, t_total = 256, 0, 0.0
-    r0 = 0
-    while t_total < seconds_target and total_rows < w.N:
-        t0 = time.perf_counter()
-        oracle.sage_attention(q, k, v, lay, False, True, oracle.PV_FP16, sm, heads=[(0, 0)],
-                              rows=(r0, r0 + rows))
-        t_total += time.perf_counter() - t0
-        total_rows += rows
-        r0 += rows
-    value = 4.0 * total_rows * w.N * w.d / t_total / 1e12
-    return {"value": value, "unit": "TOPS", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{total_rows} query rows x {w.N} keys of head (0,0), d={w.d}, "
-                      f"non-causal, FP16 PV, quantization of the head included "
+    case = _oracle_case(args)
+    W = case[0]
+    t_total, ops, rows, it, heads = 0.0, 0.0, 256, 0, set()
+    while t_total < seconds_target and it < 64:
+        dt, n_ops, head = _oracle_sample(case, it, rows)
+        t_total += dt
+        ops += n_ops
+        heads.add(head)
+        it += 1
+    return {"value": ops / t_total / 1e12, "unit": "TOPS", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{it} slices of {rows} query rows x all their keys over {len(heads)} "
+                      f"heads of {_workload_name(W)}, quantization of each head included "
                       f"({t_total:.1f} s of CPU work)"}
 
 
 def _workload(args):
-    """The headline workload, optionally overridden (smaller cases for profiling)."""
+    """The workload to time: the headline point by default, one of the other target
+    workloads with --workload, optionally overridden (smaller cases for profiling)."""
+    from quantized_attention_03_b200 import inputs
     W = dict(WORKLOAD)
+    if args.workload == "llm_prefill":
+        w = inputs.llm_prefill()
+    elif args.workload == "video_dit":
+        w = inputs.video_dit()
+    elif args.workload == "varlen":
+        w = inputs.varlen()
+    elif args.workload == "sweep":
+        n = args.N or 16384
+        w = inputs.sweep(n, args.d or 128, args.causal)
+    else:
+        w = None
+    if w is not None:
+        W.update(B=w.B, H=w.H, N=w.N, d=w.d, causal=w.causal, pv_mode=w.pv_modes[0])
+        W["gen"] = w
     for key in ("B", "N", "d"):
-        if getattr(args, key) is not None:
+        if getattr(args, key) is not None and args.workload in ("headline", "sweep"):
             W[key] = getattr(args, key)
     if args.causal:
         W["causal"] = True
@@ -227,6 +270,10 @@ def _workload(args):
 
 
 def _workload_name(W):
+    if W.get("varlen"):
+        return (f"packed varlen {len(W['lens'])} sequences (lengths {W['lens']}) H={W['H']} "
+                f"d={W['d']} {'causal' if W['causal'] else 'non-causal'} PV={W['pv_mode']} "
+                f"smooth_k")
     return (f"B={W['B']} H={W['H']} N={W['N']} d={W['d']} "
             f"{'causal' if W['causal'] else 'non-causal'} PV={W['pv_mode']} smooth_k")
 
@@ -260,9 +307,11 @@ def run_ours(args):
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
 
     W = _workload(args)
+    if args.workload == "varlen":
+        return run_varlen(args, W, dist, world, rank, local)
     B, H, N, d = W["B"], W["H"], W["N"], W["d"]
-    w = inputs.sweep(N, d, W["causal"])
-    qc, kc, vc = inputs.make_dense(w, B=B)
+    w = W.get("gen") or inputs.sweep(N, d, W["causal"])
+    qc, kc, vc = inputs.make_dense(w, B=B, N=N)
     q, k, v = qc.cuda(), kc.cuda(), vc.cuda()
     pv = sage.SAGE_PV_FP16 if W["pv_mode"] == "fp16" else sage.SAGE_PV_FP8
     vq, vscale = v, None
@@ -396,7 +445,8 @@ def run_ours(args):
     if os.path.exists(traffic_file):
         with open(traffic_file) as f:
             tr = json.load(f)
-        if tr.get("kernel_source_hash") == _kernel_hash():
+        if (tr.get("kernel_source_hash") == _kernel_hash() and args.workload == "headline"
+                and (B, H, N, d, W["causal"], W["pv_mode"]) == (2, 32, 16384, 128, False, "fp16")):
             roofline["traffic"] = tr.get("bytes_per_launch")
 
     if rank == 0:
@@ -404,13 +454,14 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "s8+f16", "data": "synthetic",
-            "config": {"workload": "sequence-length sweep point " + _workload_name(W) +
+            "dtype": "s8+f8" if pv == sage.SAGE_PV_FP8 else "s8+f16", "data": "synthetic",
+            "config": {"workload": (args.workload if args.workload != "headline" else
+                                    "sequence-length sweep point") + " " + _workload_name(W) +
                                    " (per GPU)",
                        "B": B, "H": H, "N": N, "d": d, "causal": W["causal"],
                        "pv_mode": W["pv_mode"], "smooth_k": W["smooth_k"],
                        "parallelism": f"replicas x{world}",
-                       "l2": "inputs larger than L2 (Q, K, V 268 MB each); no flush"},
+                       "l2": _l2_note(elem_bytes)},
             "roofline": roofline,
             "e2e": {"value": e2e_value, "unit": "TOPS",
                     "h2d_bytes_per_step": 3 * elem_bytes, "d2h_bytes_per_step": elem_bytes,
@@ -419,11 +470,124 @@ def run_ours(args):
             "clocks": clocks.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+            line["cpu_baseline"] = cpu_baseline(args, args.cpu_seconds)
         print(json.dumps(line))
     if dist is not None:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def run_varlen(args, W, dist, world, rank, local):
+    """Packed varlen workload through sage_attn_varlen_fwd (quantization and attention
+    in one call with caller scratch); the attention kernel is not timed separately."""
+    import torch
+    import quantized_attention_03_b200 as sage
+    from quantized_attention_03_b200 import inputs
+
+    w = W["gen"]
+    qc, kc, vc, cu = inputs.make_varlen(w)
+    lens = [int(x) for x in (cu[1:] - cu[:-1])]
+    W.update(varlen=True, lens=lens)
+    T, H, d = qc.shape
+    nseq, maxlen = len(lens), max(lens)
+    pv = sage.SAGE_PV_FP16 if W["pv_mode"] == "fp16" else sage.SAGE_PV_FP8
+    q, k, v, cud = qc.cuda(), kc.cuda(), vc.cuda(), cu.cuda()
+    out = torch.empty_like(q)
+    need = sage.sage_workspace_size(nseq, H, maxlen, T, d, pv)
+    ws = torch.empty(need, dtype=torch.uint8, device=q.device)
+    stream = torch.cuda.current_stream()
+    ops = inputs.varlen_ops(lens, H, d, W["causal"])
+
+    def step(qq=q, kk=k, vv=v, oo=out):
+        sage.sage_attn_varlen_fwd(qq, kk, vv, oo, cud, nseq, T, maxlen, H, d, W["causal"], True,
+                                  pv, 0.0, ws, need, stream)
+
+    clocks = ClockSampler(local)
+    clocks.__enter__()
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if sage.sage_get_device_status() != 0:
+        raise RuntimeError("device status after warm-up")
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.mark("t0")
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks.mark("t1")
+    clocks.__exit__(None, None, None)
+    if sage.sage_get_device_status() != 0:
+        raise RuntimeError("device status after timing")
+    total_ms = max_over_ranks(e0.elapsed_time(e1), dist, q.device)
+    value = weak_scaling_tops(ops, args.steps, world, total_ms)
+
+    e2e_steps = 0 if args.no_e2e else max(3, args.steps // 4)
+    qh, kh, vh = (t.pin_memory() for t in (qc, kc, vc))
+    oh = torch.empty_like(qc).pin_memory()
+    qd, kd, vd, od = (torch.empty_like(q) for _ in range(4))
+
+    def e2e_step():
+        qd.copy_(qh, non_blocking=True)
+        kd.copy_(kh, non_blocking=True)
+        vd.copy_(vh, non_blocking=True)
+        step(qd, kd, vd, od)
+        oh.copy_(od, non_blocking=True)
+
+    if e2e_steps:
+        e2e_step()
+    torch.cuda.synchronize()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    s1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(max(s0.elapsed_time(s1), 1e-9), dist, q.device)
+    e2e_value = weak_scaling_tops(ops, e2e_steps, world, e2e_ms) if e2e_steps else None
+
+    peaks, src = _peaks()
+    bf16 = peaks["bf16_tflops_sustained"]
+    int8_peak = 2.0 * bf16
+    pv_peak = bf16 if pv == sage.SAGE_PV_FP16 else 2.0 * bf16
+    mixed = 1.0 / (0.5 / int8_peak + 0.5 / pv_peak)
+    if rank == 0:
+        elem_bytes = q.numel() * 2
+        line = {
+            "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "s8+f8" if pv == sage.SAGE_PV_FP8 else "s8+f16", "data": "synthetic",
+            "config": {"workload": "varlen " + _workload_name(W) + " (per GPU)",
+                       "H": H, "d": d, "T": T, "lens": lens, "causal": W["causal"],
+                       "pv_mode": W["pv_mode"], "parallelism": f"replicas x{world}",
+                       "l2": _l2_note(q.numel() * 2)},
+            "roofline": {"bound": "tensor", "achieved": value / world, "peak": mixed,
+                         "unit": "TOPS", "frac": value / world / mixed, "traffic": None,
+                         "kernel": "whole varlen step (quantization + attention in one call; "
+                                   "the attention kernel is not timed separately)"},
+            "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": 3 * elem_bytes,
+                    "d2h_bytes_per_step": elem_bytes, "steps": e2e_steps},
+            "gpu_launches": 3 * args.steps,   # column statistics, quantization, attention
+            "clocks": clocks.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            line["cpu_baseline"] = cpu_baseline(args, args.cpu_seconds)
+        print(json.dumps(line))
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def _l2_note(tensor_bytes: int) -> str:
+    mb = tensor_bytes / 1e6
+    if 3 * tensor_bytes > 126e6:
+        return f"inputs larger than L2 (Q, K, V {mb:.0f} MB each); no flush"
+    return f"inputs fit in L2 (Q, K, V {mb:.0f} MB each); no flush, so L2-resident"
 
 
 def _kernel_hash():
@@ -447,6 +611,9 @@ def main():
     ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="headline",
+                    choices=["headline", "llm_prefill", "video_dit", "sweep", "varlen"],
+                    help="headline: B2 H32 N16384 d128 non-causal FP16 PV (the metric's point)")
     ap.add_argument("--ref-rows", type=int, default=64)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")

@@ -64,14 +64,30 @@ typedef enum {
 
 enum { SAGE_PV_FP16 = 0, SAGE_PV_FP8 = 1 };
 
+/*
+ * Smoothing flags, passed in the `smooth_k` argument of the fused entry points
+ * (sage_attn_fwd, sage_attn_fwd_ws, sage_attn_varlen_fwd, sage_attn_fwd_noalloc):
+ *   SAGE_SMOOTH_K (1): step 1 above. 0 and 1 keep their plain boolean meaning.
+ *   SAGE_SMOOTH_V (2): smooth V in FP8 mode (「4比特量化三倍加速不掉点！清华即插即用的SageAttention迎来升级」, 技术方案,
+ *     the paragraph after item (4)): V <- V - mean(V), the mean per channel over the
+ *     tokens of one head (per sequence in varlen, summed in fp64 and rounded once to
+ *     fp32), the E4M3 codes and per-channel scales taken of the smoothed V, and mean(V)
+ *     added to every output row. Softmax rows sum to one, so the exact result is
+ *     unchanged; the E4M3 range is no longer spent on a channel offset.
+ * Other bits give SAGE_ERR_INVALID_ARG; SAGE_SMOOTH_V with SAGE_PV_FP16 gives
+ * SAGE_ERR_UNSUPPORTED (fp16 V is not quantized, so there is nothing to smooth for).
+ */
+enum { SAGE_SMOOTH_K = 1, SAGE_SMOOTH_V = 2 };
+
 /* Opaque CUDA stream (binary-compatible with cudaStream_t). */
 typedef struct CUstream_st *sage_stream_t;
 
 /*
  * Bytes of scratch the fused entry points need for one call: INT8 codes of Q and K,
  * their block scales, the K mean (and its fp64 column sums), and in FP8 mode the E4M3
- * codes of V with their per-channel scales. Dense: nseq = B, max_seqlen = N,
- * total_tokens = B*N.
+ * codes of V with their per-channel scales and the V column statistics (sum, max,
+ * min) smooth V needs. Dense: nseq = B, max_seqlen = N, total_tokens = B*N. The size
+ * does not depend on the smoothing flags.
  */
 SAGE_API size_t sage_workspace_size(int nseq, int H, int max_seqlen, int total_tokens, int d,
                            int pv_mode);
@@ -115,6 +131,22 @@ SAGE_API sage_status_t sage_quant_v_fp8_varlen(const void *v, const int32_t *cu_
                                       uint8_t *v_e4m3, float *v_scale, sage_stream_t stream);
 
 /*
+ * Smooth V, then V to E4M3 (the SAGE_SMOOTH_V step on its own): v_mean [B,H,d] fp32 =
+ * mean over tokens of V[b,h,:,c] (fp64 sum, rounded once); x = fp32(V) - v_mean (one
+ * fp32 subtraction); v_scale = amax|x|/448 per channel; v_e4m3 = E4M3 of fp32 x/v_scale
+ * as in sage_quant_v_fp8. A channel with x all zero (a constant channel) has scale 0
+ * and codes 0. Uses a small stream-ordered allocation for the column statistics.
+ */
+SAGE_API sage_status_t sage_quant_v_fp8_smooth(const void *v, uint8_t *v_e4m3, float *v_scale,
+                                               float *v_mean, int B, int H, int N, int d,
+                                               sage_stream_t stream);
+SAGE_API sage_status_t sage_quant_v_fp8_smooth_varlen(const void *v, const int32_t *cu_seqlens,
+                                                      int nseq, int total_tokens,
+                                                      int max_seqlen, int H, int d,
+                                                      uint8_t *v_e4m3, float *v_scale,
+                                                      float *v_mean, sage_stream_t stream);
+
+/*
  * The whole forward pass (steps 1-3), dense layout: out[B,H,N,d] fp16. pv_mode selects
  * SAGE_PV_FP16 or SAGE_PV_FP8. Scratch comes from stream-ordered allocation
  * (cudaMallocAsync/cudaFreeAsync on `stream`).
@@ -153,6 +185,17 @@ SAGE_API sage_status_t sage_attn_fwd_quantized(const int8_t *q_i8, const float *
                                       const float *v_scale, void *out, int B, int H, int N,
                                       int d, int causal, int pv_mode, float sm_scale,
                                       sage_stream_t stream);
+
+/* Step 3 alone in FP8 mode with smoothed V: v_e4m3, v_scale and v_mean [B,H,d] as
+ * produced by sage_quant_v_fp8_smooth; out = O v_scale / (448 l) + v_mean per channel.
+ * Allocates nothing. */
+SAGE_API sage_status_t sage_attn_fwd_quantized_smooth_v(const int8_t *q_i8, const float *q_scale,
+                                                        const int8_t *k_i8, const float *k_scale,
+                                                        const uint8_t *v_e4m3,
+                                                        const float *v_scale, const float *v_mean,
+                                                        void *out, int B, int H, int N, int d,
+                                                        int causal, float sm_scale,
+                                                        sage_stream_t stream);
 
 /*
  * Debug: the integer score tiles S = q_i8 k_i8^T (int32, [B,H,N,N]) exactly as the

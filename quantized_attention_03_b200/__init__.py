@@ -31,6 +31,8 @@ SAGE_ERR_TIMEOUT = 6
 SAGE_ERR_BAD_SEQLENS = 7
 SAGE_PV_FP16 = 0
 SAGE_PV_FP8 = 1
+SAGE_SMOOTH_K = 1     # flags of the fused entry points' smooth_k argument
+SAGE_SMOOTH_V = 2
 
 Q_BLOCK = 128
 K_BLOCK = 64
@@ -48,12 +50,16 @@ SIGNATURES = {
     "sage_quant_qk_varlen": (_S, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _I, _P]),
     "sage_quant_v_fp8": (_S, [_P, _P, _P, _I, _I, _I, _I, _P]),
     "sage_quant_v_fp8_varlen": (_S, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
+    "sage_quant_v_fp8_smooth": (_S, [_P, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "sage_quant_v_fp8_smooth_varlen": (_S, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
     "sage_attn_fwd": (_S, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
     "sage_attn_fwd_ws": (_S, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
     "sage_attn_varlen_fwd": (_S, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P,
                                   _Z, _P]),
     "sage_attn_fwd_quantized": (_S, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F,
                                      _P]),
+    "sage_attn_fwd_quantized_smooth_v": (_S, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I,
+                                              _I, _F, _P]),
     "sage_debug_qk_int32": (_S, [_P, _P, _P, _I, _I, _I, _I, _P]),
     "sage_attn_fwd_noalloc": (_S, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
     "sage_debug_wait_timeout": (_S, [ctypes.c_ulonglong, _P]),
@@ -155,6 +161,18 @@ def sage_quant_v_fp8_varlen(v, cu_seqlens, nseq, total_tokens, max_seqlen, H, d,
                  max_seqlen, H, d, _ptr(v_e4m3), _ptr(v_scale), _stream(stream))
 
 
+def sage_quant_v_fp8_smooth(v, v_e4m3, v_scale, v_mean, B, H, N, d, stream=None):
+    return _call("sage_quant_v_fp8_smooth", _ptr(v), _ptr(v_e4m3), _ptr(v_scale), _ptr(v_mean),
+                 B, H, N, d, _stream(stream))
+
+
+def sage_quant_v_fp8_smooth_varlen(v, cu_seqlens, nseq, total_tokens, max_seqlen, H, d, v_e4m3,
+                                   v_scale, v_mean, stream=None):
+    return _call("sage_quant_v_fp8_smooth_varlen", _ptr(v), _ptr(cu_seqlens), nseq,
+                 total_tokens, max_seqlen, H, d, _ptr(v_e4m3), _ptr(v_scale), _ptr(v_mean),
+                 _stream(stream))
+
+
 def sage_attn_fwd(q, k, v, out, B, H, N, d, causal, smooth_k, pv_mode, sm_scale, stream=None):
     return _call("sage_attn_fwd", _ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, N, d, int(causal),
                  int(smooth_k), int(pv_mode), float(sm_scale), _stream(stream))
@@ -179,6 +197,13 @@ def sage_attn_fwd_quantized(q_i8, q_scale, k_i8, k_scale, v, v_scale, out, B, H,
     return _call("sage_attn_fwd_quantized", _ptr(q_i8), _ptr(q_scale), _ptr(k_i8), _ptr(k_scale),
                  _ptr(v), _ptr(v_scale), _ptr(out), B, H, N, d, int(causal), int(pv_mode),
                  float(sm_scale), _stream(stream))
+
+
+def sage_attn_fwd_quantized_smooth_v(q_i8, q_scale, k_i8, k_scale, v_e4m3, v_scale, v_mean, out,
+                                     B, H, N, d, causal, sm_scale, stream=None):
+    return _call("sage_attn_fwd_quantized_smooth_v", _ptr(q_i8), _ptr(q_scale), _ptr(k_i8),
+                 _ptr(k_scale), _ptr(v_e4m3), _ptr(v_scale), _ptr(v_mean), _ptr(out), B, H, N,
+                 d, int(causal), float(sm_scale), _stream(stream))
 
 
 def sage_debug_qk_int32(q_i8, k_i8, s_out, B, H, N, d, stream=None):
@@ -223,27 +248,33 @@ def _check_status(stream=None):
         raise SageError("device", code)
 
 
+def _smooth_flags(smooth_k: bool, smooth_v: bool) -> int:
+    return (SAGE_SMOOTH_K if smooth_k else 0) | (SAGE_SMOOTH_V if smooth_v else 0)
+
+
 def sageattn(q, k, v, causal: bool = False, smooth_k: bool = True, pv_mode: int = SAGE_PV_FP16,
-             sm_scale: float = 0.0, out=None, stream=None):
+             sm_scale: float = 0.0, out=None, stream=None, smooth_v: bool = False):
     """O = SageAttention(q, k, v) for fp16 CUDA tensors [B, H, N, d]."""
     import torch
     B, H, N, d = q.shape
     if out is None:
         out = torch.empty_like(q)
-    sage_attn_fwd(q, k, v, out, B, H, N, d, causal, smooth_k, pv_mode, sm_scale, stream)
+    sage_attn_fwd(q, k, v, out, B, H, N, d, causal, _smooth_flags(smooth_k, smooth_v), pv_mode,
+                  sm_scale, stream)
     return out
 
 
 def sageattn_varlen(q, k, v, cu_seqlens, max_seqlen: int, causal: bool = False,
                     smooth_k: bool = True, pv_mode: int = SAGE_PV_FP16, sm_scale: float = 0.0,
-                    out=None, stream=None):
+                    out=None, stream=None, smooth_v: bool = False):
     """SageAttention over packed sequences: q, k, v [T, H, d], cu_seqlens int32 [nseq+1]."""
     import torch
     T, H, d = q.shape
     if out is None:
         out = torch.empty_like(q)
     sage_attn_varlen_fwd(q, k, v, out, cu_seqlens, cu_seqlens.numel() - 1, T, max_seqlen, H, d,
-                         causal, smooth_k, pv_mode, sm_scale, None, 0, stream)
+                         causal, _smooth_flags(smooth_k, smooth_v), pv_mode, sm_scale, None, 0,
+                         stream)
     return out
 
 
@@ -279,32 +310,50 @@ def quant_qk_varlen(q, k, cu_seqlens, max_seqlen: int, smooth_k: bool = True, st
     return z
 
 
-def quant_v_fp8(v, stream=None):
-    """Dense V -> (E4M3 codes as uint8 [B,H,N,d], per-channel scales [B,H,d])."""
+def quant_v_fp8(v, stream=None, smooth_v: bool = False):
+    """Dense V -> (E4M3 codes as uint8 [B,H,N,d], per-channel scales [B,H,d]); with
+    smooth_v, a third result: the channel mean of V [B,H,d] the codes are taken from."""
     import torch
     B, H, N, d = v.shape
     codes = torch.empty(v.shape, dtype=torch.uint8, device=v.device)
     scales = torch.empty((B, H, d), dtype=torch.float32, device=v.device)
-    sage_quant_v_fp8(v, codes, scales, B, H, N, d, stream)
-    return codes, scales
+    if not smooth_v:
+        sage_quant_v_fp8(v, codes, scales, B, H, N, d, stream)
+        return codes, scales
+    mean = torch.empty((B, H, d), dtype=torch.float32, device=v.device)
+    sage_quant_v_fp8_smooth(v, codes, scales, mean, B, H, N, d, stream)
+    return codes, scales, mean
 
 
-def quant_v_fp8_varlen(v, cu_seqlens, max_seqlen: int, stream=None):
+def quant_v_fp8_varlen(v, cu_seqlens, max_seqlen: int, stream=None, smooth_v: bool = False):
     import torch
     T, H, d = v.shape
     nseq = cu_seqlens.numel() - 1
     codes = torch.empty(v.shape, dtype=torch.uint8, device=v.device)
     scales = torch.empty((nseq, H, d), dtype=torch.float32, device=v.device)
-    sage_quant_v_fp8_varlen(v, cu_seqlens, nseq, T, max_seqlen, H, d, codes, scales, stream)
-    return codes, scales
+    if not smooth_v:
+        sage_quant_v_fp8_varlen(v, cu_seqlens, nseq, T, max_seqlen, H, d, codes, scales, stream)
+        return codes, scales
+    mean = torch.empty((nseq, H, d), dtype=torch.float32, device=v.device)
+    sage_quant_v_fp8_smooth_varlen(v, cu_seqlens, nseq, T, max_seqlen, H, d, codes, scales, mean,
+                                   stream)
+    return codes, scales, mean
 
 
 def attn_quantized(q_i8, q_scale, k_i8, k_scale, v, v_scale, causal: bool = False,
-                   pv_mode: int = SAGE_PV_FP16, sm_scale: float = 0.0, out=None, stream=None):
+                   pv_mode: int = SAGE_PV_FP16, sm_scale: float = 0.0, out=None, stream=None,
+                   v_mean=None):
+    """Step 3 on pre-quantized operands; v_mean (FP8 mode) selects the smooth-V epilogue."""
     import torch
     B, H, N, d = q_i8.shape
     if out is None:
         out = torch.empty(q_i8.shape, dtype=torch.float16, device=q_i8.device)
+    if v_mean is not None:
+        if pv_mode != SAGE_PV_FP8:
+            raise ValueError("v_mean needs the FP8 P.V mode")
+        sage_attn_fwd_quantized_smooth_v(q_i8, q_scale, k_i8, k_scale, v, v_scale, v_mean, out,
+                                         B, H, N, d, causal, sm_scale, stream)
+        return out
     sage_attn_fwd_quantized(q_i8, q_scale, k_i8, k_scale, v, v_scale, out, B, H, N, d, causal,
                             pv_mode, sm_scale, stream)
     return out

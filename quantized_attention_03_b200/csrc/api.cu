@@ -59,11 +59,10 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 struct Workspace {
     int8_t *q_i8 = nullptr, *k_i8 = nullptr;
     float *q_scale = nullptr, *k_scale = nullptr, *k_mean = nullptr;
-    double *ksum = nullptr;
-    uint32_t *vamax = nullptr;   // adjacent to ksum: one memset clears both
+    ColStats cs;                 // contiguous: one memset clears all of it
     uint8_t *v8 = nullptr;
-    float *v_scale = nullptr;
-    size_t stats_bytes = 0;      // bytes of [ksum | vamax]
+    float *v_scale = nullptr, *v_mean = nullptr;
+    size_t stats_bytes = 0;      // bytes of the column statistics
     size_t total = 0;
 };
 
@@ -85,12 +84,15 @@ Workspace carve(char *base, int nseq, int H, int maxlen, int total_tokens, int d
     w.k_scale = reinterpret_cast<float *>(take(heads * nkb * 4));
     w.k_mean = reinterpret_cast<float *>(take(heads * d * 4));
     const size_t stats0 = off;
-    w.ksum = reinterpret_cast<double *>(take(heads * d * 8));
+    w.cs.ksum = reinterpret_cast<double *>(take(heads * d * 8));
     if (pv_mode == SAGE_PV_FP8) {
-        w.vamax = reinterpret_cast<uint32_t *>(take(heads * d * 4));
+        w.cs.vsum = reinterpret_cast<double *>(take(heads * d * 8));
+        w.cs.vhi = reinterpret_cast<uint32_t *>(take(heads * d * 4));
+        w.cs.vneg = reinterpret_cast<uint32_t *>(take(heads * d * 4));
         w.stats_bytes = off - stats0;
         w.v8 = reinterpret_cast<uint8_t *>(take(codes));
         w.v_scale = reinterpret_cast<float *>(take(heads * d * 4));
+        w.v_mean = reinterpret_cast<float *>(take(heads * d * 4));
     } else {
         w.stats_bytes = off - stats0;
     }
@@ -109,14 +111,24 @@ sage_status_t check_shape(int nseq, int H, int maxlen, int d)
     return SAGE_OK;
 }
 
+// The smoothing flags of the fused entry points.
+sage_status_t check_smooth(int smooth, int pv_mode)
+{
+    if (smooth & ~(SAGE_SMOOTH_K | SAGE_SMOOTH_V))
+        return SAGE_ERR_INVALID_ARG;
+    if ((smooth & SAGE_SMOOTH_V) && pv_mode != SAGE_PV_FP8)
+        return SAGE_ERR_UNSUPPORTED;
+    return SAGE_OK;
+}
+
 float resolve_scale(float sm_scale, int d)
 {
     return sm_scale > 0.0f ? sm_scale : 1.0f / std::sqrt((float)d);
 }
 
-// Steps 1-3 with the given scratch; q/k/v/out already validated.
+// Steps 1-3 with the given scratch; q/k/v/out and the smoothing flags already validated.
 sage_status_t forward(const void *q, const void *k, const void *v, void *out, const SeqLayout &L,
-                      int causal, int smooth_k, int pv_mode, float sm_scale, char *ws,
+                      int causal, int smooth, int pv_mode, float sm_scale, char *ws,
                       cudaStream_t st)
 {
     sage_status_t err;
@@ -125,21 +137,27 @@ sage_status_t forward(const void *q, const void *k, const void *v, void *out, co
         return err;
     Workspace w = carve(ws, L.nseq, L.H, L.maxlen, L.total, L.d, pv_mode);
     const bool fp8 = pv_mode == SAGE_PV_FP8;
-    cudaError_t e = cudaMemsetAsync(w.ksum, 0, w.stats_bytes, st);
+    const bool sk = (smooth & SAGE_SMOOTH_K) != 0, sv = (smooth & SAGE_SMOOTH_V) != 0;
+    cudaError_t e = cudaMemsetAsync(w.cs.ksum, 0, w.stats_bytes, st);
     if (e != cudaSuccess)
         return cuda_fail(e);
     const __half *qh = static_cast<const __half *>(q);
     const __half *kh = static_cast<const __half *>(k);
     const __half *vh = static_cast<const __half *>(v);
-    if ((e = launch_colstats(kh, vh, smooth_k ? w.ksum : nullptr, fp8 ? w.vamax : nullptr, L,
-                             status, st)) != cudaSuccess)
+    ColStats cs = w.cs;
+    if (!sk)
+        cs.ksum = nullptr;
+    if (!sv)
+        cs.vsum = nullptr;
+    if ((e = launch_colstats(kh, vh, cs, L, status, st)) != cudaSuccess)
         return cuda_fail(e);
-    if ((e = launch_quant(qh, kh, vh, smooth_k ? w.ksum : nullptr, w.vamax, w.q_i8, w.q_scale,
-                          w.k_i8, w.k_scale, w.k_mean, fp8 ? w.v8 : nullptr, w.v_scale, L, status,
+    if ((e = launch_quant(qh, kh, vh, cs, w.q_i8, w.q_scale, w.k_i8, w.k_scale, w.k_mean,
+                          fp8 ? w.v8 : nullptr, w.v_scale, sv ? w.v_mean : nullptr, L, status,
                           st)) != cudaSuccess)
         return cuda_fail(e);
-    AttnArgs a{w.q_i8, w.q_scale, w.k_i8, w.k_scale, fp8 ? (const void *)w.v8 : v, w.v_scale,
-               static_cast<__half *>(out), nullptr, causal, pv_mode, resolve_scale(sm_scale, L.d)};
+    AttnArgs a{w.q_i8,     w.q_scale, w.k_i8, w.k_scale, fp8 ? (const void *)w.v8 : v,
+               w.v_scale,  sv ? w.v_mean : nullptr,     static_cast<__half *>(out),
+               nullptr,    causal,    pv_mode, resolve_scale(sm_scale, L.d)};
     sage_status_t herr;
     if ((e = launch_attention(a, L, status, st, &herr)) != cudaSuccess)
         return herr != SAGE_OK ? herr : cuda_fail(e);
@@ -160,6 +178,42 @@ sage_status_t quant_qk_entry(const void *q, const void *k, const int32_t *cu_seq
                              int total_tokens, int max_seqlen, int H, int d, int8_t *q_i8,
                              float *q_scale, int8_t *k_i8, float *k_scale, float *k_mean,
                              int smooth_k, void *workspace, size_t ws_bytes, cudaStream_t st);
+sage_status_t quant_v_entry(const void *v, const int32_t *cu_seqlens, int nseq, int total_tokens,
+                            int max_seqlen, int H, int d, uint8_t *v_e4m3, float *v_scale,
+                            float *v_mean, bool smooth, cudaStream_t st);
+
+// Step 3 alone on pre-quantized operands (dense).
+sage_status_t quantized_entry(const int8_t *q_i8, const float *q_scale, const int8_t *k_i8,
+                              const float *k_scale, const void *v, const float *v_scale,
+                              const float *v_mean, void *out, int B, int H, int N, int d,
+                              int causal, int pv_mode, float sm_scale, cudaStream_t st)
+{
+    sage_status_t r = check_shape(B, H, N, d);
+    if (r != SAGE_OK)
+        return r;
+    if (pv_mode != SAGE_PV_FP16 && pv_mode != SAGE_PV_FP8)
+        return SAGE_ERR_INVALID_ARG;
+    if (B == 0 || H == 0 || N == 0)
+        return SAGE_OK;
+    if (!q_i8 || !q_scale || !k_i8 || !k_scale || !v || !out ||
+        (pv_mode == SAGE_PV_FP8 && !v_scale))
+        return SAGE_ERR_INVALID_ARG;
+    if ((int64_t)B * N > INT32_MAX)
+        return SAGE_ERR_UNSUPPORTED;
+    if (!aligned16(q_i8) || !aligned16(k_i8) || !aligned16(v) || !aligned16(out))
+        return SAGE_ERR_MISALIGNED;
+    int *status = status_ptr(&r);
+    if (!status)
+        return r;
+    const SeqLayout L = SeqLayout::dense(B, H, N, d);
+    AttnArgs a{q_i8,   q_scale, k_i8,   k_scale, v, v_scale, v_mean, static_cast<__half *>(out),
+               nullptr, causal, pv_mode, resolve_scale(sm_scale, d)};
+    sage_status_t herr;
+    cudaError_t e = launch_attention(a, L, status, st, &herr);
+    if (e != cudaSuccess)
+        return herr != SAGE_OK ? herr : cuda_fail(e);
+    return SAGE_OK;
+}
 
 }  // namespace
 }  // namespace sage
@@ -230,18 +284,63 @@ sage_status_t quant_qk_entry(const void *q, const void *k, const int32_t *cu_seq
             ksum = static_cast<double *>(p);
             owned = true;
         }
+        ColStats cs;
+        cs.ksum = ksum;
         if ((e = cudaMemsetAsync(ksum, 0, sum_bytes, st)) != cudaSuccess ||
-            (e = launch_colstats(static_cast<const __half *>(k), nullptr, ksum, nullptr, L, status,
-                                 st)) != cudaSuccess) {
+            (e = launch_colstats(static_cast<const __half *>(k), nullptr, cs, L, status, st)) !=
+                cudaSuccess) {
             if (owned)
                 cudaFreeAsync(ksum, st);
             return cuda_fail(e);
         }
     }
-    e = launch_quant(static_cast<const __half *>(q), static_cast<const __half *>(k), nullptr, ksum,
-                     nullptr, q_i8, q_scale, k_i8, k_scale, k_mean, nullptr, nullptr, L, status, st);
+    ColStats cs;
+    cs.ksum = ksum;
+    e = launch_quant(static_cast<const __half *>(q), static_cast<const __half *>(k), nullptr, cs,
+                     q_i8, q_scale, k_i8, k_scale, k_mean, nullptr, nullptr, nullptr, L, status,
+                     st);
     if (owned)
         cudaFreeAsync(ksum, st);
+    return e == cudaSuccess ? SAGE_OK : cuda_fail(e);
+}
+
+// V to E4M3 (smooth: V - mean(V) first, the mean written to v_mean), dense or packed.
+sage_status_t quant_v_entry(const void *v, const int32_t *cu_seqlens, int nseq, int total_tokens,
+                            int max_seqlen, int H, int d, uint8_t *v_e4m3, float *v_scale,
+                            float *v_mean, bool smooth, cudaStream_t st)
+{
+    sage_status_t r = check_shape(nseq, H, max_seqlen, d);
+    if (r != SAGE_OK)
+        return r;
+    if (nseq == 0 || H == 0 || max_seqlen == 0 || total_tokens == 0)
+        return SAGE_OK;
+    if (!v || !v_e4m3 || !v_scale || (smooth && !v_mean) || total_tokens < 0)
+        return SAGE_ERR_INVALID_ARG;
+    if (!aligned16(v) || !aligned16(v_e4m3))
+        return SAGE_ERR_MISALIGNED;
+    int *status = status_ptr(&r);
+    if (!status)
+        return r;
+    const SeqLayout L = cu_seqlens ? SeqLayout::packed(cu_seqlens, nseq, total_tokens, max_seqlen, H, d)
+                                   : SeqLayout::dense(nseq, H, max_seqlen, d);
+    // [vsum (fp64) | vhi | vneg] per (sequence, head, channel)
+    const size_t n = (size_t)nseq * H * d;
+    const size_t bytes = n * (8 + 4 + 4);
+    void *p = nullptr;
+    cudaError_t e;
+    if ((e = cudaMallocAsync(&p, bytes, st)) != cudaSuccess)
+        return cuda_fail(e);
+    ColStats cs;
+    cs.vsum = smooth ? static_cast<double *>(p) : nullptr;
+    cs.vhi = reinterpret_cast<uint32_t *>(static_cast<char *>(p) + n * 8);
+    cs.vneg = cs.vhi + n;
+    if ((e = cudaMemsetAsync(p, 0, bytes, st)) == cudaSuccess &&
+        (e = launch_colstats(nullptr, static_cast<const __half *>(v), cs, L, status, st)) ==
+            cudaSuccess)
+        e = launch_quant(nullptr, nullptr, static_cast<const __half *>(v), cs, nullptr, nullptr,
+                         nullptr, nullptr, nullptr, v_e4m3, v_scale, smooth ? v_mean : nullptr,
+                         L, status, st);
+    cudaFreeAsync(p, st);
     return e == cudaSuccess ? SAGE_OK : cuda_fail(e);
 }
 }  // namespace
@@ -272,44 +371,40 @@ sage_status_t sage_quant_qk_ws(const void *q, const void *k, int8_t *q_i8, float
                           smooth_k, workspace, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
+sage_status_t sage_quant_v_fp8_smooth_varlen(const void *v, const int32_t *cu_seqlens, int nseq,
+                                             int total_tokens, int max_seqlen, int H, int d,
+                                             uint8_t *v_e4m3, float *v_scale, float *v_mean,
+                                             sage_stream_t stream)
+{
+    return quant_v_entry(v, cu_seqlens, nseq, total_tokens, max_seqlen, H, d, v_e4m3, v_scale,
+                         v_mean, true, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sage_status_t sage_quant_v_fp8_smooth(const void *v, uint8_t *v_e4m3, float *v_scale,
+                                      float *v_mean, int B, int H, int N, int d,
+                                      sage_stream_t stream)
+{
+    if (B > 0 && N > 0 && (int64_t)B * N > INT32_MAX)
+        return SAGE_ERR_UNSUPPORTED;
+    return quant_v_entry(v, nullptr, B, B * N, N, H, d, v_e4m3, v_scale, v_mean, true,
+                         reinterpret_cast<cudaStream_t>(stream));
+}
+
 sage_status_t sage_quant_v_fp8_varlen(const void *v, const int32_t *cu_seqlens, int nseq,
                                       int total_tokens, int max_seqlen, int H, int d,
                                       uint8_t *v_e4m3, float *v_scale, sage_stream_t stream)
 {
-    sage_status_t r = check_shape(nseq, H, max_seqlen, d);
-    if (r != SAGE_OK)
-        return r;
-    if (nseq == 0 || H == 0 || max_seqlen == 0 || total_tokens == 0)
-        return SAGE_OK;
-    if (!v || !v_e4m3 || !v_scale || total_tokens < 0)
-        return SAGE_ERR_INVALID_ARG;
-    if (!aligned16(v) || !aligned16(v_e4m3))
-        return SAGE_ERR_MISALIGNED;
-    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    int *status = status_ptr(&r);
-    if (!status)
-        return r;
-    const SeqLayout L = cu_seqlens ? SeqLayout::packed(cu_seqlens, nseq, total_tokens, max_seqlen, H, d)
-                                   : SeqLayout::dense(nseq, H, max_seqlen, d);
-    void *p = nullptr;
-    const size_t bytes = (size_t)nseq * H * d * 4;
-    cudaError_t e;
-    if ((e = cudaMallocAsync(&p, bytes, st)) != cudaSuccess)
-        return cuda_fail(e);
-    uint32_t *vamax = static_cast<uint32_t *>(p);
-    if ((e = cudaMemsetAsync(vamax, 0, bytes, st)) == cudaSuccess &&
-        (e = launch_colstats(nullptr, static_cast<const __half *>(v), nullptr, vamax, L, status,
-                             st)) == cudaSuccess)
-        e = launch_quant(nullptr, nullptr, static_cast<const __half *>(v), nullptr, vamax, nullptr,
-                         nullptr, nullptr, nullptr, nullptr, v_e4m3, v_scale, L, status, st);
-    cudaFreeAsync(p, st);
-    return e == cudaSuccess ? SAGE_OK : cuda_fail(e);
+    return quant_v_entry(v, cu_seqlens, nseq, total_tokens, max_seqlen, H, d, v_e4m3, v_scale,
+                         nullptr, false, reinterpret_cast<cudaStream_t>(stream));
 }
 
 sage_status_t sage_quant_v_fp8(const void *v, uint8_t *v_e4m3, float *v_scale, int B, int H,
                                int N, int d, sage_stream_t stream)
 {
-    return sage_quant_v_fp8_varlen(v, nullptr, B, B * N, N, H, d, v_e4m3, v_scale, stream);
+    if (B > 0 && N > 0 && (int64_t)B * N > INT32_MAX)
+        return SAGE_ERR_UNSUPPORTED;
+    return quant_v_entry(v, nullptr, B, B * N, N, H, d, v_e4m3, v_scale, nullptr, false,
+                         reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"
@@ -327,6 +422,8 @@ sage_status_t attn_entry(const void *q, const void *k, const void *v, void *out,
         return r;
     if (pv_mode != SAGE_PV_FP16 && pv_mode != SAGE_PV_FP8)
         return SAGE_ERR_INVALID_ARG;
+    if ((r = check_smooth(smooth_k, pv_mode)) != SAGE_OK)
+        return r;
     if (total_tokens < 0)
         return SAGE_ERR_INVALID_ARG;
     if (nseq == 0 || H == 0 || max_seqlen == 0 || total_tokens == 0)
@@ -400,29 +497,22 @@ sage_status_t sage_attn_fwd_quantized(const int8_t *q_i8, const float *q_scale,
                                       int d, int causal, int pv_mode, float sm_scale,
                                       sage_stream_t stream)
 {
-    sage_status_t r = check_shape(B, H, N, d);
-    if (r != SAGE_OK)
-        return r;
-    if (pv_mode != SAGE_PV_FP16 && pv_mode != SAGE_PV_FP8)
+    return quantized_entry(q_i8, q_scale, k_i8, k_scale, v, v_scale, nullptr, out, B, H, N, d,
+                           causal, pv_mode, sm_scale, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sage_status_t sage_attn_fwd_quantized_smooth_v(const int8_t *q_i8, const float *q_scale,
+                                               const int8_t *k_i8, const float *k_scale,
+                                               const uint8_t *v_e4m3, const float *v_scale,
+                                               const float *v_mean, void *out, int B, int H,
+                                               int N, int d, int causal, float sm_scale,
+                                               sage_stream_t stream)
+{
+    if (v_mean == nullptr && B > 0 && H > 0 && N > 0)
         return SAGE_ERR_INVALID_ARG;
-    if (B == 0 || H == 0 || N == 0)
-        return SAGE_OK;
-    if (!q_i8 || !q_scale || !k_i8 || !k_scale || !v || !out ||
-        (pv_mode == SAGE_PV_FP8 && !v_scale))
-        return SAGE_ERR_INVALID_ARG;
-    if (!aligned16(q_i8) || !aligned16(k_i8) || !aligned16(v) || !aligned16(out))
-        return SAGE_ERR_MISALIGNED;
-    int *status = status_ptr(&r);
-    if (!status)
-        return r;
-    const SeqLayout L = SeqLayout::dense(B, H, N, d);
-    AttnArgs a{q_i8, q_scale, k_i8, k_scale, v, v_scale, static_cast<__half *>(out), nullptr,
-               causal, pv_mode, resolve_scale(sm_scale, d)};
-    sage_status_t herr;
-    cudaError_t e = launch_attention(a, L, status, reinterpret_cast<cudaStream_t>(stream), &herr);
-    if (e != cudaSuccess)
-        return herr != SAGE_OK ? herr : cuda_fail(e);
-    return SAGE_OK;
+    return quantized_entry(q_i8, q_scale, k_i8, k_scale, v_e4m3, v_scale, v_mean, out, B, H, N,
+                           d, causal, SAGE_PV_FP8, sm_scale,
+                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 sage_status_t sage_debug_qk_int32(const int8_t *q_i8, const int8_t *k_i8, int32_t *s_out, int B,
@@ -454,7 +544,7 @@ sage_status_t sage_debug_qk_int32(const int8_t *q_i8, const int8_t *k_i8, int32_
         const float *ks = qs + (size_t)B * H * nqb;
         const void *vz = ws + sc_bytes;
         __half *o = reinterpret_cast<__half *>(ws + sc_bytes + align256(elems * 2));
-        AttnArgs a{q_i8, qs, k_i8, ks, vz, nullptr, o, s_out, 0, SAGE_PV_FP16, 1.0f};
+        AttnArgs a{q_i8, qs, k_i8, ks, vz, nullptr, nullptr, o, s_out, 0, SAGE_PV_FP16, 1.0f};
         sage_status_t herr;
         e = launch_attention(a, SeqLayout::dense(B, H, N, d), status, st, &herr);
         if (e != cudaSuccess && herr != SAGE_OK) {
@@ -569,6 +659,8 @@ extern "C" sage_status_t sage_attn_fwd_noalloc(const void *q, const void *k, con
         return r;
     if (pv_mode != SAGE_PV_FP16 && pv_mode != SAGE_PV_FP8)
         return SAGE_ERR_INVALID_ARG;
+    if ((r = check_smooth(smooth_k, pv_mode)) != SAGE_OK)
+        return r;
     if (B == 0 || H == 0 || N == 0)
         return SAGE_OK;
     if ((int64_t)B * N > INT32_MAX)
@@ -589,8 +681,8 @@ extern "C" sage_status_t sage_attn_fwd_noalloc(const void *q, const void *k, con
     char *ws = nullptr;
     if ((r = noalloc_scratch(&ws)) != SAGE_OK)
         return r;
-    // forward() zeroes the only scratch that must start at zero (the K column sums and
-    // V maxima) before its kernels run; everything else is written before it is read.
+    // forward() zeroes the only scratch that must start at zero (the K and V column
+    // statistics) before its kernels run; everything else is written before it is read.
     return forward(q, k, v, out, SeqLayout::dense(B, H, N, d), causal, smooth_k, pv_mode,
                    sm_scale, ws, reinterpret_cast<cudaStream_t>(stream));
 }

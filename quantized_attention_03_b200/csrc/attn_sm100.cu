@@ -117,6 +117,7 @@ struct KParams {
     const float *q_scale;
     const float *k_scale;
     const float *v_scale;
+    const float *v_mean;   // FP8 with smooth V: added to every output row; else nullptr
     __half *out;
     int32_t *s_dump;
     SeqLayout L;
@@ -463,6 +464,9 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
                             if constexpr (FP8)
                                 sc = __ldg(p.v_scale + sh * D + ch * 32 + c + e) * inv_l;
                             f[e] = __uint_as_float(r[c + e]) * sc;
+                            if constexpr (FP8)
+                                if (p.v_mean != nullptr)
+                                    f[e] += __ldg(p.v_mean + sh * D + ch * 32 + c + e);
                         }
                         uint4 u;
                         u.x = pack_half2(f[0], f[1]);
@@ -701,6 +705,7 @@ cudaError_t run(const AttnArgs &a, const SeqLayout &L, int *status, cudaStream_t
     p.q_scale = a.q_scale;
     p.k_scale = a.k_scale;
     p.v_scale = a.v_scale;
+    p.v_mean = a.v_mean;
     p.out = a.out;
     p.s_dump = a.s_dump;
     p.L = L;

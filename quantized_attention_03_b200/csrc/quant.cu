@@ -3,12 +3,15 @@
 // 「SageAttention：低比特量化Attention，实现推理加速」, section 技术方案: K <- K - mean(K) with the mean per channel
 // over tokens; Q and K quantized to INT8 per block of FlashAttention size (Q: 128
 // tokens, K: 64 tokens) with one fp32 scale amax/127 per block. "SageAttention2"
-// article, 技术方案 (4): V in E4M3, here with one fp32 scale (amax/448) per channel.
+// article, 技术方案 (4): V in E4M3, here with one fp32 scale (amax/448) per channel;
+// the paragraph after (4): optionally V <- V - mean(V) first (smooth V).
 //
 // Two HBM-bound passes:
-//   colstats: per-(sequence, head, channel) reductions over tokens: fp64 sums of K
-//             (exact for |K| N < 2^29, so the mean does not depend on summation order)
-//             and the fp32 amax of |V|. Row chunks of 512 tokens, fp64 atomics.
+//   colstats: per-(sequence, head, channel) reductions over tokens: fp64 sums of K and
+//             V (exact for |x| N < 2^29, so the means do not depend on summation
+//             order) and the max and min of V. Row chunks of 512 tokens, atomics.
+//             amax |fl(V - mean)| = max(fl(max V - mean), fl(mean - min V)) exactly,
+//             because fp32 rounding is monotonic, so V needs no third pass.
 //   quant:    one CTA per 128-token chunk of Q (one Q block), K (two K blocks) or V;
 //             16-byte vector loads/stores, warp-shuffle amax. Codes are the rounding of
 //             the IEEE fp32 quotient x / scale, computed as x * (1 / scale) with an exact
@@ -41,12 +44,11 @@ __device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8])
 template <int D>
 __global__ void __launch_bounds__(kThreads) colstats_kernel(const __half *__restrict__ k,
                                                             const __half *__restrict__ v,
-                                                            double *__restrict__ ksum,
-                                                            uint32_t *__restrict__ vamax,
-                                                            SeqLayout L, int *status)
+                                                            ColStats cs, SeqLayout L, int *status)
 {
     constexpr int kGroups = D / 8;              // 16-byte column groups per row
     constexpr int kRowsPerPass = kThreads / kGroups;
+    constexpr int kWarps = kThreads / 32;
     const int s = blockIdx.z, h = blockIdx.y;
     int start, len;
     if (!L.range(s, start, len, status))
@@ -56,52 +58,78 @@ __global__ void __launch_bounds__(kThreads) colstats_kernel(const __half *__rest
         return;
     const int r_end = min(len, r_begin + kColChunk);
     const int g = threadIdx.x % kGroups, r0 = threadIdx.x / kGroups;
+    const bool do_k = cs.ksum != nullptr, do_v = cs.vhi != nullptr, do_vsum = cs.vsum != nullptr;
 
-    double acc[8];
-    float amx[8];
+    double ks[8], vs[8];
+    float hi[8], ng[8];                          // max V and max -V
 #pragma unroll
     for (int i = 0; i < 8; i++) {
-        acc[i] = 0.0;
-        amx[i] = 0.0f;
+        ks[i] = vs[i] = 0.0;
+        hi[i] = ng[i] = -INFINITY;
     }
     for (int r = r_begin + r0; r < r_end; r += kRowsPerPass) {
         const int64_t off = L.offset(s, start, h, r) + g * 8;
         float f[8];
-        if (ksum != nullptr) {
+        if (do_k) {
             unpack8(__ldg(reinterpret_cast<const uint4 *>(k + off)), f);
 #pragma unroll
             for (int i = 0; i < 8; i++)
-                acc[i] += (double)f[i];
+                ks[i] += (double)f[i];
         }
-        if (vamax != nullptr) {
+        if (do_v) {
             unpack8(__ldg(reinterpret_cast<const uint4 *>(v + off)), f);
 #pragma unroll
-            for (int i = 0; i < 8; i++)
-                amx[i] = fmaxf(amx[i], fabsf(f[i]));
+            for (int i = 0; i < 8; i++) {
+                hi[i] = fmaxf(hi[i], f[i]);
+                ng[i] = fmaxf(ng[i], -f[i]);
+                if (do_vsum)
+                    vs[i] += (double)f[i];
+            }
         }
     }
 
-    __shared__ double s_sum[kRowsPerPass][D];
-    __shared__ float s_max[kRowsPerPass][D];
+    // lanes kGroups apart hold the same columns: fold them, then one row per warp
 #pragma unroll
-    for (int i = 0; i < 8; i++) {
-        s_sum[r0][g * 8 + i] = acc[i];
-        s_max[r0][g * 8 + i] = amx[i];
+    for (int o = kGroups; o < 32; o <<= 1)
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            ks[i] += __shfl_xor_sync(0xffffffffu, ks[i], o);
+            vs[i] += __shfl_xor_sync(0xffffffffu, vs[i], o);
+            hi[i] = fmaxf(hi[i], __shfl_xor_sync(0xffffffffu, hi[i], o));
+            ng[i] = fmaxf(ng[i], __shfl_xor_sync(0xffffffffu, ng[i], o));
+        }
+    __shared__ double s_ks[kWarps][D], s_vs[kWarps][D];
+    __shared__ float s_hi[kWarps][D], s_ng[kWarps][D];
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (lane < kGroups) {
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            s_ks[warp][g * 8 + i] = ks[i];
+            s_vs[warp][g * 8 + i] = vs[i];
+            s_hi[warp][g * 8 + i] = hi[i];
+            s_ng[warp][g * 8 + i] = ng[i];
+        }
     }
     __syncthreads();
     if (threadIdx.x < D) {
         const int c = threadIdx.x;
-        double t = 0.0;
-        float m = 0.0f;
-        for (int r = 0; r < kRowsPerPass; r++) {
-            t += s_sum[r][c];
-            m = fmaxf(m, s_max[r][c]);
+        double tk = 0.0, tv = 0.0;
+        float mh = -INFINITY, mn = -INFINITY;
+        for (int w = 0; w < kWarps; w++) {
+            tk += s_ks[w][c];
+            tv += s_vs[w][c];
+            mh = fmaxf(mh, s_hi[w][c]);
+            mn = fmaxf(mn, s_ng[w][c]);
         }
         const int64_t o = ((int64_t)s * L.H + h) * D + c;
-        if (ksum != nullptr)
-            atomicAdd(ksum + o, t);
-        if (vamax != nullptr)
-            atomicMax(vamax + o, __float_as_uint(m));   // non-negative floats order as ints
+        if (do_k)
+            atomicAdd(cs.ksum + o, tk);
+        if (do_v) {
+            if (do_vsum)
+                atomicAdd(cs.vsum + o, tv);
+            atomicMax(cs.vhi + o, float_key(__float_as_uint(mh)));
+            atomicMax(cs.vneg + o, float_key(__float_as_uint(mn)));
+        }
     }
 }
 
@@ -161,9 +189,9 @@ __device__ __forceinline__ float e4m3_quotient(float x, float s, float r)
 template <int D>
 __global__ void __launch_bounds__(kThreads) quant_kernel(
     const __half *__restrict__ q, const __half *__restrict__ k, const __half *__restrict__ v,
-    const double *__restrict__ ksum, const uint32_t *__restrict__ vamax, int8_t *__restrict__ q_i8,
-    float *__restrict__ q_scale, int8_t *__restrict__ k_i8, float *__restrict__ k_scale,
-    float *__restrict__ k_mean, uint8_t *__restrict__ v_e4m3, float *__restrict__ v_scale,
+    ColStats cs, int8_t *__restrict__ q_i8, float *__restrict__ q_scale,
+    int8_t *__restrict__ k_i8, float *__restrict__ k_scale, float *__restrict__ k_mean,
+    uint8_t *__restrict__ v_e4m3, float *__restrict__ v_scale, float *__restrict__ v_mean,
     SeqLayout L, int nqb, int nkb, int part0, int *status)
 {
     constexpr int kHalf = D / 2;          // elements per thread (two threads per token)
@@ -171,6 +199,8 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(
     __shared__ float s_red[8];
     __shared__ float s_aux[D];            // K mean or V scale per channel
     __shared__ float s_rcp[D];            // fl(1 / V scale) per channel
+    __shared__ float s_vmu[D];            // V mean per channel (0 without smooth V)
+    const double *ksum = cs.ksum;
 
     const int s = blockIdx.z, h = blockIdx.y;
     int start, len;
@@ -188,6 +218,11 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(
     if (row0 >= len) {                    // padding block of a short sequence
         if (kind == 1 && chunk == 0 && threadIdx.x < D)
             k_mean[sh * D + threadIdx.x] = 0.0f;
+        if (kind == 2 && chunk == 0 && threadIdx.x < D) {   // empty sequence
+            v_scale[sh * D + threadIdx.x] = 0.0f;
+            if (v_mean != nullptr)
+                v_mean[sh * D + threadIdx.x] = 0.0f;
+        }
         if (threadIdx.x == 0) {
             if (kind == 0)
                 q_scale[sh * nqb + chunk] = 0.0f;
@@ -210,11 +245,21 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(
     }
     if (kind == 2 && threadIdx.x < D) {
         const int c = threadIdx.x;
-        const float sv = __fdiv_rn(__uint_as_float(vamax[sh * D + c]), 448.0f);
+        const int64_t o = sh * D + c;
+        const float mu = cs.vsum ? (float)(cs.vsum[o] / (double)len) : 0.0f;
+        const float vmax = __uint_as_float(key_bits(cs.vhi[o]));
+        const float vnegmax = __uint_as_float(key_bits(cs.vneg[o]));   // -min V
+        // the largest |fl(V - mu)|: rounding is monotonic, so it is at max V or min V
+        const float amax = fmaxf(__fsub_rn(vmax, mu), __fadd_rn(vnegmax, mu));
+        const float sv = __fdiv_rn(amax, 448.0f);
         s_aux[c] = sv;
         s_rcp[c] = sv != 0.0f ? __fdiv_rn(1.0f, sv) : 0.0f;
-        if (chunk == 0)
-            v_scale[sh * D + c] = sv;
+        s_vmu[c] = mu;
+        if (chunk == 0) {
+            v_scale[o] = sv;
+            if (v_mean != nullptr)
+                v_mean[o] = mu;
+        }
     }
     __syncthreads();
 
@@ -245,8 +290,10 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(
             float qv[4];
 #pragma unroll
             for (int e = 0; e < 4; e++) {
-                const float sv = s_aux[col0 + i + e];
-                qv[e] = sv != 0.0f ? e4m3_quotient(x[i + e], sv, s_rcp[col0 + i + e]) : 0.0f;
+                const int c = col0 + i + e;
+                const float sv = s_aux[c];
+                const float xs = __fsub_rn(x[i + e], s_vmu[c]);
+                qv[e] = sv != 0.0f ? e4m3_quotient(xs, sv, s_rcp[c]) : 0.0f;
             }
             const uint32_t lo = pack_e4m3x2(qv[0], qv[1]);
             const uint32_t hi = pack_e4m3x2(qv[2], qv[3]);
@@ -305,23 +352,22 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(
 
 }  // namespace
 
-cudaError_t launch_colstats(const __half *k, const __half *v, double *ksum, uint32_t *vamax,
+cudaError_t launch_colstats(const __half *k, const __half *v, const ColStats &cs,
                             const SeqLayout &L, int *status, cudaStream_t st)
 {
-    if (ksum == nullptr && vamax == nullptr)
+    if (cs.ksum == nullptr && cs.vhi == nullptr)
         return cudaSuccess;
     dim3 grid((L.maxlen + kColChunk - 1) / kColChunk, L.H, L.nseq);
     if (L.d == 128)
-        colstats_kernel<128><<<grid, kThreads, 0, st>>>(k, v, ksum, vamax, L, status);
+        colstats_kernel<128><<<grid, kThreads, 0, st>>>(k, v, cs, L, status);
     else
-        colstats_kernel<64><<<grid, kThreads, 0, st>>>(k, v, ksum, vamax, L, status);
+        colstats_kernel<64><<<grid, kThreads, 0, st>>>(k, v, cs, L, status);
     return cudaGetLastError();
 }
 
-// Quantizes Q and K (q_i8 != nullptr) and/or V (v_e4m3 != nullptr) in one launch.
-cudaError_t launch_quant(const __half *q, const __half *k, const __half *v, const double *ksum,
-                         const uint32_t *vamax, int8_t *q_i8, float *q_scale, int8_t *k_i8,
-                         float *k_scale, float *k_mean, uint8_t *v_e4m3, float *v_scale,
+cudaError_t launch_quant(const __half *q, const __half *k, const __half *v, const ColStats &cs,
+                         int8_t *q_i8, float *q_scale, int8_t *k_i8, float *k_scale,
+                         float *k_mean, uint8_t *v_e4m3, float *v_scale, float *v_mean,
                          const SeqLayout &L, int *status, cudaStream_t st)
 {
     const int nqb = (L.maxlen + kQBlock - 1) / kQBlock;
@@ -332,12 +378,12 @@ cudaError_t launch_quant(const __half *q, const __half *k, const __half *v, cons
         return cudaSuccess;
     dim3 grid(nqb * (part1 - part0), L.H, L.nseq);
     if (L.d == 128)
-        quant_kernel<128><<<grid, kThreads, 0, st>>>(q, k, v, ksum, vamax, q_i8, q_scale, k_i8,
-                                                     k_scale, k_mean, v_e4m3, v_scale, L, nqb,
+        quant_kernel<128><<<grid, kThreads, 0, st>>>(q, k, v, cs, q_i8, q_scale, k_i8, k_scale,
+                                                     k_mean, v_e4m3, v_scale, v_mean, L, nqb,
                                                      nkb, part0, status);
     else
-        quant_kernel<64><<<grid, kThreads, 0, st>>>(q, k, v, ksum, vamax, q_i8, q_scale, k_i8,
-                                                    k_scale, k_mean, v_e4m3, v_scale, L, nqb,
+        quant_kernel<64><<<grid, kThreads, 0, st>>>(q, k, v, cs, q_i8, q_scale, k_i8, k_scale,
+                                                    k_mean, v_e4m3, v_scale, v_mean, L, nqb,
                                                     nkb, part0, status);
     return cudaGetLastError();
 }

@@ -64,12 +64,36 @@ struct SeqLayout {
 // Device status bits are 1 << sage_status_t; the host reports the lowest set.
 __host__ __device__ constexpr int status_bit(sage_status_t s) { return 1 << (int)s; }
 
+// Per-(sequence, head, channel) reductions over tokens, each [nseq, H, d], zeroed by the
+// caller before colstats accumulates into them. A null member is not computed.
+//   ksum, vsum: fp64 sums of K and V (exact, so the means are order-independent);
+//   vhi, vneg:  max V and max -V as order-preserving keys (float_key) for atomicMax.
+struct ColStats {
+    double *ksum = nullptr;
+    double *vsum = nullptr;
+    uint32_t *vhi = nullptr;
+    uint32_t *vneg = nullptr;
+};
+
+// Unsigned key whose integer order is the float order (for atomicMax on floats of any
+// sign); key 0 is below every float.
+__host__ __device__ inline uint32_t float_key(uint32_t bits)
+{
+    return (bits & 0x80000000u) ? ~bits : (bits | 0x80000000u);
+}
+__host__ __device__ inline uint32_t key_bits(uint32_t key)
+{
+    return (key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key;
+}
+
 // Launchers (quant.cu, attn_sm100.cu). All return cudaSuccess or the launch error.
-cudaError_t launch_colstats(const __half *k, const __half *v, double *ksum, uint32_t *vamax,
+cudaError_t launch_colstats(const __half *k, const __half *v, const ColStats &cs,
                             const SeqLayout &L, int *status, cudaStream_t st);
-cudaError_t launch_quant(const __half *q, const __half *k, const __half *v, const double *ksum,
-                         const uint32_t *vamax, int8_t *q_i8, float *q_scale, int8_t *k_i8,
-                         float *k_scale, float *k_mean, uint8_t *v_e4m3, float *v_scale,
+// Quantizes Q and K (q_i8 != nullptr) and/or V (v_e4m3 != nullptr). K is smoothed when
+// cs.ksum is set, V when cs.vsum is set (its mean goes to v_mean if that is set).
+cudaError_t launch_quant(const __half *q, const __half *k, const __half *v, const ColStats &cs,
+                         int8_t *q_i8, float *q_scale, int8_t *k_i8, float *k_scale,
+                         float *k_mean, uint8_t *v_e4m3, float *v_scale, float *v_mean,
                          const SeqLayout &L, int *status, cudaStream_t st);
 
 struct AttnArgs {
@@ -79,6 +103,7 @@ struct AttnArgs {
     const float *k_scale;
     const void *v;        // fp16 V or E4M3 codes
     const float *v_scale; // FP8 mode
+    const float *v_mean;  // FP8 mode with smooth V, else nullptr
     __half *out;
     int32_t *s_dump;      // debug: int32 scores [nseq,H,maxlen,maxlen] or nullptr
     int causal;

@@ -48,8 +48,8 @@ FAKE = 0x10000          # 16-byte aligned, never dereferenced: validation fails 
 MIS = 0x10008           # 8-byte aligned only
 
 
-def _fwd(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, B=1, H=1, N=128, d=64, pv=0):
-    return lib.sage_attn_fwd(q, k, v, o, B, H, N, d, 0, 1, pv, 0.0, None)
+def _fwd(lib, q=FAKE, k=FAKE, v=FAKE, o=FAKE, B=1, H=1, N=128, d=64, pv=0, smooth=1):
+    return lib.sage_attn_fwd(q, k, v, o, B, H, N, d, 0, smooth, pv, 0.0, None)
 
 
 def test_host_validation(lib):
@@ -61,6 +61,23 @@ def test_host_validation(lib):
     assert _fwd(lib, v=MIS) == sage.SAGE_ERR_MISALIGNED
     assert _fwd(lib, o=MIS) == sage.SAGE_ERR_MISALIGNED
     assert _fwd(lib, H=70000) == sage.SAGE_ERR_UNSUPPORTED
+
+
+def test_smoothing_flags(lib):
+    # smooth V needs FP8 P.V (fp16 V is never quantized); unknown bits are rejected
+    assert _fwd(lib, smooth=sage.SAGE_SMOOTH_V, pv=0) == sage.SAGE_ERR_UNSUPPORTED
+    assert _fwd(lib, smooth=3, pv=0) == sage.SAGE_ERR_UNSUPPORTED
+    assert _fwd(lib, smooth=4, pv=1) == sage.SAGE_ERR_INVALID_ARG
+    assert _fwd(lib, smooth=-1, pv=1) == sage.SAGE_ERR_INVALID_ARG
+    assert _fwd(lib, smooth=3, pv=1, q=0) == sage.SAGE_ERR_INVALID_ARG      # flags accepted
+    assert lib.sage_attn_fwd_noalloc(FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 0, 2, 0, 0.0,
+                                     None) == sage.SAGE_ERR_UNSUPPORTED
+    # the pre-quantized smooth-V entry needs the V mean
+    assert lib.sage_attn_fwd_quantized_smooth_v(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE,
+                                                1, 1, 128, 64, 0, 0.0, None) == \
+        sage.SAGE_ERR_INVALID_ARG
+    assert lib.sage_quant_v_fp8_smooth(FAKE, FAKE, FAKE, None, 1, 1, 128, 64, None) == \
+        sage.SAGE_ERR_INVALID_ARG
 
 
 def test_empty_inputs_are_noops(lib):

@@ -201,3 +201,98 @@ def test_fp8_relative_l1_is_reported():
     r = rel_l1(got, exact)
     print(f"FP8 PV relative L1 vs fp64: {r:.4f}")
     assert r < 0.06
+
+
+# ------------------------------------------------------------ smooth V (FP8 P.V mode)
+
+
+def _offset_v(v, d, seed, amp=6.0):
+    """V with a per-channel offset of up to +-amp (outputs stay below 16 in magnitude, so
+    the fp16 output rounding stays inside the max |error| bound)."""
+    g = torch.Generator().manual_seed(seed)
+    off = (torch.rand(d, generator=g) * 2 - 1) * amp
+    return (v.float() + off).half()
+
+
+SMOOTH_V_CASES = [(1, 64, False), (129, 128, True), (300, 64, True), (513, 128, False),
+                  (1000, 128, True)]
+
+
+@pytest.mark.parametrize("N,d,causal", SMOOTH_V_CASES)
+def test_smooth_v_small_full_compare(N, d, causal):
+    B, H = 2, 2
+    w = inputs.Workload("t", 300 + N + d, B, H, N, d, causal, 2.0)
+    q, k, v = inputs.make_dense(w)
+    v = _offset_v(v, d, 301 + N)
+    out = sage.sageattn(q.cuda(), k.cuda(), v.cuda(), causal, True, sage.SAGE_PV_FP8,
+                        smooth_v=True)
+    plain = sage.sageattn(q.cuda(), k.cuda(), v.cuda(), causal, True, sage.SAGE_PV_FP8)
+    assert sage.sage_get_device_status() == 0
+    got, raw = _np(out), _np(plain)
+    lay = oracle.Layout.dense(B, H, N, d)
+    ref = oracle.sage_attention(q.numpy(), k.numpy(), v.numpy(), lay, causal, True,
+                                oracle.PV_FP8, smooth_v=True)
+    tag = f"smooth V N={N} d={d} causal={causal}"
+    assert_vs_oracle(got, ref, tag)
+    exact = oracle.attn_fp64(q.numpy(), k.numpy(), v.numpy(), lay, causal, 1 / math.sqrt(d))
+    assert_vs_fp64(got, exact, True, tag)
+    if N > 1:   # the smoothed V codes spend their range on the spread, not on the offset
+        assert rel_l1(got, exact) < rel_l1(raw, exact)
+
+
+def test_smooth_v_quantized_entry_matches_fused():
+    B, H, N, d = 2, 3, 700, 128
+    w = inputs.Workload("t", 71, B, H, N, d, True, 1.0)
+    q, k, v = inputs.make_dense(w)
+    qd, kd, vd = q.cuda(), k.cuda(), _offset_v(v, d, 72).cuda()
+    fused = sage.sageattn(qd, kd, vd, True, True, sage.SAGE_PV_FP8, smooth_v=True)
+    z = sage.quant_qk(qd, kd, True)
+    codes, scales, mean = sage.quant_v_fp8(vd, smooth_v=True)
+    split = sage.attn_quantized(z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], codes, scales,
+                                True, sage.SAGE_PV_FP8, v_mean=mean)
+    need = sage.sage_workspace_size(B, H, N, B * N, d, sage.SAGE_PV_FP8)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    out_ws = torch.empty_like(qd)
+    sage.sage_attn_fwd_ws(qd, kd, vd, out_ws, B, H, N, d, 1,
+                          sage.SAGE_SMOOTH_K | sage.SAGE_SMOOTH_V, sage.SAGE_PV_FP8, 0.0, ws, need)
+    assert sage.sage_get_device_status() == 0
+    assert torch.equal(fused, split) and torch.equal(fused, out_ws)
+
+
+def test_smooth_v_varlen_full_compare():
+    H, d = 4, 64
+    lens = [1, 200, 129, 0, 700, 64]
+    w = inputs.Workload("t", 81, 0, H, 0, d, True, 2.0, nseq=len(lens))
+    q, k, v, cu = inputs.make_varlen(w, lens=lens)
+    v = _offset_v(v, d, 82)
+    out = sage.sageattn_varlen(q.cuda(), k.cuda(), v.cuda(), cu.cuda(), max(lens), True, True,
+                               sage.SAGE_PV_FP8, smooth_v=True)
+    assert sage.sage_get_device_status() == 0
+    got = _np(out)
+    lay = oracle.Layout.packed(cu.tolist(), H, d)
+    ref = oracle.sage_attention(q.numpy(), k.numpy(), v.numpy(), lay, True, True, oracle.PV_FP8,
+                                smooth_v=True)
+    assert_vs_oracle(got, ref, "varlen smooth V")
+    exact = oracle.attn_fp64(q.numpy(), k.numpy(), v.numpy(), lay, True, 1 / math.sqrt(d))
+    assert_vs_fp64(got, exact, True, "varlen smooth V")
+
+
+def test_smooth_v_full_size_video_dit_sampled():
+    w = inputs.video_dit()
+    q, k, v = inputs.make_dense(w)
+    v = _offset_v(v, w.d, 91)
+    got = _np(sage.sageattn(q.cuda(), k.cuda(), v.cuda(), False, True, sage.SAGE_PV_FP8,
+                            smooth_v=True))
+    assert sage.sage_get_device_status() == 0
+    lay = oracle.Layout.dense(w.B, w.H, w.N, w.d)
+    qn, kn, vn = q.numpy(), k.numpy(), v.numpy()
+    for h in (0, w.H - 1):
+        for r0, r1 in _sample_rows(w.N):
+            ref = oracle.sage_attention(qn, kn, vn, lay, False, True, oracle.PV_FP8,
+                                        heads=[(0, h)], rows=(r0, r1), smooth_v=True)
+            exact = oracle.attn_fp64(qn, kn, vn, lay, False, 1 / math.sqrt(w.d), heads=[(0, h)],
+                                     rows=(r0, r1))
+            mask = ~np.isnan(ref)
+            tag = f"video_dit smooth V head {h} rows {r0}:{r1}"
+            assert_vs_oracle(got[mask], ref[mask], tag)
+            assert_vs_fp64(got[mask], exact[mask], True, tag)

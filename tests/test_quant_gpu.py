@@ -127,3 +127,45 @@ def test_quant_qk_ws_matches_allocating_entry():
     with pytest.raises(sage.SageError):
         sage.sage_quant_qk_ws(q, k, got["q_i8"], got["q_scale"], got["k_i8"], got["k_scale"],
                               got["k_mean"], B, H, N, d, True, ws, ws.numel() - 8)
+
+
+def _v_with_offsets(B, H, N, d, seed):
+    w = inputs.Workload("t", seed, B, H, N, d, False, 1.0)
+    _, _, v = inputs.make_dense(w)
+    g = torch.Generator().manual_seed(seed)
+    v = (v.float() + torch.randn(d, generator=g) * 8.0).half()   # channel offsets
+    v[0, 0, :, 1] = 2.5                     # a constant channel: V - mean = 0
+    v[0, -1, :, 2] = 0                      # an all-zero channel
+    v[-1, 0, :, 3] = -v[-1, 0, :, 3].abs() - 1.0   # an all-negative channel
+    return v
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("N", [1, 300])
+def test_quant_v_fp8_smooth_bit_exact(d, N):
+    B, H = 2, 2
+    v = _v_with_offsets(B, H, N, d, 31 + d + N)
+    codes, scales, mean = sage.quant_v_fp8(v.cuda(), smooth_v=True)
+    lay = oracle.Layout.dense(B, H, N, d)
+    rm = oracle.v_mean(v.numpy(), lay)
+    rc, rs = oracle.quant_v_fp8(v.numpy(), lay, mu=rm)
+    assert np.array_equal(_np(mean), rm)
+    assert np.array_equal(_np(scales), rs)
+    assert np.array_equal(_np(codes), rc)
+    assert sage.sage_get_device_status() == 0
+
+
+def test_quant_v_fp8_smooth_varlen_bit_exact():
+    H, d = 3, 128
+    lens = [1, 129, 640, 0, 64]
+    w = inputs.Workload("t", 41, 0, H, 0, d, True, 2.0, nseq=len(lens))
+    _, _, v, cu = inputs.make_varlen(w, lens=lens)
+    v = (v.float() + torch.linspace(-30, 30, d)).half()
+    codes, scales, mean = sage.quant_v_fp8_varlen(v.cuda(), cu.cuda(), max(lens), smooth_v=True)
+    lay = oracle.Layout.packed(cu.tolist(), H, d)
+    rm = oracle.v_mean(v.numpy(), lay)
+    rc, rs = oracle.quant_v_fp8(v.numpy(), lay, mu=rm)
+    assert np.array_equal(_np(mean), rm)
+    assert np.array_equal(_np(scales), rs)
+    assert np.array_equal(_np(codes), rc)
+    assert sage.sage_get_device_status() == 0

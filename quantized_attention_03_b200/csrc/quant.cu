@@ -12,11 +12,11 @@
 //             order) and the max and min of V. Row chunks of 512 tokens, atomics.
 //             amax |fl(V - mean)| = max(fl(max V - mean), fl(mean - min V)) exactly,
 //             because fp32 rounding is monotonic, so V needs no third pass.
-//   quant:    one CTA per 128-token chunk of Q (one Q block), K (two K blocks) or V;
-//             16-byte vector loads/stores, warp-shuffle amax. Codes are the rounding of
-//             the IEEE fp32 quotient x / scale, computed as x * (1 / scale) with an exact
-//             division only where the two could round differently, so they match the
-//             definition bit for bit without a division per element.
+//   quant:    one CTA per 128-token chunk of Q (one Q block), K (two K blocks) or V,
+//             staged in shared memory by bulk copies; warp-shuffle amax. Codes are the
+//             rounding of the IEEE fp32 quotient x / scale, computed as x * (1 / scale)
+//             with an exact division only where the two could round differently, so
+//             they match the definition bit for bit without a division per element.
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
@@ -29,6 +29,7 @@ namespace {
 
 constexpr int kColChunk = 512;   // tokens per colstats CTA
 constexpr int kThreads = 256;
+constexpr uint64_t kWaitNs = 2000000000ull;   // bound on the wait for a chunk's bulk copy
 
 __device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8])
 {
@@ -41,7 +42,8 @@ __device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8])
     }
 }
 
-template <int D>
+// DO_K: fp64 sums of K; DO_V: max and max of -V, plus fp64 sums of V when cs.vsum is set.
+template <int D, bool DO_K, bool DO_V>
 __global__ void __launch_bounds__(kThreads) colstats_kernel(const __half *__restrict__ k,
                                                             const __half *__restrict__ v,
                                                             ColStats cs, SeqLayout L, int *status)
@@ -58,7 +60,8 @@ __global__ void __launch_bounds__(kThreads) colstats_kernel(const __half *__rest
         return;
     const int r_end = min(len, r_begin + kColChunk);
     const int g = threadIdx.x % kGroups, r0 = threadIdx.x / kGroups;
-    const bool do_k = cs.ksum != nullptr, do_v = cs.vhi != nullptr, do_vsum = cs.vsum != nullptr;
+    constexpr bool do_k = DO_K, do_v = DO_V;
+    const bool do_vsum = DO_V && cs.vsum != nullptr;
 
     double ks[8], vs[8];
     float hi[8], ng[8];                          // max V and max -V
@@ -67,25 +70,51 @@ __global__ void __launch_bounds__(kThreads) colstats_kernel(const __half *__rest
         ks[i] = vs[i] = 0.0;
         hi[i] = ng[i] = -INFINITY;
     }
-    for (int r = r_begin + r0; r < r_end; r += kRowsPerPass) {
-        const int64_t off = L.offset(s, start, h, r) + g * 8;
+    auto add_k = [&](const uint4 &u) {
         float f[8];
-        if (do_k) {
-            unpack8(__ldg(reinterpret_cast<const uint4 *>(k + off)), f);
+        unpack8(u, f);
 #pragma unroll
-            for (int i = 0; i < 8; i++)
-                ks[i] += (double)f[i];
-        }
-        if (do_v) {
-            unpack8(__ldg(reinterpret_cast<const uint4 *>(v + off)), f);
+        for (int i = 0; i < 8; i++)
+            ks[i] += (double)f[i];
+    };
+    auto add_v = [&](const uint4 &u) {
+        float f[8];
+        unpack8(u, f);
 #pragma unroll
-            for (int i = 0; i < 8; i++) {
-                hi[i] = fmaxf(hi[i], f[i]);
-                ng[i] = fmaxf(ng[i], -f[i]);
-                if (do_vsum)
-                    vs[i] += (double)f[i];
-            }
+        for (int i = 0; i < 8; i++) {
+            hi[i] = fmaxf(hi[i], f[i]);
+            ng[i] = fmaxf(ng[i], -f[i]);
+            if (do_vsum)
+                vs[i] += (double)f[i];
         }
+    };
+    // four rows per iteration, so that four 16-byte loads per tensor are in flight
+    constexpr int kUnroll = 4;
+    int r = r_begin + r0;
+    for (; r + (kUnroll - 1) * kRowsPerPass < r_end; r += kUnroll * kRowsPerPass) {
+        uint4 uk[kUnroll], uv[kUnroll];
+#pragma unroll
+        for (int j = 0; j < kUnroll; j++) {
+            const int64_t off = L.offset(s, start, h, r + j * kRowsPerPass) + g * 8;
+            if (do_k)
+                uk[j] = __ldg(reinterpret_cast<const uint4 *>(k + off));
+            if (do_v)
+                uv[j] = __ldg(reinterpret_cast<const uint4 *>(v + off));
+        }
+#pragma unroll
+        for (int j = 0; j < kUnroll; j++) {
+            if (do_k)
+                add_k(uk[j]);
+            if (do_v)
+                add_v(uv[j]);
+        }
+    }
+    for (; r < r_end; r += kRowsPerPass) {
+        const int64_t off = L.offset(s, start, h, r) + g * 8;
+        if (do_k)
+            add_k(__ldg(reinterpret_cast<const uint4 *>(k + off)));
+        if (do_v)
+            add_v(__ldg(reinterpret_cast<const uint4 *>(v + off)));
     }
 
     // lanes kGroups apart hold the same columns: fold them, then one row per warp
@@ -133,24 +162,6 @@ __global__ void __launch_bounds__(kThreads) colstats_kernel(const __half *__rest
     }
 }
 
-// Block-wide max over `nthreads` consecutive threads starting at warp `w0`.
-template <int NWARPS>
-__device__ __forceinline__ float group_max(float x, float *s_red, int w0)
-{
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-        x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    if (lane == 0)
-        s_red[warp] = x;
-    __syncthreads();
-    float m = 0.0f;
-#pragma unroll
-    for (int i = 0; i < NWARPS; i++)
-        m = fmaxf(m, s_red[w0 + i]);
-    return m;
-}
-
 constexpr float kRound = 12582912.0f;            // 1.5 * 2^23: adding it rounds to an integer
 constexpr int kRoundBits = 0x4B400000;
 
@@ -172,6 +183,44 @@ __device__ __forceinline__ int8_t int8_code(float x, float s, float r)
     return (int8_t)c;
 }
 
+// The eight codes int8_code(x, s, r) of x[0..3] (pairs), packed little-endian. The
+// product x * r, rounded to an integer by the 1.5 * 2^23 bias, is computed on packed
+// fp32 pairs; the code is the low byte of the biased float's bits (their integer part
+// is 0x4B400000 + code). No clamp is needed: s = fl(amax / 127) and r = fl(1 / s) give
+// |x r| <= 127 (1 + 2^-22) < 127.5. Elements within 2^-15 of a tie are redone with the
+// exact quotient (rare).
+__device__ __forceinline__ uint2 int8_codes8(const float2 (&x)[4], float s, float r)
+{
+    if (s == 0.0f)
+        return make_uint2(0u, 0u);
+    constexpr float kTie = 0.5f - 3.0517578125e-05f;
+    uint32_t bits[8];
+    bool tie = false;
+#pragma unroll
+    for (int j = 0; j < 4; j++) {
+        const float2 t = mul2(x[j], make_float2(r, r));
+        const float2 b = add2(t, make_float2(kRound, kRound));
+        const float2 n = add2(b, make_float2(-kRound, -kRound));
+        const float2 d = fma2(n, make_float2(-1.0f, -1.0f), t);   // t - round(t), exact
+        tie |= (fabsf(d.x) > kTie) | (fabsf(d.y) > kTie);
+        bits[2 * j] = __float_as_uint(b.x);
+        bits[2 * j + 1] = __float_as_uint(b.y);
+    }
+    if (tie) {
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            bits[2 * j] = (uint8_t)int8_code(x[j].x, s, r);
+            bits[2 * j + 1] = (uint8_t)int8_code(x[j].y, s, r);
+        }
+    }
+    uint2 w;
+    w.x = __byte_perm(__byte_perm(bits[0], bits[1], 0x0040), __byte_perm(bits[2], bits[3], 0x0040),
+                      0x5410);
+    w.y = __byte_perm(__byte_perm(bits[4], bits[5], 0x0040), __byte_perm(bits[6], bits[7], 0x0040),
+                      0x5410);
+    return w;
+}
+
 // fl(x / s) for the E4M3 encoder, with r = fl(1 / s): the product x * r differs from the
 // IEEE quotient by at most a few ulps, which changes the E4M3 rounding only next to a
 // rounding midpoint of a normal E4M3 binade (low 20 mantissa bits near 1 << 19) or in the
@@ -186,21 +235,31 @@ __device__ __forceinline__ float e4m3_quotient(float x, float s, float r)
     return q;
 }
 
+// One CTA per 128-token chunk of one (sequence, head): a Q block, a pair of K blocks or
+// a V chunk. The chunk (128 rows x D fp16, 32 KB at D = 128) comes into shared memory
+// with bulk copies (one for the dense layout, one per row for the packed layout) issued
+// at CTA start, so every resident CTA keeps its whole chunk in flight. Thread t then
+// owns the 16-byte column group t % (D/8) of rows t / (D/8) + i (256 / (D/8)), which
+// makes the shared-memory reads conflict-free and fixes the thread's 8 channels.
 template <int D>
-__global__ void __launch_bounds__(kThreads) quant_kernel(
+__global__ void __launch_bounds__(kThreads, 4) quant_kernel(
     const __half *__restrict__ q, const __half *__restrict__ k, const __half *__restrict__ v,
     ColStats cs, int8_t *__restrict__ q_i8, float *__restrict__ q_scale,
     int8_t *__restrict__ k_i8, float *__restrict__ k_scale, float *__restrict__ k_mean,
     uint8_t *__restrict__ v_e4m3, float *__restrict__ v_scale, float *__restrict__ v_mean,
     SeqLayout L, int nqb, int nkb, int part0, int *status)
 {
-    constexpr int kHalf = D / 2;          // elements per thread (two threads per token)
-    constexpr int kVec = kHalf / 8;       // 16-byte loads per thread
-    __shared__ float s_red[8];
-    __shared__ float s_aux[D];            // K mean or V scale per channel
-    __shared__ float s_rcp[D];            // fl(1 / V scale) per channel
-    __shared__ float s_vmu[D];            // V mean per channel (0 without smooth V)
-    const double *ksum = cs.ksum;
+    constexpr int kGpr = D / 8;                      // 16-byte groups per row
+    constexpr int kRowStep = kThreads / kGpr;        // rows between a thread's groups
+    constexpr int kSteps = kQBlock / kRowStep;       // groups per thread
+    constexpr int kHalfSteps = kKBlock / kRowStep;   // those in the first 64-row K block
+    constexpr int kWarps = kThreads / 32;
+    __shared__ __align__(128) uint4 s_x[kQBlock * kGpr];
+    __shared__ __align__(8) uint64_t s_bar;
+    __shared__ float s_red[2][kWarps];
+    __shared__ float s_mu[D];             // K mean or V mean per channel
+    __shared__ float s_sc[D];             // V scale per channel
+    __shared__ float s_rc[D];             // fl(1 / V scale) per channel
 
     const int s = blockIdx.z, h = blockIdx.y;
     int start, len;
@@ -211,9 +270,6 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(
     const int kind = part0 + (int)blockIdx.x / nqb;
     const int chunk = (int)blockIdx.x % nqb;
     const int row0 = chunk * kQBlock;
-    const int row = row0 + threadIdx.x / 2;
-    const int col0 = (threadIdx.x & 1) * kHalf;
-    const bool valid = row < len;
 
     if (row0 >= len) {                    // padding block of a short sequence
         if (kind == 1 && chunk == 0 && threadIdx.x < D)
@@ -235,11 +291,30 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(
         }
         return;
     }
+    const int nrows = min(kQBlock, len - row0);
+    const __half *src = kind == 0 ? q : (kind == 1 ? k : v);
 
+    // ---- the chunk into shared memory
+    if (threadIdx.x == 0) {
+        mbar_init(&s_bar, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        mbar_arrive_expect_tx(&s_bar, (uint32_t)(nrows * D * 2));
+        if (L.cu == nullptr)       // rows of one head are contiguous
+            bulk_load_g2s(s_x, src + L.offset(s, start, h, row0), (uint32_t)(nrows * D * 2),
+                          &s_bar);
+    }
+    if (L.cu != nullptr && (int)threadIdx.x < nrows)
+        bulk_load_g2s(s_x + threadIdx.x * kGpr, src + L.offset(s, start, h, row0 + threadIdx.x),
+                      D * 2, &s_bar);
+
+    // ---- per-channel statistics while the copy is in flight
     if (kind == 1 && threadIdx.x < D) {
         const int c = threadIdx.x;
-        const float mu = ksum ? (float)(ksum[sh * D + c] / (double)len) : 0.0f;
-        s_aux[c] = mu;
+        const float mu = cs.ksum ? (float)(cs.ksum[sh * D + c] / (double)len) : 0.0f;
+        s_mu[c] = mu;
         if (chunk == 0)
             k_mean[sh * D + c] = mu;
     }
@@ -252,102 +327,151 @@ __global__ void __launch_bounds__(kThreads) quant_kernel(
         // the largest |fl(V - mu)|: rounding is monotonic, so it is at max V or min V
         const float amax = fmaxf(__fsub_rn(vmax, mu), __fadd_rn(vnegmax, mu));
         const float sv = __fdiv_rn(amax, 448.0f);
-        s_aux[c] = sv;
-        s_rcp[c] = sv != 0.0f ? __fdiv_rn(1.0f, sv) : 0.0f;
-        s_vmu[c] = mu;
+        s_sc[c] = sv;
+        s_rc[c] = sv != 0.0f ? __fdiv_rn(1.0f, sv) : 0.0f;
+        s_mu[c] = mu;
         if (chunk == 0) {
             v_scale[o] = sv;
             if (v_mean != nullptr)
                 v_mean[o] = mu;
         }
     }
+    if (kind == 0 && threadIdx.x < D)
+        s_mu[threadIdx.x] = 0.0f;
     __syncthreads();
 
-    const int64_t off = L.offset(s, start, h, row) + col0;
-    const __half *src = kind == 0 ? q : (kind == 1 ? k : v);
-    float x[kHalf];
+    const int cg = threadIdx.x % kGpr, r_in = threadIdx.x / kGpr;
+    const int c0 = cg * 8;
+    float mu[8];
 #pragma unroll
-    for (int i = 0; i < kVec; i++) {
-        float f[8];
-        if (valid)
-            unpack8(__ldg(reinterpret_cast<const uint4 *>(src + off) + i), f);
-        else
-#pragma unroll
-            for (int e = 0; e < 8; e++)
-                f[e] = 0.0f;
-#pragma unroll
-        for (int e = 0; e < 8; e++)
-            x[i * 8 + e] = f[e];
-    }
+    for (int e = 0; e < 8; e++)
+        mu[e] = s_mu[c0 + e];
+
+    if (!mbar_wait(&s_bar, 0, nullptr, status, status_bit(SAGE_ERR_TIMEOUT), kWaitNs))
+        return;
 
     if (kind == 2) {
-        // E4M3 codes with the per-channel scale
-        if (!valid)
-            return;
-        uint32_t w[kHalf / 4];
+        float sc[8], rc[8];
 #pragma unroll
-        for (int i = 0; i < kHalf; i += 4) {
-            float qv[4];
-#pragma unroll
-            for (int e = 0; e < 4; e++) {
-                const int c = col0 + i + e;
-                const float sv = s_aux[c];
-                const float xs = __fsub_rn(x[i + e], s_vmu[c]);
-                qv[e] = sv != 0.0f ? e4m3_quotient(xs, sv, s_rcp[c]) : 0.0f;
-            }
-            const uint32_t lo = pack_e4m3x2(qv[0], qv[1]);
-            const uint32_t hi = pack_e4m3x2(qv[2], qv[3]);
-            w[i / 4] = lo | (hi << 16);
+        for (int e = 0; e < 8; e++) {
+            sc[e] = s_sc[c0 + e];
+            rc[e] = s_rc[c0 + e];
         }
-        uint4 *dst = reinterpret_cast<uint4 *>(v_e4m3 + off);
 #pragma unroll
-        for (int i = 0; i < kHalf / 16; i++)
-            dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
+        for (int i = 0; i < kSteps; i++) {
+            const int row = i * kRowStep + r_in;
+            if (row >= nrows)
+                break;
+            float f[8];
+            unpack8(s_x[row * kGpr + cg], f);
+            float qv[8];
+#pragma unroll
+            for (int e = 0; e < 8; e++) {
+                const float xs = __fsub_rn(f[e], mu[e]);
+                qv[e] = sc[e] != 0.0f ? e4m3_quotient(xs, sc[e], rc[e]) : 0.0f;
+            }
+            uint2 w;
+            w.x = (uint32_t)pack_e4m3x2(qv[0], qv[1]) | ((uint32_t)pack_e4m3x2(qv[2], qv[3]) << 16);
+            w.y = (uint32_t)pack_e4m3x2(qv[4], qv[5]) | ((uint32_t)pack_e4m3x2(qv[6], qv[7]) << 16);
+            *reinterpret_cast<uint2 *>(v_e4m3 + L.offset(s, start, h, row0 + row) + c0) = w;
+        }
         return;
     }
 
-    float amax = 0.0f;
-    if (kind == 1) {
+    // ---- Q / K: block amax (K: one per 64-row half), then codes.
+    // Pass 1 keeps per-channel fp16 extrema only: fp32 rounding is monotonic, so the
+    // largest |fl(x - mu)| of a block is max(fl(max x - mu), fl(mu - min x)) over its
+    // channels (Q: mu = 0, i.e. max |x|).
+    const __half2 kNegInf = __halves2half2(__ushort_as_half(0xFC00), __ushort_as_half(0xFC00));
+    const __half2 kPosInf = __halves2half2(__ushort_as_half(0x7C00), __ushort_as_half(0x7C00));
+    __half2 hi[2][4], lo[2][4];
 #pragma unroll
-        for (int i = 0; i < kHalf; i++)
-            x[i] = __fsub_rn(x[i], s_aux[col0 + i]);
-    }
-    if (valid) {
+    for (int b = 0; b < 2; b++)
 #pragma unroll
-        for (int i = 0; i < kHalf; i++)
-            amax = fmaxf(amax, fabsf(x[i]));
+        for (int j = 0; j < 4; j++) {
+            hi[b][j] = kNegInf;
+            lo[b][j] = kPosInf;
+        }
+#pragma unroll
+    for (int i = 0; i < kSteps; i++) {
+        const int row = i * kRowStep + r_in;
+        const int b = i < kHalfSteps ? 0 : 1;
+        if (row < nrows) {
+            const uint4 u = s_x[row * kGpr + cg];
+            const __half2 *x2 = reinterpret_cast<const __half2 *>(&u);
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                hi[b][j] = __hmax2(hi[b][j], x2[j]);
+                lo[b][j] = __hmin2(lo[b][j], x2[j]);
+            }
+        }
     }
-
-    float scale;
+    float am[2] = {0.0f, 0.0f};
+#pragma unroll
+    for (int b = 0; b < 2; b++)
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            const float2 hf = __half22float2(hi[b][j]), lf = __half22float2(lo[b][j]);
+            am[b] = fmaxf(am[b], fmaxf(__fsub_rn(hf.x, mu[2 * j]), __fsub_rn(mu[2 * j], lf.x)));
+            am[b] = fmaxf(am[b],
+                          fmaxf(__fsub_rn(hf.y, mu[2 * j + 1]), __fsub_rn(mu[2 * j + 1], lf.y)));
+        }
+    float a0 = am[0], a1 = am[1];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        a0 = fmaxf(a0, __shfl_xor_sync(0xffffffffu, a0, o));
+        a1 = fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, o));
+    }
+    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+    if (lane == 0) {
+        s_red[0][warp] = a0;
+        s_red[1][warp] = a1;
+    }
+    __syncthreads();
+    float A0 = 0.0f, A1 = 0.0f;
+#pragma unroll
+    for (int w = 0; w < kWarps; w++) {
+        A0 = fmaxf(A0, s_red[0][w]);
+        A1 = fmaxf(A1, s_red[1][w]);
+    }
+    float sc0, sc1;
     if (kind == 0) {
-        scale = __fdiv_rn(group_max<8>(amax, s_red, 0), 127.0f);
+        sc0 = sc1 = __fdiv_rn(fmaxf(A0, A1), 127.0f);
         if (threadIdx.x == 0)
-            q_scale[sh * nqb + chunk] = scale;
+            q_scale[sh * nqb + chunk] = sc0;
     } else {
-        const int half_blk = threadIdx.x / 128;    // 64-token K block within the chunk
-        scale = __fdiv_rn(group_max<4>(amax, s_red, half_blk * 4), 127.0f);
-        const int kb = 2 * chunk + half_blk;
-        if ((threadIdx.x & 127) == 0 && kb < nkb)
-            k_scale[sh * nkb + kb] = scale;
+        sc0 = __fdiv_rn(A0, 127.0f);
+        sc1 = __fdiv_rn(A1, 127.0f);
+        if (threadIdx.x == 0) {
+            if (2 * chunk < nkb)
+                k_scale[sh * nkb + 2 * chunk] = sc0;
+            if (2 * chunk + 1 < nkb)
+                k_scale[sh * nkb + 2 * chunk + 1] = sc1;
+        }
     }
-    if (!valid)
-        return;
-
-    const float rcp = scale != 0.0f ? __fdiv_rn(1.0f, scale) : 0.0f;
-    uint32_t w[kHalf / 4];
+    const float rc0 = sc0 != 0.0f ? __fdiv_rn(1.0f, sc0) : 0.0f;
+    const float rc1 = sc1 != 0.0f ? __fdiv_rn(1.0f, sc1) : 0.0f;
+    float2 nmu[4];                        // -mu (Q: -0, so that x + nmu = x exactly)
 #pragma unroll
-    for (int i = 0; i < kHalf; i += 4) {
-        const uint32_t b0 = (uint8_t)int8_code(x[i], scale, rcp);
-        const uint32_t b1 = (uint8_t)int8_code(x[i + 1], scale, rcp);
-        const uint32_t b2 = (uint8_t)int8_code(x[i + 2], scale, rcp);
-        const uint32_t b3 = (uint8_t)int8_code(x[i + 3], scale, rcp);
-        w[i / 4] = b0 | (b1 << 8) | (b2 << 16) | (b3 << 24);
+    for (int j = 0; j < 4; j++)
+        nmu[j] = make_float2(-mu[2 * j], -mu[2 * j + 1]);
+    int8_t *dst = kind == 0 ? q_i8 : k_i8;
+#pragma unroll
+    for (int i = 0; i < kSteps; i++) {
+        const int row = i * kRowStep + r_in;
+        if (row >= nrows)
+            break;
+        const float scale = i < kHalfSteps ? sc0 : sc1;
+        const float rcp = i < kHalfSteps ? rc0 : rc1;
+        float f[8];
+        unpack8(s_x[row * kGpr + cg], f);
+        float2 x[4];
+#pragma unroll
+        for (int j = 0; j < 4; j++)
+            x[j] = add2(make_float2(f[2 * j], f[2 * j + 1]), nmu[j]);
+        const uint2 w = int8_codes8(x, scale, rcp);
+        *reinterpret_cast<uint2 *>(dst + L.offset(s, start, h, row0 + row) + c0) = w;
     }
-    int8_t *dst8 = (kind == 0 ? q_i8 : k_i8) + off;
-    uint4 *dst = reinterpret_cast<uint4 *>(dst8);
-#pragma unroll
-    for (int i = 0; i < kHalf / 16; i++)
-        dst[i] = make_uint4(w[4 * i], w[4 * i + 1], w[4 * i + 2], w[4 * i + 3]);
 }
 
 }  // namespace
@@ -358,10 +482,22 @@ cudaError_t launch_colstats(const __half *k, const __half *v, const ColStats &cs
     if (cs.ksum == nullptr && cs.vhi == nullptr)
         return cudaSuccess;
     dim3 grid((L.maxlen + kColChunk - 1) / kColChunk, L.H, L.nseq);
-    if (L.d == 128)
-        colstats_kernel<128><<<grid, kThreads, 0, st>>>(k, v, cs, L, status);
-    else
-        colstats_kernel<64><<<grid, kThreads, 0, st>>>(k, v, cs, L, status);
+    const bool dk = cs.ksum != nullptr, dv = cs.vhi != nullptr;
+    if (L.d == 128) {
+        if (dk && dv)
+            colstats_kernel<128, true, true><<<grid, kThreads, 0, st>>>(k, v, cs, L, status);
+        else if (dk)
+            colstats_kernel<128, true, false><<<grid, kThreads, 0, st>>>(k, v, cs, L, status);
+        else
+            colstats_kernel<128, false, true><<<grid, kThreads, 0, st>>>(k, v, cs, L, status);
+    } else {
+        if (dk && dv)
+            colstats_kernel<64, true, true><<<grid, kThreads, 0, st>>>(k, v, cs, L, status);
+        else if (dk)
+            colstats_kernel<64, true, false><<<grid, kThreads, 0, st>>>(k, v, cs, L, status);
+        else
+            colstats_kernel<64, false, true><<<grid, kThreads, 0, st>>>(k, v, cs, L, status);
+    }
     return cudaGetLastError();
 }
 

@@ -349,14 +349,16 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
             };
             // FP16 mode streams each chunk of P to shared memory as it is produced (the
             // P.V wait comes first); FP8 mode, whose P tile is half the size, packs the
-            // whole row in registers and stores it after the wait.
+            // whole row in registers and stores it after the wait. (Streaming FP8 P, with
+            // one buffer or with two, measured slower.)
             constexpr bool kStreamP = !FP8;
             if constexpr (kStreamP) {
                 if (!(ok = await_pv_and_rescale()))
                     break;
             }
-            constexpr int kWords = FP8 ? C::BN / 4 : C::BN / 2;
-            uint32_t pw[kStreamP ? 1 : kWords];
+            constexpr int kWords = FP8 ? C::BN / 4 : 1;
+            uint32_t pw[kWords];
+            const uint32_t pbuf = smem_u32(sP) + i * C::kPBytes;
 
             // p = 2^(S sc - m): S to fp32 exactly through the magic bias
             // (|S| <= 127^2 d < 2^22), one packed FFMA, ex2; each 16-key chunk is packed to
@@ -364,8 +366,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
             // 16-byte chunk c of row r sits at chunk c ^ (r % 8) of the row's 128-byte line.
             auto tile_exp = [&](auto masked) {
                 constexpr bool MASKED = decltype(masked)::value;
-                [[maybe_unused]] const uint32_t prow =
-                    smem_u32(sP) + i * C::kPBytes + row_in_tile * 128;
+                [[maybe_unused]] const uint32_t prow = pbuf + row_in_tile * 128;
                 [[maybe_unused]] const uint32_t sw = row_in_tile & 7;
                 float2 lsum2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
@@ -428,7 +429,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
             if constexpr (!kStreamP) {
                 if (!(ok = await_pv_and_rescale()))
                     break;
-                const uint32_t prow = smem_u32(sP) + i * C::kPBytes + row_in_tile * 128;
+                const uint32_t prow = pbuf + row_in_tile * 128;
                 const uint32_t sw = row_in_tile & 7;
 #pragma unroll
                 for (int c = 0; c < kWords / 4; c++)

@@ -47,9 +47,9 @@ def lib():
         L.oracle_head_channel_mean.argtypes = [P, i64, i64, i32, P]
         L.oracle_head_quant_int8.argtypes = [P, P, i64, i64, i32, i32, P, P]
         L.oracle_head_quant_v_fp8.argtypes = [P, P, i64, i64, i32, P, P]
-        L.oracle_head_attn_quant.argtypes = [P, P, P, P, P, P, P, i64, i64, i32, i32, i32, f64,
-                                             i32, i64, i64, P]
-        L.oracle_head_attn_fp64.argtypes = [P, P, P, i64, i64, i32, i32, f64, i64, i64, P]
+        L.oracle_head_attn_quant.argtypes = [P, P, P, P, P, P, P, i64, i64, i64, i32, i32, i32,
+                                             f64, i32, i64, i64, P]
+        L.oracle_head_attn_fp64.argtypes = [P, P, P, i64, i64, i64, i32, i32, f64, i64, i64, P]
         L.oracle_f16_to_f64.argtypes = [ctypes.c_uint16]
         L.oracle_f16_to_f64.restype = f64
         L.oracle_round_f16.argtypes = [f64]
@@ -169,13 +169,16 @@ def quant_int8(x: np.ndarray, layout: Layout, blk: int, mu: Optional[np.ndarray]
     return codes, scales
 
 
-def quant_qk(q: np.ndarray, k: np.ndarray, layout: Layout, smooth_k: bool = True, heads=None):
+def quant_qk(q: np.ndarray, k: np.ndarray, layout: Layout, smooth_k: bool = True, heads=None,
+             kv_layout: Optional[Layout] = None):
     """Smooth K, then per-block INT8 of Q (128 tokens) and K (64 tokens), for every (or
-    each selected) head."""
-    zeros = np.zeros((layout.nseq, layout.H, layout.d), np.float32)
-    mu = k_mean(k, layout, heads) if smooth_k else zeros
+    each selected) head. ``kv_layout`` places K when it has its own lengths (default:
+    the layout of Q)."""
+    kvl = layout if kv_layout is None else kv_layout
+    zeros = np.zeros((kvl.nseq, kvl.H, kvl.d), np.float32)
+    mu = k_mean(k, kvl, heads) if smooth_k else zeros
     q_i8, q_scale = quant_int8(q, layout, Q_BLOCK, None, heads)
-    k_i8, k_scale = quant_int8(k, layout, K_BLOCK, mu if smooth_k else None, heads)
+    k_i8, k_scale = quant_int8(k, kvl, K_BLOCK, mu if smooth_k else None, heads)
     return dict(q_i8=q_i8, q_scale=q_scale, k_i8=k_i8, k_scale=k_scale, k_mean=mu)
 
 
@@ -196,11 +199,15 @@ def quant_v_fp8(v: np.ndarray, layout: Layout, heads=None, mu: Optional[np.ndarr
 def attn_quant(q_i8, q_scale, k_i8, k_scale, v, v_scale, layout: Layout, causal: bool,
                pv_mode: int, sm_scale: float, tile_n: int = 128, heads=None,
                rows: Optional[Tuple[int, int]] = None,
-               v_mean: Optional[np.ndarray] = None) -> np.ndarray:
+               v_mean: Optional[np.ndarray] = None,
+               kv_layout: Optional[Layout] = None) -> np.ndarray:
     """Quantized attention from codes and scales; fp16 output, NaN where not computed.
 
     ``v`` is fp16 V (FP16 mode) or its E4M3 codes as uint8 (FP8 mode); ``v_mean``
-    [nseq, H, d] (FP8 mode, smooth V) is added to every output row."""
+    [nseq, H, d] (FP8 mode, smooth V) is added to every output row. ``kv_layout`` places
+    K and V when their lengths differ from Q's (causal masks align at the bottom right)."""
+    kvl = layout if kv_layout is None else kv_layout
+    assert kvl.stride == layout.stride and kvl.nseq == layout.nseq
     out = np.full(q_i8.shape, np.nan, np.float16)
     ob = out.view(np.uint16)
     if pv_mode == PV_FP16:
@@ -210,27 +217,31 @@ def attn_quant(q_i8, q_scale, k_i8, k_scale, v, v_scale, layout: Layout, causal:
         assert vv.dtype == np.uint8
     nqb, nkb = q_scale.shape[2], k_scale.shape[2]
     r0, r1 = rows if rows is not None else (0, layout.maxlen)
-    for s, h, off, n in layout.heads(heads):
+    for (s, h, off, n), (_, _, koff, nk) in zip(layout.heads(heads), kvl.heads(heads)):
         sh = s * layout.H + h
         vsp = _ptr(v_scale, sh * layout.d) if v_scale is not None else None
         vmp = _ptr(v_mean, sh * layout.d) if v_mean is not None else None
-        lib().oracle_head_attn_quant(_ptr(q_i8, off), _ptr(q_scale, sh * nqb), _ptr(k_i8, off),
-                                     _ptr(k_scale, sh * nkb), _ptr(vv, off), vsp, vmp, n,
+        lib().oracle_head_attn_quant(_ptr(q_i8, off), _ptr(q_scale, sh * nqb), _ptr(k_i8, koff),
+                                     _ptr(k_scale, sh * nkb), _ptr(vv, koff), vsp, vmp, n, nk,
                                      layout.stride, layout.d, int(causal), int(pv_mode),
                                      float(sm_scale), int(tile_n), r0, r1, _ptr(ob, off))
     return out
 
 
 def attn_fp64(q, k, v, layout: Layout, causal: bool, sm_scale: float, heads=None,
-              rows: Optional[Tuple[int, int]] = None) -> np.ndarray:
-    """Exact attention in fp64 (inputs of any float dtype, upcast exactly)."""
+              rows: Optional[Tuple[int, int]] = None,
+              kv_layout: Optional[Layout] = None) -> np.ndarray:
+    """Exact attention in fp64 (inputs of any float dtype, upcast exactly); ``kv_layout``
+    as in attn_quant."""
+    kvl = layout if kv_layout is None else kv_layout
+    assert kvl.stride == layout.stride and kvl.nseq == layout.nseq
     q64 = np.ascontiguousarray(q, np.float64)
     k64 = np.ascontiguousarray(k, np.float64)
     v64 = np.ascontiguousarray(v, np.float64)
     out = np.full(q64.shape, np.nan, np.float64)
     r0, r1 = rows if rows is not None else (0, layout.maxlen)
-    for s, h, off, n in layout.heads(heads):
-        lib().oracle_head_attn_fp64(_ptr(q64, off), _ptr(k64, off), _ptr(v64, off), n,
+    for (s, h, off, n), (_, _, koff, nk) in zip(layout.heads(heads), kvl.heads(heads)):
+        lib().oracle_head_attn_fp64(_ptr(q64, off), _ptr(k64, koff), _ptr(v64, koff), n, nk,
                                     layout.stride, layout.d, int(causal), float(sm_scale),
                                     r0, r1, _ptr(out, off))
     return out
@@ -243,17 +254,19 @@ def default_sm_scale(d: int, sm_scale: Optional[float] = None) -> float:
 def sage_attention(q, k, v, layout: Layout, causal: bool = False, smooth_k: bool = True,
                    pv_mode: int = PV_FP16, sm_scale: Optional[float] = None,
                    tile_n: int = 128, heads=None, rows=None,
-                   smooth_v: bool = False) -> np.ndarray:
+                   smooth_v: bool = False, kv_layout: Optional[Layout] = None) -> np.ndarray:
     """The whole method from fp16 Q, K, V: smooth K (and, in FP8 mode, optionally V),
-    quantize, quantized attention."""
+    quantize, quantized attention. ``kv_layout`` places K and V when their lengths differ
+    from Q's."""
     if smooth_v and pv_mode != PV_FP8:
         raise ValueError("smooth V applies to the FP8 P.V mode")
+    kvl = layout if kv_layout is None else kv_layout
     sm = default_sm_scale(layout.d, sm_scale)
-    z = quant_qk(q, k, layout, smooth_k, heads)
+    z = quant_qk(q, k, layout, smooth_k, heads, kvl)
     if pv_mode == PV_FP8:
-        vm = channel_mean(v, layout, heads) if smooth_v else None
-        v8, vs = quant_v_fp8(v, layout, heads, vm)
+        vm = channel_mean(v, kvl, heads) if smooth_v else None
+        v8, vs = quant_v_fp8(v, kvl, heads, vm)
         return attn_quant(z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], v8, vs, layout,
-                          causal, PV_FP8, sm, tile_n, heads, rows, vm)
+                          causal, PV_FP8, sm, tile_n, heads, rows, vm, kvl)
     return attn_quant(z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], v, None, layout,
-                      causal, PV_FP16, sm, tile_n, heads, rows)
+                      causal, PV_FP16, sm, tile_n, heads, rows, None, kvl)

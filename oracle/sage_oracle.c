@@ -245,11 +245,15 @@ void oracle_head_quant_v_fp8(const uint16_t *V, const float *mu, int64_t n, int6
 enum { ORACLE_PV_FP16 = 0, ORACLE_PV_FP8 = 1 };
 
 /*
- * Quantized attention for query rows [r0, r1) of one head of length n, following the
- * method's steps in order:
+ * Quantized attention for query rows [r0, r1) of one head with nq queries and nk keys
+ * (nq = nk for self-attention; nq < nk for queries that are the last nq positions of a
+ * longer sequence, e.g. prefill against cached keys), following the method's steps in
+ * order:
  *   S_int[i,j] = sum_c q[i,c] k[j,c] in integers (INT32 range is never exceeded);
  *   t[i,j] = S_int * sq[i/128] * sk[j/64] * sm_scale * log2(e)  (base-2 logits);
- *   causal: j > i is masked out;
+ *   causal: key j is visible to query i when j <= i + (nk - nq) (the mask aligned at
+ *   the bottom-right corner; the square mask j <= i when nq = nk); a query that sees no
+ *   key (only when nq > nk) gets a zero output row;
  *   online softmax over KV tiles [j0, j0+tile_n) in ascending order, all in fp64:
  *     m' = max(m, max_j t), alpha = 2^(m - m') (0 when m = -inf),
  *     p_j = 2^(t_j - m'),  l = alpha l + sum p_j,
@@ -262,18 +266,28 @@ enum { ORACLE_PV_FP16 = 0, ORACLE_PV_FP8 = 1 };
  */
 void oracle_head_attn_quant(const int8_t *qc, const float *qs, const int8_t *kc,
                             const float *ks, const void *v, const float *vs, const float *vm,
-                            int64_t n, int64_t stride, int d, int causal, int pv_mode,
-                            double sm_scale, int tile_n, int64_t r0, int64_t r1, uint16_t *out)
+                            int64_t nq, int64_t nk, int64_t stride, int d, int causal,
+                            int pv_mode, double sm_scale, int tile_n, int64_t r0, int64_t r1,
+                            uint16_t *out)
 {
     const double log2e = 1.4426950408889634073599246810019;   /* 1/ln 2 */
-    if (r1 > n)
-        r1 = n;
+    if (r1 > nq)
+        r1 = nq;
 #pragma omp parallel for schedule(dynamic, 4)
     for (int64_t i = r0; i < r1; i++) {
         double *O = (double *)calloc((size_t)d, sizeof(double));
         double *t = (double *)malloc((size_t)tile_n * sizeof(double));
         double m = -INFINITY, l = 0.0;
-        int64_t jend = causal ? i + 1 : n;               /* keys j < jend are visible */
+        int64_t jend = causal ? i + 1 + (nk - nq) : nk;  /* keys j < jend are visible */
+        if (jend > nk)
+            jend = nk;
+        if (jend <= 0) {                                  /* no visible key: zero row */
+            for (int c = 0; c < d; c++)
+                out[i * stride + c] = 0;
+            free(O);
+            free(t);
+            continue;
+        }
         for (int64_t j0 = 0; j0 < jend; j0 += tile_n) {
             int64_t j1 = j0 + tile_n < jend ? j0 + tile_n : jend;
             double tmax = -INFINITY;
@@ -321,19 +335,28 @@ void oracle_head_attn_quant(const int8_t *qc, const float *qs, const int8_t *kc,
 /* ---------------------------------------------------------------- exact attention */
 
 /*
- * O = softmax(sm_scale Q K^T + causal mask) V for rows [r0, r1) of one head, all in
- * fp64 (two passes: row max, then normalized weights). Inputs are fp64 so the smoothing
- * invariant can be checked with K - mean(K) exactly. Output at out[i*stride + c].
+ * O = softmax(sm_scale Q K^T + causal mask) V for rows [r0, r1) of one head with nq
+ * queries and nk keys, all in fp64 (two passes: row max, then normalized weights); the
+ * causal mask is the bottom-right one of oracle_head_attn_quant, and a query with no
+ * visible key gets a zero row. Inputs are fp64 so the smoothing invariant can be
+ * checked with K - mean(K) exactly. Output at out[i*stride + c].
  */
-void oracle_head_attn_fp64(const double *Q, const double *K, const double *V, int64_t n,
-                           int64_t stride, int d, int causal, double sm_scale, int64_t r0,
-                           int64_t r1, double *out)
+void oracle_head_attn_fp64(const double *Q, const double *K, const double *V, int64_t nq,
+                           int64_t nk, int64_t stride, int d, int causal, double sm_scale,
+                           int64_t r0, int64_t r1, double *out)
 {
-    if (r1 > n)
-        r1 = n;
+    if (r1 > nq)
+        r1 = nq;
 #pragma omp parallel for schedule(dynamic, 4)
     for (int64_t i = r0; i < r1; i++) {
-        int64_t jend = causal ? i + 1 : n;
+        int64_t jend = causal ? i + 1 + (nk - nq) : nk;
+        if (jend > nk)
+            jend = nk;
+        if (jend <= 0) {
+            for (int c = 0; c < d; c++)
+                out[i * stride + c] = 0.0;
+            continue;
+        }
         double *s = (double *)malloc((size_t)jend * sizeof(double));
         double mx = -INFINITY;
         for (int64_t j = 0; j < jend; j++) {

@@ -307,3 +307,113 @@ def test_smooth_v_rejected_in_fp16_mode():
     with pytest.raises(ValueError):
         oracle.sage_attention(x, x, x, Layout.dense(1, 1, 4, d), False, True, PV_FP16, 0.25,
                               smooth_v=True)
+
+
+# Queries that are the last Nq positions of a longer sequence (Nq != Nk: prefill against
+# cached keys, or decode with Nq = 1): the causal mask aligns at the bottom right, query i
+# sees keys j <= i + Nk - Nq.
+
+def _bottom_right_mask(nq, nk):
+    i = np.arange(nq)[:, None]
+    j = np.arange(nk)[None, :]
+    return j <= i + (nk - nq)
+
+
+@pytest.mark.parametrize("nq,nk", [(70, 200), (1, 130), (128, 128), (200, 70)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_fp64_kv_matches_torch_sdpa_with_mask(nq, nk, causal):
+    B, H, d = 1, 2, 16
+    q = _rand16((B, H, nq, d), 151)
+    k, v = _rand16((B, H, nk, d), 152), _rand16((B, H, nk, d), 153)
+    sm = 1 / math.sqrt(d)
+    got = oracle.attn_fp64(q, k, v, Layout.dense(B, H, nq, d), causal, sm,
+                           kv_layout=Layout.dense(B, H, nk, d))
+    mask = torch.from_numpy(_bottom_right_mask(nq, nk)) if causal else None
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        *(torch.from_numpy(x.astype(np.float64)) for x in (q, k, v)), attn_mask=mask, scale=sm)
+    ref = ref.numpy()
+    if causal and nq > nk:        # rows without a visible key: zero here, NaN in torch
+        dead = ~_bottom_right_mask(nq, nk).any(axis=1)
+        assert dead.sum() == nq - nk
+        assert np.all(got[:, :, dead] == 0)
+        got, ref = got[:, :, ~dead], ref[:, :, ~dead]
+    assert np.allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_kv_rows_are_the_tail_of_the_square_problem():
+    # the last Nq queries of a causal square problem see exactly the keys the Nq x Nk
+    # problem gives them: fp64 rows agree bit for bit
+    N, nq, d = 300, 90, 32
+    q, k, v = (_rand16((1, 1, N, d), s) for s in (161, 162, 163))
+    sm = 1 / math.sqrt(d)
+    full = oracle.attn_fp64(q, k, v, Layout.dense(1, 1, N, d), True, sm)
+    tail = oracle.attn_fp64(np.ascontiguousarray(q[:, :, N - nq:]), k, v,
+                            Layout.dense(1, 1, nq, d), True, sm,
+                            kv_layout=Layout.dense(1, 1, N, d))
+    assert np.array_equal(tail, full[:, :, N - nq:])
+
+
+@pytest.mark.parametrize("pv_mode", [PV_FP16, PV_FP8])
+def test_quantized_kv_decode_and_equal_lengths(pv_mode):
+    d, nk = 64, 700
+    k, v = _rand16((1, 2, nk, d), 171), _rand16((1, 2, nk, d), 172)
+    kvl = Layout.dense(1, 2, nk, d)
+    # decode: one query sees every key, so causal and non-causal agree exactly
+    q1 = _rand16((1, 2, 1, d), 173)
+    l1 = Layout.dense(1, 2, 1, d)
+    a = oracle.sage_attention(q1, k, v, l1, True, True, pv_mode, kv_layout=kvl)
+    b = oracle.sage_attention(q1, k, v, l1, False, True, pv_mode, kv_layout=kvl)
+    assert np.array_equal(a, b)
+    exact = oracle.attn_fp64(q1, k, v, l1, False, 1 / math.sqrt(d), kv_layout=kvl)
+    assert _cos(a, exact) > (0.9999 if pv_mode == PV_FP16 else 0.999)
+    # Nq = Nk through the separate layout is the self-attention path, bit for bit
+    q = _rand16((1, 2, nk, d), 174)
+    same = oracle.sage_attention(q, k, v, kvl, True, True, pv_mode, kv_layout=kvl)
+    base = oracle.sage_attention(q, k, v, kvl, True, True, pv_mode)
+    assert np.array_equal(same, base)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_quantized_kv_tracks_fp64(causal):
+    nq, nk, d = 200, 900, 64
+    q = _rand16((1, 2, nq, d), 181)
+    k = (_rand16((1, 2, nk, d), 182).astype(np.float32) + _rand16((d,), 183, 2.0)).astype(np.float16)
+    v = _rand16((1, 2, nk, d), 184)
+    lq, lk = Layout.dense(1, 2, nq, d), Layout.dense(1, 2, nk, d)
+    sm = 1 / math.sqrt(d)
+    o = oracle.sage_attention(q, k, v, lq, causal, True, PV_FP16, sm, kv_layout=lk)
+    exact = oracle.attn_fp64(q, k, v, lq, causal, sm, kv_layout=lk)
+    assert _cos(o, exact) > 0.9999 and _rel_l1(o, exact) < 0.02
+    # the K mean is taken over the keys, not the queries: using Q's length for it fails
+    zq = oracle.quant_qk(q, k, lq, True, kv_layout=lk)
+    mu = k.astype(np.float64).mean(axis=2).astype(np.float32)
+    assert np.array_equal(zq["k_mean"], mu)
+
+
+def test_quantized_kv_more_queries_than_keys():
+    nq, nk, d = 300, 100, 32
+    q = _rand16((1, 1, nq, d), 191)
+    k, v = _rand16((1, 1, nk, d), 192), _rand16((1, 1, nk, d), 193)
+    lq, lk = Layout.dense(1, 1, nq, d), Layout.dense(1, 1, nk, d)
+    o = oracle.sage_attention(q, k, v, lq, True, True, PV_FP16, 0.2, kv_layout=lk)
+    assert np.all(o[0, 0, :nq - nk] == 0)                 # no visible key
+    exact = oracle.attn_fp64(q, k, v, lq, True, 0.2, kv_layout=lk)
+    assert _cos(o[0, 0, nq - nk:], exact[0, 0, nq - nk:]) > 0.9999
+
+
+def test_varlen_kv_equals_per_sequence_dense():
+    H, d = 2, 32
+    lq, lk = [70, 1, 129], [200, 333, 129]
+    cq = np.concatenate([[0], np.cumsum(lq)])
+    ck = np.concatenate([[0], np.cumsum(lk)])
+    q = _rand16((int(cq[-1]), H, d), 201)
+    k, v = _rand16((int(ck[-1]), H, d), 202), _rand16((int(ck[-1]), H, d), 203)
+    o = oracle.sage_attention(q, k, v, Layout.packed(cq, H, d), True, True, PV_FP16, 0.2,
+                              kv_layout=Layout.packed(ck, H, d))
+    for s in range(3):
+        sq, sk = slice(cq[s], cq[s + 1]), slice(ck[s], ck[s + 1])
+        dq = np.ascontiguousarray(q[sq].transpose(1, 0, 2))[None]
+        dk, dv = (np.ascontiguousarray(x[sk].transpose(1, 0, 2))[None] for x in (k, v))
+        od = oracle.sage_attention(dq, dk, dv, Layout.dense(1, H, lq[s], d), True, True,
+                                   PV_FP16, 0.2, kv_layout=Layout.dense(1, H, lk[s], d))
+        assert np.array_equal(o[sq].transpose(1, 0, 2), od[0])

@@ -92,6 +92,11 @@ typedef struct CUstream_st *sage_stream_t;
 SAGE_API size_t sage_workspace_size(int nseq, int H, int max_seqlen, int total_tokens, int d,
                            int pv_mode);
 
+/* sage_workspace_size for queries and keys of different lengths (the *_kv entry points):
+ * max_seqlen_q / total_q for Q and the output, max_seqlen_k / total_k for K and V. */
+SAGE_API size_t sage_workspace_size_kv(int nseq, int H, int max_seqlen_q, int max_seqlen_k,
+                                       int total_q, int total_k, int d, int pv_mode);
+
 /*
  * Steps 1-2 on their own (dense): k_mean[b,h,c] = mean over tokens of K[b,h,:,c]
  * (zeros when smooth_k == 0), q_i8/q_scale = per-128-token INT8 of Q, k_i8/k_scale =
@@ -118,6 +123,14 @@ SAGE_API sage_status_t sage_quant_qk_varlen(const void *q, const void *k, const 
                                    int nseq, int total_tokens, int max_seqlen, int H, int d,
                                    int8_t *q_i8, float *q_scale, int8_t *k_i8, float *k_scale,
                                    float *k_mean, int smooth_k, sage_stream_t stream);
+
+/* sage_quant_qk for Q [B,H,Nq,d] and K [B,H,Nk,d] of different lengths: q_scale is
+ * [B,H,ceil(Nq/128)], k_scale [B,H,ceil(Nk/64)], and the K mean is taken over the Nk
+ * keys. */
+SAGE_API sage_status_t sage_quant_qk_kv(const void *q, const void *k, int8_t *q_i8,
+                                        float *q_scale, int8_t *k_i8, float *k_scale,
+                                        float *k_mean, int B, int H, int Nq, int Nk, int d,
+                                        int smooth_k, sage_stream_t stream);
 
 /*
  * V to FP8 E4M3 (「4比特量化三倍加速不掉点！清华即插即用的SageAttention迎来升级」, 技术方案 (4)) with one fp32 scale per
@@ -176,6 +189,37 @@ SAGE_API sage_status_t sage_attn_varlen_fwd(const void *q, const void *k, const 
                                    size_t ws_bytes, sage_stream_t stream);
 
 /*
+ * Queries and keys of different lengths (dense): q and out are [B,H,Nq,d], k and v are
+ * [B,H,Nk,d], e.g. the last Nq tokens of a sequence attending to all Nk = past + Nq of
+ * its keys (prefill against cached keys; Nq = 1 is a decode step). With causal, query i
+ * sees keys j <= i + (Nk - Nq): the mask is aligned at the bottom-right corner and is
+ * the square mask when Nq = Nk. A query that sees no key (only if Nq > Nk) gets a zero
+ * output row, and Nk = 0 gives a zero output. workspace may be NULL (stream-ordered
+ * allocation) or caller scratch of sage_workspace_size_kv(B, H, Nq, Nk, B*Nq, B*Nk, d,
+ * pv_mode) bytes, 256-byte aligned. The pages only recommend the causal mode for the
+ * decoding stage of language models (「如何将SageAttention量化注意力机制集成到你的AI项目中获得2-5倍速度提升」, section
+ * 语言模型推理加速); queries fewer than keys and the bottom-right alignment are the
+ * usual reading of that use.
+ */
+SAGE_API sage_status_t sage_attn_fwd_kv(const void *q, const void *k, const void *v, void *out,
+                                        int B, int H, int Nq, int Nk, int d, int causal,
+                                        int smooth_k, int pv_mode, float sm_scale,
+                                        void *workspace, size_t ws_bytes, sage_stream_t stream);
+
+/* sage_attn_fwd_kv on packed sequences: q/out [total_q,H,d] with cu_seqlens_q, k/v
+ * [total_k,H,d] with cu_seqlens_k (both int32 [nseq+1] on the device); sequence s has
+ * cu_seqlens_q[s+1]-cu_seqlens_q[s] queries and cu_seqlens_k[s+1]-cu_seqlens_k[s] keys,
+ * bounded by max_seqlen_q and max_seqlen_k. */
+SAGE_API sage_status_t sage_attn_varlen_fwd_kv(const void *q, const void *k, const void *v,
+                                               void *out, const int32_t *cu_seqlens_q,
+                                               const int32_t *cu_seqlens_k, int nseq,
+                                               int total_q, int total_k, int max_seqlen_q,
+                                               int max_seqlen_k, int H, int d, int causal,
+                                               int smooth_k, int pv_mode, float sm_scale,
+                                               void *workspace, size_t ws_bytes,
+                                               sage_stream_t stream);
+
+/*
  * Step 3 alone on pre-quantized operands (dense): q_i8/q_scale and k_i8/k_scale as
  * produced by sage_quant_qk; v is fp16 V (SAGE_PV_FP16, v_scale ignored) or E4M3 codes
  * with per-channel v_scale (SAGE_PV_FP8). Allocates nothing.
@@ -196,6 +240,16 @@ SAGE_API sage_status_t sage_attn_fwd_quantized_smooth_v(const int8_t *q_i8, cons
                                                         void *out, int B, int H, int N, int d,
                                                         int causal, float sm_scale,
                                                         sage_stream_t stream);
+
+/* Step 3 alone with Nq queries and Nk keys (codes and scales from sage_quant_qk_kv; V
+ * codes from sage_quant_v_fp8[_smooth] with N = Nk); v_mean selects the smooth-V
+ * epilogue (FP8 only) or is NULL. */
+SAGE_API sage_status_t sage_attn_fwd_quantized_kv(const int8_t *q_i8, const float *q_scale,
+                                                  const int8_t *k_i8, const float *k_scale,
+                                                  const void *v, const float *v_scale,
+                                                  const float *v_mean, void *out, int B, int H,
+                                                  int Nq, int Nk, int d, int causal, int pv_mode,
+                                                  float sm_scale, sage_stream_t stream);
 
 /*
  * Debug: the integer score tiles S = q_i8 k_i8^T (int32, [B,H,N,N]) exactly as the

@@ -45,6 +45,13 @@ _Z = ctypes.c_size_t
 _S = ctypes.c_int  # sage_status_t
 SIGNATURES = {
     "sage_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
+    "sage_workspace_size_kv": (_Z, [_I, _I, _I, _I, _I, _I, _I, _I]),
+    "sage_quant_qk_kv": (_S, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
+    "sage_attn_fwd_kv": (_S, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
+    "sage_attn_varlen_fwd_kv": (_S, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I,
+                                     _I, _F, _P, _Z, _P]),
+    "sage_attn_fwd_quantized_kv": (_S, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
+                                        _I, _F, _P]),
     "sage_quant_qk": (_S, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "sage_quant_qk_ws": (_S, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]),
     "sage_quant_qk_varlen": (_S, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _I, _P]),
@@ -129,6 +136,41 @@ def _call(name: str, *args):
 
 def sage_workspace_size(nseq, H, max_seqlen, total_tokens, d, pv_mode) -> int:
     return int(lib().sage_workspace_size(nseq, H, max_seqlen, total_tokens, d, pv_mode))
+
+
+def sage_workspace_size_kv(nseq, H, max_seqlen_q, max_seqlen_k, total_q, total_k, d,
+                           pv_mode) -> int:
+    return int(lib().sage_workspace_size_kv(nseq, H, max_seqlen_q, max_seqlen_k, total_q, total_k,
+                                            d, pv_mode))
+
+
+def sage_quant_qk_kv(q, k, q_i8, q_scale, k_i8, k_scale, k_mean, B, H, Nq, Nk, d, smooth_k,
+                     stream=None):
+    return _call("sage_quant_qk_kv", _ptr(q), _ptr(k), _ptr(q_i8), _ptr(q_scale), _ptr(k_i8),
+                 _ptr(k_scale), _ptr(k_mean), B, H, Nq, Nk, d, int(smooth_k), _stream(stream))
+
+
+def sage_attn_fwd_kv(q, k, v, out, B, H, Nq, Nk, d, causal, smooth_k, pv_mode, sm_scale,
+                     workspace=None, ws_bytes=0, stream=None):
+    return _call("sage_attn_fwd_kv", _ptr(q), _ptr(k), _ptr(v), _ptr(out), B, H, Nq, Nk, d,
+                 int(causal), int(smooth_k), int(pv_mode), float(sm_scale), _ptr(workspace),
+                 int(ws_bytes), _stream(stream))
+
+
+def sage_attn_varlen_fwd_kv(q, k, v, out, cu_seqlens_q, cu_seqlens_k, nseq, total_q, total_k,
+                            max_seqlen_q, max_seqlen_k, H, d, causal, smooth_k, pv_mode, sm_scale,
+                            workspace=None, ws_bytes=0, stream=None):
+    return _call("sage_attn_varlen_fwd_kv", _ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                 _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), nseq, total_q, total_k, max_seqlen_q,
+                 max_seqlen_k, H, d, int(causal), int(smooth_k), int(pv_mode), float(sm_scale),
+                 _ptr(workspace), int(ws_bytes), _stream(stream))
+
+
+def sage_attn_fwd_quantized_kv(q_i8, q_scale, k_i8, k_scale, v, v_scale, v_mean, out, B, H, Nq,
+                               Nk, d, causal, pv_mode, sm_scale, stream=None):
+    return _call("sage_attn_fwd_quantized_kv", _ptr(q_i8), _ptr(q_scale), _ptr(k_i8),
+                 _ptr(k_scale), _ptr(v), _ptr(v_scale), _ptr(v_mean), _ptr(out), B, H, Nq, Nk, d,
+                 int(causal), int(pv_mode), float(sm_scale), _stream(stream))
 
 
 def sage_quant_qk(q, k, q_i8, q_scale, k_i8, k_scale, k_mean, B, H, N, d, smooth_k, stream=None):
@@ -254,13 +296,36 @@ def _smooth_flags(smooth_k: bool, smooth_v: bool) -> int:
 
 def sageattn(q, k, v, causal: bool = False, smooth_k: bool = True, pv_mode: int = SAGE_PV_FP16,
              sm_scale: float = 0.0, out=None, stream=None, smooth_v: bool = False):
-    """O = SageAttention(q, k, v) for fp16 CUDA tensors [B, H, N, d]."""
+    """O = SageAttention(q, k, v) for fp16 CUDA tensors q [B, H, Nq, d], k and v
+    [B, H, Nk, d] (Nq != Nk: sage_attn_fwd_kv, causal mask aligned at the bottom right)."""
     import torch
-    B, H, N, d = q.shape
+    B, H, Nq, d = q.shape
+    Nk = k.shape[2]
     if out is None:
         out = torch.empty_like(q)
-    sage_attn_fwd(q, k, v, out, B, H, N, d, causal, _smooth_flags(smooth_k, smooth_v), pv_mode,
-                  sm_scale, stream)
+    flags = _smooth_flags(smooth_k, smooth_v)
+    if Nq == Nk:
+        sage_attn_fwd(q, k, v, out, B, H, Nq, d, causal, flags, pv_mode, sm_scale, stream)
+    else:
+        sage_attn_fwd_kv(q, k, v, out, B, H, Nq, Nk, d, causal, flags, pv_mode, sm_scale, None, 0,
+                         stream)
+    return out
+
+
+def sageattn_varlen_kv(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
+                       causal: bool = False, smooth_k: bool = True,
+                       pv_mode: int = SAGE_PV_FP16, sm_scale: float = 0.0, out=None,
+                       stream=None, smooth_v: bool = False):
+    """Packed sequences with their own query and key lengths: q [Tq, H, d], k and v
+    [Tk, H, d], cu_seqlens_q / cu_seqlens_k int32 [nseq+1] on the device."""
+    import torch
+    Tq, H, d = q.shape
+    Tk = k.shape[0]
+    if out is None:
+        out = torch.empty_like(q)
+    sage_attn_varlen_fwd_kv(q, k, v, out, cu_seqlens_q, cu_seqlens_k, cu_seqlens_q.numel() - 1,
+                            Tq, Tk, max_seqlen_q, max_seqlen_k, H, d, causal,
+                            _smooth_flags(smooth_k, smooth_v), pv_mode, sm_scale, None, 0, stream)
     return out
 
 
@@ -279,17 +344,23 @@ def sageattn_varlen(q, k, v, cu_seqlens, max_seqlen: int, causal: bool = False,
 
 
 def quant_qk(q, k, smooth_k: bool = True, stream=None):
-    """Dense smooth-K + per-block INT8: dict of q_i8, q_scale, k_i8, k_scale, k_mean."""
+    """Dense smooth-K + per-block INT8: dict of q_i8, q_scale, k_i8, k_scale, k_mean
+    (q [B,H,Nq,d] and k [B,H,Nk,d] may differ in length)."""
     import torch
     B, H, N, d = q.shape
+    Nk = k.shape[2]
     dev = q.device
     z = dict(q_i8=torch.empty(q.shape, dtype=torch.int8, device=dev),
              q_scale=torch.empty((B, H, math.ceil(N / Q_BLOCK)), dtype=torch.float32, device=dev),
              k_i8=torch.empty(k.shape, dtype=torch.int8, device=dev),
-             k_scale=torch.empty((B, H, math.ceil(N / K_BLOCK)), dtype=torch.float32, device=dev),
+             k_scale=torch.empty((B, H, math.ceil(Nk / K_BLOCK)), dtype=torch.float32, device=dev),
              k_mean=torch.empty((B, H, d), dtype=torch.float32, device=dev))
-    sage_quant_qk(q, k, z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], z["k_mean"], B, H, N, d,
-                  smooth_k, stream)
+    if N == Nk:
+        sage_quant_qk(q, k, z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], z["k_mean"], B, H, N,
+                      d, smooth_k, stream)
+    else:
+        sage_quant_qk_kv(q, k, z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], z["k_mean"], B,
+                         H, N, Nk, d, smooth_k, stream)
     return z
 
 
@@ -346,8 +417,13 @@ def attn_quantized(q_i8, q_scale, k_i8, k_scale, v, v_scale, causal: bool = Fals
     """Step 3 on pre-quantized operands; v_mean (FP8 mode) selects the smooth-V epilogue."""
     import torch
     B, H, N, d = q_i8.shape
+    Nk = k_i8.shape[2]
     if out is None:
         out = torch.empty(q_i8.shape, dtype=torch.float16, device=q_i8.device)
+    if Nk != N:
+        sage_attn_fwd_quantized_kv(q_i8, q_scale, k_i8, k_scale, v, v_scale, v_mean, out, B, H, N,
+                                   Nk, d, causal, pv_mode, sm_scale, stream)
+        return out
     if v_mean is not None:
         if pv_mode != SAGE_PV_FP8:
             raise ValueError("v_mean needs the FP8 P.V mode")

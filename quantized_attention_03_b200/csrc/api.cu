@@ -66,11 +66,13 @@ struct Workspace {
     size_t total = 0;
 };
 
-Workspace carve(char *base, int nseq, int H, int maxlen, int total_tokens, int d, int pv_mode)
+// Queries: max_q / total_q tokens per (sequence) / in all; keys and values: max_k / total_k.
+Workspace carve(char *base, int nseq, int H, int max_q, int max_k, int total_q, int total_k,
+                int d, int pv_mode)
 {
     Workspace w;
-    const size_t codes = (size_t)total_tokens * H * d;
-    const size_t nqb = (maxlen + kQBlock - 1) / kQBlock, nkb = (maxlen + kKBlock - 1) / kKBlock;
+    const size_t qcodes = (size_t)total_q * H * d, kcodes = (size_t)total_k * H * d;
+    const size_t nqb = (max_q + kQBlock - 1) / kQBlock, nkb = (max_k + kKBlock - 1) / kKBlock;
     const size_t heads = (size_t)nseq * H;
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -78,8 +80,8 @@ Workspace carve(char *base, int nseq, int H, int maxlen, int total_tokens, int d
         off += align256(bytes);
         return p;
     };
-    w.q_i8 = reinterpret_cast<int8_t *>(take(codes));
-    w.k_i8 = reinterpret_cast<int8_t *>(take(codes));
+    w.q_i8 = reinterpret_cast<int8_t *>(take(qcodes));
+    w.k_i8 = reinterpret_cast<int8_t *>(take(kcodes));
     w.q_scale = reinterpret_cast<float *>(take(heads * nqb * 4));
     w.k_scale = reinterpret_cast<float *>(take(heads * nkb * 4));
     w.k_mean = reinterpret_cast<float *>(take(heads * d * 4));
@@ -90,7 +92,7 @@ Workspace carve(char *base, int nseq, int H, int maxlen, int total_tokens, int d
         w.cs.vhi = reinterpret_cast<uint32_t *>(take(heads * d * 4));
         w.cs.vneg = reinterpret_cast<uint32_t *>(take(heads * d * 4));
         w.stats_bytes = off - stats0;
-        w.v8 = reinterpret_cast<uint8_t *>(take(codes));
+        w.v8 = reinterpret_cast<uint8_t *>(take(kcodes));
         w.v_scale = reinterpret_cast<float *>(take(heads * d * 4));
         w.v_mean = reinterpret_cast<float *>(take(heads * d * 4));
     } else {
@@ -127,15 +129,16 @@ float resolve_scale(float sm_scale, int d)
 }
 
 // Steps 1-3 with the given scratch; q/k/v/out and the smoothing flags already validated.
+// Queries in layout L, keys and values in LK (the same layout for self-attention).
 sage_status_t forward(const void *q, const void *k, const void *v, void *out, const SeqLayout &L,
-                      int causal, int smooth, int pv_mode, float sm_scale, char *ws,
-                      cudaStream_t st)
+                      const SeqLayout &LK, int causal, int smooth, int pv_mode, float sm_scale,
+                      char *ws, cudaStream_t st)
 {
     sage_status_t err;
     int *status = status_ptr(&err);
     if (!status)
         return err;
-    Workspace w = carve(ws, L.nseq, L.H, L.maxlen, L.total, L.d, pv_mode);
+    Workspace w = carve(ws, L.nseq, L.H, L.maxlen, LK.maxlen, L.total, LK.total, L.d, pv_mode);
     const bool fp8 = pv_mode == SAGE_PV_FP8;
     const bool sk = (smooth & SAGE_SMOOTH_K) != 0, sv = (smooth & SAGE_SMOOTH_V) != 0;
     cudaError_t e = cudaMemsetAsync(w.cs.ksum, 0, w.stats_bytes, st);
@@ -149,17 +152,17 @@ sage_status_t forward(const void *q, const void *k, const void *v, void *out, co
         cs.ksum = nullptr;
     if (!sv)
         cs.vsum = nullptr;
-    if ((e = launch_colstats(kh, vh, cs, L, status, st)) != cudaSuccess)
+    if ((e = launch_colstats(kh, vh, cs, LK, status, st)) != cudaSuccess)
         return cuda_fail(e);
     if ((e = launch_quant(qh, kh, vh, cs, w.q_i8, w.q_scale, w.k_i8, w.k_scale, w.k_mean,
-                          fp8 ? w.v8 : nullptr, w.v_scale, sv ? w.v_mean : nullptr, L, status,
-                          st)) != cudaSuccess)
+                          fp8 ? w.v8 : nullptr, w.v_scale, sv ? w.v_mean : nullptr, L, LK,
+                          status, st)) != cudaSuccess)
         return cuda_fail(e);
     AttnArgs a{w.q_i8,     w.q_scale, w.k_i8, w.k_scale, fp8 ? (const void *)w.v8 : v,
                w.v_scale,  sv ? w.v_mean : nullptr,     static_cast<__half *>(out),
                nullptr,    causal,    pv_mode, resolve_scale(sm_scale, L.d)};
     sage_status_t herr;
-    if ((e = launch_attention(a, L, status, st, &herr)) != cudaSuccess)
+    if ((e = launch_attention(a, L, LK, status, st, &herr)) != cudaSuccess)
         return herr != SAGE_OK ? herr : cuda_fail(e);
     return SAGE_OK;
 }
@@ -174,42 +177,81 @@ sage_status_t alloc_ws(size_t bytes, cudaStream_t st, char **p)
     return SAGE_OK;
 }
 
-sage_status_t quant_qk_entry(const void *q, const void *k, const int32_t *cu_seqlens, int nseq,
-                             int total_tokens, int max_seqlen, int H, int d, int8_t *q_i8,
+// Shapes of one call: nseq sequences (dense: B), H heads, head dim d; queries have
+// max_q tokens per sequence and total_q in all, keys and values max_k and total_k;
+// cu_q / cu_k are the device cu_seqlens of a packed layout, or nullptr for dense.
+struct Shape {
+    const int32_t *cu_q, *cu_k;
+    int nseq, H, d, max_q, max_k, total_q, total_k;
+    SeqLayout lq() const
+    {
+        return cu_q ? SeqLayout::packed(cu_q, nseq, total_q, max_q, H, d)
+                    : SeqLayout::dense(nseq, H, max_q, d);
+    }
+    SeqLayout lk() const
+    {
+        return cu_k ? SeqLayout::packed(cu_k, nseq, total_k, max_k, H, d)
+                    : SeqLayout::dense(nseq, H, max_k, d);
+    }
+    bool empty() const { return nseq == 0 || H == 0 || max_q == 0 || total_q == 0; }
+};
+
+Shape dense_shape(int B, int H, int Nq, int Nk, int d)
+{
+    return Shape{nullptr, nullptr, B, H, d, Nq, Nk, B * Nq, B * Nk};
+}
+
+// Host-side checks shared by the entry points: sizes, the head dim and the grid limits.
+sage_status_t check_shape2(const Shape &sh)
+{
+    sage_status_t r = check_shape(sh.nseq, sh.H, sh.max_q, sh.d);
+    if (r != SAGE_OK)
+        return r;
+    if (sh.max_k < 0 || sh.total_q < 0 || sh.total_k < 0)
+        return SAGE_ERR_INVALID_ARG;
+    return SAGE_OK;
+}
+
+// B*N fits the int32 token counts of the dense layout.
+bool dense_fits(int B, int N) { return !(B > 0 && N > 0 && (int64_t)B * N > INT32_MAX); }
+
+sage_status_t quant_qk_entry(const void *q, const void *k, const Shape &sh, int8_t *q_i8,
                              float *q_scale, int8_t *k_i8, float *k_scale, float *k_mean,
                              int smooth_k, void *workspace, size_t ws_bytes, cudaStream_t st);
 sage_status_t quant_v_entry(const void *v, const int32_t *cu_seqlens, int nseq, int total_tokens,
                             int max_seqlen, int H, int d, uint8_t *v_e4m3, float *v_scale,
                             float *v_mean, bool smooth, cudaStream_t st);
 
-// Step 3 alone on pre-quantized operands (dense).
+// Step 3 alone on pre-quantized operands (dense; Nq queries, Nk keys).
 sage_status_t quantized_entry(const int8_t *q_i8, const float *q_scale, const int8_t *k_i8,
                               const float *k_scale, const void *v, const float *v_scale,
-                              const float *v_mean, void *out, int B, int H, int N, int d,
-                              int causal, int pv_mode, float sm_scale, cudaStream_t st)
+                              const float *v_mean, void *out, int B, int H, int Nq, int Nk,
+                              int d, int causal, int pv_mode, float sm_scale, cudaStream_t st)
 {
-    sage_status_t r = check_shape(B, H, N, d);
+    sage_status_t r = check_shape(B, H, Nq, d);
     if (r != SAGE_OK)
         return r;
+    if (Nk < 0)
+        return SAGE_ERR_INVALID_ARG;
     if (pv_mode != SAGE_PV_FP16 && pv_mode != SAGE_PV_FP8)
         return SAGE_ERR_INVALID_ARG;
-    if (B == 0 || H == 0 || N == 0)
+    if (B == 0 || H == 0 || Nq == 0)
         return SAGE_OK;
-    if (!q_i8 || !q_scale || !k_i8 || !k_scale || !v || !out ||
-        (pv_mode == SAGE_PV_FP8 && !v_scale))
+    if (!q_i8 || !q_scale || !out || (Nk > 0 && (!k_i8 || !k_scale || !v)) ||
+        (pv_mode == SAGE_PV_FP8 && Nk > 0 && !v_scale))
         return SAGE_ERR_INVALID_ARG;
-    if ((int64_t)B * N > INT32_MAX)
+    if (!dense_fits(B, Nq) || !dense_fits(B, Nk))
         return SAGE_ERR_UNSUPPORTED;
     if (!aligned16(q_i8) || !aligned16(k_i8) || !aligned16(v) || !aligned16(out))
         return SAGE_ERR_MISALIGNED;
     int *status = status_ptr(&r);
     if (!status)
         return r;
-    const SeqLayout L = SeqLayout::dense(B, H, N, d);
+    const Shape sh = dense_shape(B, H, Nq, Nk, d);
     AttnArgs a{q_i8,   q_scale, k_i8,   k_scale, v, v_scale, v_mean, static_cast<__half *>(out),
                nullptr, causal, pv_mode, resolve_scale(sm_scale, d)};
     sage_status_t herr;
-    cudaError_t e = launch_attention(a, L, status, st, &herr);
+    cudaError_t e = launch_attention(a, sh.lq(), sh.lk(), status, st, &herr);
     if (e != cudaSuccess)
         return herr != SAGE_OK ? herr : cuda_fail(e);
     return SAGE_OK;
@@ -224,19 +266,37 @@ extern "C" {
 
 size_t sage_workspace_size(int nseq, int H, int max_seqlen, int total_tokens, int d, int pv_mode)
 {
-    if (nseq < 0 || H < 0 || max_seqlen < 0 || total_tokens < 0)
+    return sage_workspace_size_kv(nseq, H, max_seqlen, max_seqlen, total_tokens, total_tokens, d,
+                                  pv_mode);
+}
+
+size_t sage_workspace_size_kv(int nseq, int H, int max_seqlen_q, int max_seqlen_k,
+                              int total_q, int total_k, int d, int pv_mode)
+{
+    if (nseq < 0 || H < 0 || max_seqlen_q < 0 || max_seqlen_k < 0 || total_q < 0 || total_k < 0)
         return 0;
-    return carve(nullptr, nseq, H, max_seqlen, total_tokens, d, pv_mode).total;
+    return carve(nullptr, nseq, H, max_seqlen_q, max_seqlen_k, total_q, total_k, d, pv_mode)
+        .total;
 }
 
 sage_status_t sage_quant_qk(const void *q, const void *k, int8_t *q_i8, float *q_scale,
                             int8_t *k_i8, float *k_scale, float *k_mean, int B, int H, int N,
                             int d, int smooth_k, sage_stream_t stream)
 {
-    if (B > 0 && N > 0 && (int64_t)B * N > INT32_MAX)
+    if (!dense_fits(B, N))
         return SAGE_ERR_UNSUPPORTED;
-    return quant_qk_entry(q, k, nullptr, B, B * N, N, H, d, q_i8, q_scale, k_i8, k_scale, k_mean,
+    return quant_qk_entry(q, k, dense_shape(B, H, N, N, d), q_i8, q_scale, k_i8, k_scale, k_mean,
                           smooth_k, nullptr, 0, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sage_status_t sage_quant_qk_kv(const void *q, const void *k, int8_t *q_i8, float *q_scale,
+                               int8_t *k_i8, float *k_scale, float *k_mean, int B, int H, int Nq,
+                               int Nk, int d, int smooth_k, sage_stream_t stream)
+{
+    if (!dense_fits(B, Nq) || !dense_fits(B, Nk))
+        return SAGE_ERR_UNSUPPORTED;
+    return quant_qk_entry(q, k, dense_shape(B, H, Nq, Nk, d), q_i8, q_scale, k_i8, k_scale,
+                          k_mean, smooth_k, nullptr, 0, reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"
@@ -245,21 +305,21 @@ namespace sage {
 namespace {
 // Steps 1-2 with optional caller scratch for the fp64 K column sums (nullptr: a
 // stream-ordered allocation is made and released).
-sage_status_t quant_qk_entry(const void *q, const void *k, const int32_t *cu_seqlens, int nseq,
-                             int total_tokens, int max_seqlen, int H, int d, int8_t *q_i8,
+sage_status_t quant_qk_entry(const void *q, const void *k, const Shape &sh, int8_t *q_i8,
                              float *q_scale, int8_t *k_i8, float *k_scale, float *k_mean,
                              int smooth_k, void *workspace, size_t ws_bytes, cudaStream_t st)
 {
-    sage_status_t r = check_shape(nseq, H, max_seqlen, d);
+    sage_status_t r = check_shape2(sh);
     if (r != SAGE_OK)
         return r;
-    if (nseq == 0 || H == 0 || max_seqlen == 0 || total_tokens == 0)
+    const bool has_q = sh.max_q > 0 && sh.total_q > 0, has_k = sh.max_k > 0 && sh.total_k > 0;
+    if (sh.nseq == 0 || sh.H == 0 || (!has_q && !has_k))
         return SAGE_OK;
-    if (!q || !k || !q_i8 || !q_scale || !k_i8 || !k_scale || !k_mean || total_tokens < 0)
+    if ((has_q && (!q || !q_i8 || !q_scale)) || (has_k && (!k || !k_i8 || !k_scale || !k_mean)))
         return SAGE_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(q_i8) || !aligned16(k_i8))
         return SAGE_ERR_MISALIGNED;
-    const size_t sum_bytes = (size_t)nseq * H * d * 8;
+    const size_t sum_bytes = (size_t)sh.nseq * sh.H * sh.d * 8;
     if (workspace != nullptr && smooth_k) {
         if (ws_bytes < sum_bytes)
             return SAGE_ERR_WORKSPACE;
@@ -269,12 +329,11 @@ sage_status_t quant_qk_entry(const void *q, const void *k, const int32_t *cu_seq
     int *status = status_ptr(&r);
     if (!status)
         return r;
-    const SeqLayout L = cu_seqlens ? SeqLayout::packed(cu_seqlens, nseq, total_tokens, max_seqlen, H, d)
-                                   : SeqLayout::dense(nseq, H, max_seqlen, d);
+    const SeqLayout Lq = sh.lq(), Lk = sh.lk();
     double *ksum = nullptr;
     bool owned = false;
     cudaError_t e;
-    if (smooth_k) {
+    if (smooth_k && has_k) {
         if (workspace != nullptr) {
             ksum = static_cast<double *>(workspace);
         } else {
@@ -287,7 +346,7 @@ sage_status_t quant_qk_entry(const void *q, const void *k, const int32_t *cu_seq
         ColStats cs;
         cs.ksum = ksum;
         if ((e = cudaMemsetAsync(ksum, 0, sum_bytes, st)) != cudaSuccess ||
-            (e = launch_colstats(static_cast<const __half *>(k), nullptr, cs, L, status, st)) !=
+            (e = launch_colstats(static_cast<const __half *>(k), nullptr, cs, Lk, status, st)) !=
                 cudaSuccess) {
             if (owned)
                 cudaFreeAsync(ksum, st);
@@ -297,8 +356,8 @@ sage_status_t quant_qk_entry(const void *q, const void *k, const int32_t *cu_seq
     ColStats cs;
     cs.ksum = ksum;
     e = launch_quant(static_cast<const __half *>(q), static_cast<const __half *>(k), nullptr, cs,
-                     q_i8, q_scale, k_i8, k_scale, k_mean, nullptr, nullptr, nullptr, L, status,
-                     st);
+                     q_i8, q_scale, k_i8, k_scale, k_mean, nullptr, nullptr, nullptr, Lq, Lk,
+                     status, st);
     if (owned)
         cudaFreeAsync(ksum, st);
     return e == cudaSuccess ? SAGE_OK : cuda_fail(e);
@@ -339,7 +398,7 @@ sage_status_t quant_v_entry(const void *v, const int32_t *cu_seqlens, int nseq, 
             cudaSuccess)
         e = launch_quant(nullptr, nullptr, static_cast<const __half *>(v), cs, nullptr, nullptr,
                          nullptr, nullptr, nullptr, v_e4m3, v_scale, smooth ? v_mean : nullptr,
-                         L, status, st);
+                         L, L, status, st);
     cudaFreeAsync(p, st);
     return e == cudaSuccess ? SAGE_OK : cuda_fail(e);
 }
@@ -353,8 +412,9 @@ sage_status_t sage_quant_qk_varlen(const void *q, const void *k, const int32_t *
                                    int8_t *q_i8, float *q_scale, int8_t *k_i8, float *k_scale,
                                    float *k_mean, int smooth_k, sage_stream_t stream)
 {
-    return quant_qk_entry(q, k, cu_seqlens, nseq, total_tokens, max_seqlen, H, d, q_i8, q_scale,
-                          k_i8, k_scale, k_mean, smooth_k, nullptr, 0,
+    const Shape sh{cu_seqlens, cu_seqlens, nseq, H, d, max_seqlen, max_seqlen, total_tokens,
+                   total_tokens};
+    return quant_qk_entry(q, k, sh, q_i8, q_scale, k_i8, k_scale, k_mean, smooth_k, nullptr, 0,
                           reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -365,9 +425,9 @@ sage_status_t sage_quant_qk_ws(const void *q, const void *k, int8_t *q_i8, float
 {
     if (workspace == nullptr && smooth_k && !(B == 0 || H == 0 || N == 0))
         return SAGE_ERR_WORKSPACE;
-    if (B > 0 && N > 0 && (int64_t)B * N > INT32_MAX)
+    if (!dense_fits(B, N))
         return SAGE_ERR_UNSUPPORTED;
-    return quant_qk_entry(q, k, nullptr, B, B * N, N, H, d, q_i8, q_scale, k_i8, k_scale, k_mean,
+    return quant_qk_entry(q, k, dense_shape(B, H, N, N, d), q_i8, q_scale, k_i8, k_scale, k_mean,
                           smooth_k, workspace, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -411,43 +471,44 @@ sage_status_t sage_quant_v_fp8(const void *v, uint8_t *v_e4m3, float *v_scale, i
 
 namespace sage {
 namespace {
-// Dense (cu_seqlens == nullptr) or packed forward pass with optional caller scratch.
-sage_status_t attn_entry(const void *q, const void *k, const void *v, void *out,
-                         const int32_t *cu_seqlens, int nseq, int total_tokens, int max_seqlen,
-                         int H, int d, int causal, int smooth_k, int pv_mode, float sm_scale,
-                         void *workspace, size_t ws_bytes, sage_stream_t stream)
+// Dense or packed forward pass with optional caller scratch.
+sage_status_t attn_entry(const void *q, const void *k, const void *v, void *out, const Shape &sh,
+                         int causal, int smooth_k, int pv_mode, float sm_scale, void *workspace,
+                         size_t ws_bytes, sage_stream_t stream)
 {
-    sage_status_t r = check_shape(nseq, H, max_seqlen, d);
+    sage_status_t r = check_shape2(sh);
     if (r != SAGE_OK)
         return r;
     if (pv_mode != SAGE_PV_FP16 && pv_mode != SAGE_PV_FP8)
         return SAGE_ERR_INVALID_ARG;
     if ((r = check_smooth(smooth_k, pv_mode)) != SAGE_OK)
         return r;
-    if (total_tokens < 0)
-        return SAGE_ERR_INVALID_ARG;
-    if (nseq == 0 || H == 0 || max_seqlen == 0 || total_tokens == 0)
+    if (sh.empty())
         return SAGE_OK;
-    if (!q || !k || !v || !out)
+    const bool no_keys = sh.max_k == 0 || sh.total_k == 0;
+    if (!q || !out || (!no_keys && (!k || !v)))
         return SAGE_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
         return SAGE_ERR_MISALIGNED;
-    const size_t need = sage_workspace_size(nseq, H, max_seqlen, total_tokens, d, pv_mode);
     cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-    const SeqLayout L = cu_seqlens ? SeqLayout::packed(cu_seqlens, nseq, total_tokens, max_seqlen, H, d)
-                                   : SeqLayout::dense(nseq, H, max_seqlen, d);
+    if (no_keys) {   // no query sees a key: the output is zero
+        cudaError_t e = cudaMemsetAsync(out, 0, (size_t)sh.total_q * sh.H * sh.d * 2, st);
+        return e == cudaSuccess ? SAGE_OK : cuda_fail(e);
+    }
+    const size_t need = sage_workspace_size_kv(sh.nseq, sh.H, sh.max_q, sh.max_k, sh.total_q,
+                                               sh.total_k, sh.d, pv_mode);
     if (workspace != nullptr) {
         if (ws_bytes < need)
             return SAGE_ERR_WORKSPACE;
         if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
             return SAGE_ERR_MISALIGNED;
-        return forward(q, k, v, out, L, causal, smooth_k, pv_mode, sm_scale,
+        return forward(q, k, v, out, sh.lq(), sh.lk(), causal, smooth_k, pv_mode, sm_scale,
                        static_cast<char *>(workspace), st);
     }
     char *ws = nullptr;
     if ((r = alloc_ws(need, st, &ws)) != SAGE_OK)
         return r;
-    r = forward(q, k, v, out, L, causal, smooth_k, pv_mode, sm_scale, ws, st);
+    r = forward(q, k, v, out, sh.lq(), sh.lk(), causal, smooth_k, pv_mode, sm_scale, ws, st);
     cudaFreeAsync(ws, st);
     return r;
 }
@@ -464,8 +525,26 @@ sage_status_t sage_attn_varlen_fwd(const void *q, const void *k, const void *v, 
 {
     if (cu_seqlens == nullptr && nseq > 0 && total_tokens > 0)
         return SAGE_ERR_INVALID_ARG;
-    return attn_entry(q, k, v, out, cu_seqlens, nseq, total_tokens, max_seqlen, H, d, causal,
-                      smooth_k, pv_mode, sm_scale, workspace, ws_bytes, stream);
+    const Shape sh{cu_seqlens, cu_seqlens, nseq, H, d, max_seqlen, max_seqlen, total_tokens,
+                   total_tokens};
+    return attn_entry(q, k, v, out, sh, causal, smooth_k, pv_mode, sm_scale, workspace,
+                      ws_bytes, stream);
+}
+
+sage_status_t sage_attn_varlen_fwd_kv(const void *q, const void *k, const void *v, void *out,
+                                      const int32_t *cu_seqlens_q, const int32_t *cu_seqlens_k,
+                                      int nseq, int total_q, int total_k, int max_seqlen_q,
+                                      int max_seqlen_k, int H, int d, int causal, int smooth_k,
+                                      int pv_mode, float sm_scale, void *workspace,
+                                      size_t ws_bytes, sage_stream_t stream)
+{
+    if (nseq > 0 && ((cu_seqlens_q == nullptr && total_q > 0) ||
+                     (cu_seqlens_k == nullptr && total_k > 0)))
+        return SAGE_ERR_INVALID_ARG;
+    const Shape sh{cu_seqlens_q, cu_seqlens_k, nseq, H, d, max_seqlen_q, max_seqlen_k, total_q,
+                   total_k};
+    return attn_entry(q, k, v, out, sh, causal, smooth_k, pv_mode, sm_scale, workspace,
+                      ws_bytes, stream);
 }
 
 sage_status_t sage_attn_fwd_ws(const void *q, const void *k, const void *v, void *out, int B,
@@ -475,9 +554,9 @@ sage_status_t sage_attn_fwd_ws(const void *q, const void *k, const void *v, void
 {
     if (workspace == nullptr && !(B == 0 || H == 0 || N == 0))
         return SAGE_ERR_WORKSPACE;
-    if (B > 0 && N > 0 && (int64_t)B * N > INT32_MAX)
+    if (!dense_fits(B, N))
         return SAGE_ERR_UNSUPPORTED;
-    return attn_entry(q, k, v, out, nullptr, B, B * N, N, H, d, causal, smooth_k, pv_mode,
+    return attn_entry(q, k, v, out, dense_shape(B, H, N, N, d), causal, smooth_k, pv_mode,
                       sm_scale, workspace, ws_bytes, stream);
 }
 
@@ -485,10 +564,21 @@ sage_status_t sage_attn_fwd(const void *q, const void *k, const void *v, void *o
                             int N, int d, int causal, int smooth_k, int pv_mode, float sm_scale,
                             sage_stream_t stream)
 {
-    if (B > 0 && N > 0 && (int64_t)B * N > INT32_MAX)
+    if (!dense_fits(B, N))
         return SAGE_ERR_UNSUPPORTED;
-    return attn_entry(q, k, v, out, nullptr, B, B * N, N, H, d, causal, smooth_k, pv_mode,
+    return attn_entry(q, k, v, out, dense_shape(B, H, N, N, d), causal, smooth_k, pv_mode,
                       sm_scale, nullptr, 0, stream);
+}
+
+sage_status_t sage_attn_fwd_kv(const void *q, const void *k, const void *v, void *out, int B,
+                               int H, int Nq, int Nk, int d, int causal, int smooth_k,
+                               int pv_mode, float sm_scale, void *workspace, size_t ws_bytes,
+                               sage_stream_t stream)
+{
+    if (!dense_fits(B, Nq) || !dense_fits(B, Nk))
+        return SAGE_ERR_UNSUPPORTED;
+    return attn_entry(q, k, v, out, dense_shape(B, H, Nq, Nk, d), causal, smooth_k, pv_mode,
+                      sm_scale, workspace, ws_bytes, stream);
 }
 
 sage_status_t sage_attn_fwd_quantized(const int8_t *q_i8, const float *q_scale,
@@ -497,8 +587,20 @@ sage_status_t sage_attn_fwd_quantized(const int8_t *q_i8, const float *q_scale,
                                       int d, int causal, int pv_mode, float sm_scale,
                                       sage_stream_t stream)
 {
-    return quantized_entry(q_i8, q_scale, k_i8, k_scale, v, v_scale, nullptr, out, B, H, N, d,
-                           causal, pv_mode, sm_scale, reinterpret_cast<cudaStream_t>(stream));
+    return quantized_entry(q_i8, q_scale, k_i8, k_scale, v, v_scale, nullptr, out, B, H, N, N,
+                           d, causal, pv_mode, sm_scale, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sage_status_t sage_attn_fwd_quantized_kv(const int8_t *q_i8, const float *q_scale,
+                                         const int8_t *k_i8, const float *k_scale, const void *v,
+                                         const float *v_scale, const float *v_mean, void *out,
+                                         int B, int H, int Nq, int Nk, int d, int causal,
+                                         int pv_mode, float sm_scale, sage_stream_t stream)
+{
+    if (v_mean != nullptr && pv_mode != SAGE_PV_FP8)
+        return SAGE_ERR_UNSUPPORTED;
+    return quantized_entry(q_i8, q_scale, k_i8, k_scale, v, v_scale, v_mean, out, B, H, Nq, Nk,
+                           d, causal, pv_mode, sm_scale, reinterpret_cast<cudaStream_t>(stream));
 }
 
 sage_status_t sage_attn_fwd_quantized_smooth_v(const int8_t *q_i8, const float *q_scale,
@@ -511,7 +613,7 @@ sage_status_t sage_attn_fwd_quantized_smooth_v(const int8_t *q_i8, const float *
     if (v_mean == nullptr && B > 0 && H > 0 && N > 0)
         return SAGE_ERR_INVALID_ARG;
     return quantized_entry(q_i8, q_scale, k_i8, k_scale, v_e4m3, v_scale, v_mean, out, B, H, N,
-                           d, causal, SAGE_PV_FP8, sm_scale,
+                           N, d, causal, SAGE_PV_FP8, sm_scale,
                            reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -546,7 +648,8 @@ sage_status_t sage_debug_qk_int32(const int8_t *q_i8, const int8_t *k_i8, int32_
         __half *o = reinterpret_cast<__half *>(ws + sc_bytes + align256(elems * 2));
         AttnArgs a{q_i8, qs, k_i8, ks, vz, nullptr, nullptr, o, s_out, 0, SAGE_PV_FP16, 1.0f};
         sage_status_t herr;
-        e = launch_attention(a, SeqLayout::dense(B, H, N, d), status, st, &herr);
+        const SeqLayout L = SeqLayout::dense(B, H, N, d);
+        e = launch_attention(a, L, L, status, st, &herr);
         if (e != cudaSuccess && herr != SAGE_OK) {
             cudaFreeAsync(ws, st);
             return herr;
@@ -683,6 +786,7 @@ extern "C" sage_status_t sage_attn_fwd_noalloc(const void *q, const void *k, con
         return r;
     // forward() zeroes the only scratch that must start at zero (the K and V column
     // statistics) before its kernels run; everything else is written before it is read.
-    return forward(q, k, v, out, SeqLayout::dense(B, H, N, d), causal, smooth_k, pv_mode,
+    const SeqLayout L = SeqLayout::dense(B, H, N, d);
+    return forward(q, k, v, out, L, L, causal, smooth_k, pv_mode,
                    sm_scale, ws, reinterpret_cast<cudaStream_t>(stream));
 }

@@ -120,7 +120,8 @@ struct KParams {
     const float *v_mean;   // FP8 with smooth V: added to every output row; else nullptr
     __half *out;
     int32_t *s_dump;
-    SeqLayout L;
+    SeqLayout L;         // queries (and the output)
+    SeqLayout LK;        // keys and values (L again for self-attention)
     int nqb, nkb;        // scale blocks per (sequence, head) row of the scale arrays
     int causal;
     float sc_log2;       // sm_scale * log2(e)
@@ -169,16 +170,31 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
     uint8_t *smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
 
     const SeqLayout &L = p.L;
+    const SeqLayout &LK = p.LK;
     const int s = blockIdx.z, h = blockIdx.y;
-    int start, len;
-    if (!L.range(s, start, len, p.status))
+    int start, len, kstart, klen;
+    if (!L.range(s, start, len, p.status) || !LK.range(s, kstart, klen, p.status))
         return;
     const int cta_x = p.causal ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
     const int qt0 = cta_x * NQT;
     if (qt0 * C::BM >= len)
         return;                                    // whole CTA beyond this sequence
     const int last_row = min(len, (qt0 + NQT) * C::BM) - 1;
-    const int nkv = p.causal ? last_row / C::BN + 1 : (len + C::BN - 1) / C::BN;
+    // causal: query i sees keys j <= i + koff (bottom-right aligned; koff = 0 when the
+    // queries and keys are the same sequence)
+    const int koff = klen - len;
+    const int nkt = (klen + C::BN - 1) / C::BN;
+    const int nkv = !p.causal ? nkt : (last_row + koff < 0 ? 0 : min(nkt, (last_row + koff) / C::BN + 1));
+    if (nkv == 0) {
+        // no query row of this CTA sees a key: its output rows are zero
+        const int r0 = qt0 * C::BM, nrow = last_row + 1 - r0;
+        for (int idx = threadIdx.x; idx < nrow * (D / 8); idx += blockDim.x) {
+            const int r = r0 + idx / (D / 8);
+            *reinterpret_cast<uint4 *>(p.out + L.offset(s, start, h, r) + (idx % (D / 8)) * 8) =
+                make_uint4(0u, 0u, 0u, 0u);
+        }
+        return;
+    }
 
     uint8_t *sQ = smem + C::kOffQ;
     uint8_t *sK = smem + C::kOffK;
@@ -239,7 +255,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
         const int64_t sh = (int64_t)s * L.H + h;
         const bool tile_valid = qt * C::BM < len;
         const float qsc = (tile_valid ? __ldg(p.q_scale + sh * p.nqb + qt) : 0.0f) * p.sc_log2;
-        const int kb_valid = (len + kKBlock - 1) / kKBlock;
+        const int kb_valid = (klen + kKBlock - 1) / kKBlock;
 
         // m_ref: the max that P is taken relative to; it moves only when the row max
         // exceeds it by more than kRescaleSlack (0 in FP8 mode, so P <= 1 and 448 P fits E4M3)
@@ -255,8 +271,9 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
             const float sc1 = qsc * (kb1 < kb_valid ? __ldg(p.k_scale + sh * p.nkb + kb1) : 0.0f);
             const int kcol0 = j * C::BN;
             const bool need_mask =
-                (kcol0 + C::BN > len) || (p.causal && kcol0 + C::BN - 1 > qt * C::BM);
-            const int col_lim = p.causal ? min(len, qrow + 1) : len;   // keys < col_lim visible
+                (kcol0 + C::BN > klen) || (p.causal && kcol0 + C::BN - 1 > qt * C::BM + koff);
+            // keys < col_lim are visible to this row
+            const int col_lim = p.causal ? min(klen, qrow + 1 + koff) : klen;
 
             // the whole 128-key score row into registers (one TMEM pass)
             uint32_t sreg[4][32];
@@ -268,9 +285,9 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
                 tmem_ld_wait(sreg[ch]);
             if constexpr (DUMP) {
                 if (qrow < len) {
-                    int32_t *drow = p.s_dump + (sh * L.maxlen + qrow) * L.maxlen;
+                    int32_t *drow = p.s_dump + (sh * L.maxlen + qrow) * LK.maxlen;
                     for (int e = 0; e < C::BN; e++)
-                        if (kcol0 + e < len)
+                        if (kcol0 + e < klen)
                             drow[kcol0 + e] = static_cast<int>(sreg[e / 32][e % 32]);
                 }
             }
@@ -445,7 +462,9 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
         // epilogue: the last P.V, normalize, round to fp16, store the row
         if (ok && (ok = warp_wait(&pv_full[i], (nkv - 1) & 1, abort, p.status))) {
             tc_fence_after();
-            const float inv_l = 1.0f / l;
+            // a row that sees no key (only when there are more queries than keys) has
+            // l = 0 and P = 0: it is written as zeros
+            const float inv_l = l > 0.0f ? 1.0f / l : 0.0f;
             __half *dst = p.out + L.offset(s, start, h, qrow);
             uint32_t orow[D / 32][32];
 #pragma unroll
@@ -466,7 +485,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
                                 sc = __ldg(p.v_scale + sh * D + ch * 32 + c + e) * inv_l;
                             f[e] = __uint_as_float(r[c + e]) * sc;
                             if constexpr (FP8)
-                                if (p.v_mean != nullptr)
+                                if (p.v_mean != nullptr && l > 0.0f)
                                     f[e] += __ldg(p.v_mean + sh * D + ch * 32 + c + e);
                         }
                         uint4 u;
@@ -497,7 +516,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
             for (int j = 0; j < nkv; j++) {
                 const int stg = j % C::STAGES;
                 const uint32_t ph = (j / C::STAGES) & 1;
-                tma_coords(L, s, start, h, j * C::BN, c1, c2);
+                tma_coords(LK, s, kstart, h, j * C::BN, c1, c2);
                 if (!mbar_wait(&k_empty[stg], ph ^ 1, abort, p.status,
                                status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs))
                     break;
@@ -684,8 +703,8 @@ bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int elem
 }
 
 template <int D, bool FP8, int NQT, bool DUMP>
-cudaError_t run(const AttnArgs &a, const SeqLayout &L, int *status, cudaStream_t st,
-                sage_status_t *host_err)
+cudaError_t run(const AttnArgs &a, const SeqLayout &L, const SeqLayout &LK, int *status,
+                cudaStream_t st, sage_status_t *host_err)
 {
     using C = Cfg<D, FP8, NQT>;
     CUtensorMap mq, mk, mv;
@@ -694,10 +713,10 @@ cudaError_t run(const AttnArgs &a, const SeqLayout &L, int *status, cudaStream_t
     const CUtensorMapSwizzle v_swz =
         C::kVRowBytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     bool ok = make_map(&mq, a.q_i8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L, D, C::BM, qk_swz) &&
-              make_map(&mk, a.k_i8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L, D, C::BN, qk_swz) &&
+              make_map(&mk, a.k_i8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, LK, D, C::BN, qk_swz) &&
               make_map(&mv, a.v,
                        FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
-                       C::kVElem, L, C::kVRowBytes / C::kVElem, C::BN, v_swz);
+                       C::kVElem, LK, C::kVRowBytes / C::kVElem, C::BN, v_swz);
     if (!ok) {
         *host_err = SAGE_ERR_CUDA;
         return cudaErrorInvalidValue;
@@ -710,8 +729,9 @@ cudaError_t run(const AttnArgs &a, const SeqLayout &L, int *status, cudaStream_t
     p.out = a.out;
     p.s_dump = a.s_dump;
     p.L = L;
+    p.LK = LK;
     p.nqb = (L.maxlen + kQBlock - 1) / kQBlock;
-    p.nkb = (L.maxlen + kKBlock - 1) / kKBlock;
+    p.nkb = (LK.maxlen + kKBlock - 1) / kKBlock;
     p.causal = a.causal;
     p.sc_log2 = a.sm_scale * kLog2e;
     p.status = status;
@@ -729,21 +749,25 @@ cudaError_t run(const AttnArgs &a, const SeqLayout &L, int *status, cudaStream_t
 
 }  // namespace
 
-cudaError_t launch_attention(const AttnArgs &a, const SeqLayout &L, int *status, cudaStream_t st,
-                             sage_status_t *host_err)
+cudaError_t launch_attention(const AttnArgs &a, const SeqLayout &L, const SeqLayout &LK,
+                             int *status, cudaStream_t st, sage_status_t *host_err)
 {
     *host_err = SAGE_OK;
+    if (L.nseq != LK.nseq || L.H != LK.H || L.d != LK.d) {
+        *host_err = SAGE_ERR_INVALID_ARG;
+        return cudaErrorInvalidValue;
+    }
     const bool fp8 = a.pv_mode == SAGE_PV_FP8;
     if (a.s_dump != nullptr) {
         if (L.d == 128)
-            return run<128, false, 2, true>(a, L, status, st, host_err);
-        return run<64, false, 2, true>(a, L, status, st, host_err);
+            return run<128, false, 2, true>(a, L, LK, status, st, host_err);
+        return run<64, false, 2, true>(a, L, LK, status, st, host_err);
     }
     if (L.d == 128)
-        return fp8 ? run<128, true, 2, false>(a, L, status, st, host_err)
-                   : run<128, false, 2, false>(a, L, status, st, host_err);
-    return fp8 ? run<64, true, 2, false>(a, L, status, st, host_err)
-               : run<64, false, 2, false>(a, L, status, st, host_err);
+        return fp8 ? run<128, true, 2, false>(a, L, LK, status, st, host_err)
+                   : run<128, false, 2, false>(a, L, LK, status, st, host_err);
+    return fp8 ? run<64, true, 2, false>(a, L, LK, status, st, host_err)
+               : run<64, false, 2, false>(a, L, LK, status, st, host_err);
 }
 
 }  // namespace sage

@@ -247,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 4) quant_kernel(
     ColStats cs, int8_t *__restrict__ q_i8, float *__restrict__ q_scale,
     int8_t *__restrict__ k_i8, float *__restrict__ k_scale, float *__restrict__ k_mean,
     uint8_t *__restrict__ v_e4m3, float *__restrict__ v_scale, float *__restrict__ v_mean,
-    SeqLayout L, int nqb, int nkb, int part0, int *status)
+    SeqLayout Lq, SeqLayout Lk, int with_q, int nkc, int *status)
 {
     constexpr int kGpr = D / 8;                      // 16-byte groups per row
     constexpr int kRowStep = kThreads / kGpr;        // rows between a thread's groups
@@ -261,14 +261,26 @@ __global__ void __launch_bounds__(kThreads, 4) quant_kernel(
     __shared__ float s_sc[D];             // V scale per channel
     __shared__ float s_rc[D];             // fl(1 / V scale) per channel
 
+    // 0: Q block, 1: K pair of blocks, 2: V chunk. grid.x spans the parts in order:
+    // [Q chunks of Lq | K chunks of Lk] when with_q, then [V chunks of Lk] if any.
+    const int nqb = (Lq.maxlen + kQBlock - 1) / kQBlock;   // Q scale blocks per head
+    const int nkb = (Lk.maxlen + kKBlock - 1) / kKBlock;   // K scale blocks per head
+    int kind, chunk = (int)blockIdx.x;
+    if (with_q && chunk < nqb) {
+        kind = 0;
+    } else {
+        if (with_q)
+            chunk -= nqb;
+        kind = (with_q && chunk < nkc) ? 1 : 2;
+        if (kind == 2 && with_q)
+            chunk -= nkc;
+    }
+    const SeqLayout &L = kind == 0 ? Lq : Lk;
     const int s = blockIdx.z, h = blockIdx.y;
     int start, len;
     if (!L.range(s, start, len, status))
         return;
     const int64_t sh = (int64_t)s * L.H + h;
-    // 0: Q block, 1: K pair of blocks, 2: V chunk; grid.x spans consecutive parts
-    const int kind = part0 + (int)blockIdx.x / nqb;
-    const int chunk = (int)blockIdx.x % nqb;
     const int row0 = chunk * kQBlock;
 
     if (row0 >= len) {                    // padding block of a short sequence
@@ -479,7 +491,7 @@ __global__ void __launch_bounds__(kThreads, 4) quant_kernel(
 cudaError_t launch_colstats(const __half *k, const __half *v, const ColStats &cs,
                             const SeqLayout &L, int *status, cudaStream_t st)
 {
-    if (cs.ksum == nullptr && cs.vhi == nullptr)
+    if ((cs.ksum == nullptr && cs.vhi == nullptr) || L.maxlen == 0 || L.H == 0 || L.nseq == 0)
         return cudaSuccess;
     dim3 grid((L.maxlen + kColChunk - 1) / kColChunk, L.H, L.nseq);
     const bool dk = cs.ksum != nullptr, dv = cs.vhi != nullptr;
@@ -501,26 +513,31 @@ cudaError_t launch_colstats(const __half *k, const __half *v, const ColStats &cs
     return cudaGetLastError();
 }
 
+// Quantizes Q and K (q_i8 != nullptr) and/or V (v_e4m3 != nullptr) in one launch.
 cudaError_t launch_quant(const __half *q, const __half *k, const __half *v, const ColStats &cs,
                          int8_t *q_i8, float *q_scale, int8_t *k_i8, float *k_scale,
                          float *k_mean, uint8_t *v_e4m3, float *v_scale, float *v_mean,
-                         const SeqLayout &L, int *status, cudaStream_t st)
+                         const SeqLayout &Lq, const SeqLayout &Lk, int *status,
+                         cudaStream_t st)
 {
-    const int nqb = (L.maxlen + kQBlock - 1) / kQBlock;
-    const int nkb = (L.maxlen + kKBlock - 1) / kKBlock;
-    const int part0 = q_i8 != nullptr ? 0 : 2;
-    const int part1 = v_e4m3 != nullptr ? 3 : 2;
-    if (part1 <= part0)
+    const int with_q = q_i8 != nullptr ? 1 : 0;
+    const bool with_v = v_e4m3 != nullptr;
+    const int nqc = (Lq.maxlen + kQBlock - 1) / kQBlock;     // 128-token chunks
+    const int nkc = (Lk.maxlen + kQBlock - 1) / kQBlock;
+    const int nx = (with_q ? nqc + nkc : 0) + (with_v ? nkc : 0);
+    if (nx == 0 || Lk.H == 0 || Lk.nseq == 0)
         return cudaSuccess;
-    dim3 grid(nqb * (part1 - part0), L.H, L.nseq);
-    if (L.d == 128)
+    if (with_q && (Lq.nseq != Lk.nseq || Lq.H != Lk.H || Lq.d != Lk.d))
+        return cudaErrorInvalidValue;
+    dim3 grid(nx, Lk.H, Lk.nseq);
+    if (Lk.d == 128)
         quant_kernel<128><<<grid, kThreads, 0, st>>>(q, k, v, cs, q_i8, q_scale, k_i8, k_scale,
-                                                     k_mean, v_e4m3, v_scale, v_mean, L, nqb,
-                                                     nkb, part0, status);
+                                                     k_mean, v_e4m3, v_scale, v_mean, Lq, Lk,
+                                                     with_q, nkc, status);
     else
         quant_kernel<64><<<grid, kThreads, 0, st>>>(q, k, v, cs, q_i8, q_scale, k_i8, k_scale,
-                                                    k_mean, v_e4m3, v_scale, v_mean, L, nqb,
-                                                    nkb, part0, status);
+                                                    k_mean, v_e4m3, v_scale, v_mean, Lq, Lk,
+                                                    with_q, nkc, status);
     return cudaGetLastError();
 }
 

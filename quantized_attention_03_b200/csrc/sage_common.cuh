@@ -90,11 +90,13 @@ __host__ __device__ inline uint32_t key_bits(uint32_t key)
 cudaError_t launch_colstats(const __half *k, const __half *v, const ColStats &cs,
                             const SeqLayout &L, int *status, cudaStream_t st);
 // Quantizes Q and K (q_i8 != nullptr) and/or V (v_e4m3 != nullptr). K is smoothed when
-// cs.ksum is set, V when cs.vsum is set (its mean goes to v_mean if that is set).
+// cs.ksum is set, V when cs.vsum is set (its mean goes to v_mean if that is set). Q
+// lives in layout Lq, K and V in Lk (the same layout for self-attention).
 cudaError_t launch_quant(const __half *q, const __half *k, const __half *v, const ColStats &cs,
                          int8_t *q_i8, float *q_scale, int8_t *k_i8, float *k_scale,
                          float *k_mean, uint8_t *v_e4m3, float *v_scale, float *v_mean,
-                         const SeqLayout &L, int *status, cudaStream_t st);
+                         const SeqLayout &Lq, const SeqLayout &Lk, int *status,
+                         cudaStream_t st);
 
 struct AttnArgs {
     const int8_t *q_i8;
@@ -110,8 +112,10 @@ struct AttnArgs {
     int pv_mode;
     float sm_scale;
 };
-cudaError_t launch_attention(const AttnArgs &a, const SeqLayout &L, int *status, cudaStream_t st,
-                             sage_status_t *host_err);
+// Queries in layout Lq, keys and values in Lk (the same layout for self-attention; with
+// different lengths the causal mask aligns at the bottom right).
+cudaError_t launch_attention(const AttnArgs &a, const SeqLayout &Lq, const SeqLayout &Lk,
+                             int *status, cudaStream_t st, sage_status_t *host_err);
 cudaError_t launch_wait_selftest(int *status, uint64_t timeout_ns, cudaStream_t st);
 
 }  // namespace sage

@@ -7,7 +7,8 @@ video-DiT attention with channel outliers in K, long-sequence sweeps, packed var
 Recipe (all draws on the CPU from ``torch.Generator().manual_seed(seed)``, in this order):
 
 1. (varlen only) the sequence lengths, ``randint(lo, hi + 1)`` each;
-2. Q, K, V as fp32 standard normals in the layout's shape;
+2. Q, K, V as fp32 standard normals in the layout's shape (Q with its own length when
+   the queries are fewer than the keys);
 3. the K channel offset: one length-d vector added to every token of every head. With
    ``offset_channels = c`` only c channels (``randperm(d)[:c]``) get an offset, drawn
    after the permutation. ``N(0, s^2)`` is read as variance s^2 (std s);
@@ -42,6 +43,7 @@ class Workload:
     nseq: int = 0                  # > 0: packed varlen with nseq sequences
     len_lo: int = 512
     len_hi: int = 16384
+    nq: int = 0                    # > 0: queries per sequence when fewer than the N keys
 
 
 def tiny() -> Workload:
@@ -63,6 +65,13 @@ def sweep(N: int, d: int, causal: bool) -> Workload:
                     B, 32, N, d, causal, 1.0)
 
 
+def prefill_kv() -> Workload:
+    """The last 2048 tokens of 8192-token sequences attending to all their keys (chunked
+    prefill against cached keys), causal."""
+    return Workload("LLM chunked prefill B2 H32 Nq2048 Nk8192 d128 causal", 1005, 2, 32, 8192,
+                    128, True, 1.0, nq=2048)
+
+
 def varlen() -> Workload:
     return Workload("packed varlen causal 8 seqs H32 d128", 1004, 0, 32, 0, 128, True, 2.0,
                     pv_modes=("fp8",), nseq=8)
@@ -77,13 +86,16 @@ def _offset(g: torch.Generator, d: int, std: float, channels: Optional[int]) -> 
     return off
 
 
-def make_dense(w: Workload, B: Optional[int] = None, N: Optional[int] = None):
-    """fp16 CPU tensors q, k, v of shape [B, H, N, d] (B and N may be overridden)."""
+def make_dense(w: Workload, B: Optional[int] = None, N: Optional[int] = None,
+               Nq: Optional[int] = None):
+    """fp16 CPU tensors q [B, H, Nq, d] and k, v [B, H, N, d] (B, N and Nq may be
+    overridden; Nq defaults to the workload's nq, else N)."""
     B = w.B if B is None else B
     N = w.N if N is None else N
+    Nq = (w.nq or N) if Nq is None else Nq
     g = torch.Generator().manual_seed(w.seed)
     shape = (B, w.H, N, w.d)
-    q = torch.randn(shape, generator=g)
+    q = torch.randn((B, w.H, Nq, w.d), generator=g)
     k = torch.randn(shape, generator=g)
     v = torch.randn(shape, generator=g)
     k += _offset(g, w.d, w.offset_std, w.offset_channels)
@@ -112,10 +124,37 @@ def make_varlen(w: Workload, nseq: Optional[int] = None, len_lo: Optional[int] =
     return q.half(), k.half(), v.half(), cu
 
 
+def make_varlen_kv(w: Workload, lens_q, lens_k):
+    """Packed q [Tq, H, d], k and v [Tk, H, d] with their own per-sequence lengths, and
+    int32 cu_seqlens_q, cu_seqlens_k."""
+    g = torch.Generator().manual_seed(w.seed)
+    cq = torch.zeros(len(lens_q) + 1, dtype=torch.int32)
+    ck = torch.zeros(len(lens_k) + 1, dtype=torch.int32)
+    cq[1:] = torch.cumsum(torch.as_tensor(lens_q, dtype=torch.int64), 0).to(torch.int32)
+    ck[1:] = torch.cumsum(torch.as_tensor(lens_k, dtype=torch.int64), 0).to(torch.int32)
+    q = torch.randn((int(cq[-1]), w.H, w.d), generator=g)
+    k = torch.randn((int(ck[-1]), w.H, w.d), generator=g)
+    v = torch.randn((int(ck[-1]), w.H, w.d), generator=g)
+    k += _offset(g, w.d, w.offset_std, w.offset_channels)
+    return q.half(), k.half(), v.half(), cq, ck
+
+
 def attention_ops(B: int, H: int, N: int, d: int, causal: bool) -> float:
     """Operation count of one attention forward: 4 B H N^2 d, halved for causal."""
     ops = 4.0 * B * H * N * N * d
     return ops / 2 if causal else ops
+
+
+def attention_ops_kv(B: int, H: int, Nq: int, Nk: int, d: int, causal: bool) -> float:
+    """4 d per visible (query, key) pair: B H Nq Nk 4d, or with the bottom-right causal
+    mask B H 4d times the visible pairs sum over i of min(Nk, max(0, i + 1 + Nk - Nq))."""
+    if not causal:
+        return 4.0 * B * H * Nq * Nk * d
+    off = Nk - Nq
+    lo = max(0, -off)                  # first query that sees a key
+    full = max(lo, min(Nq, Nk - off))  # queries from here on see all Nk keys
+    pairs = sum(i + 1 + off for i in range(lo, full)) + (Nq - full) * Nk
+    return 4.0 * B * H * pairs * d
 
 
 def varlen_ops(lens, H: int, d: int, causal: bool) -> float:

@@ -296,3 +296,100 @@ def test_smooth_v_full_size_video_dit_sampled():
             tag = f"video_dit smooth V head {h} rows {r0}:{r1}"
             assert_vs_oracle(got[mask], ref[mask], tag)
             assert_vs_fp64(got[mask], exact[mask], True, tag)
+
+
+# ------------------------------------- queries fewer (or more) than keys: Nq != Nk
+
+
+KV_CASES = [
+    # Nq, Nk, d, causal
+    (1, 700, 128, True), (1, 129, 64, False), (70, 300, 64, True), (128, 1000, 128, False),
+    (513, 1200, 128, True), (300, 100, 64, True), (200, 129, 128, False),
+]
+
+
+@pytest.mark.parametrize("pv", ["fp16", "fp8"])
+@pytest.mark.parametrize("Nq,Nk,d,causal", KV_CASES)
+def test_kv_small_full_compare(Nq, Nk, d, causal, pv):
+    B, H = 2, 2
+    w = inputs.Workload("t", 400 + Nq + Nk, B, H, Nk, d, causal, 2.0, nq=Nq)
+    q, k, v = inputs.make_dense(w)
+    got = _run_dense(q, k, v, causal, pv)
+    lq, lk = oracle.Layout.dense(B, H, Nq, d), oracle.Layout.dense(B, H, Nk, d)
+    ref = oracle.sage_attention(q.numpy(), k.numpy(), v.numpy(), lq, causal, True, PV[pv],
+                                kv_layout=lk)
+    tag = f"Nq={Nq} Nk={Nk} d={d} causal={causal} {pv}"
+    assert_vs_oracle(got, ref, tag)
+    exact = oracle.attn_fp64(q.numpy(), k.numpy(), v.numpy(), lq, causal, 1 / math.sqrt(d),
+                             kv_layout=lk)
+    assert_vs_fp64(got, exact, pv == "fp8", tag)
+    if causal and Nq > Nk:
+        assert not got[:, :, :Nq - Nk].any()          # queries that see no key
+
+
+def test_kv_quantized_entry_and_workspace_match_fused():
+    B, H, Nq, Nk, d = 2, 3, 300, 900, 128
+    w = inputs.Workload("t", 91, B, H, Nk, d, True, 1.0, nq=Nq)
+    q, k, v = (t.cuda() for t in inputs.make_dense(w))
+    fused = sage.sageattn(q, k, v, True, True, sage.SAGE_PV_FP8, smooth_v=True)
+    z = sage.quant_qk(q, k, True)
+    codes, scales, mean = sage.quant_v_fp8(v, smooth_v=True)
+    split = sage.attn_quantized(z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], codes, scales,
+                                True, sage.SAGE_PV_FP8, v_mean=mean)
+    need = sage.sage_workspace_size_kv(B, H, Nq, Nk, B * Nq, B * Nk, d, sage.SAGE_PV_FP8)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    out_ws = torch.empty_like(q)
+    sage.sage_attn_fwd_kv(q, k, v, out_ws, B, H, Nq, Nk, d, 1,
+                          sage.SAGE_SMOOTH_K | sage.SAGE_SMOOTH_V, sage.SAGE_PV_FP8, 0.0, ws, need)
+    assert sage.sage_get_device_status() == 0
+    assert torch.equal(fused, split) and torch.equal(fused, out_ws)
+
+
+def test_kv_no_keys_gives_zero_output():
+    q = torch.randn((1, 2, 64, 64), device="cuda").half()
+    k = torch.empty((1, 2, 0, 64), device="cuda", dtype=torch.float16)
+    out = torch.full_like(q, 7.0)
+    sage.sage_attn_fwd_kv(q, k, k, out, 1, 2, 64, 0, 64, 1, 1, sage.SAGE_PV_FP16, 0.0)
+    assert sage.sage_get_device_status() == 0
+    assert not out.any()
+
+
+@pytest.mark.parametrize("pv", ["fp16", "fp8"])
+def test_varlen_kv_full_compare(pv):
+    H, d = 4, 128
+    lens_q = [1, 200, 128, 0, 333, 64]
+    lens_k = [700, 200, 1000, 50, 129, 1]
+    w = inputs.Workload("t", 97, 0, H, 0, d, True, 2.0, nseq=len(lens_q))
+    q, k, v, cq, ck = inputs.make_varlen_kv(w, lens_q, lens_k)
+    out = sage.sageattn_varlen_kv(q.cuda(), k.cuda(), v.cuda(), cq.cuda(), ck.cuda(), max(lens_q),
+                                  max(lens_k), True, True, PV[pv])
+    assert sage.sage_get_device_status() == 0
+    got = _np(out)
+    lq = oracle.Layout.packed(cq.tolist(), H, d)
+    lk = oracle.Layout.packed(ck.tolist(), H, d)
+    ref = oracle.sage_attention(q.numpy(), k.numpy(), v.numpy(), lq, True, True, PV[pv],
+                                kv_layout=lk)
+    assert_vs_oracle(got, ref, f"varlen kv {pv}")
+    exact = oracle.attn_fp64(q.numpy(), k.numpy(), v.numpy(), lq, True, 1 / math.sqrt(d),
+                             kv_layout=lk)
+    assert_vs_fp64(got, exact, pv == "fp8", f"varlen kv {pv}")
+
+
+def test_prefill_kv_config_sampled():
+    w = inputs.prefill_kv()
+    q, k, v = inputs.make_dense(w)
+    got = _run_dense(q, k, v, True, "fp16")
+    lq = oracle.Layout.dense(w.B, w.H, w.nq, w.d)
+    lk = oracle.Layout.dense(w.B, w.H, w.N, w.d)
+    qn, kn, vn = q.numpy(), k.numpy(), v.numpy()
+    for s, h in [(0, 0), (w.B - 1, w.H - 1)]:
+        for r0, r1 in _sample_rows(w.nq):
+            ref = oracle.sage_attention(qn, kn, vn, lq, True, True, oracle.PV_FP16, heads=[(s, h)],
+                                        rows=(r0, r1), kv_layout=lk)
+            exact = oracle.attn_fp64(qn, kn, vn, lq, True, 1 / math.sqrt(w.d), heads=[(s, h)],
+                                     rows=(r0, r1), kv_layout=lk)
+            mask = ~np.isnan(ref)
+            assert mask.sum() == (r1 - r0) * w.d
+            tag = f"prefill kv head {(s, h)} rows {r0}:{r1}"
+            assert_vs_oracle(got[mask], ref[mask], tag)
+            assert_vs_fp64(got[mask], exact[mask], False, tag)

@@ -169,3 +169,16 @@ def test_quant_v_fp8_smooth_varlen_bit_exact():
     assert np.array_equal(_np(scales), rs)
     assert np.array_equal(_np(codes), rc)
     assert sage.sage_get_device_status() == 0
+
+
+@pytest.mark.parametrize("Nq,Nk,d", [(1, 300, 128), (130, 1000, 64), (300, 100, 128)])
+def test_quant_qk_kv_bit_exact(Nq, Nk, d):
+    B, H = 2, 3
+    w = inputs.Workload("t", 51 + Nq, B, H, Nk, d, True, 2.0, nq=Nq)
+    q, k, _ = inputs.make_dense(w)
+    assert q.shape[2] == Nq and k.shape[2] == Nk
+    z = sage.quant_qk(q.cuda(), k.cuda(), True)
+    assert sage.sage_get_device_status() == 0
+    ref = oracle.quant_qk(q.numpy(), k.numpy(), oracle.Layout.dense(B, H, Nq, d), True,
+                          kv_layout=oracle.Layout.dense(B, H, Nk, d))
+    _check_qk(z, ref, f"kv {Nq}x{Nk}")

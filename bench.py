@@ -153,24 +153,28 @@ def _oracle_case(args):
         q, k, v, cu = inputs.make_varlen(w)
         lay = oracle.Layout.packed(cu.tolist(), w.H, w.d)
         W.update(varlen=True, lens=lay.lens)
+        kvl = lay
     else:
-        q, k, v = inputs.make_dense(w, B=1, N=W["N"])
-        lay = oracle.Layout.dense(1, w.H, W["N"], W["d"])
+        nq = W.get("Nq") or W["N"]
+        q, k, v = inputs.make_dense(w, B=1, N=W["N"], Nq=nq)
+        lay = oracle.Layout.dense(1, w.H, nq, W["d"])
+        kvl = oracle.Layout.dense(1, w.H, W["N"], W["d"])
     pv = oracle.PV_FP8 if W["pv_mode"] == "fp8" else oracle.PV_FP16
-    return W, q.numpy(), k.numpy(), v.numpy(), lay, pv
+    return W, q.numpy(), k.numpy(), v.numpy(), lay, pv, kvl
 
 
-def _sample_ops(r0: int, r1: int, n: int, d: int, causal: bool) -> float:
-    """Operations of query rows [r0, r1) of one head of length n (4 d per visible key)."""
+def _sample_ops(r0: int, r1: int, nq: int, nk: int, d: int, causal: bool) -> float:
+    """Operations of query rows [r0, r1) of one head with nq queries and nk keys (4 d per
+    visible key; the causal mask aligned at the bottom right)."""
     if not causal:
-        return 4.0 * (r1 - r0) * n * d
-    return 4.0 * d * sum(min(r + 1, n) for r in range(r0, r1))
+        return 4.0 * (r1 - r0) * nk * d
+    return 4.0 * d * sum(max(0, min(r + 1 + nk - nq, nk)) for r in range(r0, r1))
 
 
 def _oracle_sample(case, it: int, rows: int):
     """Run the oracle on `rows` query rows of one head; returns (seconds, ops, head)."""
     import oracle
-    W, q, k, v, lay, pv = case
+    W, q, k, v, lay, pv, kvl = case
     s = it % lay.nseq
     h = (it // lay.nseq) % lay.H
     n = lay.lens[s]
@@ -180,8 +184,9 @@ def _oracle_sample(case, it: int, rows: int):
     r1 = min(r0 + rows, n)
     t0 = time.perf_counter()
     oracle.sage_attention(q, k, v, lay, W["causal"], W["smooth_k"], pv,
-                          1.0 / math.sqrt(lay.d), heads=[(s, h)], rows=(r0, r1))
-    return time.perf_counter() - t0, _sample_ops(r0, r1, n, lay.d, W["causal"]), (s, h)
+                          1.0 / math.sqrt(lay.d), heads=[(s, h)], rows=(r0, r1), kv_layout=kvl)
+    return (time.perf_counter() - t0, _sample_ops(r0, r1, n, kvl.lens[s], lay.d, W["causal"]),
+            (s, h))
 
 
 def run_reference(args):
@@ -251,6 +256,8 @@ def _workload(args):
         w = inputs.video_dit()
     elif args.workload == "varlen":
         w = inputs.varlen()
+    elif args.workload == "prefill_kv":
+        w = inputs.prefill_kv()
     elif args.workload == "sweep":
         n = args.N or 16384
         w = inputs.sweep(n, args.d or 128, args.causal)
@@ -259,6 +266,8 @@ def _workload(args):
     if w is not None:
         W.update(B=w.B, H=w.H, N=w.N, d=w.d, causal=w.causal, pv_mode=w.pv_modes[0])
         W["gen"] = w
+        if w.nq:
+            W["Nq"] = w.nq
     for key in ("B", "N", "d"):
         if getattr(args, key) is not None and args.workload in ("headline", "sweep"):
             W[key] = getattr(args, key)
@@ -274,22 +283,9 @@ def _workload_name(W):
         return (f"packed varlen {len(W['lens'])} sequences (lengths {W['lens']}) H={W['H']} "
                 f"d={W['d']} {'causal' if W['causal'] else 'non-causal'} PV={W['pv_mode']} "
                 f"smooth_k")
-    return (f"B={W['B']} H={W['H']} N={W['N']} d={W['d']} "
+    nq = f" Nq={W['Nq']} Nk={W['N']}" if W.get("Nq") else ""
+    return (f"B={W['B']} H={W['H']} N={W['N']}{nq} d={W['d']} "
             f"{'causal' if W['causal'] else 'non-causal'} PV={W['pv_mode']} smooth_k")
-
-
-def _keep_pool_cached(device: int):
-    """Let the device's stream-ordered memory pool keep freed blocks (plumbing): the
-    library's own small scratch allocations then never go back to the driver between
-    steps."""
-    try:
-        from cuda.bindings import runtime as rt
-        err, pool = rt.cudaDeviceGetDefaultMemPool(device)
-        if err == rt.cudaError_t.cudaSuccess:
-            rt.cudaMemPoolSetAttribute(pool, rt.cudaMemPoolAttr.cudaMemPoolAttrReleaseThreshold,
-                                       rt.cuuint64_t(2 ** 64 - 1))
-    except Exception:
-        pass
 
 
 def run_ours(args):
@@ -299,7 +295,6 @@ def run_ours(args):
 
     world, rank, local = _dist()
     torch.cuda.set_device(local)
-    _keep_pool_cached(local)
     dist = None
     if world > 1:
         import torch.distributed as dist
@@ -310,8 +305,9 @@ def run_ours(args):
     if args.workload == "varlen":
         return run_varlen(args, W, dist, world, rank, local)
     B, H, N, d = W["B"], W["H"], W["N"], W["d"]
+    Nq = W.get("Nq") or N                  # queries per sequence (N keys)
     w = W.get("gen") or inputs.sweep(N, d, W["causal"])
-    qc, kc, vc = inputs.make_dense(w, B=B, N=N)
+    qc, kc, vc = inputs.make_dense(w, B=B, N=N, Nq=Nq)
     q, k, v = qc.cuda(), kc.cuda(), vc.cuda()
     pv = sage.SAGE_PV_FP16 if W["pv_mode"] == "fp16" else sage.SAGE_PV_FP8
     vq, vscale = v, None
@@ -320,7 +316,7 @@ def run_ours(args):
         vscale = torch.empty((B, H, d), dtype=torch.float32, device=v.device)
     sm_scale = 1.0 / math.sqrt(d)
     dev = q.device
-    nqb, nkb = math.ceil(N / 128), math.ceil(N / 64)
+    nqb, nkb = math.ceil(Nq / 128), math.ceil(N / 64)
     q_i8 = torch.empty(q.shape, dtype=torch.int8, device=dev)
     k_i8 = torch.empty(k.shape, dtype=torch.int8, device=dev)
     q_scale = torch.empty((B, H, nqb), dtype=torch.float32, device=dev)
@@ -330,16 +326,26 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
 
     ksum_ws = torch.empty(B * H * d * 8, dtype=torch.uint8, device=dev)   # fp64 K sums
+    vstat_ws = torch.empty(B * H * d * 16, dtype=torch.uint8, device=dev)  # V column statistics
 
     def quant():
-        sage.sage_quant_qk_ws(q, k, q_i8, q_scale, k_i8, k_scale, k_mean, B, H, N, d,
-                              W["smooth_k"], ksum_ws, ksum_ws.numel(), stream)
+        if Nq == N:
+            sage.sage_quant_qk_ws(q, k, q_i8, q_scale, k_i8, k_scale, k_mean, B, H, N, d,
+                                  W["smooth_k"], ksum_ws, ksum_ws.numel(), stream)
+        else:
+            sage.sage_quant_qk_kv(q, k, q_i8, q_scale, k_i8, k_scale, k_mean, B, H, Nq, N, d,
+                                  W["smooth_k"], ksum_ws, ksum_ws.numel(), stream)
         if pv == sage.SAGE_PV_FP8:
-            sage.sage_quant_v_fp8(v, vq, vscale, B, H, N, d, stream)
+            sage.sage_quant_v_fp8_ws(v, vq, vscale, None, B, H, N, d, vstat_ws, vstat_ws.numel(),
+                                     stream)
 
     def attend():
-        sage.sage_attn_fwd_quantized(q_i8, q_scale, k_i8, k_scale, vq, vscale, out, B, H, N, d,
-                                     W["causal"], pv, sm_scale, stream)
+        if Nq == N:
+            sage.sage_attn_fwd_quantized(q_i8, q_scale, k_i8, k_scale, vq, vscale, out, B, H, N,
+                                         d, W["causal"], pv, sm_scale, stream)
+        else:
+            sage.sage_attn_fwd_quantized_kv(q_i8, q_scale, k_i8, k_scale, vq, vscale, None, out,
+                                            B, H, Nq, N, d, W["causal"], pv, sm_scale, stream)
 
     def step():
         quant()
@@ -386,7 +392,8 @@ def run_ours(args):
     quant_ms = [e0.elapsed_time(e1) for (e0, e1, _) in ev]
     total_ms = max_over_ranks(total_ms, dist, dev)
 
-    ops = _ops(B, H, N, d, W["causal"])
+    ops = (_ops(B, H, N, d, W["causal"]) if Nq == N
+           else inputs.attention_ops_kv(B, H, Nq, N, d, W["causal"]))
     ms_per_step = total_ms / args.steps
     value = weak_scaling_tops(ops, args.steps, world, total_ms)
     attn_avg_ms = sum(attn_ms) / len(attn_ms)
@@ -396,14 +403,19 @@ def run_ours(args):
     e2e_steps = 0 if args.no_e2e else max(3, args.steps // 4)
     qh, kh, vh = (t.pin_memory() for t in (qc, kc, vc))
     oh = torch.empty_like(qc).pin_memory()
-    qd, kd, vd, od = (torch.empty_like(q) for _ in range(4))
+    qd, od = torch.empty_like(q), torch.empty_like(q)
+    kd, vd = torch.empty_like(k), torch.empty_like(v)
 
     def e2e_step():
         qd.copy_(qh, non_blocking=True)
         kd.copy_(kh, non_blocking=True)
         vd.copy_(vh, non_blocking=True)
-        sage.sage_attn_fwd(qd, kd, vd, od, B, H, N, d, W["causal"], W["smooth_k"], pv, sm_scale,
-                           stream)
+        if Nq == N:
+            sage.sage_attn_fwd(qd, kd, vd, od, B, H, N, d, W["causal"], W["smooth_k"], pv,
+                               sm_scale, stream)
+        else:
+            sage.sage_attn_fwd_kv(qd, kd, vd, od, B, H, Nq, N, d, W["causal"], W["smooth_k"], pv,
+                                  sm_scale, None, 0, stream)
         oh.copy_(od, non_blocking=True)
 
     if e2e_steps:
@@ -424,7 +436,8 @@ def run_ours(args):
     if status != 0:
         raise RuntimeError(f"device status after e2e: {sage.status_string(status)}")
     e2e_value = weak_scaling_tops(ops, e2e_steps, world, e2e_ms) if e2e_steps else None
-    elem_bytes = B * H * N * d * 2
+    elem_bytes = B * H * N * d * 2         # one K or V tensor
+    q_bytes = B * H * Nq * d * 2           # Q or O
 
     peaks, src = _peaks()
     bf16 = peaks["bf16_tflops_sustained"]
@@ -459,12 +472,13 @@ def run_ours(args):
                                     "sequence-length sweep point") + " " + _workload_name(W) +
                                    " (per GPU)",
                        "B": B, "H": H, "N": N, "d": d, "causal": W["causal"],
+                       **({"Nq": Nq, "Nk": N} if Nq != N else {}),
                        "pv_mode": W["pv_mode"], "smooth_k": W["smooth_k"],
                        "parallelism": f"replicas x{world}",
                        "l2": _l2_note(elem_bytes)},
             "roofline": roofline,
             "e2e": {"value": e2e_value, "unit": "TOPS",
-                    "h2d_bytes_per_step": 3 * elem_bytes, "d2h_bytes_per_step": elem_bytes,
+                    "h2d_bytes_per_step": q_bytes + 2 * elem_bytes, "d2h_bytes_per_step": q_bytes,
                     "steps": e2e_steps},
             "gpu_launches": (3 if pv == sage.SAGE_PV_FP16 else 5) * args.steps,
             "clocks": clocks.summary(),
@@ -612,7 +626,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="headline",
-                    choices=["headline", "llm_prefill", "video_dit", "sweep", "varlen"],
+                    choices=["headline", "llm_prefill", "video_dit", "sweep", "varlen",
+                             "prefill_kv"],
                     help="headline: B2 H32 N16384 d128 non-causal FP16 PV (the metric's point)")
     ap.add_argument("--ref-rows", type=int, default=64)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

@@ -29,6 +29,10 @@
  *   - Head dim d is 64 or 128. sm_scale <= 0 selects 1/sqrt(d). causal is the square
  *     mask j <= i within each sequence.
  *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *   - "Stream-ordered allocation": scratch taken with cudaMallocFromPoolAsync from a
+ *     memory pool the library creates once per device and never trims (it keeps the
+ *     largest working set it has seen), released with cudaFreeAsync on the same stream.
+ *     Callers that must not allocate use the *_ws entry points or sage_attn_fwd_noalloc.
  *     Nothing synchronizes except sage_get_device_status().
  *   - Host-detectable argument errors return before anything is enqueued. Errors that
  *     only the device can see (a bounded wait that timed out, malformed cu_seqlens) set
@@ -104,7 +108,7 @@ SAGE_API size_t sage_workspace_size_kv(int nseq, int H, int max_seqlen_q, int ma
  * for |K| N < 2^29) and rounded once to fp32; codes are round-half-even of the fp32
  * quotient x/scale clamped to [-127, 127]; an all-zero block has scale 0 and codes 0.
  * Outputs are caller-owned device buffers of the shapes in the conventions above.
- * Uses a small stream-ordered allocation (cudaMallocAsync) for the fp64 sums.
+ * Uses a small stream-ordered allocation for the fp64 sums.
  */
 SAGE_API sage_status_t sage_quant_qk(const void *q, const void *k, int8_t *q_i8, float *q_scale,
                             int8_t *k_i8, float *k_scale, float *k_mean, int B, int H, int N,
@@ -126,11 +130,13 @@ SAGE_API sage_status_t sage_quant_qk_varlen(const void *q, const void *k, const 
 
 /* sage_quant_qk for Q [B,H,Nq,d] and K [B,H,Nk,d] of different lengths: q_scale is
  * [B,H,ceil(Nq/128)], k_scale [B,H,ceil(Nk/64)], and the K mean is taken over the Nk
- * keys. */
+ * keys. workspace: NULL (a stream-ordered allocation for the fp64 K sums) or caller
+ * scratch of at least B*H*d*8 bytes, 16-byte aligned. */
 SAGE_API sage_status_t sage_quant_qk_kv(const void *q, const void *k, int8_t *q_i8,
                                         float *q_scale, int8_t *k_i8, float *k_scale,
                                         float *k_mean, int B, int H, int Nq, int Nk, int d,
-                                        int smooth_k, sage_stream_t stream);
+                                        int smooth_k, void *workspace, size_t ws_bytes,
+                                        sage_stream_t stream);
 
 /*
  * V to FP8 E4M3 (「4比特量化三倍加速不掉点！清华即插即用的SageAttention迎来升级」, 技术方案 (4)) with one fp32 scale per
@@ -142,6 +148,14 @@ SAGE_API sage_status_t sage_quant_v_fp8(const void *v, uint8_t *v_e4m3, float *v
 SAGE_API sage_status_t sage_quant_v_fp8_varlen(const void *v, const int32_t *cu_seqlens, int nseq,
                                       int total_tokens, int max_seqlen, int H, int d,
                                       uint8_t *v_e4m3, float *v_scale, sage_stream_t stream);
+
+/* sage_quant_v_fp8 (v_mean == NULL) or sage_quant_v_fp8_smooth (v_mean != NULL) with
+ * caller-owned scratch for the column statistics: at least B*H*d*16 bytes, 16-byte
+ * aligned. Allocates nothing. */
+SAGE_API sage_status_t sage_quant_v_fp8_ws(const void *v, uint8_t *v_e4m3, float *v_scale,
+                                           float *v_mean, int B, int H, int N, int d,
+                                           void *workspace, size_t ws_bytes,
+                                           sage_stream_t stream);
 
 /*
  * Smooth V, then V to E4M3 (the SAGE_SMOOTH_V step on its own): v_mean [B,H,d] fp32 =
@@ -161,8 +175,7 @@ SAGE_API sage_status_t sage_quant_v_fp8_smooth_varlen(const void *v, const int32
 
 /*
  * The whole forward pass (steps 1-3), dense layout: out[B,H,N,d] fp16. pv_mode selects
- * SAGE_PV_FP16 or SAGE_PV_FP8. Scratch comes from stream-ordered allocation
- * (cudaMallocAsync/cudaFreeAsync on `stream`).
+ * SAGE_PV_FP16 or SAGE_PV_FP8. Scratch comes from stream-ordered allocation on `stream`.
  */
 SAGE_API sage_status_t sage_attn_fwd(const void *q, const void *k, const void *v, void *out, int B,
                             int H, int N, int d, int causal, int smooth_k, int pv_mode,

@@ -46,7 +46,7 @@ _S = ctypes.c_int  # sage_status_t
 SIGNATURES = {
     "sage_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
     "sage_workspace_size_kv": (_Z, [_I, _I, _I, _I, _I, _I, _I, _I]),
-    "sage_quant_qk_kv": (_S, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P]),
+    "sage_quant_qk_kv": (_S, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _Z, _P]),
     "sage_attn_fwd_kv": (_S, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
     "sage_attn_varlen_fwd_kv": (_S, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I,
                                      _I, _F, _P, _Z, _P]),
@@ -58,6 +58,7 @@ SIGNATURES = {
     "sage_quant_v_fp8": (_S, [_P, _P, _P, _I, _I, _I, _I, _P]),
     "sage_quant_v_fp8_varlen": (_S, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
     "sage_quant_v_fp8_smooth": (_S, [_P, _P, _P, _P, _I, _I, _I, _I, _P]),
+    "sage_quant_v_fp8_ws": (_S, [_P, _P, _P, _P, _I, _I, _I, _I, _P, _Z, _P]),
     "sage_quant_v_fp8_smooth_varlen": (_S, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P]),
     "sage_attn_fwd": (_S, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P]),
     "sage_attn_fwd_ws": (_S, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
@@ -145,9 +146,10 @@ def sage_workspace_size_kv(nseq, H, max_seqlen_q, max_seqlen_k, total_q, total_k
 
 
 def sage_quant_qk_kv(q, k, q_i8, q_scale, k_i8, k_scale, k_mean, B, H, Nq, Nk, d, smooth_k,
-                     stream=None):
+                     workspace=None, ws_bytes=0, stream=None):
     return _call("sage_quant_qk_kv", _ptr(q), _ptr(k), _ptr(q_i8), _ptr(q_scale), _ptr(k_i8),
-                 _ptr(k_scale), _ptr(k_mean), B, H, Nq, Nk, d, int(smooth_k), _stream(stream))
+                 _ptr(k_scale), _ptr(k_mean), B, H, Nq, Nk, d, int(smooth_k), _ptr(workspace),
+                 int(ws_bytes), _stream(stream))
 
 
 def sage_attn_fwd_kv(q, k, v, out, B, H, Nq, Nk, d, causal, smooth_k, pv_mode, sm_scale,
@@ -201,6 +203,12 @@ def sage_quant_v_fp8_varlen(v, cu_seqlens, nseq, total_tokens, max_seqlen, H, d,
                             v_scale, stream=None):
     return _call("sage_quant_v_fp8_varlen", _ptr(v), _ptr(cu_seqlens), nseq, total_tokens,
                  max_seqlen, H, d, _ptr(v_e4m3), _ptr(v_scale), _stream(stream))
+
+
+def sage_quant_v_fp8_ws(v, v_e4m3, v_scale, v_mean, B, H, N, d, workspace, ws_bytes,
+                        stream=None):
+    return _call("sage_quant_v_fp8_ws", _ptr(v), _ptr(v_e4m3), _ptr(v_scale), _ptr(v_mean), B, H,
+                 N, d, _ptr(workspace), int(ws_bytes), _stream(stream))
 
 
 def sage_quant_v_fp8_smooth(v, v_e4m3, v_scale, v_mean, B, H, N, d, stream=None):
@@ -360,7 +368,7 @@ def quant_qk(q, k, smooth_k: bool = True, stream=None):
                       d, smooth_k, stream)
     else:
         sage_quant_qk_kv(q, k, z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], z["k_mean"], B,
-                         H, N, Nk, d, smooth_k, stream)
+                         H, N, Nk, d, smooth_k, None, 0, stream)
     return z
 
 

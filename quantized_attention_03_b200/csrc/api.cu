@@ -53,6 +53,42 @@ int *status_ptr(sage_status_t *err)
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Stream-ordered scratch comes from one memory pool per device that the library creates
+// and never trims (release threshold = all), so that after the first calls an
+// allocation is bookkeeping only and never waits for memory to be mapped again.
+cudaMemPool_t g_pool[64] = {};
+
+cudaError_t scratch_alloc(void **p, size_t bytes, cudaStream_t st)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (dev < 0 || dev >= 64)
+        return cudaErrorInvalidDevice;
+    {
+        std::lock_guard<std::mutex> lk(g_mu);
+        if (g_pool[dev] == nullptr) {
+            cudaMemPoolProps props = {};
+            props.allocType = cudaMemAllocationTypePinned;
+            props.handleTypes = cudaMemHandleTypeNone;
+            props.location.type = cudaMemLocationTypeDevice;
+            props.location.id = dev;
+            cudaMemPool_t pool = nullptr;
+            if ((e = cudaMemPoolCreate(&pool, &props)) != cudaSuccess)
+                return e;
+            uint64_t keep = ~0ull;
+            if ((e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep)) !=
+                cudaSuccess) {
+                cudaMemPoolDestroy(pool);
+                return e;
+            }
+            g_pool[dev] = pool;
+        }
+    }
+    return cudaMallocFromPoolAsync(p, bytes ? bytes : 256, g_pool[dev], st);
+}
+
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Scratch carved from one buffer, every part 256-byte aligned.
@@ -170,7 +206,7 @@ sage_status_t forward(const void *q, const void *k, const void *v, void *out, co
 sage_status_t alloc_ws(size_t bytes, cudaStream_t st, char **p)
 {
     void *ptr = nullptr;
-    cudaError_t e = cudaMallocAsync(&ptr, bytes ? bytes : 256, st);
+    cudaError_t e = scratch_alloc(&ptr, bytes, st);
     if (e != cudaSuccess)
         return cuda_fail(e);
     *p = static_cast<char *>(ptr);
@@ -220,7 +256,8 @@ sage_status_t quant_qk_entry(const void *q, const void *k, const Shape &sh, int8
                              int smooth_k, void *workspace, size_t ws_bytes, cudaStream_t st);
 sage_status_t quant_v_entry(const void *v, const int32_t *cu_seqlens, int nseq, int total_tokens,
                             int max_seqlen, int H, int d, uint8_t *v_e4m3, float *v_scale,
-                            float *v_mean, bool smooth, cudaStream_t st);
+                            float *v_mean, bool smooth, void *workspace, size_t ws_bytes,
+                            cudaStream_t st);
 
 // Step 3 alone on pre-quantized operands (dense; Nq queries, Nk keys).
 sage_status_t quantized_entry(const int8_t *q_i8, const float *q_scale, const int8_t *k_i8,
@@ -291,12 +328,14 @@ sage_status_t sage_quant_qk(const void *q, const void *k, int8_t *q_i8, float *q
 
 sage_status_t sage_quant_qk_kv(const void *q, const void *k, int8_t *q_i8, float *q_scale,
                                int8_t *k_i8, float *k_scale, float *k_mean, int B, int H, int Nq,
-                               int Nk, int d, int smooth_k, sage_stream_t stream)
+                               int Nk, int d, int smooth_k, void *workspace, size_t ws_bytes,
+                               sage_stream_t stream)
 {
     if (!dense_fits(B, Nq) || !dense_fits(B, Nk))
         return SAGE_ERR_UNSUPPORTED;
     return quant_qk_entry(q, k, dense_shape(B, H, Nq, Nk, d), q_i8, q_scale, k_i8, k_scale,
-                          k_mean, smooth_k, nullptr, 0, reinterpret_cast<cudaStream_t>(stream));
+                          k_mean, smooth_k, workspace, ws_bytes,
+                          reinterpret_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"
@@ -338,7 +377,7 @@ sage_status_t quant_qk_entry(const void *q, const void *k, const Shape &sh, int8
             ksum = static_cast<double *>(workspace);
         } else {
             void *p = nullptr;
-            if ((e = cudaMallocAsync(&p, sum_bytes, st)) != cudaSuccess)
+            if ((e = scratch_alloc(&p, sum_bytes, st)) != cudaSuccess)
                 return cuda_fail(e);
             ksum = static_cast<double *>(p);
             owned = true;
@@ -363,10 +402,13 @@ sage_status_t quant_qk_entry(const void *q, const void *k, const Shape &sh, int8
     return e == cudaSuccess ? SAGE_OK : cuda_fail(e);
 }
 
-// V to E4M3 (smooth: V - mean(V) first, the mean written to v_mean), dense or packed.
+// V to E4M3 (smooth: V - mean(V) first, the mean written to v_mean), dense or packed,
+// with caller scratch for the column statistics or (workspace == nullptr) a
+// stream-ordered allocation.
 sage_status_t quant_v_entry(const void *v, const int32_t *cu_seqlens, int nseq, int total_tokens,
                             int max_seqlen, int H, int d, uint8_t *v_e4m3, float *v_scale,
-                            float *v_mean, bool smooth, cudaStream_t st)
+                            float *v_mean, bool smooth, void *workspace, size_t ws_bytes,
+                            cudaStream_t st)
 {
     sage_status_t r = check_shape(nseq, H, max_seqlen, d);
     if (r != SAGE_OK)
@@ -377,17 +419,23 @@ sage_status_t quant_v_entry(const void *v, const int32_t *cu_seqlens, int nseq, 
         return SAGE_ERR_INVALID_ARG;
     if (!aligned16(v) || !aligned16(v_e4m3))
         return SAGE_ERR_MISALIGNED;
+    // [vsum (fp64) | vhi | vneg] per (sequence, head, channel)
+    const size_t n = (size_t)nseq * H * d;
+    const size_t bytes = n * (8 + 4 + 4);
+    if (workspace != nullptr) {
+        if (ws_bytes < bytes)
+            return SAGE_ERR_WORKSPACE;
+        if ((reinterpret_cast<uintptr_t>(workspace) & 15u) != 0)
+            return SAGE_ERR_MISALIGNED;
+    }
     int *status = status_ptr(&r);
     if (!status)
         return r;
     const SeqLayout L = cu_seqlens ? SeqLayout::packed(cu_seqlens, nseq, total_tokens, max_seqlen, H, d)
                                    : SeqLayout::dense(nseq, H, max_seqlen, d);
-    // [vsum (fp64) | vhi | vneg] per (sequence, head, channel)
-    const size_t n = (size_t)nseq * H * d;
-    const size_t bytes = n * (8 + 4 + 4);
-    void *p = nullptr;
+    void *p = workspace;
     cudaError_t e;
-    if ((e = cudaMallocAsync(&p, bytes, st)) != cudaSuccess)
+    if (p == nullptr && (e = scratch_alloc(&p, bytes, st)) != cudaSuccess)
         return cuda_fail(e);
     ColStats cs;
     cs.vsum = smooth ? static_cast<double *>(p) : nullptr;
@@ -399,7 +447,8 @@ sage_status_t quant_v_entry(const void *v, const int32_t *cu_seqlens, int nseq, 
         e = launch_quant(nullptr, nullptr, static_cast<const __half *>(v), cs, nullptr, nullptr,
                          nullptr, nullptr, nullptr, v_e4m3, v_scale, smooth ? v_mean : nullptr,
                          L, L, status, st);
-    cudaFreeAsync(p, st);
+    if (workspace == nullptr)
+        cudaFreeAsync(p, st);
     return e == cudaSuccess ? SAGE_OK : cuda_fail(e);
 }
 }  // namespace
@@ -437,7 +486,7 @@ sage_status_t sage_quant_v_fp8_smooth_varlen(const void *v, const int32_t *cu_se
                                              sage_stream_t stream)
 {
     return quant_v_entry(v, cu_seqlens, nseq, total_tokens, max_seqlen, H, d, v_e4m3, v_scale,
-                         v_mean, true, reinterpret_cast<cudaStream_t>(stream));
+                         v_mean, true, nullptr, 0, reinterpret_cast<cudaStream_t>(stream));
 }
 
 sage_status_t sage_quant_v_fp8_smooth(const void *v, uint8_t *v_e4m3, float *v_scale,
@@ -446,8 +495,8 @@ sage_status_t sage_quant_v_fp8_smooth(const void *v, uint8_t *v_e4m3, float *v_s
 {
     if (B > 0 && N > 0 && (int64_t)B * N > INT32_MAX)
         return SAGE_ERR_UNSUPPORTED;
-    return quant_v_entry(v, nullptr, B, B * N, N, H, d, v_e4m3, v_scale, v_mean, true,
-                         reinterpret_cast<cudaStream_t>(stream));
+    return quant_v_entry(v, nullptr, B, B * N, N, H, d, v_e4m3, v_scale, v_mean, true, nullptr,
+                         0, reinterpret_cast<cudaStream_t>(stream));
 }
 
 sage_status_t sage_quant_v_fp8_varlen(const void *v, const int32_t *cu_seqlens, int nseq,
@@ -455,7 +504,7 @@ sage_status_t sage_quant_v_fp8_varlen(const void *v, const int32_t *cu_seqlens, 
                                       uint8_t *v_e4m3, float *v_scale, sage_stream_t stream)
 {
     return quant_v_entry(v, cu_seqlens, nseq, total_tokens, max_seqlen, H, d, v_e4m3, v_scale,
-                         nullptr, false, reinterpret_cast<cudaStream_t>(stream));
+                         nullptr, false, nullptr, 0, reinterpret_cast<cudaStream_t>(stream));
 }
 
 sage_status_t sage_quant_v_fp8(const void *v, uint8_t *v_e4m3, float *v_scale, int B, int H,
@@ -463,7 +512,20 @@ sage_status_t sage_quant_v_fp8(const void *v, uint8_t *v_e4m3, float *v_scale, i
 {
     if (B > 0 && N > 0 && (int64_t)B * N > INT32_MAX)
         return SAGE_ERR_UNSUPPORTED;
-    return quant_v_entry(v, nullptr, B, B * N, N, H, d, v_e4m3, v_scale, nullptr, false,
+    return quant_v_entry(v, nullptr, B, B * N, N, H, d, v_e4m3, v_scale, nullptr, false, nullptr,
+                         0, reinterpret_cast<cudaStream_t>(stream));
+}
+
+sage_status_t sage_quant_v_fp8_ws(const void *v, uint8_t *v_e4m3, float *v_scale, float *v_mean,
+                                  int B, int H, int N, int d, void *workspace, size_t ws_bytes,
+                                  sage_stream_t stream)
+{
+    if (workspace == nullptr && !(B == 0 || H == 0 || N == 0))
+        return SAGE_ERR_WORKSPACE;
+    if (!dense_fits(B, N))
+        return SAGE_ERR_UNSUPPORTED;
+    return quant_v_entry(v, nullptr, B, B * N, N, H, d, v_e4m3, v_scale, v_mean,
+                         v_mean != nullptr, workspace, ws_bytes,
                          reinterpret_cast<cudaStream_t>(stream));
 }
 

@@ -182,3 +182,21 @@ def test_quant_qk_kv_bit_exact(Nq, Nk, d):
     ref = oracle.quant_qk(q.numpy(), k.numpy(), oracle.Layout.dense(B, H, Nq, d), True,
                           kv_layout=oracle.Layout.dense(B, H, Nk, d))
     _check_qk(z, ref, f"kv {Nq}x{Nk}")
+
+
+def test_quant_v_fp8_ws_matches_allocating_entries():
+    B, H, N, d = 2, 3, 500, 128
+    v = _v_with_offsets(B, H, N, d, 61).cuda()
+    ws = torch.empty(B * H * d * 16, dtype=torch.uint8, device="cuda")
+    for smooth in (False, True):
+        ref = sage.quant_v_fp8(v, smooth_v=smooth)
+        codes = torch.empty_like(ref[0])
+        scales = torch.empty_like(ref[1])
+        mean = torch.empty_like(ref[1]) if smooth else None
+        sage.sage_quant_v_fp8_ws(v, codes, scales, mean, B, H, N, d, ws, ws.numel())
+        assert sage.sage_get_device_status() == 0
+        assert torch.equal(codes, ref[0]) and torch.equal(scales, ref[1])
+        if smooth:
+            assert torch.equal(mean, ref[2])
+    with pytest.raises(sage.SageError):
+        sage.sage_quant_v_fp8_ws(v, codes, scales, None, B, H, N, d, ws, ws.numel() - 16)

@@ -29,6 +29,8 @@ from . import build as _build
 
 Q_BLOCK = 128   # Q tokens per INT8 scale block
 K_BLOCK = 64    # K tokens per INT8 scale block
+Q_FINE = 1      # finer groups: one Q scale per token ...
+K_FINE = 32     # ... and one K scale per 32 tokens
 PV_FP16 = 0
 PV_FP8 = 1
 
@@ -48,7 +50,7 @@ def lib():
         L.oracle_head_quant_int8.argtypes = [P, P, i64, i64, i32, i32, P, P]
         L.oracle_head_quant_v_fp8.argtypes = [P, P, i64, i64, i32, P, P]
         L.oracle_head_attn_quant.argtypes = [P, P, P, P, P, P, P, i64, i64, i64, i32, i32, i32,
-                                             f64, i32, i64, i64, P]
+                                             f64, i32, i32, i32, i64, i64, P]
         L.oracle_head_attn_fp64.argtypes = [P, P, P, i64, i64, i64, i32, i32, f64, i64, i64, P]
         L.oracle_f16_to_f64.argtypes = [ctypes.c_uint16]
         L.oracle_f16_to_f64.restype = f64
@@ -170,15 +172,16 @@ def quant_int8(x: np.ndarray, layout: Layout, blk: int, mu: Optional[np.ndarray]
 
 
 def quant_qk(q: np.ndarray, k: np.ndarray, layout: Layout, smooth_k: bool = True, heads=None,
-             kv_layout: Optional[Layout] = None):
+             kv_layout: Optional[Layout] = None, fine: bool = False):
     """Smooth K, then per-block INT8 of Q (128 tokens) and K (64 tokens), for every (or
-    each selected) head. ``kv_layout`` places K when it has its own lengths (default:
-    the layout of Q)."""
+    each selected) head; with ``fine``, one Q scale per token and one K scale per 32
+    tokens. ``kv_layout`` places K when it has its own lengths (default: Q's layout)."""
     kvl = layout if kv_layout is None else kv_layout
     zeros = np.zeros((kvl.nseq, kvl.H, kvl.d), np.float32)
     mu = k_mean(k, kvl, heads) if smooth_k else zeros
-    q_i8, q_scale = quant_int8(q, layout, Q_BLOCK, None, heads)
-    k_i8, k_scale = quant_int8(k, kvl, K_BLOCK, mu if smooth_k else None, heads)
+    q_i8, q_scale = quant_int8(q, layout, Q_FINE if fine else Q_BLOCK, None, heads)
+    k_i8, k_scale = quant_int8(k, kvl, K_FINE if fine else K_BLOCK, mu if smooth_k else None,
+                               heads)
     return dict(q_i8=q_i8, q_scale=q_scale, k_i8=k_i8, k_scale=k_scale, k_mean=mu)
 
 
@@ -200,8 +203,9 @@ def attn_quant(q_i8, q_scale, k_i8, k_scale, v, v_scale, layout: Layout, causal:
                pv_mode: int, sm_scale: float, tile_n: int = 128, heads=None,
                rows: Optional[Tuple[int, int]] = None,
                v_mean: Optional[np.ndarray] = None,
-               kv_layout: Optional[Layout] = None) -> np.ndarray:
+               kv_layout: Optional[Layout] = None, fine: bool = False) -> np.ndarray:
     """Quantized attention from codes and scales; fp16 output, NaN where not computed.
+    ``fine``: the scales are per Q token and per 32 K tokens (quant_qk(fine=True)).
 
     ``v`` is fp16 V (FP16 mode) or its E4M3 codes as uint8 (FP8 mode); ``v_mean``
     [nseq, H, d] (FP8 mode, smooth V) is added to every output row. ``kv_layout`` places
@@ -224,7 +228,9 @@ def attn_quant(q_i8, q_scale, k_i8, k_scale, v, v_scale, layout: Layout, causal:
         lib().oracle_head_attn_quant(_ptr(q_i8, off), _ptr(q_scale, sh * nqb), _ptr(k_i8, koff),
                                      _ptr(k_scale, sh * nkb), _ptr(vv, koff), vsp, vmp, n, nk,
                                      layout.stride, layout.d, int(causal), int(pv_mode),
-                                     float(sm_scale), int(tile_n), r0, r1, _ptr(ob, off))
+                                     float(sm_scale), int(tile_n),
+                                     Q_FINE if fine else Q_BLOCK, K_FINE if fine else K_BLOCK,
+                                     r0, r1, _ptr(ob, off))
     return out
 
 
@@ -254,19 +260,20 @@ def default_sm_scale(d: int, sm_scale: Optional[float] = None) -> float:
 def sage_attention(q, k, v, layout: Layout, causal: bool = False, smooth_k: bool = True,
                    pv_mode: int = PV_FP16, sm_scale: Optional[float] = None,
                    tile_n: int = 128, heads=None, rows=None,
-                   smooth_v: bool = False, kv_layout: Optional[Layout] = None) -> np.ndarray:
+                   smooth_v: bool = False, kv_layout: Optional[Layout] = None,
+                   fine: bool = False) -> np.ndarray:
     """The whole method from fp16 Q, K, V: smooth K (and, in FP8 mode, optionally V),
     quantize, quantized attention. ``kv_layout`` places K and V when their lengths differ
-    from Q's."""
+    from Q's; ``fine`` selects per-token Q and per-32-token K scales."""
     if smooth_v and pv_mode != PV_FP8:
         raise ValueError("smooth V applies to the FP8 P.V mode")
     kvl = layout if kv_layout is None else kv_layout
     sm = default_sm_scale(layout.d, sm_scale)
-    z = quant_qk(q, k, layout, smooth_k, heads, kvl)
+    z = quant_qk(q, k, layout, smooth_k, heads, kvl, fine)
     if pv_mode == PV_FP8:
         vm = channel_mean(v, kvl, heads) if smooth_v else None
         v8, vs = quant_v_fp8(v, kvl, heads, vm)
         return attn_quant(z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], v8, vs, layout,
-                          causal, PV_FP8, sm, tile_n, heads, rows, vm, kvl)
+                          causal, PV_FP8, sm, tile_n, heads, rows, vm, kvl, fine)
     return attn_quant(z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], v, None, layout,
-                      causal, PV_FP16, sm, tile_n, heads, rows, None, kvl)
+                      causal, PV_FP16, sm, tile_n, heads, rows, None, kvl, fine)

@@ -250,7 +250,9 @@ enum { ORACLE_PV_FP16 = 0, ORACLE_PV_FP8 = 1 };
  * longer sequence, e.g. prefill against cached keys), following the method's steps in
  * order:
  *   S_int[i,j] = sum_c q[i,c] k[j,c] in integers (INT32 range is never exceeded);
- *   t[i,j] = S_int * sq[i/128] * sk[j/64] * sm_scale * log2(e)  (base-2 logits);
+ *   t[i,j] = S_int * sq[i/qg] * sk[j/kg] * sm_scale * log2(e)  (base-2 logits), where
+ *   qg and kg are the tokens per Q and K scale (128 and 64 for per-block scales, 1 and
+ *   32 for the finer groups);
  *   causal: key j is visible to query i when j <= i + (nk - nq) (the mask aligned at
  *   the bottom-right corner; the square mask j <= i when nq = nk); a query that sees no
  *   key (only when nq > nk) gets a zero output row;
@@ -267,8 +269,8 @@ enum { ORACLE_PV_FP16 = 0, ORACLE_PV_FP8 = 1 };
 void oracle_head_attn_quant(const int8_t *qc, const float *qs, const int8_t *kc,
                             const float *ks, const void *v, const float *vs, const float *vm,
                             int64_t nq, int64_t nk, int64_t stride, int d, int causal,
-                            int pv_mode, double sm_scale, int tile_n, int64_t r0, int64_t r1,
-                            uint16_t *out)
+                            int pv_mode, double sm_scale, int tile_n, int qg, int kg,
+                            int64_t r0, int64_t r1, uint16_t *out)
 {
     const double log2e = 1.4426950408889634073599246810019;   /* 1/ln 2 */
     if (r1 > nq)
@@ -295,7 +297,7 @@ void oracle_head_attn_quant(const int8_t *qc, const float *qs, const int8_t *kc,
                 int32_t S = 0;
                 for (int c = 0; c < d; c++)
                     S += (int32_t)qc[i * stride + c] * (int32_t)kc[j * stride + c];
-                t[j - j0] = (double)S * (double)qs[i / 128] * (double)ks[j / 64] * sm_scale * log2e;
+                t[j - j0] = (double)S * (double)qs[i / qg] * (double)ks[j / kg] * sm_scale * log2e;
                 if (t[j - j0] > tmax)
                     tmax = t[j - j0];
             }

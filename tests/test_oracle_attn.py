@@ -417,3 +417,55 @@ def test_varlen_kv_equals_per_sequence_dense():
         od = oracle.sage_attention(dq, dk, dv, Layout.dense(1, H, lq[s], d), True, True,
                                    PV_FP16, 0.2, kv_layout=Layout.dense(1, H, lk[s], d))
         assert np.array_equal(o[sq].transpose(1, 0, 2), od[0])
+
+
+# Finer scale groups ([SA2] 技术方案 (2), restated for this tensor-core layout: one Q
+# scale per query row and one K scale per 32 keys).
+
+@pytest.mark.parametrize("pv_mode", [PV_FP16, PV_FP8])
+def test_fine_single_tile_equals_plain_softmax(pv_mode):
+    N, d = 200, 32
+    q, k, v = (_rand16((1, 1, N, d), s) for s in (211, 212, 213))
+    lay = Layout.dense(1, 1, N, d)
+    sm = 1 / math.sqrt(d)
+    z = oracle.quant_qk(q, k, lay, True, fine=True)
+    if pv_mode == PV_FP8:
+        vq, vs = oracle.quant_v_fp8(v, lay)
+    else:
+        vq, vs = v, None
+    got = oracle.attn_quant(z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], vq, vs, lay, False,
+                            pv_mode, sm, tile_n=256, fine=True)
+    # closed form with the scales expanded per row and per 32 keys
+    qc = z["q_i8"][0, 0].astype(np.int64)
+    kc = z["k_i8"][0, 0].astype(np.int64)
+    S = qc @ kc.T
+    t = (S * z["q_scale"][0, 0][:, None].astype(np.float64)
+         * z["k_scale"][0, 0][np.arange(N) // 32][None, :].astype(np.float64) * sm / math.log(2))
+    p = np.exp2(t - t.max(axis=1, keepdims=True))
+    if pv_mode == PV_FP16:
+        O = p.astype(np.float16).astype(np.float64) @ vq[0, 0].astype(np.float64) / p.sum(1, keepdims=True)
+    else:
+        P = torch.from_numpy(448 * p).to(torch.float32).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+        vv = torch.from_numpy(vq[0, 0]).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+        O = P @ vv * vs[0, 0][None, :] / (448 * p.sum(1, keepdims=True))
+    ref = O.astype(np.float16).astype(np.float64)
+    diff = np.abs(got[0, 0].astype(np.float64) - ref)
+    assert diff.max() <= 2 * np.spacing(np.abs(ref).astype(np.float16)).astype(np.float64).max()
+
+
+def test_fine_groups_beat_blocks_on_row_outliers():
+    # query rows of very different magnitude (and a K block with a loud 32-key half): one
+    # scale per row/32 keys tracks fp64 much better than one per 128/64 tokens
+    N, d = 512, 64
+    q, k, v = (_rand16((1, 1, N, d), s) for s in (221, 222, 223))
+    rowmag = np.where(np.arange(N) % 16 == 0, 24.0, 0.25)
+    q = (q.astype(np.float64) * rowmag[None, None, :, None]).astype(np.float16)
+    kmag = np.where((np.arange(N) // 32) % 2 == 0, 6.0, 0.5)
+    k = (k.astype(np.float64) * kmag[None, None, :, None]).astype(np.float16)
+    lay = Layout.dense(1, 1, N, d)
+    sm = 1 / math.sqrt(d)
+    exact = oracle.attn_fp64(q, k, v, lay, False, sm)
+    fine = oracle.sage_attention(q, k, v, lay, False, True, PV_FP16, sm, fine=True)
+    block = oracle.sage_attention(q, k, v, lay, False, True, PV_FP16, sm)
+    assert _rel_l1(fine, exact) < 0.5 * _rel_l1(block, exact)
+    assert _cos(fine, exact) > 0.999

@@ -171,3 +171,23 @@ def test_v_fp8_smoothed_per_channel():
     # the offsets are gone: smoothed scales are far below the raw ones on offset channels
     _, raw = oracle.quant_v_fp8(v, lay)
     assert np.all(scales[0, :, [0, 1, 4]] < 0.2 * raw[0, :, [0, 1, 4]])
+
+
+def test_fine_groups_scales():
+    # finer groups ([SA2] 技术方案 (2), restated for one scale per query row and per 32
+    # keys): every Q token gets amax/127 of its own row, every 32 K tokens of their block
+    N, d = 100, 16
+    lay = Layout.dense(1, 2, N, d)
+    q = _rand16((1, 2, N, d), 31) * (2.0 ** np.arange(N) % 7)[None, None, :, None].astype(np.float16)
+    k = _rand16((1, 2, N, d), 32)
+    z = oracle.quant_qk(q, k, lay, True, fine=True)
+    qa = np.abs(q.astype(np.float32)).max(axis=3)
+    assert z["q_scale"].shape == (1, 2, N)
+    assert np.array_equal(z["q_scale"], (qa / np.float32(127)).astype(np.float32))
+    kf = k.astype(np.float32) - z["k_mean"][:, :, None, :]
+    assert z["k_scale"].shape == (1, 2, 4)
+    for b in range(4):
+        blk = np.abs(kf[:, :, 32 * b:min(N, 32 * b + 32)]).max(axis=(2, 3))
+        assert np.array_equal(z["k_scale"][:, :, b], (blk / np.float32(127)).astype(np.float32))
+    # every row of Q spends the full code range
+    assert np.all(np.abs(z["q_i8"]).max(axis=3)[qa > 0] == 127)

@@ -468,4 +468,4 @@ def test_fine_groups_beat_blocks_on_row_outliers():
     fine = oracle.sage_attention(q, k, v, lay, False, True, PV_FP16, sm, fine=True)
     block = oracle.sage_attention(q, k, v, lay, False, True, PV_FP16, sm)
     assert _rel_l1(fine, exact) < 0.5 * _rel_l1(block, exact)
-    assert _cos(fine, exact) > 0.999
+    assert _rel_l1(fine, exact) < 0.02

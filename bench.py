@@ -184,7 +184,8 @@ def _oracle_sample(case, it: int, rows: int):
     r1 = min(r0 + rows, n)
     t0 = time.perf_counter()
     oracle.sage_attention(q, k, v, lay, W["causal"], W["smooth_k"], pv,
-                          1.0 / math.sqrt(lay.d), heads=[(s, h)], rows=(r0, r1), kv_layout=kvl)
+                          1.0 / math.sqrt(lay.d), heads=[(s, h)], rows=(r0, r1), kv_layout=kvl,
+                          fine=W.get("fine", False))
     return (time.perf_counter() - t0, _sample_ops(r0, r1, n, kvl.lens[s], lay.d, W["causal"]),
             (s, h))
 
@@ -275,6 +276,7 @@ def _workload(args):
         W["causal"] = True
     if args.pv is not None:
         W["pv_mode"] = args.pv
+    W["fine"] = bool(args.fine)
     return W
 
 
@@ -285,7 +287,8 @@ def _workload_name(W):
                 f"smooth_k")
     nq = f" Nq={W['Nq']} Nk={W['N']}" if W.get("Nq") else ""
     return (f"B={W['B']} H={W['H']} N={W['N']}{nq} d={W['d']} "
-            f"{'causal' if W['causal'] else 'non-causal'} PV={W['pv_mode']} smooth_k")
+            f"{'causal' if W['causal'] else 'non-causal'} PV={W['pv_mode']} smooth_k"
+            f"{' fine-groups' if W.get('fine') else ''}")
 
 
 def run_ours(args):
@@ -316,7 +319,9 @@ def run_ours(args):
         vscale = torch.empty((B, H, d), dtype=torch.float32, device=v.device)
     sm_scale = 1.0 / math.sqrt(d)
     dev = q.device
-    nqb, nkb = math.ceil(Nq / 128), math.ceil(N / 64)
+    fine = W["fine"]
+    nqb, nkb = (Nq, math.ceil(N / 32)) if fine else (math.ceil(Nq / 128), math.ceil(N / 64))
+    qk_flags = (sage.SAGE_SMOOTH_K if W["smooth_k"] else 0) | (sage.SAGE_QK_FINE if fine else 0)
     q_i8 = torch.empty(q.shape, dtype=torch.int8, device=dev)
     k_i8 = torch.empty(k.shape, dtype=torch.int8, device=dev)
     q_scale = torch.empty((B, H, nqb), dtype=torch.float32, device=dev)
@@ -329,23 +334,24 @@ def run_ours(args):
     vstat_ws = torch.empty(B * H * d * 16, dtype=torch.uint8, device=dev)  # V column statistics
 
     def quant():
-        if Nq == N:
+        if Nq == N and not fine:
             sage.sage_quant_qk_ws(q, k, q_i8, q_scale, k_i8, k_scale, k_mean, B, H, N, d,
                                   W["smooth_k"], ksum_ws, ksum_ws.numel(), stream)
         else:
             sage.sage_quant_qk_kv(q, k, q_i8, q_scale, k_i8, k_scale, k_mean, B, H, Nq, N, d,
-                                  W["smooth_k"], ksum_ws, ksum_ws.numel(), stream)
+                                  qk_flags, ksum_ws, ksum_ws.numel(), stream)
         if pv == sage.SAGE_PV_FP8:
             sage.sage_quant_v_fp8_ws(v, vq, vscale, None, B, H, N, d, vstat_ws, vstat_ws.numel(),
                                      stream)
 
     def attend():
-        if Nq == N:
+        if Nq == N and not fine:
             sage.sage_attn_fwd_quantized(q_i8, q_scale, k_i8, k_scale, vq, vscale, out, B, H, N,
                                          d, W["causal"], pv, sm_scale, stream)
         else:
             sage.sage_attn_fwd_quantized_kv(q_i8, q_scale, k_i8, k_scale, vq, vscale, None, out,
-                                            B, H, Nq, N, d, W["causal"], pv, sm_scale, stream)
+                                            B, H, Nq, N, d, W["causal"], pv, sm_scale,
+                                            sage.SAGE_QK_FINE if fine else 0, stream)
 
     def step():
         quant()
@@ -410,11 +416,11 @@ def run_ours(args):
         qd.copy_(qh, non_blocking=True)
         kd.copy_(kh, non_blocking=True)
         vd.copy_(vh, non_blocking=True)
-        if Nq == N:
+        if Nq == N and not fine:
             sage.sage_attn_fwd(qd, kd, vd, od, B, H, N, d, W["causal"], W["smooth_k"], pv,
                                sm_scale, stream)
         else:
-            sage.sage_attn_fwd_kv(qd, kd, vd, od, B, H, Nq, N, d, W["causal"], W["smooth_k"], pv,
+            sage.sage_attn_fwd_kv(qd, kd, vd, od, B, H, Nq, N, d, W["causal"], qk_flags, pv,
                                   sm_scale, None, 0, stream)
         oh.copy_(od, non_blocking=True)
 
@@ -513,7 +519,8 @@ def run_varlen(args, W, dist, world, rank, local):
     ops = inputs.varlen_ops(lens, H, d, W["causal"])
 
     def step(qq=q, kk=k, vv=v, oo=out):
-        sage.sage_attn_varlen_fwd(qq, kk, vv, oo, cud, nseq, T, maxlen, H, d, W["causal"], True,
+        flags = sage.SAGE_SMOOTH_K | (sage.SAGE_QK_FINE if W["fine"] else 0)
+        sage.sage_attn_varlen_fwd(qq, kk, vv, oo, cud, nseq, T, maxlen, H, d, W["causal"], flags,
                                   pv, 0.0, ws, need, stream)
 
     clocks = ClockSampler(local)
@@ -638,6 +645,8 @@ def main():
     ap.add_argument("--d", type=int, default=None, choices=[64, 128])
     ap.add_argument("--causal", action="store_true")
     ap.add_argument("--pv", choices=["fp16", "fp8"], default=None)
+    ap.add_argument("--fine", action="store_true",
+                    help="one Q scale per token and one K scale per 32 tokens")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

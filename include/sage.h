@@ -69,8 +69,9 @@ typedef enum {
 enum { SAGE_PV_FP16 = 0, SAGE_PV_FP8 = 1 };
 
 /*
- * Smoothing flags, passed in the `smooth_k` argument of the fused entry points
- * (sage_attn_fwd, sage_attn_fwd_ws, sage_attn_varlen_fwd, sage_attn_fwd_noalloc):
+ * Option flags, passed in the `smooth_k` argument of the fused entry points
+ * (sage_attn_fwd, sage_attn_fwd_ws, sage_attn_varlen_fwd, sage_attn_fwd_noalloc and the
+ * *_kv forms) and of the Q/K quantization entry points:
  *   SAGE_SMOOTH_K (1): step 1 above. 0 and 1 keep their plain boolean meaning.
  *   SAGE_SMOOTH_V (2): smooth V in FP8 mode (「4比特量化三倍加速不掉点！清华即插即用的SageAttention迎来升级」, 技术方案,
  *     the paragraph after item (4)): V <- V - mean(V), the mean per channel over the
@@ -78,10 +79,16 @@ enum { SAGE_PV_FP16 = 0, SAGE_PV_FP8 = 1 };
  *     fp32), the E4M3 codes and per-channel scales taken of the smoothed V, and mean(V)
  *     added to every output row. Softmax rows sum to one, so the exact result is
  *     unchanged; the E4M3 range is no longer spent on a channel offset.
- * Other bits give SAGE_ERR_INVALID_ARG; SAGE_SMOOTH_V with SAGE_PV_FP16 gives
+ *   SAGE_QK_FINE (8): finer quantization groups ("SageAttention2" article, 技术方案 (2),
+ *     which groups tokens by the threads that hold them in the tensor-core layout): here
+ *     every query row is held by one thread, so Q gets one scale per token, and K one
+ *     scale per 32 tokens (the tensor-memory load width). q_scale is then
+ *     [nseq, H, maxlen_q] and k_scale [nseq, H, ceil(maxlen_k / 32)].
+ * Other bits give SAGE_ERR_INVALID_ARG (the Q/K quantization entry points accept only
+ * SAGE_SMOOTH_K and SAGE_QK_FINE); SAGE_SMOOTH_V with SAGE_PV_FP16 gives
  * SAGE_ERR_UNSUPPORTED (fp16 V is not quantized, so there is nothing to smooth for).
  */
-enum { SAGE_SMOOTH_K = 1, SAGE_SMOOTH_V = 2 };
+enum { SAGE_SMOOTH_K = 1, SAGE_SMOOTH_V = 2, SAGE_QK_FINE = 8 };
 
 /* Opaque CUDA stream (binary-compatible with cudaStream_t). */
 typedef struct CUstream_st *sage_stream_t;
@@ -256,13 +263,15 @@ SAGE_API sage_status_t sage_attn_fwd_quantized_smooth_v(const int8_t *q_i8, cons
 
 /* Step 3 alone with Nq queries and Nk keys (codes and scales from sage_quant_qk_kv; V
  * codes from sage_quant_v_fp8[_smooth] with N = Nk); v_mean selects the smooth-V
- * epilogue (FP8 only) or is NULL. */
+ * epilogue (FP8 only) or is NULL; flags is 0 or SAGE_QK_FINE (the scale layout the codes
+ * were made with). */
 SAGE_API sage_status_t sage_attn_fwd_quantized_kv(const int8_t *q_i8, const float *q_scale,
                                                   const int8_t *k_i8, const float *k_scale,
                                                   const void *v, const float *v_scale,
                                                   const float *v_mean, void *out, int B, int H,
                                                   int Nq, int Nk, int d, int causal, int pv_mode,
-                                                  float sm_scale, sage_stream_t stream);
+                                                  float sm_scale, int flags,
+                                                  sage_stream_t stream);
 
 /*
  * Debug: the integer score tiles S = q_i8 k_i8^T (int32, [B,H,N,N]) exactly as the

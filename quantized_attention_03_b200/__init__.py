@@ -33,6 +33,7 @@ SAGE_PV_FP16 = 0
 SAGE_PV_FP8 = 1
 SAGE_SMOOTH_K = 1     # flags of the fused entry points' smooth_k argument
 SAGE_SMOOTH_V = 2
+SAGE_QK_FINE = 8
 
 Q_BLOCK = 128
 K_BLOCK = 64
@@ -51,7 +52,7 @@ SIGNATURES = {
     "sage_attn_varlen_fwd_kv": (_S, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I,
                                      _I, _F, _P, _Z, _P]),
     "sage_attn_fwd_quantized_kv": (_S, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
-                                        _I, _F, _P]),
+                                        _I, _F, _I, _P]),
     "sage_quant_qk": (_S, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "sage_quant_qk_ws": (_S, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]),
     "sage_quant_qk_varlen": (_S, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _I, _P]),
@@ -169,10 +170,10 @@ def sage_attn_varlen_fwd_kv(q, k, v, out, cu_seqlens_q, cu_seqlens_k, nseq, tota
 
 
 def sage_attn_fwd_quantized_kv(q_i8, q_scale, k_i8, k_scale, v, v_scale, v_mean, out, B, H, Nq,
-                               Nk, d, causal, pv_mode, sm_scale, stream=None):
+                               Nk, d, causal, pv_mode, sm_scale, flags=0, stream=None):
     return _call("sage_attn_fwd_quantized_kv", _ptr(q_i8), _ptr(q_scale), _ptr(k_i8),
                  _ptr(k_scale), _ptr(v), _ptr(v_scale), _ptr(v_mean), _ptr(out), B, H, Nq, Nk, d,
-                 int(causal), int(pv_mode), float(sm_scale), _stream(stream))
+                 int(causal), int(pv_mode), float(sm_scale), int(flags), _stream(stream))
 
 
 def sage_quant_qk(q, k, q_i8, q_scale, k_i8, k_scale, k_mean, B, H, N, d, smooth_k, stream=None):
@@ -298,12 +299,14 @@ def _check_status(stream=None):
         raise SageError("device", code)
 
 
-def _smooth_flags(smooth_k: bool, smooth_v: bool) -> int:
-    return (SAGE_SMOOTH_K if smooth_k else 0) | (SAGE_SMOOTH_V if smooth_v else 0)
+def _smooth_flags(smooth_k: bool, smooth_v: bool, fine: bool = False) -> int:
+    return ((SAGE_SMOOTH_K if smooth_k else 0) | (SAGE_SMOOTH_V if smooth_v else 0)
+            | (SAGE_QK_FINE if fine else 0))
 
 
 def sageattn(q, k, v, causal: bool = False, smooth_k: bool = True, pv_mode: int = SAGE_PV_FP16,
-             sm_scale: float = 0.0, out=None, stream=None, smooth_v: bool = False):
+             sm_scale: float = 0.0, out=None, stream=None, smooth_v: bool = False,
+             fine: bool = False):
     """O = SageAttention(q, k, v) for fp16 CUDA tensors q [B, H, Nq, d], k and v
     [B, H, Nk, d] (Nq != Nk: sage_attn_fwd_kv, causal mask aligned at the bottom right)."""
     import torch
@@ -311,7 +314,7 @@ def sageattn(q, k, v, causal: bool = False, smooth_k: bool = True, pv_mode: int 
     Nk = k.shape[2]
     if out is None:
         out = torch.empty_like(q)
-    flags = _smooth_flags(smooth_k, smooth_v)
+    flags = _smooth_flags(smooth_k, smooth_v, fine)
     if Nq == Nk:
         sage_attn_fwd(q, k, v, out, B, H, Nq, d, causal, flags, pv_mode, sm_scale, stream)
     else:
@@ -351,41 +354,46 @@ def sageattn_varlen(q, k, v, cu_seqlens, max_seqlen: int, causal: bool = False,
     return out
 
 
-def quant_qk(q, k, smooth_k: bool = True, stream=None):
-    """Dense smooth-K + per-block INT8: dict of q_i8, q_scale, k_i8, k_scale, k_mean
-    (q [B,H,Nq,d] and k [B,H,Nk,d] may differ in length)."""
+def quant_qk(q, k, smooth_k: bool = True, stream=None, fine: bool = False):
+    """Dense smooth-K + INT8: dict of q_i8, q_scale, k_i8, k_scale, k_mean (q [B,H,Nq,d]
+    and k [B,H,Nk,d] may differ in length; fine: per-token Q and per-32-token K scales)."""
     import torch
     B, H, N, d = q.shape
     Nk = k.shape[2]
     dev = q.device
+    qg, kg = (1, 32) if fine else (Q_BLOCK, K_BLOCK)
     z = dict(q_i8=torch.empty(q.shape, dtype=torch.int8, device=dev),
-             q_scale=torch.empty((B, H, math.ceil(N / Q_BLOCK)), dtype=torch.float32, device=dev),
+             q_scale=torch.empty((B, H, math.ceil(N / qg)), dtype=torch.float32, device=dev),
              k_i8=torch.empty(k.shape, dtype=torch.int8, device=dev),
-             k_scale=torch.empty((B, H, math.ceil(Nk / K_BLOCK)), dtype=torch.float32, device=dev),
+             k_scale=torch.empty((B, H, math.ceil(Nk / kg)), dtype=torch.float32, device=dev),
              k_mean=torch.empty((B, H, d), dtype=torch.float32, device=dev))
-    if N == Nk:
+    flags = (SAGE_SMOOTH_K if smooth_k else 0) | (SAGE_QK_FINE if fine else 0)
+    if N == Nk and not fine:
         sage_quant_qk(q, k, z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], z["k_mean"], B, H, N,
                       d, smooth_k, stream)
     else:
         sage_quant_qk_kv(q, k, z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], z["k_mean"], B,
-                         H, N, Nk, d, smooth_k, None, 0, stream)
+                         H, N, Nk, d, flags, None, 0, stream)
     return z
 
 
-def quant_qk_varlen(q, k, cu_seqlens, max_seqlen: int, smooth_k: bool = True, stream=None):
+def quant_qk_varlen(q, k, cu_seqlens, max_seqlen: int, smooth_k: bool = True, stream=None,
+                    fine: bool = False):
     import torch
     T, H, d = q.shape
     nseq = cu_seqlens.numel() - 1
     dev = q.device
+    qg, kg = (1, 32) if fine else (Q_BLOCK, K_BLOCK)
     z = dict(q_i8=torch.empty(q.shape, dtype=torch.int8, device=dev),
-             q_scale=torch.empty((nseq, H, math.ceil(max_seqlen / Q_BLOCK)), dtype=torch.float32,
+             q_scale=torch.empty((nseq, H, math.ceil(max_seqlen / qg)), dtype=torch.float32,
                                  device=dev),
              k_i8=torch.empty(k.shape, dtype=torch.int8, device=dev),
-             k_scale=torch.empty((nseq, H, math.ceil(max_seqlen / K_BLOCK)), dtype=torch.float32,
+             k_scale=torch.empty((nseq, H, math.ceil(max_seqlen / kg)), dtype=torch.float32,
                                  device=dev),
              k_mean=torch.empty((nseq, H, d), dtype=torch.float32, device=dev))
+    flags = (SAGE_SMOOTH_K if smooth_k else 0) | (SAGE_QK_FINE if fine else 0)
     sage_quant_qk_varlen(q, k, cu_seqlens, nseq, T, max_seqlen, H, d, z["q_i8"], z["q_scale"],
-                         z["k_i8"], z["k_scale"], z["k_mean"], smooth_k, stream)
+                         z["k_i8"], z["k_scale"], z["k_mean"], flags, stream)
     return z
 
 
@@ -421,16 +429,18 @@ def quant_v_fp8_varlen(v, cu_seqlens, max_seqlen: int, stream=None, smooth_v: bo
 
 def attn_quantized(q_i8, q_scale, k_i8, k_scale, v, v_scale, causal: bool = False,
                    pv_mode: int = SAGE_PV_FP16, sm_scale: float = 0.0, out=None, stream=None,
-                   v_mean=None):
-    """Step 3 on pre-quantized operands; v_mean (FP8 mode) selects the smooth-V epilogue."""
+                   v_mean=None, fine: bool = False):
+    """Step 3 on pre-quantized operands; v_mean (FP8 mode) selects the smooth-V epilogue,
+    fine the per-token Q / per-32-token K scale layout."""
     import torch
     B, H, N, d = q_i8.shape
     Nk = k_i8.shape[2]
     if out is None:
         out = torch.empty(q_i8.shape, dtype=torch.float16, device=q_i8.device)
-    if Nk != N:
+    if Nk != N or fine:
         sage_attn_fwd_quantized_kv(q_i8, q_scale, k_i8, k_scale, v, v_scale, v_mean, out, B, H, N,
-                                   Nk, d, causal, pv_mode, sm_scale, stream)
+                                   Nk, d, causal, pv_mode, sm_scale,
+                                   SAGE_QK_FINE if fine else 0, stream)
         return out
     if v_mean is not None:
         if pv_mode != SAGE_PV_FP8:

@@ -108,7 +108,9 @@ Workspace carve(char *base, int nseq, int H, int max_q, int max_k, int total_q, 
 {
     Workspace w;
     const size_t qcodes = (size_t)total_q * H * d, kcodes = (size_t)total_k * H * d;
-    const size_t nqb = (max_q + kQBlock - 1) / kQBlock, nkb = (max_k + kKBlock - 1) / kKBlock;
+    // scale rows sized for the finer groups (one Q scale per token, one K scale per 32
+    // tokens), which also hold the per-block scales
+    const size_t nqb = (size_t)max_q, nkb = (max_k + 31) / 32;
     const size_t heads = (size_t)nseq * H;
     size_t off = 0;
     auto take = [&](size_t bytes) {
@@ -149,10 +151,10 @@ sage_status_t check_shape(int nseq, int H, int maxlen, int d)
     return SAGE_OK;
 }
 
-// The smoothing flags of the fused entry points.
+// The option flags of the fused entry points.
 sage_status_t check_smooth(int smooth, int pv_mode)
 {
-    if (smooth & ~(SAGE_SMOOTH_K | SAGE_SMOOTH_V))
+    if (smooth & ~(SAGE_SMOOTH_K | SAGE_SMOOTH_V | SAGE_QK_FINE))
         return SAGE_ERR_INVALID_ARG;
     if ((smooth & SAGE_SMOOTH_V) && pv_mode != SAGE_PV_FP8)
         return SAGE_ERR_UNSUPPORTED;
@@ -177,6 +179,7 @@ sage_status_t forward(const void *q, const void *k, const void *v, void *out, co
     Workspace w = carve(ws, L.nseq, L.H, L.maxlen, LK.maxlen, L.total, LK.total, L.d, pv_mode);
     const bool fp8 = pv_mode == SAGE_PV_FP8;
     const bool sk = (smooth & SAGE_SMOOTH_K) != 0, sv = (smooth & SAGE_SMOOTH_V) != 0;
+    const bool fine = (smooth & SAGE_QK_FINE) != 0;
     cudaError_t e = cudaMemsetAsync(w.cs.ksum, 0, w.stats_bytes, st);
     if (e != cudaSuccess)
         return cuda_fail(e);
@@ -192,11 +195,11 @@ sage_status_t forward(const void *q, const void *k, const void *v, void *out, co
         return cuda_fail(e);
     if ((e = launch_quant(qh, kh, vh, cs, w.q_i8, w.q_scale, w.k_i8, w.k_scale, w.k_mean,
                           fp8 ? w.v8 : nullptr, w.v_scale, sv ? w.v_mean : nullptr, L, LK,
-                          status, st)) != cudaSuccess)
+                          fine, status, st)) != cudaSuccess)
         return cuda_fail(e);
     AttnArgs a{w.q_i8,     w.q_scale, w.k_i8, w.k_scale, fp8 ? (const void *)w.v8 : v,
                w.v_scale,  sv ? w.v_mean : nullptr,     static_cast<__half *>(out),
-               nullptr,    causal,    pv_mode, resolve_scale(sm_scale, L.d)};
+               nullptr,    causal,    pv_mode, resolve_scale(sm_scale, L.d), fine ? 1 : 0};
     sage_status_t herr;
     if ((e = launch_attention(a, L, LK, status, st, &herr)) != cudaSuccess)
         return herr != SAGE_OK ? herr : cuda_fail(e);
@@ -263,7 +266,8 @@ sage_status_t quant_v_entry(const void *v, const int32_t *cu_seqlens, int nseq, 
 sage_status_t quantized_entry(const int8_t *q_i8, const float *q_scale, const int8_t *k_i8,
                               const float *k_scale, const void *v, const float *v_scale,
                               const float *v_mean, void *out, int B, int H, int Nq, int Nk,
-                              int d, int causal, int pv_mode, float sm_scale, cudaStream_t st)
+                              int d, int causal, int pv_mode, float sm_scale, bool fine,
+                              cudaStream_t st)
 {
     sage_status_t r = check_shape(B, H, Nq, d);
     if (r != SAGE_OK)
@@ -286,7 +290,7 @@ sage_status_t quantized_entry(const int8_t *q_i8, const float *q_scale, const in
         return r;
     const Shape sh = dense_shape(B, H, Nq, Nk, d);
     AttnArgs a{q_i8,   q_scale, k_i8,   k_scale, v, v_scale, v_mean, static_cast<__half *>(out),
-               nullptr, causal, pv_mode, resolve_scale(sm_scale, d)};
+               nullptr, causal, pv_mode, resolve_scale(sm_scale, d), fine ? 1 : 0};
     sage_status_t herr;
     cudaError_t e = launch_attention(a, sh.lq(), sh.lk(), status, st, &herr);
     if (e != cudaSuccess)
@@ -351,6 +355,11 @@ sage_status_t quant_qk_entry(const void *q, const void *k, const Shape &sh, int8
     sage_status_t r = check_shape2(sh);
     if (r != SAGE_OK)
         return r;
+    // the flags word: SAGE_SMOOTH_K (1, the original boolean) and SAGE_QK_FINE
+    if (smooth_k & ~(SAGE_SMOOTH_K | SAGE_QK_FINE))
+        return SAGE_ERR_INVALID_ARG;
+    const bool fine = (smooth_k & SAGE_QK_FINE) != 0;
+    smooth_k &= SAGE_SMOOTH_K;
     const bool has_q = sh.max_q > 0 && sh.total_q > 0, has_k = sh.max_k > 0 && sh.total_k > 0;
     if (sh.nseq == 0 || sh.H == 0 || (!has_q && !has_k))
         return SAGE_OK;
@@ -396,7 +405,7 @@ sage_status_t quant_qk_entry(const void *q, const void *k, const Shape &sh, int8
     cs.ksum = ksum;
     e = launch_quant(static_cast<const __half *>(q), static_cast<const __half *>(k), nullptr, cs,
                      q_i8, q_scale, k_i8, k_scale, k_mean, nullptr, nullptr, nullptr, Lq, Lk,
-                     status, st);
+                     fine, status, st);
     if (owned)
         cudaFreeAsync(ksum, st);
     return e == cudaSuccess ? SAGE_OK : cuda_fail(e);
@@ -446,7 +455,7 @@ sage_status_t quant_v_entry(const void *v, const int32_t *cu_seqlens, int nseq, 
             cudaSuccess)
         e = launch_quant(nullptr, nullptr, static_cast<const __half *>(v), cs, nullptr, nullptr,
                          nullptr, nullptr, nullptr, v_e4m3, v_scale, smooth ? v_mean : nullptr,
-                         L, L, status, st);
+                         L, L, false, status, st);
     if (workspace == nullptr)
         cudaFreeAsync(p, st);
     return e == cudaSuccess ? SAGE_OK : cuda_fail(e);
@@ -472,7 +481,7 @@ sage_status_t sage_quant_qk_ws(const void *q, const void *k, int8_t *q_i8, float
                                int d, int smooth_k, void *workspace, size_t ws_bytes,
                                sage_stream_t stream)
 {
-    if (workspace == nullptr && smooth_k && !(B == 0 || H == 0 || N == 0))
+    if (workspace == nullptr && (smooth_k & SAGE_SMOOTH_K) && !(B == 0 || H == 0 || N == 0))
         return SAGE_ERR_WORKSPACE;
     if (!dense_fits(B, N))
         return SAGE_ERR_UNSUPPORTED;
@@ -650,19 +659,24 @@ sage_status_t sage_attn_fwd_quantized(const int8_t *q_i8, const float *q_scale,
                                       sage_stream_t stream)
 {
     return quantized_entry(q_i8, q_scale, k_i8, k_scale, v, v_scale, nullptr, out, B, H, N, N,
-                           d, causal, pv_mode, sm_scale, reinterpret_cast<cudaStream_t>(stream));
+                           d, causal, pv_mode, sm_scale, false,
+                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 sage_status_t sage_attn_fwd_quantized_kv(const int8_t *q_i8, const float *q_scale,
                                          const int8_t *k_i8, const float *k_scale, const void *v,
                                          const float *v_scale, const float *v_mean, void *out,
                                          int B, int H, int Nq, int Nk, int d, int causal,
-                                         int pv_mode, float sm_scale, sage_stream_t stream)
+                                         int pv_mode, float sm_scale, int flags,
+                                         sage_stream_t stream)
 {
+    if (flags & ~SAGE_QK_FINE)
+        return SAGE_ERR_INVALID_ARG;
     if (v_mean != nullptr && pv_mode != SAGE_PV_FP8)
         return SAGE_ERR_UNSUPPORTED;
     return quantized_entry(q_i8, q_scale, k_i8, k_scale, v, v_scale, v_mean, out, B, H, Nq, Nk,
-                           d, causal, pv_mode, sm_scale, reinterpret_cast<cudaStream_t>(stream));
+                           d, causal, pv_mode, sm_scale, (flags & SAGE_QK_FINE) != 0,
+                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 sage_status_t sage_attn_fwd_quantized_smooth_v(const int8_t *q_i8, const float *q_scale,
@@ -675,7 +689,7 @@ sage_status_t sage_attn_fwd_quantized_smooth_v(const int8_t *q_i8, const float *
     if (v_mean == nullptr && B > 0 && H > 0 && N > 0)
         return SAGE_ERR_INVALID_ARG;
     return quantized_entry(q_i8, q_scale, k_i8, k_scale, v_e4m3, v_scale, v_mean, out, B, H, N,
-                           N, d, causal, SAGE_PV_FP8, sm_scale,
+                           N, d, causal, SAGE_PV_FP8, sm_scale, false,
                            reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -708,7 +722,7 @@ sage_status_t sage_debug_qk_int32(const int8_t *q_i8, const int8_t *k_i8, int32_
         const float *ks = qs + (size_t)B * H * nqb;
         const void *vz = ws + sc_bytes;
         __half *o = reinterpret_cast<__half *>(ws + sc_bytes + align256(elems * 2));
-        AttnArgs a{q_i8, qs, k_i8, ks, vz, nullptr, nullptr, o, s_out, 0, SAGE_PV_FP16, 1.0f};
+        AttnArgs a{q_i8, qs, k_i8, ks, vz, nullptr, nullptr, o, s_out, 0, SAGE_PV_FP16, 1.0f, 0};
         sage_status_t herr;
         const SeqLayout L = SeqLayout::dense(B, H, N, d);
         e = launch_attention(a, L, L, status, st, &herr);

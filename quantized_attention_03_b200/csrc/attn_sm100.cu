@@ -122,7 +122,7 @@ struct KParams {
     int32_t *s_dump;
     SeqLayout L;         // queries (and the output)
     SeqLayout LK;        // keys and values (L again for self-attention)
-    int nqb, nkb;        // scale blocks per (sequence, head) row of the scale arrays
+    int nqb, nkb;        // scales per (sequence, head) row of the scale arrays
     int causal;
     float sc_log2;       // sm_scale * log2(e)
     int *status;
@@ -159,7 +159,9 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     return ok;
 }
 
-template <int D, bool FP8, int NQT, bool DUMP>
+// FINE: one Q scale per query row and one K scale per 32 keys; else one Q scale per
+// 128-row tile and one K scale per 64 keys.
+template <int D, bool FP8, int NQT, bool DUMP, bool FINE>
 __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const KParams p)
@@ -253,9 +255,12 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
         const uint32_t tS = tmem_base + lane_off + i * C::BN;
         const uint32_t tO = tmem_base + lane_off + NQT * C::BN + i * D;
         const int64_t sh = (int64_t)s * L.H + h;
-        const bool tile_valid = qt * C::BM < len;
-        const float qsc = (tile_valid ? __ldg(p.q_scale + sh * p.nqb + qt) : 0.0f) * p.sc_log2;
-        const int kb_valid = (klen + kKBlock - 1) / kKBlock;
+        // this row's Q scale (one per query tile, or one per token)
+        const int qidx = FINE ? qrow : qt;
+        const bool q_valid = (FINE ? qrow : qt * C::BM) < len;
+        const float qsc = (q_valid ? __ldg(p.q_scale + sh * p.nqb + qidx) : 0.0f) * p.sc_log2;
+        constexpr int kKGroups = FINE ? 4 : 2;        // K scales per 128-key tile
+        const int kb_valid = (klen + C::BN / kKGroups - 1) / (C::BN / kKGroups);
 
         // m_ref: the max that P is taken relative to; it moves only when the row max
         // exceeds it by more than kRescaleSlack (0 in FP8 mode, so P <= 1 and 448 P fits E4M3)
@@ -266,9 +271,13 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
             if (!(ok = warp_wait(&s_full[i], j & 1, abort, p.status)))
                 break;
             tc_fence_after();
-            const int kb0 = 2 * j, kb1 = 2 * j + 1;
-            const float sc0 = qsc * (kb0 < kb_valid ? __ldg(p.k_scale + sh * p.nkb + kb0) : 0.0f);
-            const float sc1 = qsc * (kb1 < kb_valid ? __ldg(p.k_scale + sh * p.nkb + kb1) : 0.0f);
+            // dequantization factor of each K scale group of the tile
+            float sck[kKGroups];
+#pragma unroll
+            for (int c = 0; c < kKGroups; c++) {
+                const int kb = kKGroups * j + c;
+                sck[c] = qsc * (kb < kb_valid ? __ldg(p.k_scale + sh * p.nkb + kb) : 0.0f);
+            }
             const int kcol0 = j * C::BN;
             const bool need_mask =
                 (kcol0 + C::BN > klen) || (p.causal && kcol0 + C::BN - 1 > qt * C::BM + koff);
@@ -303,8 +312,11 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
             float alpha = 1.0f, bias = 0.0f;
             auto tile_max = [&](auto masked) {
                 constexpr bool MASKED = decltype(masked)::value;
-                // integer maxima of the two 64-key halves (each K block has its own scale)
-                int im[2] = {INT_MIN, INT_MIN};
+                // integer maxima of the K scale groups (each has its own scale)
+                int im[kKGroups];
+#pragma unroll
+                for (int c = 0; c < kKGroups; c++)
+                    im[c] = INT_MIN;
 #pragma unroll
                 for (int ch = 0; ch < 4; ch++) {
                     const uint32_t keep = MASKED ? chunk_mask(col_lim - kcol0 - ch * 32) : ~0u;
@@ -317,13 +329,14 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
                         else
                             mx[e & 3] = max(mx[e & 3], v);
                     }
-                    im[ch / 2] = max(im[ch / 2], max(max(mx[0], mx[1]), max(mx[2], mx[3])));
+                    const int g = ch * kKGroups / 4;      // the 32 columns' K group
+                    im[g] = max(im[g], max(max(mx[0], mx[1]), max(mx[2], mx[3])));
                 }
                 float tmax = -INFINITY;
-                if (im[0] != INT_MIN)
-                    tmax = static_cast<float>(im[0]) * sc0;
-                if (im[1] != INT_MIN)
-                    tmax = fmaxf(tmax, static_cast<float>(im[1]) * sc1);
+#pragma unroll
+                for (int c = 0; c < kKGroups; c++)
+                    if (im[c] != INT_MIN)
+                        tmax = fmaxf(tmax, static_cast<float>(im[c]) * sck[c]);
                 const float m_new = tmax > m_ref + C::kRescaleSlack ? tmax : m_ref;
                 alpha = m_new == m_ref ? 1.0f : ex2_approx(m_ref - m_new);
                 bias = FP8 ? m_new - kLog2_448 : m_new;
@@ -388,7 +401,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
                 float2 lsum2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
                 for (int ch = 0; ch < 8; ch++) {
-                    const float sc = ch < 4 ? sc0 : sc1;
+                    const float sc = sck[ch * kKGroups / 8];
                     const uint32_t keep =
                         MASKED ? chunk_mask(col_lim - kcol0 - ch * 16) & 0xffffu : 0xffffu;
                     float pe[16];
@@ -702,7 +715,7 @@ bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int elem
     return r == CUDA_SUCCESS;
 }
 
-template <int D, bool FP8, int NQT, bool DUMP>
+template <int D, bool FP8, int NQT, bool DUMP, bool FINE>
 cudaError_t run(const AttnArgs &a, const SeqLayout &L, const SeqLayout &LK, int *status,
                 cudaStream_t st, sage_status_t *host_err)
 {
@@ -730,13 +743,14 @@ cudaError_t run(const AttnArgs &a, const SeqLayout &L, const SeqLayout &LK, int 
     p.s_dump = a.s_dump;
     p.L = L;
     p.LK = LK;
-    p.nqb = (L.maxlen + kQBlock - 1) / kQBlock;
-    p.nkb = (LK.maxlen + kKBlock - 1) / kKBlock;
+    const int q_grp = FINE ? 1 : kQBlock, k_grp = FINE ? 32 : kKBlock;
+    p.nqb = (L.maxlen + q_grp - 1) / q_grp;
+    p.nkb = (LK.maxlen + k_grp - 1) / k_grp;
     p.causal = a.causal;
     p.sc_log2 = a.sm_scale * kLog2e;
     p.status = status;
 
-    auto kern = attn_kernel<D, FP8, NQT, DUMP>;
+    auto kern = attn_kernel<D, FP8, NQT, DUMP, FINE>;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess)
@@ -760,14 +774,21 @@ cudaError_t launch_attention(const AttnArgs &a, const SeqLayout &L, const SeqLay
     const bool fp8 = a.pv_mode == SAGE_PV_FP8;
     if (a.s_dump != nullptr) {
         if (L.d == 128)
-            return run<128, false, 2, true>(a, L, LK, status, st, host_err);
-        return run<64, false, 2, true>(a, L, LK, status, st, host_err);
+            return run<128, false, 2, true, false>(a, L, LK, status, st, host_err);
+        return run<64, false, 2, true, false>(a, L, LK, status, st, host_err);
+    }
+    if (a.fine) {
+        if (L.d == 128)
+            return fp8 ? run<128, true, 2, false, true>(a, L, LK, status, st, host_err)
+                       : run<128, false, 2, false, true>(a, L, LK, status, st, host_err);
+        return fp8 ? run<64, true, 2, false, true>(a, L, LK, status, st, host_err)
+                   : run<64, false, 2, false, true>(a, L, LK, status, st, host_err);
     }
     if (L.d == 128)
-        return fp8 ? run<128, true, 2, false>(a, L, LK, status, st, host_err)
-                   : run<128, false, 2, false>(a, L, LK, status, st, host_err);
-    return fp8 ? run<64, true, 2, false>(a, L, LK, status, st, host_err)
-               : run<64, false, 2, false>(a, L, LK, status, st, host_err);
+        return fp8 ? run<128, true, 2, false, false>(a, L, LK, status, st, host_err)
+                   : run<128, false, 2, false, false>(a, L, LK, status, st, host_err);
+    return fp8 ? run<64, true, 2, false, false>(a, L, LK, status, st, host_err)
+               : run<64, false, 2, false, false>(a, L, LK, status, st, host_err);
 }
 
 }  // namespace sage

@@ -235,13 +235,147 @@ __device__ __forceinline__ float e4m3_quotient(float x, float s, float r)
     return q;
 }
 
+// Codes of one 128-token chunk of Q or K (already in shared memory) with one scale per G
+// rows: G = 128 (a Q block), 64 (a K block), 32 (finer K groups) or 1 (one scale per
+// token). Thread (cg, r_in) owns the 16-byte column group cg of rows r_in + i * kRowStep;
+// mu holds its 8 channels' means (0 for Q), scale_out the head's scale row of nsc
+// entries.
+template <int D, int G>
+__device__ __forceinline__ void qk_chunk(const uint4 *s_x, const float (&mu)[8], int cg,
+                                         int r_in, int nrows, int row0, int chunk,
+                                         float *scale_out, int nsc, int8_t *dst,
+                                         const SeqLayout &L, int s, int start, int h,
+                                         float (*s_red)[kThreads / 32])
+{
+    constexpr int kGpr = D / 8;
+    constexpr int kRowStep = kThreads / kGpr;
+    constexpr int kSteps = kQBlock / kRowStep;
+    constexpr int kWarps = kThreads / 32;
+    const int c0 = cg * 8;
+    float sc[kSteps], rc[kSteps];
+    if constexpr (G == 1) {
+        // one scale per row: the row's kGpr 16-byte groups sit in consecutive lanes
+#pragma unroll
+        for (int i = 0; i < kSteps; i++) {
+            const int row = i * kRowStep + r_in;
+            float m = 0.0f;
+            if (row < nrows) {
+                float f[8];
+                unpack8(s_x[row * kGpr + cg], f);
+#pragma unroll
+                for (int e = 0; e < 8; e++)
+                    m = fmaxf(m, fabsf(__fsub_rn(f[e], mu[e])));
+            }
+#pragma unroll
+            for (int o = 1; o < kGpr; o <<= 1)
+                m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            sc[i] = __fdiv_rn(m, 127.0f);
+            rc[i] = sc[i] != 0.0f ? __fdiv_rn(1.0f, sc[i]) : 0.0f;
+            if (cg == 0 && row0 + row < nsc)
+                scale_out[row0 + row] = sc[i];          // rows past the sequence: 0
+        }
+    } else {
+        // one scale per G rows. fp32 rounding is monotonic, so the largest |fl(x - mu)| of a
+        // group is max(fl(max x - mu), fl(mu - min x)) over its channels: pass 1 keeps
+        // per-channel fp16 extrema only (Q: mu = 0, i.e. max |x|)
+        constexpr int kGroups = kQBlock / G;
+        constexpr int kStepsPerGroup = G / kRowStep;
+        static_assert(G % kRowStep == 0, "a group spans whole row steps");
+        const __half2 kNegInf =
+            __halves2half2(__ushort_as_half(0xFC00), __ushort_as_half(0xFC00));
+        const __half2 kPosInf =
+            __halves2half2(__ushort_as_half(0x7C00), __ushort_as_half(0x7C00));
+        __half2 hi[kGroups][4], lo[kGroups][4];
+#pragma unroll
+        for (int g = 0; g < kGroups; g++)
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                hi[g][j] = kNegInf;
+                lo[g][j] = kPosInf;
+            }
+#pragma unroll
+        for (int i = 0; i < kSteps; i++) {
+            const int row = i * kRowStep + r_in;
+            const int g = i / kStepsPerGroup;
+            if (row < nrows) {
+                const uint4 u = s_x[row * kGpr + cg];
+                const __half2 *x2 = reinterpret_cast<const __half2 *>(&u);
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    hi[g][j] = __hmax2(hi[g][j], x2[j]);
+                    lo[g][j] = __hmin2(lo[g][j], x2[j]);
+                }
+            }
+        }
+        float am[kGroups];
+#pragma unroll
+        for (int g = 0; g < kGroups; g++) {
+            am[g] = 0.0f;
+#pragma unroll
+            for (int j = 0; j < 4; j++) {
+                const float2 hf = __half22float2(hi[g][j]), lf = __half22float2(lo[g][j]);
+                am[g] = fmaxf(am[g],
+                              fmaxf(__fsub_rn(hf.x, mu[2 * j]), __fsub_rn(mu[2 * j], lf.x)));
+                am[g] = fmaxf(am[g], fmaxf(__fsub_rn(hf.y, mu[2 * j + 1]),
+                                           __fsub_rn(mu[2 * j + 1], lf.y)));
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+                am[g] = fmaxf(am[g], __shfl_xor_sync(0xffffffffu, am[g], o));
+        }
+        const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
+        if (lane == 0)
+#pragma unroll
+            for (int g = 0; g < kGroups; g++)
+                s_red[g][warp] = am[g];
+        __syncthreads();
+        float sg[kGroups], rg[kGroups];
+#pragma unroll
+        for (int g = 0; g < kGroups; g++) {
+            float A = 0.0f;
+#pragma unroll
+            for (int w = 0; w < kWarps; w++)
+                A = fmaxf(A, s_red[g][w]);
+            sg[g] = __fdiv_rn(A, 127.0f);
+            rg[g] = sg[g] != 0.0f ? __fdiv_rn(1.0f, sg[g]) : 0.0f;
+            if (threadIdx.x == 0 && chunk * kGroups + g < nsc)
+                scale_out[chunk * kGroups + g] = sg[g];
+        }
+#pragma unroll
+        for (int i = 0; i < kSteps; i++) {
+            sc[i] = sg[i / kStepsPerGroup];
+            rc[i] = rg[i / kStepsPerGroup];
+        }
+    }
+    float2 nmu[4];                        // -mu (Q: -0, so that x + nmu = x exactly)
+#pragma unroll
+    for (int j = 0; j < 4; j++)
+        nmu[j] = make_float2(-mu[2 * j], -mu[2 * j + 1]);
+#pragma unroll
+    for (int i = 0; i < kSteps; i++) {
+        const int row = i * kRowStep + r_in;
+        if (row >= nrows)
+            break;
+        float f[8];
+        unpack8(s_x[row * kGpr + cg], f);
+        float2 x[4];
+#pragma unroll
+        for (int j = 0; j < 4; j++)
+            x[j] = add2(make_float2(f[2 * j], f[2 * j + 1]), nmu[j]);
+        const uint2 w = int8_codes8(x, sc[i], rc[i]);
+        *reinterpret_cast<uint2 *>(dst + L.offset(s, start, h, row0 + row) + c0) = w;
+    }
+}
+
 // One CTA per 128-token chunk of one (sequence, head): a Q block, a pair of K blocks or
 // a V chunk. The chunk (128 rows x D fp16, 32 KB at D = 128) comes into shared memory
 // with bulk copies (one for the dense layout, one per row for the packed layout) issued
 // at CTA start, so every resident CTA keeps its whole chunk in flight. Thread t then
 // owns the 16-byte column group t % (D/8) of rows t / (D/8) + i (256 / (D/8)), which
 // makes the shared-memory reads conflict-free and fixes the thread's 8 channels.
-template <int D>
+// FINE: one Q scale per token and one K scale per 32 tokens; else per-block scales (Q:
+// 128 tokens, K: 64 tokens).
+template <int D, bool FINE>
 __global__ void __launch_bounds__(kThreads, 4) quant_kernel(
     const __half *__restrict__ q, const __half *__restrict__ k, const __half *__restrict__ v,
     ColStats cs, int8_t *__restrict__ q_i8, float *__restrict__ q_scale,
@@ -252,25 +386,27 @@ __global__ void __launch_bounds__(kThreads, 4) quant_kernel(
     constexpr int kGpr = D / 8;                      // 16-byte groups per row
     constexpr int kRowStep = kThreads / kGpr;        // rows between a thread's groups
     constexpr int kSteps = kQBlock / kRowStep;       // groups per thread
-    constexpr int kHalfSteps = kKBlock / kRowStep;   // those in the first 64-row K block
     constexpr int kWarps = kThreads / 32;
+    constexpr int kQG = FINE ? 1 : kQBlock;          // tokens per Q scale
+    constexpr int kKG = FINE ? 32 : kKBlock;         // tokens per K scale
     __shared__ __align__(128) uint4 s_x[kQBlock * kGpr];
     __shared__ __align__(8) uint64_t s_bar;
-    __shared__ float s_red[2][kWarps];
+    __shared__ float s_red[4][kWarps];
     __shared__ float s_mu[D];             // K mean or V mean per channel
     __shared__ float s_sc[D];             // V scale per channel
     __shared__ float s_rc[D];             // fl(1 / V scale) per channel
 
     // 0: Q block, 1: K pair of blocks, 2: V chunk. grid.x spans the parts in order:
     // [Q chunks of Lq | K chunks of Lk] when with_q, then [V chunks of Lk] if any.
-    const int nqb = (Lq.maxlen + kQBlock - 1) / kQBlock;   // Q scale blocks per head
-    const int nkb = (Lk.maxlen + kKBlock - 1) / kKBlock;   // K scale blocks per head
+    const int nqc = (Lq.maxlen + kQBlock - 1) / kQBlock;   // 128-token Q chunks per head
+    const int nqb = (Lq.maxlen + kQG - 1) / kQG;           // Q scales per head
+    const int nkb = (Lk.maxlen + kKG - 1) / kKG;           // K scales per head
     int kind, chunk = (int)blockIdx.x;
-    if (with_q && chunk < nqb) {
+    if (with_q && chunk < nqc) {
         kind = 0;
     } else {
         if (with_q)
-            chunk -= nqb;
+            chunk -= nqc;
         kind = (with_q && chunk < nkc) ? 1 : 2;
         if (kind == 2 && with_q)
             chunk -= nkc;
@@ -291,15 +427,12 @@ __global__ void __launch_bounds__(kThreads, 4) quant_kernel(
             if (v_mean != nullptr)
                 v_mean[sh * D + threadIdx.x] = 0.0f;
         }
-        if (threadIdx.x == 0) {
-            if (kind == 0)
-                q_scale[sh * nqb + chunk] = 0.0f;
-            if (kind == 1) {
-                if (2 * chunk < nkb)
-                    k_scale[sh * nkb + 2 * chunk] = 0.0f;
-                if (2 * chunk + 1 < nkb)
-                    k_scale[sh * nkb + 2 * chunk + 1] = 0.0f;
-            }
+        if (kind != 2) {                  // the chunk's scale entries are 0
+            const int G = kind == 0 ? kQG : kKG, nsc = kind == 0 ? nqb : nkb;
+            float *so = (kind == 0 ? q_scale : k_scale) + sh * nsc;
+            const int e = row0 / G + (int)threadIdx.x;
+            if ((int)threadIdx.x < kQBlock / G && e < nsc)
+                so[e] = 0.0f;
         }
         return;
     }
@@ -390,100 +523,13 @@ __global__ void __launch_bounds__(kThreads, 4) quant_kernel(
         return;
     }
 
-    // ---- Q / K: block amax (K: one per 64-row half), then codes.
-    // Pass 1 keeps per-channel fp16 extrema only: fp32 rounding is monotonic, so the
-    // largest |fl(x - mu)| of a block is max(fl(max x - mu), fl(mu - min x)) over its
-    // channels (Q: mu = 0, i.e. max |x|).
-    const __half2 kNegInf = __halves2half2(__ushort_as_half(0xFC00), __ushort_as_half(0xFC00));
-    const __half2 kPosInf = __halves2half2(__ushort_as_half(0x7C00), __ushort_as_half(0x7C00));
-    __half2 hi[2][4], lo[2][4];
-#pragma unroll
-    for (int b = 0; b < 2; b++)
-#pragma unroll
-        for (int j = 0; j < 4; j++) {
-            hi[b][j] = kNegInf;
-            lo[b][j] = kPosInf;
-        }
-#pragma unroll
-    for (int i = 0; i < kSteps; i++) {
-        const int row = i * kRowStep + r_in;
-        const int b = i < kHalfSteps ? 0 : 1;
-        if (row < nrows) {
-            const uint4 u = s_x[row * kGpr + cg];
-            const __half2 *x2 = reinterpret_cast<const __half2 *>(&u);
-#pragma unroll
-            for (int j = 0; j < 4; j++) {
-                hi[b][j] = __hmax2(hi[b][j], x2[j]);
-                lo[b][j] = __hmin2(lo[b][j], x2[j]);
-            }
-        }
-    }
-    float am[2] = {0.0f, 0.0f};
-#pragma unroll
-    for (int b = 0; b < 2; b++)
-#pragma unroll
-        for (int j = 0; j < 4; j++) {
-            const float2 hf = __half22float2(hi[b][j]), lf = __half22float2(lo[b][j]);
-            am[b] = fmaxf(am[b], fmaxf(__fsub_rn(hf.x, mu[2 * j]), __fsub_rn(mu[2 * j], lf.x)));
-            am[b] = fmaxf(am[b],
-                          fmaxf(__fsub_rn(hf.y, mu[2 * j + 1]), __fsub_rn(mu[2 * j + 1], lf.y)));
-        }
-    float a0 = am[0], a1 = am[1];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        a0 = fmaxf(a0, __shfl_xor_sync(0xffffffffu, a0, o));
-        a1 = fmaxf(a1, __shfl_xor_sync(0xffffffffu, a1, o));
-    }
-    const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-    if (lane == 0) {
-        s_red[0][warp] = a0;
-        s_red[1][warp] = a1;
-    }
-    __syncthreads();
-    float A0 = 0.0f, A1 = 0.0f;
-#pragma unroll
-    for (int w = 0; w < kWarps; w++) {
-        A0 = fmaxf(A0, s_red[0][w]);
-        A1 = fmaxf(A1, s_red[1][w]);
-    }
-    float sc0, sc1;
-    if (kind == 0) {
-        sc0 = sc1 = __fdiv_rn(fmaxf(A0, A1), 127.0f);
-        if (threadIdx.x == 0)
-            q_scale[sh * nqb + chunk] = sc0;
-    } else {
-        sc0 = __fdiv_rn(A0, 127.0f);
-        sc1 = __fdiv_rn(A1, 127.0f);
-        if (threadIdx.x == 0) {
-            if (2 * chunk < nkb)
-                k_scale[sh * nkb + 2 * chunk] = sc0;
-            if (2 * chunk + 1 < nkb)
-                k_scale[sh * nkb + 2 * chunk + 1] = sc1;
-        }
-    }
-    const float rc0 = sc0 != 0.0f ? __fdiv_rn(1.0f, sc0) : 0.0f;
-    const float rc1 = sc1 != 0.0f ? __fdiv_rn(1.0f, sc1) : 0.0f;
-    float2 nmu[4];                        // -mu (Q: -0, so that x + nmu = x exactly)
-#pragma unroll
-    for (int j = 0; j < 4; j++)
-        nmu[j] = make_float2(-mu[2 * j], -mu[2 * j + 1]);
-    int8_t *dst = kind == 0 ? q_i8 : k_i8;
-#pragma unroll
-    for (int i = 0; i < kSteps; i++) {
-        const int row = i * kRowStep + r_in;
-        if (row >= nrows)
-            break;
-        const float scale = i < kHalfSteps ? sc0 : sc1;
-        const float rcp = i < kHalfSteps ? rc0 : rc1;
-        float f[8];
-        unpack8(s_x[row * kGpr + cg], f);
-        float2 x[4];
-#pragma unroll
-        for (int j = 0; j < 4; j++)
-            x[j] = add2(make_float2(f[2 * j], f[2 * j + 1]), nmu[j]);
-        const uint2 w = int8_codes8(x, scale, rcp);
-        *reinterpret_cast<uint2 *>(dst + L.offset(s, start, h, row0 + row) + c0) = w;
-    }
+    // ---- Q / K codes
+    if (kind == 0)
+        qk_chunk<D, kQG>(s_x, mu, cg, r_in, nrows, row0, chunk, q_scale + sh * nqb, nqb, q_i8, L,
+                         s, start, h, s_red);
+    else
+        qk_chunk<D, kKG>(s_x, mu, cg, r_in, nrows, row0, chunk, k_scale + sh * nkb, nkb, k_i8, L,
+                         s, start, h, s_red);
 }
 
 }  // namespace
@@ -517,7 +563,7 @@ cudaError_t launch_colstats(const __half *k, const __half *v, const ColStats &cs
 cudaError_t launch_quant(const __half *q, const __half *k, const __half *v, const ColStats &cs,
                          int8_t *q_i8, float *q_scale, int8_t *k_i8, float *k_scale,
                          float *k_mean, uint8_t *v_e4m3, float *v_scale, float *v_mean,
-                         const SeqLayout &Lq, const SeqLayout &Lk, int *status,
+                         const SeqLayout &Lq, const SeqLayout &Lk, bool fine, int *status,
                          cudaStream_t st)
 {
     const int with_q = q_i8 != nullptr ? 1 : 0;
@@ -530,14 +576,10 @@ cudaError_t launch_quant(const __half *q, const __half *k, const __half *v, cons
     if (with_q && (Lq.nseq != Lk.nseq || Lq.H != Lk.H || Lq.d != Lk.d))
         return cudaErrorInvalidValue;
     dim3 grid(nx, Lk.H, Lk.nseq);
-    if (Lk.d == 128)
-        quant_kernel<128><<<grid, kThreads, 0, st>>>(q, k, v, cs, q_i8, q_scale, k_i8, k_scale,
-                                                     k_mean, v_e4m3, v_scale, v_mean, Lq, Lk,
-                                                     with_q, nkc, status);
-    else
-        quant_kernel<64><<<grid, kThreads, 0, st>>>(q, k, v, cs, q_i8, q_scale, k_i8, k_scale,
-                                                    k_mean, v_e4m3, v_scale, v_mean, Lq, Lk,
-                                                    with_q, nkc, status);
+    auto kern = Lk.d == 128 ? (fine ? quant_kernel<128, true> : quant_kernel<128, false>)
+                            : (fine ? quant_kernel<64, true> : quant_kernel<64, false>);
+    kern<<<grid, kThreads, 0, st>>>(q, k, v, cs, q_i8, q_scale, k_i8, k_scale, k_mean, v_e4m3,
+                                    v_scale, v_mean, Lq, Lk, with_q, nkc, status);
     return cudaGetLastError();
 }
 

@@ -91,11 +91,13 @@ cudaError_t launch_colstats(const __half *k, const __half *v, const ColStats &cs
                             const SeqLayout &L, int *status, cudaStream_t st);
 // Quantizes Q and K (q_i8 != nullptr) and/or V (v_e4m3 != nullptr). K is smoothed when
 // cs.ksum is set, V when cs.vsum is set (its mean goes to v_mean if that is set). Q
-// lives in layout Lq, K and V in Lk (the same layout for self-attention).
+// lives in layout Lq, K and V in Lk (the same layout for self-attention). fine: one Q
+// scale per token and one K scale per 32 tokens (q_scale [nseq,H,maxq], k_scale
+// [nseq,H,ceil(maxk/32)]); else per-block scales (128 Q tokens, 64 K tokens).
 cudaError_t launch_quant(const __half *q, const __half *k, const __half *v, const ColStats &cs,
                          int8_t *q_i8, float *q_scale, int8_t *k_i8, float *k_scale,
                          float *k_mean, uint8_t *v_e4m3, float *v_scale, float *v_mean,
-                         const SeqLayout &Lq, const SeqLayout &Lk, int *status,
+                         const SeqLayout &Lq, const SeqLayout &Lk, bool fine, int *status,
                          cudaStream_t st);
 
 struct AttnArgs {
@@ -111,6 +113,7 @@ struct AttnArgs {
     int causal;
     int pv_mode;
     float sm_scale;
+    int fine;             // scales per Q token and per 32 K tokens (else per block)
 };
 // Queries in layout Lq, keys and values in Lk (the same layout for self-attention; with
 // different lengths the causal mask aligns at the bottom right).

@@ -393,3 +393,60 @@ def test_prefill_kv_config_sampled():
             tag = f"prefill kv head {(s, h)} rows {r0}:{r1}"
             assert_vs_oracle(got[mask], ref[mask], tag)
             assert_vs_fp64(got[mask], exact[mask], False, tag)
+
+
+# --------------------------------- finer scale groups (per Q token, per 32 K tokens)
+
+
+FINE_ATTN = [(1, 1, 128, False), (129, 129, 64, True), (513, 513, 128, False),
+             (300, 1000, 128, True), (640, 640, 64, True)]
+
+
+@pytest.mark.parametrize("pv", ["fp16", "fp8"])
+@pytest.mark.parametrize("Nq,Nk,d,causal", FINE_ATTN)
+def test_fine_small_full_compare(Nq, Nk, d, causal, pv):
+    B, H = 2, 2
+    w = inputs.Workload("t", 500 + Nq + Nk, B, H, Nk, d, causal, 2.0, nq=Nq)
+    q, k, v = inputs.make_dense(w)
+    out = sage.sageattn(q.cuda(), k.cuda(), v.cuda(), causal, True, PV[pv], fine=True)
+    assert sage.sage_get_device_status() == 0
+    got = _np(out)
+    lq, lk = oracle.Layout.dense(B, H, Nq, d), oracle.Layout.dense(B, H, Nk, d)
+    ref = oracle.sage_attention(q.numpy(), k.numpy(), v.numpy(), lq, causal, True, PV[pv],
+                                kv_layout=lk, fine=True)
+    tag = f"fine Nq={Nq} Nk={Nk} d={d} causal={causal} {pv}"
+    assert_vs_oracle(got, ref, tag)
+    exact = oracle.attn_fp64(q.numpy(), k.numpy(), v.numpy(), lq, causal, 1 / math.sqrt(d),
+                             kv_layout=lk)
+    assert_vs_fp64(got, exact, pv == "fp8", tag)
+
+
+def test_fine_quantized_entry_matches_fused():
+    B, H, N, d = 2, 3, 700, 128
+    w = inputs.Workload("t", 101, B, H, N, d, True, 1.0)
+    q, k, v = (t.cuda() for t in inputs.make_dense(w))
+    fused = sage.sageattn(q, k, v, True, True, sage.SAGE_PV_FP16, fine=True)
+    z = sage.quant_qk(q, k, True, fine=True)
+    split = sage.attn_quantized(z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], v, None, True,
+                                sage.SAGE_PV_FP16, fine=True)
+    assert sage.sage_get_device_status() == 0
+    assert torch.equal(fused, split)
+
+
+def test_fine_groups_more_accurate_on_row_outliers():
+    N, d = 1024, 128
+    g = torch.Generator().manual_seed(111)
+    q = torch.randn((1, 4, N, d), generator=g)
+    q *= torch.where(torch.arange(N) % 16 == 0, 24.0, 0.25)[None, None, :, None]
+    k = torch.randn((1, 4, N, d), generator=g)
+    k *= torch.where((torch.arange(N) // 32) % 2 == 0, 6.0, 0.5)[None, None, :, None]
+    v = torch.randn((1, 4, N, d), generator=g)
+    q, k, v = q.half(), k.half(), v.half()
+    fine = _np(sage.sageattn(q.cuda(), k.cuda(), v.cuda(), False, True, sage.SAGE_PV_FP16,
+                             fine=True))
+    block = _np(sage.sageattn(q.cuda(), k.cuda(), v.cuda(), False, True, sage.SAGE_PV_FP16))
+    assert sage.sage_get_device_status() == 0
+    exact = oracle.attn_fp64(q.numpy(), k.numpy(), v.numpy(), oracle.Layout.dense(1, 4, N, d),
+                             False, 1 / math.sqrt(d))
+    assert rel_l1(fine, exact) < 0.5 * rel_l1(block, exact)
+    assert rel_l1(fine, exact) < 0.02

@@ -200,3 +200,30 @@ def test_quant_v_fp8_ws_matches_allocating_entries():
             assert torch.equal(mean, ref[2])
     with pytest.raises(sage.SageError):
         sage.sage_quant_v_fp8_ws(v, codes, scales, None, B, H, N, d, ws, ws.numel() - 16)
+
+
+FINE_CASES = [(1, 2, 256, 64, 256), (2, 3, 300, 128, 300), (1, 2, 17, 128, 17),
+              (2, 2, 200, 64, 700), (1, 1, 1, 128, 33)]
+
+
+@pytest.mark.parametrize("B,H,Nq,d,Nk", FINE_CASES)
+def test_quant_qk_fine_bit_exact(B, H, Nq, d, Nk):
+    w = inputs.Workload("t", 81 + Nq + Nk, B, H, Nk, d, False, 2.0, nq=Nq)
+    q, k, _ = inputs.make_dense(w)
+    z = sage.quant_qk(q.cuda(), k.cuda(), True, fine=True)
+    assert sage.sage_get_device_status() == 0
+    ref = oracle.quant_qk(q.numpy(), k.numpy(), oracle.Layout.dense(B, H, Nq, d), True,
+                          kv_layout=oracle.Layout.dense(B, H, Nk, d), fine=True)
+    _check_qk(z, ref, f"fine {B}x{H}x{Nq}x{Nk}x{d}")
+
+
+def test_quant_fine_varlen_bit_exact():
+    H, d = 4, 128
+    lens = [1, 127, 128, 0, 700, 33]
+    w = inputs.Workload("t", 88, 0, H, 0, d, True, 2.0, nseq=len(lens))
+    q, k, v, cu = inputs.make_varlen(w, lens=lens)
+    z = sage.quant_qk_varlen(q.cuda(), k.cuda(), cu.cuda(), max(lens), True, fine=True)
+    assert sage.sage_get_device_status() == 0
+    ref = oracle.quant_qk(q.numpy(), k.numpy(), oracle.Layout.packed(cu.tolist(), H, d), True,
+                          fine=True)
+    _check_qk(z, ref, "fine varlen")

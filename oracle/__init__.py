@@ -49,8 +49,9 @@ def lib():
         L.oracle_head_channel_mean.argtypes = [P, i64, i64, i32, P]
         L.oracle_head_quant_int8.argtypes = [P, P, i64, i64, i32, i32, P, P]
         L.oracle_head_quant_v_fp8.argtypes = [P, P, i64, i64, i32, P, P]
-        L.oracle_head_attn_quant.argtypes = [P, P, P, P, P, P, P, i64, i64, i64, i32, i32, i32,
-                                             f64, i32, i32, i32, i64, i64, P]
+        L.oracle_head_attn_quant.argtypes = [P, P, P, P, P, P, P, P, i64, i64, i64, i32, i32,
+                                             i32, f64, i32, i32, i32, i64, i64, P]
+        L.oracle_head_q_comp.argtypes = [P, P, P, i64, i64, i32, P]
         L.oracle_head_attn_fp64.argtypes = [P, P, P, i64, i64, i64, i32, i32, f64, i64, i64, P]
         L.oracle_f16_to_f64.argtypes = [ctypes.c_uint16]
         L.oracle_f16_to_f64.restype = f64
@@ -171,18 +172,38 @@ def quant_int8(x: np.ndarray, layout: Layout, blk: int, mu: Optional[np.ndarray]
     return codes, scales
 
 
+def q_comp(k: np.ndarray, kv_layout: Layout, muk: Optional[np.ndarray], muq: np.ndarray,
+           heads=None) -> np.ndarray:
+    """Smooth-Q compensation mean(Q) K^T per key: [nseq, H, maxlen_k] fp32."""
+    kb = _bits16(k)
+    comp = np.zeros((kv_layout.nseq, kv_layout.H, kv_layout.maxlen), np.float32)
+    for s, h, off, n in kv_layout.heads(heads):
+        sh = s * kv_layout.H + h
+        mkp = _ptr(muk, sh * kv_layout.d) if muk is not None else None
+        lib().oracle_head_q_comp(_ptr(kb, off), mkp, _ptr(muq, sh * kv_layout.d), n,
+                                 kv_layout.stride, kv_layout.d, _ptr(comp, sh * kv_layout.maxlen))
+    return comp
+
+
 def quant_qk(q: np.ndarray, k: np.ndarray, layout: Layout, smooth_k: bool = True, heads=None,
-             kv_layout: Optional[Layout] = None, fine: bool = False):
+             kv_layout: Optional[Layout] = None, fine: bool = False, smooth_q: bool = False):
     """Smooth K, then per-block INT8 of Q (128 tokens) and K (64 tokens), for every (or
     each selected) head; with ``fine``, one Q scale per token and one K scale per 32
-    tokens. ``kv_layout`` places K when it has its own lengths (default: Q's layout)."""
+    tokens. ``kv_layout`` places K when it has its own lengths (default: Q's layout).
+    ``smooth_q``: Q - mean(Q) is quantized and the compensation mean(Q) K^T is returned
+    as ``q_comp`` [nseq, H, maxlen_k] (with the Q mean as ``q_mean``)."""
     kvl = layout if kv_layout is None else kv_layout
     zeros = np.zeros((kvl.nseq, kvl.H, kvl.d), np.float32)
     mu = k_mean(k, kvl, heads) if smooth_k else zeros
-    q_i8, q_scale = quant_int8(q, layout, Q_FINE if fine else Q_BLOCK, None, heads)
+    muq = channel_mean(q, layout, heads) if smooth_q else None
+    q_i8, q_scale = quant_int8(q, layout, Q_FINE if fine else Q_BLOCK, muq, heads)
     k_i8, k_scale = quant_int8(k, kvl, K_FINE if fine else K_BLOCK, mu if smooth_k else None,
                                heads)
-    return dict(q_i8=q_i8, q_scale=q_scale, k_i8=k_i8, k_scale=k_scale, k_mean=mu)
+    z = dict(q_i8=q_i8, q_scale=q_scale, k_i8=k_i8, k_scale=k_scale, k_mean=mu)
+    if smooth_q:
+        z["q_mean"] = muq
+        z["q_comp"] = q_comp(k, kvl, mu if smooth_k else None, muq, heads)
+    return z
 
 
 def quant_v_fp8(v: np.ndarray, layout: Layout, heads=None, mu: Optional[np.ndarray] = None):
@@ -203,9 +224,11 @@ def attn_quant(q_i8, q_scale, k_i8, k_scale, v, v_scale, layout: Layout, causal:
                pv_mode: int, sm_scale: float, tile_n: int = 128, heads=None,
                rows: Optional[Tuple[int, int]] = None,
                v_mean: Optional[np.ndarray] = None,
-               kv_layout: Optional[Layout] = None, fine: bool = False) -> np.ndarray:
+               kv_layout: Optional[Layout] = None, fine: bool = False,
+               q_comp: Optional[np.ndarray] = None) -> np.ndarray:
     """Quantized attention from codes and scales; fp16 output, NaN where not computed.
-    ``fine``: the scales are per Q token and per 32 K tokens (quant_qk(fine=True)).
+    ``fine``: the scales are per Q token and per 32 K tokens (quant_qk(fine=True));
+    ``q_comp`` [nseq, H, maxlen_k]: the smooth-Q compensation added to the scores.
 
     ``v`` is fp16 V (FP16 mode) or its E4M3 codes as uint8 (FP8 mode); ``v_mean``
     [nseq, H, d] (FP8 mode, smooth V) is added to every output row. ``kv_layout`` places
@@ -225,8 +248,9 @@ def attn_quant(q_i8, q_scale, k_i8, k_scale, v, v_scale, layout: Layout, causal:
         sh = s * layout.H + h
         vsp = _ptr(v_scale, sh * layout.d) if v_scale is not None else None
         vmp = _ptr(v_mean, sh * layout.d) if v_mean is not None else None
+        cp = _ptr(q_comp, sh * kvl.maxlen) if q_comp is not None else None
         lib().oracle_head_attn_quant(_ptr(q_i8, off), _ptr(q_scale, sh * nqb), _ptr(k_i8, koff),
-                                     _ptr(k_scale, sh * nkb), _ptr(vv, koff), vsp, vmp, n, nk,
+                                     _ptr(k_scale, sh * nkb), _ptr(vv, koff), vsp, vmp, cp, n, nk,
                                      layout.stride, layout.d, int(causal), int(pv_mode),
                                      float(sm_scale), int(tile_n),
                                      Q_FINE if fine else Q_BLOCK, K_FINE if fine else K_BLOCK,
@@ -261,19 +285,21 @@ def sage_attention(q, k, v, layout: Layout, causal: bool = False, smooth_k: bool
                    pv_mode: int = PV_FP16, sm_scale: Optional[float] = None,
                    tile_n: int = 128, heads=None, rows=None,
                    smooth_v: bool = False, kv_layout: Optional[Layout] = None,
-                   fine: bool = False) -> np.ndarray:
-    """The whole method from fp16 Q, K, V: smooth K (and, in FP8 mode, optionally V),
-    quantize, quantized attention. ``kv_layout`` places K and V when their lengths differ
-    from Q's; ``fine`` selects per-token Q and per-32-token K scales."""
+                   fine: bool = False, smooth_q: bool = False) -> np.ndarray:
+    """The whole method from fp16 Q, K, V: smooth K (and, in FP8 mode, optionally V;
+    optionally Q, with the mean(Q) K^T compensation), quantize, quantized attention.
+    ``kv_layout`` places K and V when their lengths differ from Q's; ``fine`` selects
+    per-token Q and per-32-token K scales."""
     if smooth_v and pv_mode != PV_FP8:
         raise ValueError("smooth V applies to the FP8 P.V mode")
     kvl = layout if kv_layout is None else kv_layout
     sm = default_sm_scale(layout.d, sm_scale)
-    z = quant_qk(q, k, layout, smooth_k, heads, kvl, fine)
+    z = quant_qk(q, k, layout, smooth_k, heads, kvl, fine, smooth_q)
+    qc = z.get("q_comp")
     if pv_mode == PV_FP8:
         vm = channel_mean(v, kvl, heads) if smooth_v else None
         v8, vs = quant_v_fp8(v, kvl, heads, vm)
         return attn_quant(z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], v8, vs, layout,
-                          causal, PV_FP8, sm, tile_n, heads, rows, vm, kvl, fine)
+                          causal, PV_FP8, sm, tile_n, heads, rows, vm, kvl, fine, qc)
     return attn_quant(z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], v, None, layout,
-                      causal, PV_FP16, sm, tile_n, heads, rows, None, kvl, fine)
+                      causal, PV_FP16, sm, tile_n, heads, rows, None, kvl, fine, qc)

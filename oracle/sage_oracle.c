@@ -21,6 +21,9 @@
  *   - Smooth V (FP8 mode): V <- V - mean(V) with the mean per channel over the tokens
  *     of one head, the attention run on the smoothed V, and mean(V) added to the
  *     output. (Same section, the paragraph after item (4).)
+ *   - Smooth Q: Q <- Q - mean(Q) (per channel over the query tokens of one head) before
+ *     quantizing, and the vector-matrix product mean(Q) K^T added back to the scores.
+ *     (Same section, item (1).)
  *   - The exact reference O = softmax(sm_scale Q K^T + mask) V in fp64, and the
  *     smoothing invariant softmax(QK^T) = softmax(Q(K - mean K)^T) it must satisfy.
  *
@@ -240,6 +243,29 @@ void oracle_head_quant_v_fp8(const uint16_t *V, const float *mu, int64_t n, int6
     }
 }
 
+/* ------------------------------------------------ smooth Q: score compensation */
+
+/*
+ * comp[j] = sum over c of muq[c] * (fp32(K[j,c]) - muk[c]) for the n keys of one head:
+ * the mean(Q) K^T term that smoothing Q removes from the scores, with K as it enters
+ * the INT8 quantization (smoothed by muk when that is not NULL, one fp32 subtraction).
+ * The sum is taken in fp64 and rounded once to fp32.
+ */
+void oracle_head_q_comp(const uint16_t *K, const float *muk, const float *muq, int64_t n,
+                        int64_t stride, int d, float *comp)
+{
+    for (int64_t j = 0; j < n; j++) {
+        double acc = 0.0;
+        for (int c = 0; c < d; c++) {
+            float x = (float)oracle_f16_to_f64(K[j * stride + c]);
+            if (muk)
+                x = x - muk[c];
+            acc += (double)muq[c] * (double)x;
+        }
+        comp[j] = (float)acc;
+    }
+}
+
 /* ----------------------------------------------------------- quantized attention */
 
 enum { ORACLE_PV_FP16 = 0, ORACLE_PV_FP8 = 1 };
@@ -250,9 +276,10 @@ enum { ORACLE_PV_FP16 = 0, ORACLE_PV_FP8 = 1 };
  * longer sequence, e.g. prefill against cached keys), following the method's steps in
  * order:
  *   S_int[i,j] = sum_c q[i,c] k[j,c] in integers (INT32 range is never exceeded);
- *   t[i,j] = S_int * sq[i/qg] * sk[j/kg] * sm_scale * log2(e)  (base-2 logits), where
- *   qg and kg are the tokens per Q and K scale (128 and 64 for per-block scales, 1 and
- *   32 for the finer groups);
+ *   t[i,j] = (S_int * sq[i/qg] * sk[j/kg] + comp[j]) * sm_scale * log2(e) (base-2
+ *   logits), where qg and kg are the tokens per Q and K scale (128 and 64 for per-block
+ *   scales, 1 and 32 for the finer groups) and comp is the smooth-Q compensation
+ *   (NULL: none);
  *   causal: key j is visible to query i when j <= i + (nk - nq) (the mask aligned at
  *   the bottom-right corner; the square mask j <= i when nq = nk); a query that sees no
  *   key (only when nq > nk) gets a zero output row;
@@ -268,7 +295,8 @@ enum { ORACLE_PV_FP16 = 0, ORACLE_PV_FP8 = 1 };
  */
 void oracle_head_attn_quant(const int8_t *qc, const float *qs, const int8_t *kc,
                             const float *ks, const void *v, const float *vs, const float *vm,
-                            int64_t nq, int64_t nk, int64_t stride, int d, int causal,
+                            const float *comp, int64_t nq, int64_t nk, int64_t stride, int d,
+                            int causal,
                             int pv_mode, double sm_scale, int tile_n, int qg, int kg,
                             int64_t r0, int64_t r1, uint16_t *out)
 {
@@ -297,7 +325,10 @@ void oracle_head_attn_quant(const int8_t *qc, const float *qs, const int8_t *kc,
                 int32_t S = 0;
                 for (int c = 0; c < d; c++)
                     S += (int32_t)qc[i * stride + c] * (int32_t)kc[j * stride + c];
-                t[j - j0] = (double)S * (double)qs[i / qg] * (double)ks[j / kg] * sm_scale * log2e;
+                double sij = (double)S * (double)qs[i / qg] * (double)ks[j / kg];
+                if (comp)
+                    sij += (double)comp[j];
+                t[j - j0] = sij * sm_scale * log2e;
                 if (t[j - j0] > tmax)
                     tmax = t[j - j0];
             }

@@ -469,3 +469,98 @@ def test_fine_groups_beat_blocks_on_row_outliers():
     block = oracle.sage_attention(q, k, v, lay, False, True, PV_FP16, sm)
     assert _rel_l1(fine, exact) < 0.5 * _rel_l1(block, exact)
     assert _rel_l1(fine, exact) < 0.02
+
+
+# Smooth Q (「4比特量化三倍加速不掉点！清华即插即用的SageAttention迎来升级」, 技术方案 (1)): Q - mean(Q) is quantized and the
+# vector-matrix product mean(Q) K^T is added back to the scores.
+
+def _q_with_channel_offsets(N, d, seed, amp=8.0):
+    q = _rand16((1, 2, N, d), seed).astype(np.float64)
+    off = np.random.default_rng(seed + 1).uniform(-amp, amp, d)
+    return (q + off).astype(np.float16)
+
+
+def test_smooth_q_compensation_closed_form():
+    N, d = 150, 32
+    q = _q_with_channel_offsets(N, d, 231)
+    k = (_rand16((1, 2, N, d), 232).astype(np.float64) + 3.0).astype(np.float16)
+    lay = Layout.dense(1, 2, N, d)
+    z = oracle.quant_qk(q, k, lay, True, smooth_q=True)
+    muq = q.astype(np.float64).mean(axis=2).astype(np.float32)
+    assert np.array_equal(z["q_mean"], muq)
+    ks = k.astype(np.float32) - z["k_mean"][:, :, None, :]          # K as it is quantized
+    ref = np.einsum("bhc,bhnc->bhn", muq.astype(np.float64), ks.astype(np.float64))
+    assert np.allclose(z["q_comp"], ref, rtol=1e-6, atol=1e-6)
+    # the Q codes reconstruct Q - mean(Q), not Q, within half a scale step
+    qs = q.astype(np.float32) - muq[:, :, None, :]
+    for blk in range(2):
+        rows = slice(128 * blk, min(N, 128 * blk + 128))
+        sc = z["q_scale"][:, :, blk][:, :, None, None]
+        rec = sc * z["q_i8"][:, :, rows].astype(np.float32)
+        assert np.all(np.abs(rec - qs[:, :, rows]) <= sc * 0.5001 + 1e-6)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("pv_mode", [PV_FP16, PV_FP8])
+def test_smooth_q_single_tile_closed_form(causal, pv_mode):
+    N, d = 200, 32
+    q = _q_with_channel_offsets(N, d, 241)[:, :1]
+    k, v = (_rand16((1, 1, N, d), s) for s in (242, 243))
+    lay = Layout.dense(1, 1, N, d)
+    sm = 1 / math.sqrt(d)
+    z = oracle.quant_qk(q, k, lay, True, smooth_q=True)
+    vq, vs = (oracle.quant_v_fp8(v, lay) if pv_mode == PV_FP8 else (v, None))
+    got = oracle.attn_quant(z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], vq, vs, lay,
+                            causal, pv_mode, sm, tile_n=256, q_comp=z["q_comp"])
+    qc = z["q_i8"][0, 0].astype(np.int64)
+    kc = z["k_i8"][0, 0].astype(np.int64)
+    sq = z["q_scale"][0, 0][np.arange(N) // 128].astype(np.float64)
+    sk = z["k_scale"][0, 0][np.arange(N) // 64].astype(np.float64)
+    t = ((qc @ kc.T) * sq[:, None] * sk[None, :] + z["q_comp"][0, 0][None, :]) * sm / math.log(2)
+    if causal:
+        t[np.triu_indices(N, 1)] = -np.inf
+    p = np.exp2(t - t.max(axis=1, keepdims=True))
+    if pv_mode == PV_FP16:
+        O = p.astype(np.float16).astype(np.float64) @ v[0, 0].astype(np.float64) / p.sum(1, keepdims=True)
+    else:
+        P = torch.from_numpy(448 * p).to(torch.float32).to(torch.float8_e4m3fn).to(torch.float64).numpy()
+        vv = torch.from_numpy(vq[0, 0]).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+        O = P @ vv * vs[0, 0][None, :] / (448 * p.sum(1, keepdims=True))
+    ref = O.astype(np.float16).astype(np.float64)
+    diff = np.abs(got[0, 0].astype(np.float64) - ref)
+    assert diff.max() <= 2 * np.spacing(np.abs(ref).astype(np.float16)).astype(np.float64).max()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_smooth_q_needs_its_compensation(causal):
+    # with channel offsets in Q, smoothing Q keeps the scores' precision; dropping the
+    # compensation (a plausible slip) changes the result completely
+    N, d = 512, 64
+    q = _q_with_channel_offsets(N, d, 251)
+    k, v = (_rand16((1, 2, N, d), s) for s in (252, 253))
+    lay = Layout.dense(1, 2, N, d)
+    sm = 1 / math.sqrt(d)
+    exact = oracle.attn_fp64(q, k, v, lay, causal, sm)
+    sq = oracle.sage_attention(q, k, v, lay, causal, True, PV_FP16, sm, smooth_q=True)
+    plain = oracle.sage_attention(q, k, v, lay, causal, True, PV_FP16, sm)
+    assert _cos(sq, exact) > 0.9999 and _rel_l1(sq, exact) < 0.02
+    assert _rel_l1(sq, exact) < 0.7 * _rel_l1(plain, exact)
+    z = oracle.quant_qk(q, k, lay, True, smooth_q=True)
+    dropped = oracle.attn_quant(z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], v, None, lay,
+                                causal, PV_FP16, sm)
+    assert _rel_l1(dropped, exact) > 0.2
+
+
+def test_smooth_q_is_a_no_op_for_zero_mean_q():
+    # Q whose every channel sums to zero exactly: mean(Q) = 0, so the codes, the
+    # compensation (all zero) and the output equal plain smooth-K attention bit for bit
+    N, d = 256, 32
+    h = _rand16((1, 1, N // 2, d), 261)
+    q = np.concatenate([h, -h], axis=2)
+    k, v = (_rand16((1, 1, N, d), s) for s in (262, 263))
+    lay = Layout.dense(1, 1, N, d)
+    z = oracle.quant_qk(q, k, lay, True, smooth_q=True)
+    assert not z["q_mean"].any() and not z["q_comp"].any()
+    a = oracle.sage_attention(q, k, v, lay, True, True, PV_FP16, smooth_q=True)
+    b = oracle.sage_attention(q, k, v, lay, True, True, PV_FP16)
+    assert np.array_equal(a, b)

@@ -79,16 +79,24 @@ enum { SAGE_PV_FP16 = 0, SAGE_PV_FP8 = 1 };
  *     fp32), the E4M3 codes and per-channel scales taken of the smoothed V, and mean(V)
  *     added to every output row. Softmax rows sum to one, so the exact result is
  *     unchanged; the E4M3 range is no longer spent on a channel offset.
+ *   SAGE_SMOOTH_Q (4): smooth Q ("SageAttention2" article, 技术方案 (1)): Q <- Q - mean(Q),
+ *     the mean per channel over the query tokens of one head (fp64 sum, rounded once),
+ *     and the vector-matrix product mean(Q) K^T (with K as it is quantized, i.e.
+ *     smoothed) added back to every score row: comp[j] = sum_c mean(Q)[c] K'[j,c] in
+ *     fp32, and the base-2 logit is (S q_scale k_scale + comp[j]) sm_scale log2(e). The
+ *     compensation varies along a row, so the kernel takes the exact row max of the
+ *     dequantized scores instead of the integer max; it costs some throughput.
  *   SAGE_QK_FINE (8): finer quantization groups ("SageAttention2" article, 技术方案 (2),
  *     which groups tokens by the threads that hold them in the tensor-core layout): here
  *     every query row is held by one thread, so Q gets one scale per token, and K one
  *     scale per 32 tokens (the tensor-memory load width). q_scale is then
  *     [nseq, H, maxlen_q] and k_scale [nseq, H, ceil(maxlen_k / 32)].
- * Other bits give SAGE_ERR_INVALID_ARG (the Q/K quantization entry points accept only
- * SAGE_SMOOTH_K and SAGE_QK_FINE); SAGE_SMOOTH_V with SAGE_PV_FP16 gives
- * SAGE_ERR_UNSUPPORTED (fp16 V is not quantized, so there is nothing to smooth for).
+ * Other bits give SAGE_ERR_INVALID_ARG (sage_quant_qk, _ws and _varlen accept only
+ * SAGE_SMOOTH_K and SAGE_QK_FINE; sage_quant_qk_kv also SAGE_SMOOTH_Q); SAGE_SMOOTH_V
+ * with SAGE_PV_FP16 gives SAGE_ERR_UNSUPPORTED (fp16 V is not quantized, so there is
+ * nothing to smooth for).
  */
-enum { SAGE_SMOOTH_K = 1, SAGE_SMOOTH_V = 2, SAGE_QK_FINE = 8 };
+enum { SAGE_SMOOTH_K = 1, SAGE_SMOOTH_V = 2, SAGE_SMOOTH_Q = 4, SAGE_QK_FINE = 8 };
 
 /* Opaque CUDA stream (binary-compatible with cudaStream_t). */
 typedef struct CUstream_st *sage_stream_t;
@@ -135,15 +143,19 @@ SAGE_API sage_status_t sage_quant_qk_varlen(const void *q, const void *k, const 
                                    int8_t *q_i8, float *q_scale, int8_t *k_i8, float *k_scale,
                                    float *k_mean, int smooth_k, sage_stream_t stream);
 
-/* sage_quant_qk for Q [B,H,Nq,d] and K [B,H,Nk,d] of different lengths: q_scale is
- * [B,H,ceil(Nq/128)], k_scale [B,H,ceil(Nk/64)], and the K mean is taken over the Nk
- * keys. workspace: NULL (a stream-ordered allocation for the fp64 K sums) or caller
- * scratch of at least B*H*d*8 bytes, 16-byte aligned. */
+/* Steps 1-2 in general form: Q [B,H,Nq,d] and K [B,H,Nk,d] (Nq may differ from Nk; the
+ * K mean is taken over the Nk keys), flags = SAGE_SMOOTH_K | SAGE_SMOOTH_Q |
+ * SAGE_QK_FINE. Scales: q_scale [B,H,ceil(Nq/128)] and k_scale [B,H,ceil(Nk/64)], or
+ * with SAGE_QK_FINE [B,H,Nq] and [B,H,ceil(Nk/32)]. With SAGE_SMOOTH_Q the Q codes are
+ * those of Q - q_mean, q_mean [B,H,d] and the score compensation q_comp
+ * [B,H,ceil(Nk/128)*128] (entries past Nk are 0) are written; otherwise both may be
+ * NULL. workspace: NULL (a stream-ordered allocation for the fp64 column sums) or caller
+ * scratch of at least B*H*d*8 bytes (B*H*d*16 with SAGE_SMOOTH_Q), 16-byte aligned. */
 SAGE_API sage_status_t sage_quant_qk_kv(const void *q, const void *k, int8_t *q_i8,
                                         float *q_scale, int8_t *k_i8, float *k_scale,
-                                        float *k_mean, int B, int H, int Nq, int Nk, int d,
-                                        int smooth_k, void *workspace, size_t ws_bytes,
-                                        sage_stream_t stream);
+                                        float *k_mean, float *q_mean, float *q_comp, int B,
+                                        int H, int Nq, int Nk, int d, int flags,
+                                        void *workspace, size_t ws_bytes, sage_stream_t stream);
 
 /*
  * V to FP8 E4M3 (「4比特量化三倍加速不掉点！清华即插即用的SageAttention迎来升级」, 技术方案 (4)) with one fp32 scale per
@@ -263,15 +275,16 @@ SAGE_API sage_status_t sage_attn_fwd_quantized_smooth_v(const int8_t *q_i8, cons
 
 /* Step 3 alone with Nq queries and Nk keys (codes and scales from sage_quant_qk_kv; V
  * codes from sage_quant_v_fp8[_smooth] with N = Nk); v_mean selects the smooth-V
- * epilogue (FP8 only) or is NULL; flags is 0 or SAGE_QK_FINE (the scale layout the codes
+ * epilogue (FP8 only) or is NULL; q_comp (16-byte aligned) is the smooth-Q compensation
+ * of sage_quant_qk_kv or NULL; flags is 0 or SAGE_QK_FINE (the scale layout the codes
  * were made with). */
 SAGE_API sage_status_t sage_attn_fwd_quantized_kv(const int8_t *q_i8, const float *q_scale,
                                                   const int8_t *k_i8, const float *k_scale,
                                                   const void *v, const float *v_scale,
-                                                  const float *v_mean, void *out, int B, int H,
-                                                  int Nq, int Nk, int d, int causal, int pv_mode,
-                                                  float sm_scale, int flags,
-                                                  sage_stream_t stream);
+                                                  const float *v_mean, const float *q_comp,
+                                                  void *out, int B, int H, int Nq, int Nk, int d,
+                                                  int causal, int pv_mode, float sm_scale,
+                                                  int flags, sage_stream_t stream);
 
 /*
  * Debug: the integer score tiles S = q_i8 k_i8^T (int32, [B,H,N,N]) exactly as the

@@ -33,6 +33,7 @@ SAGE_PV_FP16 = 0
 SAGE_PV_FP8 = 1
 SAGE_SMOOTH_K = 1     # flags of the fused entry points' smooth_k argument
 SAGE_SMOOTH_V = 2
+SAGE_SMOOTH_Q = 4
 SAGE_QK_FINE = 8
 
 Q_BLOCK = 128
@@ -47,12 +48,13 @@ _S = ctypes.c_int  # sage_status_t
 SIGNATURES = {
     "sage_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
     "sage_workspace_size_kv": (_Z, [_I, _I, _I, _I, _I, _I, _I, _I]),
-    "sage_quant_qk_kv": (_S, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _Z, _P]),
+    "sage_quant_qk_kv": (_S, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _Z,
+                              _P]),
     "sage_attn_fwd_kv": (_S, [_P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _F, _P, _Z, _P]),
     "sage_attn_varlen_fwd_kv": (_S, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I,
                                      _I, _F, _P, _Z, _P]),
-    "sage_attn_fwd_quantized_kv": (_S, [_P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I,
-                                        _I, _F, _I, _P]),
+    "sage_attn_fwd_quantized_kv": (_S, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I,
+                                        _I, _I, _F, _I, _P]),
     "sage_quant_qk": (_S, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "sage_quant_qk_ws": (_S, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]),
     "sage_quant_qk_varlen": (_S, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _I, _P]),
@@ -146,11 +148,11 @@ def sage_workspace_size_kv(nseq, H, max_seqlen_q, max_seqlen_k, total_q, total_k
                                             d, pv_mode))
 
 
-def sage_quant_qk_kv(q, k, q_i8, q_scale, k_i8, k_scale, k_mean, B, H, Nq, Nk, d, smooth_k,
-                     workspace=None, ws_bytes=0, stream=None):
+def sage_quant_qk_kv(q, k, q_i8, q_scale, k_i8, k_scale, k_mean, q_mean, q_comp, B, H, Nq, Nk,
+                     d, flags, workspace=None, ws_bytes=0, stream=None):
     return _call("sage_quant_qk_kv", _ptr(q), _ptr(k), _ptr(q_i8), _ptr(q_scale), _ptr(k_i8),
-                 _ptr(k_scale), _ptr(k_mean), B, H, Nq, Nk, d, int(smooth_k), _ptr(workspace),
-                 int(ws_bytes), _stream(stream))
+                 _ptr(k_scale), _ptr(k_mean), _ptr(q_mean), _ptr(q_comp), B, H, Nq, Nk, d,
+                 int(flags), _ptr(workspace), int(ws_bytes), _stream(stream))
 
 
 def sage_attn_fwd_kv(q, k, v, out, B, H, Nq, Nk, d, causal, smooth_k, pv_mode, sm_scale,
@@ -169,11 +171,12 @@ def sage_attn_varlen_fwd_kv(q, k, v, out, cu_seqlens_q, cu_seqlens_k, nseq, tota
                  _ptr(workspace), int(ws_bytes), _stream(stream))
 
 
-def sage_attn_fwd_quantized_kv(q_i8, q_scale, k_i8, k_scale, v, v_scale, v_mean, out, B, H, Nq,
-                               Nk, d, causal, pv_mode, sm_scale, flags=0, stream=None):
+def sage_attn_fwd_quantized_kv(q_i8, q_scale, k_i8, k_scale, v, v_scale, v_mean, q_comp, out, B,
+                               H, Nq, Nk, d, causal, pv_mode, sm_scale, flags=0, stream=None):
     return _call("sage_attn_fwd_quantized_kv", _ptr(q_i8), _ptr(q_scale), _ptr(k_i8),
-                 _ptr(k_scale), _ptr(v), _ptr(v_scale), _ptr(v_mean), _ptr(out), B, H, Nq, Nk, d,
-                 int(causal), int(pv_mode), float(sm_scale), int(flags), _stream(stream))
+                 _ptr(k_scale), _ptr(v), _ptr(v_scale), _ptr(v_mean), _ptr(q_comp), _ptr(out), B,
+                 H, Nq, Nk, d, int(causal), int(pv_mode), float(sm_scale), int(flags),
+                 _stream(stream))
 
 
 def sage_quant_qk(q, k, q_i8, q_scale, k_i8, k_scale, k_mean, B, H, N, d, smooth_k, stream=None):
@@ -299,14 +302,15 @@ def _check_status(stream=None):
         raise SageError("device", code)
 
 
-def _smooth_flags(smooth_k: bool, smooth_v: bool, fine: bool = False) -> int:
+def _smooth_flags(smooth_k: bool, smooth_v: bool, fine: bool = False,
+                  smooth_q: bool = False) -> int:
     return ((SAGE_SMOOTH_K if smooth_k else 0) | (SAGE_SMOOTH_V if smooth_v else 0)
-            | (SAGE_QK_FINE if fine else 0))
+            | (SAGE_QK_FINE if fine else 0) | (SAGE_SMOOTH_Q if smooth_q else 0))
 
 
 def sageattn(q, k, v, causal: bool = False, smooth_k: bool = True, pv_mode: int = SAGE_PV_FP16,
              sm_scale: float = 0.0, out=None, stream=None, smooth_v: bool = False,
-             fine: bool = False):
+             fine: bool = False, smooth_q: bool = False):
     """O = SageAttention(q, k, v) for fp16 CUDA tensors q [B, H, Nq, d], k and v
     [B, H, Nk, d] (Nq != Nk: sage_attn_fwd_kv, causal mask aligned at the bottom right)."""
     import torch
@@ -314,7 +318,7 @@ def sageattn(q, k, v, causal: bool = False, smooth_k: bool = True, pv_mode: int 
     Nk = k.shape[2]
     if out is None:
         out = torch.empty_like(q)
-    flags = _smooth_flags(smooth_k, smooth_v, fine)
+    flags = _smooth_flags(smooth_k, smooth_v, fine, smooth_q)
     if Nq == Nk:
         sage_attn_fwd(q, k, v, out, B, H, Nq, d, causal, flags, pv_mode, sm_scale, stream)
     else:
@@ -354,9 +358,11 @@ def sageattn_varlen(q, k, v, cu_seqlens, max_seqlen: int, causal: bool = False,
     return out
 
 
-def quant_qk(q, k, smooth_k: bool = True, stream=None, fine: bool = False):
+def quant_qk(q, k, smooth_k: bool = True, stream=None, fine: bool = False,
+             smooth_q: bool = False):
     """Dense smooth-K + INT8: dict of q_i8, q_scale, k_i8, k_scale, k_mean (q [B,H,Nq,d]
-    and k [B,H,Nk,d] may differ in length; fine: per-token Q and per-32-token K scales)."""
+    and k [B,H,Nk,d] may differ in length; fine: per-token Q and per-32-token K scales;
+    smooth_q: also q_mean [B,H,d] and the score compensation q_comp [B,H,ceil(Nk/128)*128])."""
     import torch
     B, H, N, d = q.shape
     Nk = k.shape[2]
@@ -367,13 +373,18 @@ def quant_qk(q, k, smooth_k: bool = True, stream=None, fine: bool = False):
              k_i8=torch.empty(k.shape, dtype=torch.int8, device=dev),
              k_scale=torch.empty((B, H, math.ceil(Nk / kg)), dtype=torch.float32, device=dev),
              k_mean=torch.empty((B, H, d), dtype=torch.float32, device=dev))
-    flags = (SAGE_SMOOTH_K if smooth_k else 0) | (SAGE_QK_FINE if fine else 0)
-    if N == Nk and not fine:
+    flags = ((SAGE_SMOOTH_K if smooth_k else 0) | (SAGE_QK_FINE if fine else 0)
+             | (SAGE_SMOOTH_Q if smooth_q else 0))
+    if smooth_q:
+        z["q_mean"] = torch.empty((B, H, d), dtype=torch.float32, device=dev)
+        z["q_comp"] = torch.empty((B, H, math.ceil(Nk / 128) * 128), dtype=torch.float32,
+                                  device=dev)
+    if N == Nk and not fine and not smooth_q:
         sage_quant_qk(q, k, z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], z["k_mean"], B, H, N,
                       d, smooth_k, stream)
     else:
-        sage_quant_qk_kv(q, k, z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], z["k_mean"], B,
-                         H, N, Nk, d, flags, None, 0, stream)
+        sage_quant_qk_kv(q, k, z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], z["k_mean"],
+                         z.get("q_mean"), z.get("q_comp"), B, H, N, Nk, d, flags, None, 0, stream)
     return z
 
 
@@ -429,17 +440,17 @@ def quant_v_fp8_varlen(v, cu_seqlens, max_seqlen: int, stream=None, smooth_v: bo
 
 def attn_quantized(q_i8, q_scale, k_i8, k_scale, v, v_scale, causal: bool = False,
                    pv_mode: int = SAGE_PV_FP16, sm_scale: float = 0.0, out=None, stream=None,
-                   v_mean=None, fine: bool = False):
+                   v_mean=None, fine: bool = False, q_comp=None):
     """Step 3 on pre-quantized operands; v_mean (FP8 mode) selects the smooth-V epilogue,
-    fine the per-token Q / per-32-token K scale layout."""
+    fine the per-token Q / per-32-token K scale layout, q_comp the smooth-Q compensation."""
     import torch
     B, H, N, d = q_i8.shape
     Nk = k_i8.shape[2]
     if out is None:
         out = torch.empty(q_i8.shape, dtype=torch.float16, device=q_i8.device)
-    if Nk != N or fine:
-        sage_attn_fwd_quantized_kv(q_i8, q_scale, k_i8, k_scale, v, v_scale, v_mean, out, B, H, N,
-                                   Nk, d, causal, pv_mode, sm_scale,
+    if Nk != N or fine or q_comp is not None:
+        sage_attn_fwd_quantized_kv(q_i8, q_scale, k_i8, k_scale, v, v_scale, v_mean, q_comp, out,
+                                   B, H, N, Nk, d, causal, pv_mode, sm_scale,
                                    SAGE_QK_FINE if fine else 0, stream)
         return out
     if v_mean is not None:

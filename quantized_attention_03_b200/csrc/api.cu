@@ -98,6 +98,7 @@ struct Workspace {
     ColStats cs;                 // contiguous: one memset clears all of it
     uint8_t *v8 = nullptr;
     float *v_scale = nullptr, *v_mean = nullptr;
+    float *q_comp = nullptr;     // smooth Q: mean(Q) K^T per key, [nseq, H, comp_stride(maxk)]
     size_t stats_bytes = 0;      // bytes of the column statistics
     size_t total = 0;
 };
@@ -123,8 +124,10 @@ Workspace carve(char *base, int nseq, int H, int max_q, int max_k, int total_q, 
     w.q_scale = reinterpret_cast<float *>(take(heads * nqb * 4));
     w.k_scale = reinterpret_cast<float *>(take(heads * nkb * 4));
     w.k_mean = reinterpret_cast<float *>(take(heads * d * 4));
+    w.q_comp = reinterpret_cast<float *>(take(heads * (size_t)comp_stride(max_k) * 4));
     const size_t stats0 = off;
     w.cs.ksum = reinterpret_cast<double *>(take(heads * d * 8));
+    w.cs.qsum = reinterpret_cast<double *>(take(heads * d * 8));
     if (pv_mode == SAGE_PV_FP8) {
         w.cs.vsum = reinterpret_cast<double *>(take(heads * d * 8));
         w.cs.vhi = reinterpret_cast<uint32_t *>(take(heads * d * 4));
@@ -154,7 +157,7 @@ sage_status_t check_shape(int nseq, int H, int maxlen, int d)
 // The option flags of the fused entry points.
 sage_status_t check_smooth(int smooth, int pv_mode)
 {
-    if (smooth & ~(SAGE_SMOOTH_K | SAGE_SMOOTH_V | SAGE_QK_FINE))
+    if (smooth & ~(SAGE_SMOOTH_K | SAGE_SMOOTH_V | SAGE_SMOOTH_Q | SAGE_QK_FINE))
         return SAGE_ERR_INVALID_ARG;
     if ((smooth & SAGE_SMOOTH_V) && pv_mode != SAGE_PV_FP8)
         return SAGE_ERR_UNSUPPORTED;
@@ -179,7 +182,7 @@ sage_status_t forward(const void *q, const void *k, const void *v, void *out, co
     Workspace w = carve(ws, L.nseq, L.H, L.maxlen, LK.maxlen, L.total, LK.total, L.d, pv_mode);
     const bool fp8 = pv_mode == SAGE_PV_FP8;
     const bool sk = (smooth & SAGE_SMOOTH_K) != 0, sv = (smooth & SAGE_SMOOTH_V) != 0;
-    const bool fine = (smooth & SAGE_QK_FINE) != 0;
+    const bool fine = (smooth & SAGE_QK_FINE) != 0, sq = (smooth & SAGE_SMOOTH_Q) != 0;
     cudaError_t e = cudaMemsetAsync(w.cs.ksum, 0, w.stats_bytes, st);
     if (e != cudaSuccess)
         return cuda_fail(e);
@@ -191,15 +194,24 @@ sage_status_t forward(const void *q, const void *k, const void *v, void *out, co
         cs.ksum = nullptr;
     if (!sv)
         cs.vsum = nullptr;
+    if (!sq)
+        cs.qsum = nullptr;
     if ((e = launch_colstats(kh, vh, cs, LK, status, st)) != cudaSuccess)
         return cuda_fail(e);
+    if (sq) {                                  // Q column sums (the K-sum path over Q)
+        ColStats qs;
+        qs.ksum = cs.qsum;
+        if ((e = launch_colstats(qh, nullptr, qs, L, status, st)) != cudaSuccess)
+            return cuda_fail(e);
+    }
     if ((e = launch_quant(qh, kh, vh, cs, w.q_i8, w.q_scale, w.k_i8, w.k_scale, w.k_mean,
-                          fp8 ? w.v8 : nullptr, w.v_scale, sv ? w.v_mean : nullptr, L, LK,
-                          fine, status, st)) != cudaSuccess)
+                          fp8 ? w.v8 : nullptr, w.v_scale, sv ? w.v_mean : nullptr, nullptr,
+                          sq ? w.q_comp : nullptr, L, LK, fine, status, st)) != cudaSuccess)
         return cuda_fail(e);
     AttnArgs a{w.q_i8,     w.q_scale, w.k_i8, w.k_scale, fp8 ? (const void *)w.v8 : v,
-               w.v_scale,  sv ? w.v_mean : nullptr,     static_cast<__half *>(out),
-               nullptr,    causal,    pv_mode, resolve_scale(sm_scale, L.d), fine ? 1 : 0};
+               w.v_scale,  sv ? w.v_mean : nullptr,     sq ? w.q_comp : nullptr,
+               static_cast<__half *>(out), nullptr, causal, pv_mode,
+               resolve_scale(sm_scale, L.d), fine ? 1 : 0};
     sage_status_t herr;
     if ((e = launch_attention(a, L, LK, status, st, &herr)) != cudaSuccess)
         return herr != SAGE_OK ? herr : cuda_fail(e);
@@ -256,7 +268,8 @@ bool dense_fits(int B, int N) { return !(B > 0 && N > 0 && (int64_t)B * N > INT3
 
 sage_status_t quant_qk_entry(const void *q, const void *k, const Shape &sh, int8_t *q_i8,
                              float *q_scale, int8_t *k_i8, float *k_scale, float *k_mean,
-                             int smooth_k, void *workspace, size_t ws_bytes, cudaStream_t st);
+                             float *q_mean, float *q_comp, int flags, void *workspace,
+                             size_t ws_bytes, cudaStream_t st);
 sage_status_t quant_v_entry(const void *v, const int32_t *cu_seqlens, int nseq, int total_tokens,
                             int max_seqlen, int H, int d, uint8_t *v_e4m3, float *v_scale,
                             float *v_mean, bool smooth, void *workspace, size_t ws_bytes,
@@ -265,9 +278,9 @@ sage_status_t quant_v_entry(const void *v, const int32_t *cu_seqlens, int nseq, 
 // Step 3 alone on pre-quantized operands (dense; Nq queries, Nk keys).
 sage_status_t quantized_entry(const int8_t *q_i8, const float *q_scale, const int8_t *k_i8,
                               const float *k_scale, const void *v, const float *v_scale,
-                              const float *v_mean, void *out, int B, int H, int Nq, int Nk,
-                              int d, int causal, int pv_mode, float sm_scale, bool fine,
-                              cudaStream_t st)
+                              const float *v_mean, const float *q_comp, void *out, int B,
+                              int H, int Nq, int Nk, int d, int causal, int pv_mode,
+                              float sm_scale, bool fine, cudaStream_t st)
 {
     sage_status_t r = check_shape(B, H, Nq, d);
     if (r != SAGE_OK)
@@ -283,14 +296,17 @@ sage_status_t quantized_entry(const int8_t *q_i8, const float *q_scale, const in
         return SAGE_ERR_INVALID_ARG;
     if (!dense_fits(B, Nq) || !dense_fits(B, Nk))
         return SAGE_ERR_UNSUPPORTED;
-    if (!aligned16(q_i8) || !aligned16(k_i8) || !aligned16(v) || !aligned16(out))
+    if (!aligned16(q_i8) || !aligned16(k_i8) || !aligned16(v) || !aligned16(out) ||
+        !aligned16(q_comp))
         return SAGE_ERR_MISALIGNED;
     int *status = status_ptr(&r);
     if (!status)
         return r;
     const Shape sh = dense_shape(B, H, Nq, Nk, d);
-    AttnArgs a{q_i8,   q_scale, k_i8,   k_scale, v, v_scale, v_mean, static_cast<__half *>(out),
-               nullptr, causal, pv_mode, resolve_scale(sm_scale, d), fine ? 1 : 0};
+    AttnArgs a{q_i8,   q_scale, k_i8,   k_scale,
+               v,      v_scale, v_mean, q_comp,
+               static_cast<__half *>(out), nullptr, causal, pv_mode,
+               resolve_scale(sm_scale, d), fine ? 1 : 0};
     sage_status_t herr;
     cudaError_t e = launch_attention(a, sh.lq(), sh.lk(), status, st, &herr);
     if (e != cudaSuccess)
@@ -326,19 +342,22 @@ sage_status_t sage_quant_qk(const void *q, const void *k, int8_t *q_i8, float *q
 {
     if (!dense_fits(B, N))
         return SAGE_ERR_UNSUPPORTED;
+    if (smooth_k & ~(SAGE_SMOOTH_K | SAGE_QK_FINE))
+        return SAGE_ERR_INVALID_ARG;
     return quant_qk_entry(q, k, dense_shape(B, H, N, N, d), q_i8, q_scale, k_i8, k_scale, k_mean,
-                          smooth_k, nullptr, 0, reinterpret_cast<cudaStream_t>(stream));
+                          nullptr, nullptr, smooth_k, nullptr, 0,
+                          reinterpret_cast<cudaStream_t>(stream));
 }
 
 sage_status_t sage_quant_qk_kv(const void *q, const void *k, int8_t *q_i8, float *q_scale,
-                               int8_t *k_i8, float *k_scale, float *k_mean, int B, int H, int Nq,
-                               int Nk, int d, int smooth_k, void *workspace, size_t ws_bytes,
-                               sage_stream_t stream)
+                               int8_t *k_i8, float *k_scale, float *k_mean, float *q_mean,
+                               float *q_comp, int B, int H, int Nq, int Nk, int d, int flags,
+                               void *workspace, size_t ws_bytes, sage_stream_t stream)
 {
     if (!dense_fits(B, Nq) || !dense_fits(B, Nk))
         return SAGE_ERR_UNSUPPORTED;
     return quant_qk_entry(q, k, dense_shape(B, H, Nq, Nk, d), q_i8, q_scale, k_i8, k_scale,
-                          k_mean, smooth_k, workspace, ws_bytes,
+                          k_mean, q_mean, q_comp, flags, workspace, ws_bytes,
                           reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -346,30 +365,33 @@ sage_status_t sage_quant_qk_kv(const void *q, const void *k, int8_t *q_i8, float
 
 namespace sage {
 namespace {
-// Steps 1-2 with optional caller scratch for the fp64 K column sums (nullptr: a
-// stream-ordered allocation is made and released).
+// Steps 1-2 with optional caller scratch for the fp64 column sums of K (and of Q with
+// smooth Q); nullptr: a stream-ordered allocation is made and released.
 sage_status_t quant_qk_entry(const void *q, const void *k, const Shape &sh, int8_t *q_i8,
                              float *q_scale, int8_t *k_i8, float *k_scale, float *k_mean,
-                             int smooth_k, void *workspace, size_t ws_bytes, cudaStream_t st)
+                             float *q_mean, float *q_comp, int flags, void *workspace,
+                             size_t ws_bytes, cudaStream_t st)
 {
     sage_status_t r = check_shape2(sh);
     if (r != SAGE_OK)
         return r;
-    // the flags word: SAGE_SMOOTH_K (1, the original boolean) and SAGE_QK_FINE
-    if (smooth_k & ~(SAGE_SMOOTH_K | SAGE_QK_FINE))
+    // the flags word: SAGE_SMOOTH_K (1, the original boolean), SAGE_SMOOTH_Q, SAGE_QK_FINE
+    if (flags & ~(SAGE_SMOOTH_K | SAGE_SMOOTH_Q | SAGE_QK_FINE))
         return SAGE_ERR_INVALID_ARG;
-    const bool fine = (smooth_k & SAGE_QK_FINE) != 0;
-    smooth_k &= SAGE_SMOOTH_K;
+    const bool fine = (flags & SAGE_QK_FINE) != 0;
+    const bool sk = (flags & SAGE_SMOOTH_K) != 0, sq = (flags & SAGE_SMOOTH_Q) != 0;
     const bool has_q = sh.max_q > 0 && sh.total_q > 0, has_k = sh.max_k > 0 && sh.total_k > 0;
     if (sh.nseq == 0 || sh.H == 0 || (!has_q && !has_k))
         return SAGE_OK;
-    if ((has_q && (!q || !q_i8 || !q_scale)) || (has_k && (!k || !k_i8 || !k_scale || !k_mean)))
+    if ((has_q && (!q || !q_i8 || !q_scale)) || (has_k && (!k || !k_i8 || !k_scale || !k_mean)) ||
+        (sq && (!q_mean || !q_comp)))
         return SAGE_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(q_i8) || !aligned16(k_i8))
         return SAGE_ERR_MISALIGNED;
     const size_t sum_bytes = (size_t)sh.nseq * sh.H * sh.d * 8;
-    if (workspace != nullptr && smooth_k) {
-        if (ws_bytes < sum_bytes)
+    const size_t need = (sk || sq) ? (sq ? 2 : 1) * sum_bytes : 0;   // [K sums | Q sums]
+    if (workspace != nullptr && need) {
+        if (ws_bytes < need)
             return SAGE_ERR_WORKSPACE;
         if ((reinterpret_cast<uintptr_t>(workspace) & 15u) != 0)
             return SAGE_ERR_MISALIGNED;
@@ -378,36 +400,43 @@ sage_status_t quant_qk_entry(const void *q, const void *k, const Shape &sh, int8
     if (!status)
         return r;
     const SeqLayout Lq = sh.lq(), Lk = sh.lk();
-    double *ksum = nullptr;
+    char *sums = nullptr;
     bool owned = false;
-    cudaError_t e;
-    if (smooth_k && has_k) {
+    cudaError_t e = cudaSuccess;
+    if (need) {
         if (workspace != nullptr) {
-            ksum = static_cast<double *>(workspace);
+            sums = static_cast<char *>(workspace);
         } else {
             void *p = nullptr;
-            if ((e = scratch_alloc(&p, sum_bytes, st)) != cudaSuccess)
+            if ((e = scratch_alloc(&p, need, st)) != cudaSuccess)
                 return cuda_fail(e);
-            ksum = static_cast<double *>(p);
+            sums = static_cast<char *>(p);
             owned = true;
-        }
-        ColStats cs;
-        cs.ksum = ksum;
-        if ((e = cudaMemsetAsync(ksum, 0, sum_bytes, st)) != cudaSuccess ||
-            (e = launch_colstats(static_cast<const __half *>(k), nullptr, cs, Lk, status, st)) !=
-                cudaSuccess) {
-            if (owned)
-                cudaFreeAsync(ksum, st);
-            return cuda_fail(e);
         }
     }
     ColStats cs;
-    cs.ksum = ksum;
-    e = launch_quant(static_cast<const __half *>(q), static_cast<const __half *>(k), nullptr, cs,
-                     q_i8, q_scale, k_i8, k_scale, k_mean, nullptr, nullptr, nullptr, Lq, Lk,
-                     fine, status, st);
+    if (sk && has_k)
+        cs.ksum = reinterpret_cast<double *>(sums);
+    if (sq)
+        cs.qsum = reinterpret_cast<double *>(sums + sum_bytes);
+    if (need)
+        e = cudaMemsetAsync(sums, 0, need, st);
+    if (e == cudaSuccess && cs.ksum != nullptr) {
+        ColStats kc;
+        kc.ksum = cs.ksum;
+        e = launch_colstats(static_cast<const __half *>(k), nullptr, kc, Lk, status, st);
+    }
+    if (e == cudaSuccess && cs.qsum != nullptr) {
+        ColStats qc;
+        qc.ksum = cs.qsum;
+        e = launch_colstats(static_cast<const __half *>(q), nullptr, qc, Lq, status, st);
+    }
+    if (e == cudaSuccess)
+        e = launch_quant(static_cast<const __half *>(q), static_cast<const __half *>(k), nullptr,
+                         cs, q_i8, q_scale, k_i8, k_scale, k_mean, nullptr, nullptr, nullptr,
+                         sq ? q_mean : nullptr, sq ? q_comp : nullptr, Lq, Lk, fine, status, st);
     if (owned)
-        cudaFreeAsync(ksum, st);
+        cudaFreeAsync(sums, st);
     return e == cudaSuccess ? SAGE_OK : cuda_fail(e);
 }
 
@@ -455,7 +484,7 @@ sage_status_t quant_v_entry(const void *v, const int32_t *cu_seqlens, int nseq, 
             cudaSuccess)
         e = launch_quant(nullptr, nullptr, static_cast<const __half *>(v), cs, nullptr, nullptr,
                          nullptr, nullptr, nullptr, v_e4m3, v_scale, smooth ? v_mean : nullptr,
-                         L, L, false, status, st);
+                         nullptr, nullptr, L, L, false, status, st);
     if (workspace == nullptr)
         cudaFreeAsync(p, st);
     return e == cudaSuccess ? SAGE_OK : cuda_fail(e);
@@ -472,8 +501,10 @@ sage_status_t sage_quant_qk_varlen(const void *q, const void *k, const int32_t *
 {
     const Shape sh{cu_seqlens, cu_seqlens, nseq, H, d, max_seqlen, max_seqlen, total_tokens,
                    total_tokens};
-    return quant_qk_entry(q, k, sh, q_i8, q_scale, k_i8, k_scale, k_mean, smooth_k, nullptr, 0,
-                          reinterpret_cast<cudaStream_t>(stream));
+    if (smooth_k & ~(SAGE_SMOOTH_K | SAGE_QK_FINE))
+        return SAGE_ERR_INVALID_ARG;
+    return quant_qk_entry(q, k, sh, q_i8, q_scale, k_i8, k_scale, k_mean, nullptr, nullptr,
+                          smooth_k, nullptr, 0, reinterpret_cast<cudaStream_t>(stream));
 }
 
 sage_status_t sage_quant_qk_ws(const void *q, const void *k, int8_t *q_i8, float *q_scale,
@@ -485,8 +516,11 @@ sage_status_t sage_quant_qk_ws(const void *q, const void *k, int8_t *q_i8, float
         return SAGE_ERR_WORKSPACE;
     if (!dense_fits(B, N))
         return SAGE_ERR_UNSUPPORTED;
+    if (smooth_k & ~(SAGE_SMOOTH_K | SAGE_QK_FINE))
+        return SAGE_ERR_INVALID_ARG;
     return quant_qk_entry(q, k, dense_shape(B, H, N, N, d), q_i8, q_scale, k_i8, k_scale, k_mean,
-                          smooth_k, workspace, ws_bytes, reinterpret_cast<cudaStream_t>(stream));
+                          nullptr, nullptr, smooth_k, workspace, ws_bytes,
+                          reinterpret_cast<cudaStream_t>(stream));
 }
 
 sage_status_t sage_quant_v_fp8_smooth_varlen(const void *v, const int32_t *cu_seqlens, int nseq,
@@ -658,24 +692,24 @@ sage_status_t sage_attn_fwd_quantized(const int8_t *q_i8, const float *q_scale,
                                       int d, int causal, int pv_mode, float sm_scale,
                                       sage_stream_t stream)
 {
-    return quantized_entry(q_i8, q_scale, k_i8, k_scale, v, v_scale, nullptr, out, B, H, N, N,
-                           d, causal, pv_mode, sm_scale, false,
+    return quantized_entry(q_i8, q_scale, k_i8, k_scale, v, v_scale, nullptr, nullptr, out, B, H,
+                           N, N, d, causal, pv_mode, sm_scale, false,
                            reinterpret_cast<cudaStream_t>(stream));
 }
 
 sage_status_t sage_attn_fwd_quantized_kv(const int8_t *q_i8, const float *q_scale,
                                          const int8_t *k_i8, const float *k_scale, const void *v,
-                                         const float *v_scale, const float *v_mean, void *out,
-                                         int B, int H, int Nq, int Nk, int d, int causal,
-                                         int pv_mode, float sm_scale, int flags,
-                                         sage_stream_t stream)
+                                         const float *v_scale, const float *v_mean,
+                                         const float *q_comp, void *out, int B, int H, int Nq,
+                                         int Nk, int d, int causal, int pv_mode, float sm_scale,
+                                         int flags, sage_stream_t stream)
 {
     if (flags & ~SAGE_QK_FINE)
         return SAGE_ERR_INVALID_ARG;
     if (v_mean != nullptr && pv_mode != SAGE_PV_FP8)
         return SAGE_ERR_UNSUPPORTED;
-    return quantized_entry(q_i8, q_scale, k_i8, k_scale, v, v_scale, v_mean, out, B, H, Nq, Nk,
-                           d, causal, pv_mode, sm_scale, (flags & SAGE_QK_FINE) != 0,
+    return quantized_entry(q_i8, q_scale, k_i8, k_scale, v, v_scale, v_mean, q_comp, out, B, H,
+                           Nq, Nk, d, causal, pv_mode, sm_scale, (flags & SAGE_QK_FINE) != 0,
                            reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -688,8 +722,8 @@ sage_status_t sage_attn_fwd_quantized_smooth_v(const int8_t *q_i8, const float *
 {
     if (v_mean == nullptr && B > 0 && H > 0 && N > 0)
         return SAGE_ERR_INVALID_ARG;
-    return quantized_entry(q_i8, q_scale, k_i8, k_scale, v_e4m3, v_scale, v_mean, out, B, H, N,
-                           N, d, causal, SAGE_PV_FP8, sm_scale, false,
+    return quantized_entry(q_i8, q_scale, k_i8, k_scale, v_e4m3, v_scale, v_mean, nullptr, out,
+                           B, H, N, N, d, causal, SAGE_PV_FP8, sm_scale, false,
                            reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -722,7 +756,8 @@ sage_status_t sage_debug_qk_int32(const int8_t *q_i8, const int8_t *k_i8, int32_
         const float *ks = qs + (size_t)B * H * nqb;
         const void *vz = ws + sc_bytes;
         __half *o = reinterpret_cast<__half *>(ws + sc_bytes + align256(elems * 2));
-        AttnArgs a{q_i8, qs, k_i8, ks, vz, nullptr, nullptr, o, s_out, 0, SAGE_PV_FP16, 1.0f, 0};
+        AttnArgs a{q_i8, qs, k_i8, ks, vz, nullptr, nullptr, nullptr, o, s_out, 0, SAGE_PV_FP16,
+                   1.0f, 0};
         sage_status_t herr;
         const SeqLayout L = SeqLayout::dense(B, H, N, d);
         e = launch_attention(a, L, L, status, st, &herr);

@@ -62,14 +62,16 @@ constexpr float kLog2_448 = 8.807354922057604f;  // log2(448): E4M3 P = e4m3(448
 constexpr int kEmuEveryF16 = SAGE_EXP_EMU_EVERY;
 
 
-template <int D, bool FP8, int NQT>
+template <int D, bool FP8, int NQT, bool SQ = false>
 struct Cfg {
     static constexpr int BM = 128, BN = 128;
     static constexpr int kQBytes = BM * D;                   // int8 Q tile
     static constexpr int kKBytes = BN * D;                   // int8 K tile
     static constexpr int kVBytes = BN * D * (FP8 ? 1 : 2);   // V tile
     static constexpr int kPBytes = BM * BN * (FP8 ? 1 : 2);      // P tile (A operand of P.V)
-    static constexpr int kStageBytes = kKBytes + kVBytes;
+    // smooth Q: each stage also holds the 128 fp32 score compensations of its keys
+    static constexpr int kCompBytes = SQ ? BN * 4 : 0;
+    static constexpr int kStageBytes = kKBytes + kVBytes + kCompBytes;
     static constexpr int kBudget = 220 * 1024;
     static constexpr int kStagesFit = (kBudget - NQT * (kQBytes + kPBytes)) / kStageBytes;
     static constexpr int STAGES = kStagesFit > 4 ? 4 : kStagesFit;
@@ -86,7 +88,8 @@ struct Cfg {
     static constexpr int kOffK = kOffQ + NQT * kQBytes;
     static constexpr int kOffV = kOffK + STAGES * kKBytes;
     static constexpr int kOffP = kOffV + STAGES * kVBytes;
-    static constexpr int kOffBar = kOffP + NQT * kPBytes;
+    static constexpr int kOffB = kOffP + NQT * kPBytes;
+    static constexpr int kOffBar = kOffB + STAGES * kCompBytes;
     // barriers: q, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[NQT],
     //           p_full[NQT], pv_full[NQT], s_free[NQT], drain
     static constexpr int kNumBars = 1 + 4 * STAGES + 4 * NQT + 1;
@@ -118,6 +121,8 @@ struct KParams {
     const float *k_scale;
     const float *v_scale;
     const float *v_mean;   // FP8 with smooth V: added to every output row; else nullptr
+    const float *q_comp;   // smooth Q: score compensation per key; else nullptr
+    int ncomp;             // row stride of q_comp (whole 128-key tiles)
     __half *out;
     int32_t *s_dump;
     SeqLayout L;         // queries (and the output)
@@ -160,13 +165,14 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
 }
 
 // FINE: one Q scale per query row and one K scale per 32 keys; else one Q scale per
-// 128-row tile and one K scale per 64 keys.
-template <int D, bool FP8, int NQT, bool DUMP, bool FINE>
-__global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
+// 128-row tile and one K scale per 64 keys. SQ: smooth Q, the score of key j gets the
+// compensation mean(Q) K_j^T (p.q_comp), loaded with V into each stage.
+template <int D, bool FP8, int NQT, bool DUMP, bool FINE, bool SQ>
+__global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const KParams p)
 {
-    using C = Cfg<D, FP8, NQT>;
+    using C = Cfg<D, FP8, NQT, SQ>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_addr = smem_u32(smem_raw);
     uint8_t *smem = smem_raw + ((1024 - (raw_addr & 1023)) & 1023);
@@ -202,6 +208,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
     uint8_t *sK = smem + C::kOffK;
     uint8_t *sV = smem + C::kOffV;
     uint8_t *sP = smem + C::kOffP;
+    [[maybe_unused]] const float *sB = reinterpret_cast<const float *>(smem + C::kOffB);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
     uint64_t *bar_q = bars;
     uint64_t *k_full = bars + 1;
@@ -305,6 +312,14 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
             __syncwarp();
             if (lane == 0)
                 mbar_arrive(&s_free[i]);
+            // smooth Q: this tile's score compensations arrive with V(j); the stage is not
+            // refilled before P.V(j), which needs this tile's P first
+            [[maybe_unused]] const float *bt = sB + (j % C::STAGES) * C::BN;
+            if constexpr (SQ) {
+                if (!(ok = warp_wait(&v_full[j % C::STAGES], (j / C::STAGES) & 1, abort,
+                                     p.status)))
+                    break;
+            }
 
             // Score math of one tile, in two steps around the wait for the previous P.V.
             // Only the diagonal (causal) and the ragged last tile need the per-key
@@ -312,6 +327,41 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
             float alpha = 1.0f, bias = 0.0f;
             auto tile_max = [&](auto masked) {
                 constexpr bool MASKED = decltype(masked)::value;
+                float tmax = -INFINITY;
+                if constexpr (SQ) {
+                    // u = S sc + comp c, in place of S; its exact max (the compensation
+                    // varies along the row, so the integer max no longer orders it)
+                    const float cq = p.sc_log2;
+#pragma unroll
+                    for (int ch = 0; ch < 4; ch++) {
+                        const uint32_t keep =
+                            MASKED ? chunk_mask(col_lim - kcol0 - ch * 32) : ~0u;
+                        const float sc = sck[ch * kKGroups / 4];
+                        float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+                        for (int e = 0; e < 32; e += 4) {
+                            const float4 b4 = *reinterpret_cast<const float4 *>(bt + ch * 32 + e);
+#pragma unroll
+                            for (int hh = 0; hh < 2; hh++) {
+                                float2 x = make_float2(magic_biased(sreg[ch][e + 2 * hh]),
+                                                       magic_biased(sreg[ch][e + 2 * hh + 1]));
+                                x = add2(x, make_float2(-kMagic, -kMagic));      // exact S
+                                const float2 bc = mul2(hh ? make_float2(b4.z, b4.w)
+                                                          : make_float2(b4.x, b4.y),
+                                                       make_float2(cq, cq));
+                                float2 u = fma2(x, make_float2(sc, sc), bc);
+                                if constexpr (MASKED) {
+                                    u.x = ((keep >> (e + 2 * hh)) & 1u) ? u.x : -INFINITY;
+                                    u.y = ((keep >> (e + 2 * hh + 1)) & 1u) ? u.y : -INFINITY;
+                                }
+                                sreg[ch][e + 2 * hh] = __float_as_uint(u.x);
+                                sreg[ch][e + 2 * hh + 1] = __float_as_uint(u.y);
+                                mx[hh] = fmaxf(mx[hh], fmaxf(u.x, u.y));
+                            }
+                        }
+                        tmax = fmaxf(tmax, fmaxf(mx[0], mx[1]));
+                    }
+                } else {
                 // integer maxima of the K scale groups (each has its own scale)
                 int im[kKGroups];
 #pragma unroll
@@ -332,11 +382,11 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
                     const int g = ch * kKGroups / 4;      // the 32 columns' K group
                     im[g] = max(im[g], max(max(mx[0], mx[1]), max(mx[2], mx[3])));
                 }
-                float tmax = -INFINITY;
 #pragma unroll
                 for (int c = 0; c < kKGroups; c++)
                     if (im[c] != INT_MIN)
                         tmax = fmaxf(tmax, static_cast<float>(im[c]) * sck[c]);
+                }
                 const float m_new = tmax > m_ref + C::kRescaleSlack ? tmax : m_ref;
                 alpha = m_new == m_ref ? 1.0f : ex2_approx(m_ref - m_new);
                 bias = FP8 ? m_new - kLog2_448 : m_new;
@@ -401,16 +451,24 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
                 float2 lsum2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
                 for (int ch = 0; ch < 8; ch++) {
-                    const float sc = sck[ch * kKGroups / 8];
+                    [[maybe_unused]] const float sc = sck[ch * kKGroups / 8];
                     const uint32_t keep =
                         MASKED ? chunk_mask(col_lim - kcol0 - ch * 16) & 0xffffu : 0xffffu;
                     float pe[16];
 #pragma unroll
                     for (int e = 0; e < 16; e += 2) {
-                        float2 x = make_float2(magic_biased(sreg[ch / 2][(ch % 2) * 16 + e]),
-                                               magic_biased(sreg[ch / 2][(ch % 2) * 16 + e + 1]));
-                        x = add2(x, make_float2(-kMagic, -kMagic));          // exact S
-                        const float2 t = fma2(x, make_float2(sc, sc), make_float2(-bias, -bias));
+                        float2 t;
+                        if constexpr (SQ) {   // u = S sc + comp c is already in sreg
+                            t = add2(make_float2(__uint_as_float(sreg[ch / 2][(ch % 2) * 16 + e]),
+                                                 __uint_as_float(sreg[ch / 2][(ch % 2) * 16 + e + 1])),
+                                     make_float2(-bias, -bias));
+                        } else {
+                            float2 x =
+                                make_float2(magic_biased(sreg[ch / 2][(ch % 2) * 16 + e]),
+                                            magic_biased(sreg[ch / 2][(ch % 2) * 16 + e + 1]));
+                            x = add2(x, make_float2(-kMagic, -kMagic));      // exact S
+                            t = fma2(x, make_float2(sc, sc), make_float2(-bias, -bias));
+                        }
                         // one pair in kEmuEvery on the FMA pipe, the rest on MUFU
                         constexpr int kEmuEvery = FP8 ? 0 : kEmuEveryF16;
                         float2 pv;
@@ -540,7 +598,11 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT>::kThreads, 1)
                     issued = j + 1;   // the K load of this tile is in flight
                     break;
                 }
-                mbar_arrive_expect_tx(&v_full[stg], C::kVBytes);
+                mbar_arrive_expect_tx(&v_full[stg], C::kVBytes + C::kCompBytes);
+                if constexpr (SQ)   // the stride is whole 128-key tiles: 16-byte aligned
+                    bulk_load_g2s(smem + C::kOffB + stg * C::kCompBytes,
+                                  p.q_comp + ((int64_t)s * L.H + h) * p.ncomp + j * C::BN,
+                                  C::kCompBytes, &v_full[stg]);
 #pragma unroll
                 for (int cb = 0; cb < C::kVChunks; cb++)
                     tma_load_3d(sV + stg * C::kVBytes + cb * C::kVBoxBytes, &tmV, &v_full[stg],
@@ -715,11 +777,11 @@ bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int elem
     return r == CUDA_SUCCESS;
 }
 
-template <int D, bool FP8, int NQT, bool DUMP, bool FINE>
+template <int D, bool FP8, int NQT, bool DUMP, bool FINE, bool SQ>
 cudaError_t run(const AttnArgs &a, const SeqLayout &L, const SeqLayout &LK, int *status,
                 cudaStream_t st, sage_status_t *host_err)
 {
-    using C = Cfg<D, FP8, NQT>;
+    using C = Cfg<D, FP8, NQT, SQ>;
     CUtensorMap mq, mk, mv;
     const CUtensorMapSwizzle qk_swz =
         D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
@@ -739,6 +801,8 @@ cudaError_t run(const AttnArgs &a, const SeqLayout &L, const SeqLayout &LK, int 
     p.k_scale = a.k_scale;
     p.v_scale = a.v_scale;
     p.v_mean = a.v_mean;
+    p.q_comp = a.q_comp;
+    p.ncomp = comp_stride(LK.maxlen);
     p.out = a.out;
     p.s_dump = a.s_dump;
     p.L = L;
@@ -750,7 +814,7 @@ cudaError_t run(const AttnArgs &a, const SeqLayout &L, const SeqLayout &LK, int 
     p.sc_log2 = a.sm_scale * kLog2e;
     p.status = status;
 
-    auto kern = attn_kernel<D, FP8, NQT, DUMP, FINE>;
+    auto kern = attn_kernel<D, FP8, NQT, DUMP, FINE, SQ>;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess)
@@ -759,6 +823,28 @@ cudaError_t run(const AttnArgs &a, const SeqLayout &L, const SeqLayout &LK, int 
     dim3 grid((nqt + NQT - 1) / NQT, L.H, L.nseq);
     kern<<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, p);
     return cudaGetLastError();
+}
+
+// The instantiation for the P.V mode, the scale groups and smooth Q.
+template <int D>
+cudaError_t dispatch_d(const AttnArgs &a, const SeqLayout &L, const SeqLayout &LK, int *status,
+                       cudaStream_t st, sage_status_t *host_err)
+{
+    const bool fp8 = a.pv_mode == SAGE_PV_FP8, fine = a.fine != 0, sq = a.q_comp != nullptr;
+    auto pick = [&](auto f8, auto fn, auto q) {
+        return run<D, decltype(f8)::value, 2, false, decltype(fn)::value, decltype(q)::value>(
+            a, L, LK, status, st, host_err);
+    };
+    using T = std::true_type;
+    using F = std::false_type;
+    if (fp8) {
+        if (fine)
+            return sq ? pick(T{}, T{}, T{}) : pick(T{}, T{}, F{});
+        return sq ? pick(T{}, F{}, T{}) : pick(T{}, F{}, F{});
+    }
+    if (fine)
+        return sq ? pick(F{}, T{}, T{}) : pick(F{}, T{}, F{});
+    return sq ? pick(F{}, F{}, T{}) : pick(F{}, F{}, F{});
 }
 
 }  // namespace
@@ -771,24 +857,13 @@ cudaError_t launch_attention(const AttnArgs &a, const SeqLayout &L, const SeqLay
         *host_err = SAGE_ERR_INVALID_ARG;
         return cudaErrorInvalidValue;
     }
-    const bool fp8 = a.pv_mode == SAGE_PV_FP8;
     if (a.s_dump != nullptr) {
         if (L.d == 128)
-            return run<128, false, 2, true, false>(a, L, LK, status, st, host_err);
-        return run<64, false, 2, true, false>(a, L, LK, status, st, host_err);
+            return run<128, false, 2, true, false, false>(a, L, LK, status, st, host_err);
+        return run<64, false, 2, true, false, false>(a, L, LK, status, st, host_err);
     }
-    if (a.fine) {
-        if (L.d == 128)
-            return fp8 ? run<128, true, 2, false, true>(a, L, LK, status, st, host_err)
-                       : run<128, false, 2, false, true>(a, L, LK, status, st, host_err);
-        return fp8 ? run<64, true, 2, false, true>(a, L, LK, status, st, host_err)
-                   : run<64, false, 2, false, true>(a, L, LK, status, st, host_err);
-    }
-    if (L.d == 128)
-        return fp8 ? run<128, true, 2, false, false>(a, L, LK, status, st, host_err)
-                   : run<128, false, 2, false, false>(a, L, LK, status, st, host_err);
-    return fp8 ? run<64, true, 2, false, false>(a, L, LK, status, st, host_err)
-               : run<64, false, 2, false, false>(a, L, LK, status, st, host_err);
+    return L.d == 128 ? dispatch_d<128>(a, L, LK, status, st, host_err)
+                      : dispatch_d<64>(a, L, LK, status, st, host_err);
 }
 
 }  // namespace sage

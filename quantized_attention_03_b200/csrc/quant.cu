@@ -381,7 +381,8 @@ __global__ void __launch_bounds__(kThreads, 4) quant_kernel(
     ColStats cs, int8_t *__restrict__ q_i8, float *__restrict__ q_scale,
     int8_t *__restrict__ k_i8, float *__restrict__ k_scale, float *__restrict__ k_mean,
     uint8_t *__restrict__ v_e4m3, float *__restrict__ v_scale, float *__restrict__ v_mean,
-    SeqLayout Lq, SeqLayout Lk, int with_q, int nkc, int *status)
+    float *__restrict__ q_mean, float *__restrict__ q_comp, SeqLayout Lq, SeqLayout Lk,
+    int with_q, int nkc, int *status)
 {
     constexpr int kGpr = D / 8;                      // 16-byte groups per row
     constexpr int kRowStep = kThreads / kGpr;        // rows between a thread's groups
@@ -395,6 +396,7 @@ __global__ void __launch_bounds__(kThreads, 4) quant_kernel(
     __shared__ float s_mu[D];             // K mean or V mean per channel
     __shared__ float s_sc[D];             // V scale per channel
     __shared__ float s_rc[D];             // fl(1 / V scale) per channel
+    __shared__ float s_muq[D];            // Q mean per channel (smooth Q, K chunks)
 
     // 0: Q block, 1: K pair of blocks, 2: V chunk. grid.x spans the parts in order:
     // [Q chunks of Lq | K chunks of Lk] when with_q, then [V chunks of Lk] if any.
@@ -418,8 +420,14 @@ __global__ void __launch_bounds__(kThreads, 4) quant_kernel(
         return;
     const int64_t sh = (int64_t)s * L.H + h;
     const int row0 = chunk * kQBlock;
+    const int ncomp = comp_stride(Lk.maxlen);
+    const bool comp = kind == 1 && q_comp != nullptr;   // smooth-Q compensation of K rows
 
     if (row0 >= len) {                    // padding block of a short sequence
+        if (comp && (int)threadIdx.x < kQBlock)
+            q_comp[sh * ncomp + row0 + threadIdx.x] = 0.0f;
+        if (kind == 0 && chunk == 0 && q_mean != nullptr && threadIdx.x < D)
+            q_mean[sh * D + threadIdx.x] = 0.0f;
         if (kind == 1 && chunk == 0 && threadIdx.x < D)
             k_mean[sh * D + threadIdx.x] = 0.0f;
         if (kind == 2 && chunk == 0 && threadIdx.x < D) {   // empty sequence
@@ -481,8 +489,20 @@ __global__ void __launch_bounds__(kThreads, 4) quant_kernel(
                 v_mean[o] = mu;
         }
     }
-    if (kind == 0 && threadIdx.x < D)
-        s_mu[threadIdx.x] = 0.0f;
+    if (kind == 0 && threadIdx.x < D) {
+        const int c = threadIdx.x;
+        const float mu = cs.qsum ? (float)(cs.qsum[sh * D + c] / (double)len) : 0.0f;
+        s_mu[c] = mu;
+        if (chunk == 0 && q_mean != nullptr)
+            q_mean[sh * D + c] = mu;
+    }
+    if (comp && threadIdx.x < D) {        // the Q mean of this sequence and head
+        int qstart, qlen;
+        float mu = 0.0f;
+        if (Lq.range(s, qstart, qlen, status) && qlen > 0)
+            mu = (float)(cs.qsum[sh * D + threadIdx.x] / (double)qlen);
+        s_muq[threadIdx.x] = mu;
+    }
     __syncthreads();
 
     const int cg = threadIdx.x % kGpr, r_in = threadIdx.x / kGpr;
@@ -530,6 +550,31 @@ __global__ void __launch_bounds__(kThreads, 4) quant_kernel(
     else
         qk_chunk<D, kKG>(s_x, mu, cg, r_in, nrows, row0, chunk, k_scale + sh * nkb, nkb, k_i8, L,
                          s, start, h, s_red);
+
+    // ---- smooth Q: comp[j] = mean(Q) . (K[j] - mean(K)), the smoothed K as quantized
+    if (comp) {
+        float muq[8];
+#pragma unroll
+        for (int e = 0; e < 8; e++)
+            muq[e] = s_muq[c0 + e];
+#pragma unroll
+        for (int i = 0; i < kSteps; i++) {
+            const int row = i * kRowStep + r_in;
+            float dot = 0.0f;
+            if (row < nrows) {
+                float f[8];
+                unpack8(s_x[row * kGpr + cg], f);
+#pragma unroll
+                for (int e = 0; e < 8; e++)
+                    dot = fmaf(muq[e], __fsub_rn(f[e], mu[e]), dot);
+            }
+#pragma unroll
+            for (int o = 1; o < kGpr; o <<= 1)   // the row's kGpr column groups
+                dot += __shfl_xor_sync(0xffffffffu, dot, o);
+            if (cg == 0)
+                q_comp[sh * ncomp + row0 + row] = dot;   // rows past the sequence: 0
+        }
+    }
 }
 
 }  // namespace
@@ -563,8 +608,8 @@ cudaError_t launch_colstats(const __half *k, const __half *v, const ColStats &cs
 cudaError_t launch_quant(const __half *q, const __half *k, const __half *v, const ColStats &cs,
                          int8_t *q_i8, float *q_scale, int8_t *k_i8, float *k_scale,
                          float *k_mean, uint8_t *v_e4m3, float *v_scale, float *v_mean,
-                         const SeqLayout &Lq, const SeqLayout &Lk, bool fine, int *status,
-                         cudaStream_t st)
+                         float *q_mean, float *q_comp, const SeqLayout &Lq,
+                         const SeqLayout &Lk, bool fine, int *status, cudaStream_t st)
 {
     const int with_q = q_i8 != nullptr ? 1 : 0;
     const bool with_v = v_e4m3 != nullptr;
@@ -579,7 +624,8 @@ cudaError_t launch_quant(const __half *q, const __half *k, const __half *v, cons
     auto kern = Lk.d == 128 ? (fine ? quant_kernel<128, true> : quant_kernel<128, false>)
                             : (fine ? quant_kernel<64, true> : quant_kernel<64, false>);
     kern<<<grid, kThreads, 0, st>>>(q, k, v, cs, q_i8, q_scale, k_i8, k_scale, k_mean, v_e4m3,
-                                    v_scale, v_mean, Lq, Lk, with_q, nkc, status);
+                                    v_scale, v_mean, q_mean, q_comp, Lq, Lk, with_q, nkc,
+                                    status);
     return cudaGetLastError();
 }
 

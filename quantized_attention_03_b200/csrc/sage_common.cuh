@@ -70,6 +70,7 @@ __host__ __device__ constexpr int status_bit(sage_status_t s) { return 1 << (int
 //   vhi, vneg:  max V and max -V as order-preserving keys (float_key) for atomicMax.
 struct ColStats {
     double *ksum = nullptr;
+    double *qsum = nullptr;   // Q column sums, [nseq, H, d] of the query layout (smooth Q)
     double *vsum = nullptr;
     uint32_t *vhi = nullptr;
     uint32_t *vneg = nullptr;
@@ -90,15 +91,21 @@ __host__ __device__ inline uint32_t key_bits(uint32_t key)
 cudaError_t launch_colstats(const __half *k, const __half *v, const ColStats &cs,
                             const SeqLayout &L, int *status, cudaStream_t st);
 // Quantizes Q and K (q_i8 != nullptr) and/or V (v_e4m3 != nullptr). K is smoothed when
-// cs.ksum is set, V when cs.vsum is set (its mean goes to v_mean if that is set). Q
-// lives in layout Lq, K and V in Lk (the same layout for self-attention). fine: one Q
-// scale per token and one K scale per 32 tokens (q_scale [nseq,H,maxq], k_scale
-// [nseq,H,ceil(maxk/32)]); else per-block scales (128 Q tokens, 64 K tokens).
+// cs.ksum is set, V when cs.vsum is set (its mean goes to v_mean if that is set), Q when
+// cs.qsum is set (its mean goes to q_mean if that is set, and the compensation mean(Q)
+// K^T of every key to q_comp, [nseq, H, comp_stride(maxk)]). Q lives in layout Lq, K
+// and V in Lk (the same layout for self-attention). fine: one Q scale per token and one
+// K scale per 32 tokens (q_scale [nseq,H,maxq], k_scale [nseq,H,ceil(maxk/32)]); else
+// per-block scales (128 Q tokens, 64 K tokens).
 cudaError_t launch_quant(const __half *q, const __half *k, const __half *v, const ColStats &cs,
                          int8_t *q_i8, float *q_scale, int8_t *k_i8, float *k_scale,
                          float *k_mean, uint8_t *v_e4m3, float *v_scale, float *v_mean,
-                         const SeqLayout &Lq, const SeqLayout &Lk, bool fine, int *status,
-                         cudaStream_t st);
+                         float *q_mean, float *q_comp, const SeqLayout &Lq,
+                         const SeqLayout &Lk, bool fine, int *status, cudaStream_t st);
+
+// Row stride of the smooth-Q compensation array: the key count rounded up to whole
+// 128-key tiles, so that every tile's 512 bytes start 16-byte aligned.
+__host__ __device__ constexpr int comp_stride(int maxlen_k) { return (maxlen_k + 127) / 128 * 128; }
 
 struct AttnArgs {
     const int8_t *q_i8;
@@ -108,6 +115,7 @@ struct AttnArgs {
     const void *v;        // fp16 V or E4M3 codes
     const float *v_scale; // FP8 mode
     const float *v_mean;  // FP8 mode with smooth V, else nullptr
+    const float *q_comp;  // smooth Q: mean(Q) K^T per key, [nseq, H, comp_stride]; or nullptr
     __half *out;
     int32_t *s_dump;      // debug: int32 scores [nseq,H,maxlen,maxlen] or nullptr
     int causal;

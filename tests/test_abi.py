@@ -67,7 +67,14 @@ def test_smoothing_flags(lib):
     # smooth V needs FP8 P.V (fp16 V is never quantized); unknown bits are rejected
     assert _fwd(lib, smooth=sage.SAGE_SMOOTH_V, pv=0) == sage.SAGE_ERR_UNSUPPORTED
     assert _fwd(lib, smooth=3, pv=0) == sage.SAGE_ERR_UNSUPPORTED
-    assert _fwd(lib, smooth=4, pv=1) == sage.SAGE_ERR_INVALID_ARG
+    assert _fwd(lib, smooth=16, pv=1) == sage.SAGE_ERR_INVALID_ARG
+    # the self-attention quantization entry points take smooth K and the finer groups only
+    assert lib.sage_quant_qk(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64,
+                             sage.SAGE_SMOOTH_Q, None) == sage.SAGE_ERR_INVALID_ARG
+    # smooth Q needs the mean and compensation outputs
+    assert lib.sage_quant_qk_kv(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, None, 1, 1, 128,
+                                256, 64, sage.SAGE_SMOOTH_Q, None, 0, None) == \
+        sage.SAGE_ERR_INVALID_ARG
     assert _fwd(lib, smooth=-1, pv=1) == sage.SAGE_ERR_INVALID_ARG
     assert _fwd(lib, smooth=3, pv=1, q=0) == sage.SAGE_ERR_INVALID_ARG      # flags accepted
     assert lib.sage_attn_fwd_noalloc(FAKE, FAKE, FAKE, FAKE, 1, 1, 128, 64, 0, 2, 0, 0.0,

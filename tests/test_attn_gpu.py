@@ -450,3 +450,67 @@ def test_fine_groups_more_accurate_on_row_outliers():
                              False, 1 / math.sqrt(d))
     assert rel_l1(fine, exact) < 0.5 * rel_l1(block, exact)
     assert rel_l1(fine, exact) < 0.02
+
+
+# ----------------------------------- smooth Q with the mean(Q) K^T score compensation
+
+
+def _offset_q(q, d, seed, amp=6.0):
+    g = torch.Generator().manual_seed(seed)
+    return (q.float() + (torch.rand(d, generator=g) * 2 - 1) * amp).half()
+
+
+SQ_CASES = [
+    # Nq, Nk, d, causal, fine
+    (1, 1, 128, False, False), (300, 300, 64, True, False), (513, 513, 128, False, False),
+    (200, 900, 128, True, False), (640, 640, 64, True, True), (129, 129, 128, False, True),
+]
+
+
+@pytest.mark.parametrize("pv", ["fp16", "fp8"])
+@pytest.mark.parametrize("Nq,Nk,d,causal,fine", SQ_CASES)
+def test_smooth_q_small_full_compare(Nq, Nk, d, causal, fine, pv):
+    B, H = 2, 2
+    w = inputs.Workload("t", 600 + Nq + Nk, B, H, Nk, d, causal, 2.0, nq=Nq)
+    q, k, v = inputs.make_dense(w)
+    q = _offset_q(q, d, 601 + Nq)
+    out = sage.sageattn(q.cuda(), k.cuda(), v.cuda(), causal, True, PV[pv], fine=fine,
+                        smooth_q=True)
+    assert sage.sage_get_device_status() == 0
+    got = _np(out)
+    lq, lk = oracle.Layout.dense(B, H, Nq, d), oracle.Layout.dense(B, H, Nk, d)
+    ref = oracle.sage_attention(q.numpy(), k.numpy(), v.numpy(), lq, causal, True, PV[pv],
+                                kv_layout=lk, fine=fine, smooth_q=True)
+    tag = f"smooth Q Nq={Nq} Nk={Nk} d={d} causal={causal} fine={fine} {pv}"
+    assert_vs_oracle(got, ref, tag)
+    exact = oracle.attn_fp64(q.numpy(), k.numpy(), v.numpy(), lq, causal, 1 / math.sqrt(d),
+                             kv_layout=lk)
+    assert_vs_fp64(got, exact, pv == "fp8", tag)
+
+
+def test_smooth_q_quantized_entry_matches_fused():
+    B, H, N, d = 2, 3, 700, 128
+    w = inputs.Workload("t", 131, B, H, N, d, True, 1.0)
+    q, k, v = (t.cuda() for t in inputs.make_dense(w))
+    q = _offset_q(q.cpu(), d, 132).cuda()
+    fused = sage.sageattn(q, k, v, True, True, sage.SAGE_PV_FP16, smooth_q=True)
+    z = sage.quant_qk(q, k, True, smooth_q=True)
+    split = sage.attn_quantized(z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], v, None, True,
+                                sage.SAGE_PV_FP16, q_comp=z["q_comp"])
+    assert sage.sage_get_device_status() == 0
+    assert torch.equal(fused, split)
+
+
+def test_smooth_q_more_accurate_with_q_channel_offsets():
+    N, d = 2048, 128
+    w = inputs.Workload("t", 141, 1, 4, N, d, False, 1.0)
+    q, k, v = inputs.make_dense(w)
+    q = _offset_q(q, d, 142, amp=12.0)
+    sq = _np(sage.sageattn(q.cuda(), k.cuda(), v.cuda(), False, True, sage.SAGE_PV_FP16,
+                           smooth_q=True))
+    plain = _np(sage.sageattn(q.cuda(), k.cuda(), v.cuda(), False, True, sage.SAGE_PV_FP16))
+    assert sage.sage_get_device_status() == 0
+    exact = oracle.attn_fp64(q.numpy(), k.numpy(), v.numpy(), oracle.Layout.dense(1, 4, N, d),
+                             False, 1 / math.sqrt(d))
+    assert rel_l1(sq, exact) < 0.02
+    assert rel_l1(sq, exact) < rel_l1(plain, exact)

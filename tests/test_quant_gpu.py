@@ -227,3 +227,24 @@ def test_quant_fine_varlen_bit_exact():
     ref = oracle.quant_qk(q.numpy(), k.numpy(), oracle.Layout.packed(cu.tolist(), H, d), True,
                           fine=True)
     _check_qk(z, ref, "fine varlen")
+
+
+@pytest.mark.parametrize("Nq,Nk,d,fine", [(300, 300, 128, False), (129, 700, 64, True),
+                                          (1, 200, 128, False)])
+def test_quant_smooth_q(Nq, Nk, d, fine):
+    B, H = 2, 2
+    w = inputs.Workload("t", 121 + Nq, B, H, Nk, d, False, 2.0, nq=Nq)
+    q, k, _ = inputs.make_dense(w)
+    g = torch.Generator().manual_seed(122)
+    q = (q.float() + (torch.rand(d, generator=g) * 2 - 1) * 8.0).half()   # Q channel offsets
+    z = sage.quant_qk(q.cuda(), k.cuda(), True, fine=fine, smooth_q=True)
+    assert sage.sage_get_device_status() == 0
+    ref = oracle.quant_qk(q.numpy(), k.numpy(), oracle.Layout.dense(B, H, Nq, d), True,
+                          kv_layout=oracle.Layout.dense(B, H, Nk, d), fine=fine, smooth_q=True)
+    _check_qk(z, ref, f"smooth Q {Nq}x{Nk}")
+    assert np.array_equal(_np(z["q_mean"]), ref["q_mean"])
+    comp = _np(z["q_comp"])
+    assert comp.shape == (B, H, (Nk + 127) // 128 * 128)
+    assert not comp[:, :, Nk:].any()                     # padding past the keys is zero
+    scale = np.abs(ref["q_comp"]).max()
+    assert np.abs(comp[:, :, :Nk] - ref["q_comp"]).max() <= 1e-5 * scale

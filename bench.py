@@ -185,7 +185,7 @@ def _oracle_sample(case, it: int, rows: int):
     t0 = time.perf_counter()
     oracle.sage_attention(q, k, v, lay, W["causal"], W["smooth_k"], pv,
                           1.0 / math.sqrt(lay.d), heads=[(s, h)], rows=(r0, r1), kv_layout=kvl,
-                          fine=W.get("fine", False))
+                          fine=W.get("fine", False), smooth_q=W.get("smooth_q", False))
     return (time.perf_counter() - t0, _sample_ops(r0, r1, n, kvl.lens[s], lay.d, W["causal"]),
             (s, h))
 
@@ -277,6 +277,7 @@ def _workload(args):
     if args.pv is not None:
         W["pv_mode"] = args.pv
     W["fine"] = bool(args.fine)
+    W["smooth_q"] = bool(args.smooth_q)
     return W
 
 
@@ -288,7 +289,7 @@ def _workload_name(W):
     nq = f" Nq={W['Nq']} Nk={W['N']}" if W.get("Nq") else ""
     return (f"B={W['B']} H={W['H']} N={W['N']}{nq} d={W['d']} "
             f"{'causal' if W['causal'] else 'non-causal'} PV={W['pv_mode']} smooth_k"
-            f"{' fine-groups' if W.get('fine') else ''}")
+            f"{' fine-groups' if W.get('fine') else ''}{' smooth_q' if W.get('smooth_q') else ''}")
 
 
 def run_ours(args):
@@ -319,9 +320,11 @@ def run_ours(args):
         vscale = torch.empty((B, H, d), dtype=torch.float32, device=v.device)
     sm_scale = 1.0 / math.sqrt(d)
     dev = q.device
-    fine = W["fine"]
+    fine, sq = W["fine"], W["smooth_q"]
+    general = fine or sq or Nq != N          # the *_kv entry points
     nqb, nkb = (Nq, math.ceil(N / 32)) if fine else (math.ceil(Nq / 128), math.ceil(N / 64))
-    qk_flags = (sage.SAGE_SMOOTH_K if W["smooth_k"] else 0) | (sage.SAGE_QK_FINE if fine else 0)
+    qk_flags = ((sage.SAGE_SMOOTH_K if W["smooth_k"] else 0) | (sage.SAGE_QK_FINE if fine else 0)
+                | (sage.SAGE_SMOOTH_Q if sq else 0))
     q_i8 = torch.empty(q.shape, dtype=torch.int8, device=dev)
     k_i8 = torch.empty(k.shape, dtype=torch.int8, device=dev)
     q_scale = torch.empty((B, H, nqb), dtype=torch.float32, device=dev)
@@ -330,27 +333,30 @@ def run_ours(args):
     out = torch.empty_like(q)
     stream = torch.cuda.current_stream()
 
-    ksum_ws = torch.empty(B * H * d * 8, dtype=torch.uint8, device=dev)   # fp64 K sums
+    ksum_ws = torch.empty(B * H * d * 16, dtype=torch.uint8, device=dev)  # fp64 K (and Q) sums
+    q_mean = torch.empty((B, H, d), dtype=torch.float32, device=dev) if sq else None
+    q_comp = (torch.empty((B, H, math.ceil(N / 128) * 128), dtype=torch.float32, device=dev)
+              if sq else None)
     vstat_ws = torch.empty(B * H * d * 16, dtype=torch.uint8, device=dev)  # V column statistics
 
     def quant():
-        if Nq == N and not fine:
+        if not general:
             sage.sage_quant_qk_ws(q, k, q_i8, q_scale, k_i8, k_scale, k_mean, B, H, N, d,
                                   W["smooth_k"], ksum_ws, ksum_ws.numel(), stream)
         else:
-            sage.sage_quant_qk_kv(q, k, q_i8, q_scale, k_i8, k_scale, k_mean, B, H, Nq, N, d,
-                                  qk_flags, ksum_ws, ksum_ws.numel(), stream)
+            sage.sage_quant_qk_kv(q, k, q_i8, q_scale, k_i8, k_scale, k_mean, q_mean, q_comp, B,
+                                  H, Nq, N, d, qk_flags, ksum_ws, ksum_ws.numel(), stream)
         if pv == sage.SAGE_PV_FP8:
             sage.sage_quant_v_fp8_ws(v, vq, vscale, None, B, H, N, d, vstat_ws, vstat_ws.numel(),
                                      stream)
 
     def attend():
-        if Nq == N and not fine:
+        if not general:
             sage.sage_attn_fwd_quantized(q_i8, q_scale, k_i8, k_scale, vq, vscale, out, B, H, N,
                                          d, W["causal"], pv, sm_scale, stream)
         else:
-            sage.sage_attn_fwd_quantized_kv(q_i8, q_scale, k_i8, k_scale, vq, vscale, None, out,
-                                            B, H, Nq, N, d, W["causal"], pv, sm_scale,
+            sage.sage_attn_fwd_quantized_kv(q_i8, q_scale, k_i8, k_scale, vq, vscale, None, q_comp,
+                                            out, B, H, Nq, N, d, W["causal"], pv, sm_scale,
                                             sage.SAGE_QK_FINE if fine else 0, stream)
 
     def step():
@@ -416,7 +422,7 @@ def run_ours(args):
         qd.copy_(qh, non_blocking=True)
         kd.copy_(kh, non_blocking=True)
         vd.copy_(vh, non_blocking=True)
-        if Nq == N and not fine:
+        if not general:
             sage.sage_attn_fwd(qd, kd, vd, od, B, H, N, d, W["causal"], W["smooth_k"], pv,
                                sm_scale, stream)
         else:
@@ -519,7 +525,8 @@ def run_varlen(args, W, dist, world, rank, local):
     ops = inputs.varlen_ops(lens, H, d, W["causal"])
 
     def step(qq=q, kk=k, vv=v, oo=out):
-        flags = sage.SAGE_SMOOTH_K | (sage.SAGE_QK_FINE if W["fine"] else 0)
+        flags = (sage.SAGE_SMOOTH_K | (sage.SAGE_QK_FINE if W["fine"] else 0)
+                 | (sage.SAGE_SMOOTH_Q if W["smooth_q"] else 0))
         sage.sage_attn_varlen_fwd(qq, kk, vv, oo, cud, nseq, T, maxlen, H, d, W["causal"], flags,
                                   pv, 0.0, ws, need, stream)
 
@@ -647,6 +654,8 @@ def main():
     ap.add_argument("--pv", choices=["fp16", "fp8"], default=None)
     ap.add_argument("--fine", action="store_true",
                     help="one Q scale per token and one K scale per 32 tokens")
+    ap.add_argument("--smooth-q", action="store_true",
+                    help="smooth Q with the mean(Q) K^T score compensation")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -83,6 +83,15 @@ struct Cfg {
     static constexpr int kTmemNeed = NQT * (BN + D);
     static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128 : kTmemNeed <= 256 ? 256 : 512;
     static_assert(kTmemNeed <= 512, "TMEM budget exceeded");
+    // Registers: the kernel launches with kLaunchRegs per thread (65536 / 384, rounded
+    // down to a multiple of 8); setmaxnreg then moves them from the producer, MMA and idle
+    // warps to the softmax warps. The split draws only on the block's own registers, so
+    // the totals must match (the host checks kLaunchRegs against the compiled kernel).
+    static constexpr int kLaunchRegs = 168;
+    static constexpr int kRegSoftmax = FP8 ? 208 : 216;   // measured best per P.V mode
+    static constexpr int kRegOther = FP8 ? 88 : 72;
+    static_assert((kSoftmaxWarps * kRegSoftmax + 4 * kRegOther) * 32 <= kThreads * kLaunchRegs,
+                  "register split exceeds the launch allocation");
     // shared memory map (offsets from a 1024-byte aligned base)
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + NQT * kQBytes;
@@ -252,7 +261,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
     if (warp < C::kSoftmaxWarps) {
         // ------------------------------------------------------------ softmax warps
         if constexpr (NQT == 2)
-            asm volatile("setmaxnreg.inc.sync.aligned.u32 216;\n" ::: "memory");
+            asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(C::kRegSoftmax) : "memory");
         const int i = warp / 4;                    // query tile within the CTA
         const int quarter = warp % 4;              // TMEM lane quarter of this warp
         const int qt = qt0 + i;
@@ -572,7 +581,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
     } else if (warp == C::kProducerWarp) {
         // ----------------------------------------------------------------- producer
         if constexpr (NQT == 2)
-            asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
+            asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(C::kRegOther) : "memory");
         if (lane == 0) {
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
@@ -623,7 +632,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
     } else if (warp == C::kMmaWarp) {
         // ---------------------------------------------------------------- MMA issuer
         if constexpr (NQT == 2)
-            asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
+            asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(C::kRegOther) : "memory");
         if (lane == 0) {
             constexpr uint32_t idesc_qk = instr_desc(2 /*s32*/, 1 /*s8*/, 1 /*s8*/, 0, 0, 128, 128);
             constexpr uint32_t idesc_pv = instr_desc(1 /*f32*/, 0 /*f16|e4m3*/, 0, 0,
@@ -711,7 +720,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
         }
     } else {
         if constexpr (NQT == 2)
-            asm volatile("setmaxnreg.dec.sync.aligned.u32 72;\n" ::: "memory");
+            asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(C::kRegOther) : "memory");
     }
 
     tc_fence_before();
@@ -819,6 +828,19 @@ cudaError_t run(const AttnArgs &a, const SeqLayout &L, const SeqLayout &LK, int 
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess)
         return e;
+    // the kernel must launch with the registers the setmaxnreg split assumes (with fewer,
+    // the softmax warps' increase could never be granted); read once per instantiation
+    static std::once_flag once;
+    static int regs = 0;
+    std::call_once(once, [&] {
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, kern) == cudaSuccess)
+            regs = fa.numRegs;
+    });
+    if (regs != C::kLaunchRegs) {
+        *host_err = SAGE_ERR_UNSUPPORTED;
+        return cudaErrorInvalidConfiguration;
+    }
     const int nqt = (L.maxlen + C::BM - 1) / C::BM;
     dim3 grid((nqt + NQT - 1) / NQT, L.H, L.nseq);
     kern<<<grid, C::kThreads, C::kSmemBytes, st>>>(mq, mk, mv, p);

@@ -292,6 +292,49 @@ def _workload_name(W):
             f"{' fine-groups' if W.get('fine') else ''}{' smooth_q' if W.get('smooth_q') else ''}")
 
 
+def pipelined_e2e(steps, host_in, dev_sets, host_outs, compute, dist, dev):
+    """End-to-end steps through the public API, pipelined over three streams: the
+    host-to-device copy of step i+1 and the device-to-host copy of step i-1 overlap step
+    i's compute (two device buffer sets, two pinned output buffers). Every step copies its
+    inputs in and its result out. Returns the CUDA-event time from the first copy's start
+    to the last result's arrival, max over ranks."""
+    import torch
+    s_in, s_comp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    nb = len(dev_sets)
+    ev = {k: [torch.cuda.Event() for _ in range(nb)] for k in ("in", "comp", "out")}
+
+    def one(i):
+        b = i % nb
+        ins, out = dev_sets[b]
+        s_in.wait_event(ev["comp"][b])              # the previous step on b has read ins
+        with torch.cuda.stream(s_in):
+            for d_t, h_t in zip(ins, host_in):
+                d_t.copy_(h_t, non_blocking=True)
+        ev["in"][b].record(s_in)
+        s_comp.wait_event(ev["in"][b])
+        s_comp.wait_event(ev["out"][b])             # out of the previous step on b is home
+        compute(ins, out, s_comp)
+        ev["comp"][b].record(s_comp)
+        s_out.wait_event(ev["comp"][b])
+        with torch.cuda.stream(s_out):
+            host_outs[b].copy_(out, non_blocking=True)
+        ev["out"][b].record(s_out)
+
+    one(0)                                          # warm-up
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(s_in)
+    for i in range(steps):
+        one(i)
+    s_out.wait_stream(s_in)
+    s_out.wait_stream(s_comp)
+    t1.record(s_out)
+    torch.cuda.synchronize()
+    return max_over_ranks(max(t0.elapsed_time(t1), 1e-9), dist, dev)
+
+
 def run_ours(args):
     import torch
     import quantized_attention_03_b200 as sage
@@ -413,37 +456,23 @@ def run_ours(args):
 
     # end to end through the public API: pinned host inputs -> device -> result -> host
     e2e_steps = 0 if args.no_e2e else max(3, args.steps // 4)
-    qh, kh, vh = (t.pin_memory() for t in (qc, kc, vc))
-    oh = torch.empty_like(qc).pin_memory()
-    qd, od = torch.empty_like(q), torch.empty_like(q)
-    kd, vd = torch.empty_like(k), torch.empty_like(v)
-
-    def e2e_step():
-        qd.copy_(qh, non_blocking=True)
-        kd.copy_(kh, non_blocking=True)
-        vd.copy_(vh, non_blocking=True)
-        if not general:
-            sage.sage_attn_fwd(qd, kd, vd, od, B, H, N, d, W["causal"], W["smooth_k"], pv,
-                               sm_scale, stream)
-        else:
-            sage.sage_attn_fwd_kv(qd, kd, vd, od, B, H, Nq, N, d, W["causal"], qk_flags, pv,
-                                  sm_scale, None, 0, stream)
-        oh.copy_(od, non_blocking=True)
-
+    e2e_ms = 1e-9
     if e2e_steps:
-        e2e_step()
-    torch.cuda.synchronize()
-    if dist is not None:
-        dist.barrier()
-    s0 = torch.cuda.Event(enable_timing=True)
-    s1 = torch.cuda.Event(enable_timing=True)
-    s0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    s1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max(s0.elapsed_time(s1), 1e-9)
-    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
+        host_in = [t.pin_memory() for t in (qc, kc, vc)]
+        host_outs = [torch.empty_like(qc).pin_memory() for _ in range(2)]
+        dev_sets = [([torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)],
+                     torch.empty_like(q)) for _ in range(2)]
+
+        def compute(ins, o, st):
+            qd, kd, vd = ins
+            if not general:
+                sage.sage_attn_fwd(qd, kd, vd, o, B, H, N, d, W["causal"], W["smooth_k"], pv,
+                                   sm_scale, st)
+            else:
+                sage.sage_attn_fwd_kv(qd, kd, vd, o, B, H, Nq, N, d, W["causal"], qk_flags, pv,
+                                      sm_scale, None, 0, st)
+
+        e2e_ms = pipelined_e2e(e2e_steps, host_in, dev_sets, host_outs, compute, dist, dev)
     status = sage.sage_get_device_status()
     if status != 0:
         raise RuntimeError(f"device status after e2e: {sage.status_string(status)}")
@@ -491,7 +520,9 @@ def run_ours(args):
             "roofline": roofline,
             "e2e": {"value": e2e_value, "unit": "TOPS",
                     "h2d_bytes_per_step": q_bytes + 2 * elem_bytes, "d2h_bytes_per_step": q_bytes,
-                    "steps": e2e_steps},
+                    "steps": e2e_steps,
+                    "pipelining": "3 streams: step i+1's inputs in and step i-1's output out "
+                                  "overlap step i (sage_attn_fwd, pinned host buffers)"},
             "gpu_launches": (3 if pv == sage.SAGE_PV_FP16 else 5) * args.steps,
             "clocks": clocks.summary(),
         }
@@ -524,11 +555,11 @@ def run_varlen(args, W, dist, world, rank, local):
     stream = torch.cuda.current_stream()
     ops = inputs.varlen_ops(lens, H, d, W["causal"])
 
-    def step(qq=q, kk=k, vv=v, oo=out):
+    def step(qq=q, kk=k, vv=v, oo=out, st=stream):
         flags = (sage.SAGE_SMOOTH_K | (sage.SAGE_QK_FINE if W["fine"] else 0)
                  | (sage.SAGE_SMOOTH_Q if W["smooth_q"] else 0))
         sage.sage_attn_varlen_fwd(qq, kk, vv, oo, cud, nseq, T, maxlen, H, d, W["causal"], flags,
-                                  pv, 0.0, ws, need, stream)
+                                  pv, 0.0, ws, need, st)
 
     clocks = ClockSampler(local)
     clocks.__enter__()
@@ -555,27 +586,18 @@ def run_varlen(args, W, dist, world, rank, local):
     value = weak_scaling_tops(ops, args.steps, world, total_ms)
 
     e2e_steps = 0 if args.no_e2e else max(3, args.steps // 4)
-    qh, kh, vh = (t.pin_memory() for t in (qc, kc, vc))
-    oh = torch.empty_like(qc).pin_memory()
-    qd, kd, vd, od = (torch.empty_like(q) for _ in range(4))
 
-    def e2e_step():
-        qd.copy_(qh, non_blocking=True)
-        kd.copy_(kh, non_blocking=True)
-        vd.copy_(vh, non_blocking=True)
-        step(qd, kd, vd, od)
-        oh.copy_(od, non_blocking=True)
-
+    e2e_ms = 1e-9
     if e2e_steps:
-        e2e_step()
-    torch.cuda.synchronize()
-    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
-    s1.record(stream)
-    torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(max(s0.elapsed_time(s1), 1e-9), dist, q.device)
+        host_in = [t.pin_memory() for t in (qc, kc, vc)]
+        host_outs = [torch.empty_like(qc).pin_memory() for _ in range(2)]
+        dev_sets = [([torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)],
+                     torch.empty_like(q)) for _ in range(2)]
+
+        def compute(ins, o, st):
+            step(ins[0], ins[1], ins[2], o, st)
+
+        e2e_ms = pipelined_e2e(e2e_steps, host_in, dev_sets, host_outs, compute, dist, q.device)
     e2e_value = weak_scaling_tops(ops, e2e_steps, world, e2e_ms) if e2e_steps else None
 
     peaks, src = _peaks()
@@ -599,7 +621,9 @@ def run_varlen(args, W, dist, world, rank, local):
                          "kernel": "whole varlen step (quantization + attention in one call; "
                                    "the attention kernel is not timed separately)"},
             "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": 3 * elem_bytes,
-                    "d2h_bytes_per_step": elem_bytes, "steps": e2e_steps},
+                    "d2h_bytes_per_step": elem_bytes, "steps": e2e_steps,
+                    "pipelining": "3 streams: step i+1's inputs in and step i-1's output out "
+                                  "overlap step i (sage_attn_varlen_fwd, pinned host buffers)"},
             "gpu_launches": 3 * args.steps,   # column statistics, quantization, attention
             "clocks": clocks.summary(),
         }

@@ -564,3 +564,43 @@ def test_smooth_q_is_a_no_op_for_zero_mean_q():
     a = oracle.sage_attention(q, k, v, lay, True, True, PV_FP16, smooth_q=True)
     b = oracle.sage_attention(q, k, v, lay, True, True, PV_FP16)
     assert np.array_equal(a, b)
+
+
+def test_fp64_one_hot_dominant_score():
+    # one key far ahead of the others: the output row is that key's V row
+    N, d = 40, 16
+    q = np.zeros((1, 1, 1, d), np.float16)
+    q[..., 0] = 8
+    k = _rand16((1, 1, N, d), 271, 0.01)
+    k[0, 0, 17, 0] = 8                     # score 64 * sm above every other key
+    v = _rand16((1, 1, N, d), 272)
+    o = oracle.attn_fp64(q, k, v, Layout.dense(1, 1, 1, d), False, 1.0,
+                         kv_layout=Layout.dense(1, 1, N, d))
+    assert np.allclose(o[0, 0, 0], v[0, 0, 17].astype(np.float64), atol=1e-12)
+
+
+def test_int8_scores_beat_e4m3_scores():
+    # [SA1] 技术方案: INT8 per-block quantization of Q and K is more accurate for Q K^T than
+    # E4M3 with the same blocks (amax mapped to 127 and to 448 respectively)
+    N, d = 256, 64
+    q, k = _rand16((1, 1, N, d), 281), _rand16((1, 1, N, d), 282)
+    lay = Layout.dense(1, 1, N, d)
+    exact = q[0, 0].astype(np.float64) @ k[0, 0].astype(np.float64).T
+    z = oracle.quant_qk(q, k, lay, smooth_k=False)
+    s_i8 = (z["q_i8"][0, 0].astype(np.int64) @ z["k_i8"][0, 0].astype(np.int64).T
+            * z["q_scale"][0, 0][np.arange(N) // 128][:, None]
+            * z["k_scale"][0, 0][np.arange(N) // 64][None, :])
+
+    def e4m3_blocks(x, blk):
+        out = np.empty(x.shape, np.float64)
+        for b0 in range(0, x.shape[0], blk):
+            xb = x[b0:b0 + blk].astype(np.float32)
+            s = np.float32(np.abs(xb).max() / np.float32(448))
+            codes = np.vectorize(lambda t: oracle.e4m3_encode(float(np.float32(t) / s)))(xb)
+            out[b0:b0 + blk] = np.vectorize(oracle.e4m3_decode)(codes) * float(s)
+        return out
+
+    s_f8 = e4m3_blocks(q[0, 0], 128) @ e4m3_blocks(k[0, 0], 64).T
+    err_i8 = np.abs(s_i8 - exact).mean()
+    err_f8 = np.abs(s_f8 - exact).mean()
+    assert err_i8 < 0.6 * err_f8

@@ -87,6 +87,19 @@ def test_smoothing_flags(lib):
         sage.SAGE_ERR_INVALID_ARG
 
 
+def test_size_limits(lib):
+    # token counts are int32: B*N past 2^31 - 1 is refused before anything is enqueued
+    assert _fwd(lib, B=65535, N=65536) == sage.SAGE_ERR_UNSUPPORTED
+    assert lib.sage_attn_fwd_kv(FAKE, FAKE, FAKE, FAKE, 2, 1, 128, 2 ** 30 + 1, 64, 0, 1, 0, 0.0,
+                                None, 0, None) == sage.SAGE_ERR_UNSUPPORTED
+    assert lib.sage_attn_fwd_kv(FAKE, FAKE, FAKE, FAKE, 1, 1, 128, -1, 64, 0, 1, 0, 0.0, None, 0,
+                                None) == sage.SAGE_ERR_INVALID_ARG
+    # workspace sizes grow with the shapes and are zero for negative ones
+    assert lib.sage_workspace_size_kv(1, 1, 128, 256, 128, 256, 64, 0) > \
+        lib.sage_workspace_size_kv(1, 1, 128, 128, 128, 128, 64, 0)
+    assert lib.sage_workspace_size_kv(-1, 1, 128, 256, 128, 256, 64, 0) == 0
+
+
 def test_empty_inputs_are_noops(lib):
     assert _fwd(lib, B=0) == sage.SAGE_OK
     assert _fwd(lib, N=0) == sage.SAGE_OK

@@ -523,7 +523,10 @@ def run_ours(args):
                     "steps": e2e_steps,
                     "pipelining": "3 streams: step i+1's inputs in and step i-1's output out "
                                   "overlap step i (sage_attn_fwd, pinned host buffers)"},
-            "gpu_launches": (3 if pv == sage.SAGE_PV_FP16 else 5) * args.steps,
+            # per step: K column sums, Q/K codes, attention; + Q column sums with smooth Q;
+            # + V column statistics and V codes in FP8 mode
+            "gpu_launches": (3 + (1 if sq else 0)
+                             + (2 if pv == sage.SAGE_PV_FP8 else 0)) * args.steps,
             "clocks": clocks.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:
@@ -624,7 +627,8 @@ def run_varlen(args, W, dist, world, rank, local):
                     "d2h_bytes_per_step": elem_bytes, "steps": e2e_steps,
                     "pipelining": "3 streams: step i+1's inputs in and step i-1's output out "
                                   "overlap step i (sage_attn_varlen_fwd, pinned host buffers)"},
-            "gpu_launches": 3 * args.steps,   # column statistics, quantization, attention
+            # column statistics (K and V together), quantization, attention; + Q sums
+            "gpu_launches": (3 + (1 if W["smooth_q"] else 0)) * args.steps,
             "clocks": clocks.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:

@@ -330,9 +330,11 @@ def sageattn(q, k, v, causal: bool = False, smooth_k: bool = True, pv_mode: int 
 def sageattn_varlen_kv(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
                        causal: bool = False, smooth_k: bool = True,
                        pv_mode: int = SAGE_PV_FP16, sm_scale: float = 0.0, out=None,
-                       stream=None, smooth_v: bool = False):
+                       stream=None, smooth_v: bool = False, fine: bool = False,
+                       smooth_q: bool = False):
     """Packed sequences with their own query and key lengths: q [Tq, H, d], k and v
-    [Tk, H, d], cu_seqlens_q / cu_seqlens_k int32 [nseq+1] on the device."""
+    [Tk, H, d], cu_seqlens_q / cu_seqlens_k int32 [nseq+1] on the device. The options are
+    sageattn's."""
     import torch
     Tq, H, d = q.shape
     Tk = k.shape[0]
@@ -340,21 +342,24 @@ def sageattn_varlen_kv(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, m
         out = torch.empty_like(q)
     sage_attn_varlen_fwd_kv(q, k, v, out, cu_seqlens_q, cu_seqlens_k, cu_seqlens_q.numel() - 1,
                             Tq, Tk, max_seqlen_q, max_seqlen_k, H, d, causal,
-                            _smooth_flags(smooth_k, smooth_v), pv_mode, sm_scale, None, 0, stream)
+                            _smooth_flags(smooth_k, smooth_v, fine, smooth_q), pv_mode, sm_scale,
+                            None, 0, stream)
     return out
 
 
 def sageattn_varlen(q, k, v, cu_seqlens, max_seqlen: int, causal: bool = False,
                     smooth_k: bool = True, pv_mode: int = SAGE_PV_FP16, sm_scale: float = 0.0,
-                    out=None, stream=None, smooth_v: bool = False):
-    """SageAttention over packed sequences: q, k, v [T, H, d], cu_seqlens int32 [nseq+1]."""
+                    out=None, stream=None, smooth_v: bool = False, fine: bool = False,
+                    smooth_q: bool = False):
+    """SageAttention over packed sequences: q, k, v [T, H, d], cu_seqlens int32 [nseq+1].
+    The options are sageattn's."""
     import torch
     T, H, d = q.shape
     if out is None:
         out = torch.empty_like(q)
     sage_attn_varlen_fwd(q, k, v, out, cu_seqlens, cu_seqlens.numel() - 1, T, max_seqlen, H, d,
-                         causal, _smooth_flags(smooth_k, smooth_v), pv_mode, sm_scale, None, 0,
-                         stream)
+                         causal, _smooth_flags(smooth_k, smooth_v, fine, smooth_q), pv_mode,
+                         sm_scale, None, 0, stream)
     return out
 
 

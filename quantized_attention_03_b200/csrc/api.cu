@@ -204,7 +204,11 @@ sage_status_t forward(const void *q, const void *k, const void *v, void *out, co
         if ((e = launch_colstats(qh, nullptr, qs, L, status, st)) != cudaSuccess)
             return cuda_fail(e);
     }
-    if ((e = launch_quant(qh, kh, vh, cs, w.q_i8, w.q_scale, w.k_i8, w.k_scale, w.k_mean,
+    // With smooth Q the attention kernel quantizes its own Q tiles from fp16 (measured
+    // faster there); otherwise Q's codes come from this pass with K's.
+    const bool q_in_kernel = sq;
+    if ((e = launch_quant(qh, kh, vh, cs, q_in_kernel ? nullptr : w.q_i8,
+                          q_in_kernel ? nullptr : w.q_scale, w.k_i8, w.k_scale, w.k_mean,
                           fp8 ? w.v8 : nullptr, w.v_scale, sv ? w.v_mean : nullptr, nullptr,
                           sq ? w.q_comp : nullptr, L, LK, fine, status, st)) != cudaSuccess)
         return cuda_fail(e);
@@ -212,6 +216,10 @@ sage_status_t forward(const void *q, const void *k, const void *v, void *out, co
                w.v_scale,  sv ? w.v_mean : nullptr,     sq ? w.q_comp : nullptr,
                static_cast<__half *>(out), nullptr, causal, pv_mode,
                resolve_scale(sm_scale, L.d), fine ? 1 : 0};
+    if (q_in_kernel) {
+        a.q16 = qh;
+        a.qsum = cs.qsum;
+    }
     sage_status_t herr;
     if ((e = launch_attention(a, L, LK, status, st, &herr)) != cudaSuccess)
         return herr != SAGE_OK ? herr : cuda_fail(e);

@@ -42,6 +42,7 @@
 #include <cstdio>
 #include <mutex>
 
+#include "quant_codes.cuh"
 #include "sage_common.cuh"
 #include "sm100_ptx.cuh"
 
@@ -140,6 +141,8 @@ struct KParams {
     int causal;
     float sc_log2;       // sm_scale * log2(e)
     int *status;
+    const __half *q16;   // QIN: fp16 Q, quantized in the prologue
+    const double *qsum;  // QIN with smooth Q: fp64 column sums of Q
 };
 
 __device__ __forceinline__ void tma_coords(const SeqLayout &L, int s, int start, int h, int row,
@@ -173,10 +176,83 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
     return ok;
 }
 
+// The INT8 codes and the scale of this thread's query row (QIN): Q is read as fp16, made
+// smooth (x - mean(Q), SQ), and quantized with one scale per 128-row tile (the
+// warpgroup's amax) or per row (FINE) exactly as the quantization kernel does it; the
+// codes go to the Q tile in shared memory in the layout its TMA copy would give (rows of
+// D bytes, 16-byte chunks XOR-swizzled by the row: 128-byte swizzle for D = 128, 64-byte
+// for D = 64). scratch: this warpgroup's 4 + D floats of shared memory. Returns the
+// row's scale (0 for rows past the sequence, and for a tile with no row in it).
+template <int D, bool FINE, bool SQ>
+__device__ __forceinline__ float quantize_q_row(const __half *__restrict__ src, bool valid,
+                                                const double *__restrict__ qsum, int len,
+                                                uint8_t *tile, int row, int i, float *scratch)
+{
+    const int quarter = row / 32, lane = row % 32;
+    float *s_amax = scratch;          // one per warp
+    float *s_mu = scratch + 4;        // mean(Q) per channel
+    if constexpr (SQ) {
+        for (int c = row; c < D; c += 128)
+            s_mu[c] = (float)(qsum[c] / (double)len);
+        named_bar_sync(1 + i, 128);
+    }
+    uint4 raw[D / 8];
+#pragma unroll
+    for (int g = 0; g < D / 8; g++)
+        raw[g] = valid ? __ldg(reinterpret_cast<const uint4 *>(src) + g) : make_uint4(0, 0, 0, 0);
+    // amax |fl(x - mu)| over the row (mu = 0 without smooth Q: max |x|, exact)
+    float amax = 0.0f;
+#pragma unroll
+    for (int g = 0; g < D / 8; g++) {
+        float f[8];
+        unpack8(raw[g], f);
+#pragma unroll
+        for (int e = 0; e < 8; e++)
+            amax = fmaxf(amax, fabsf(SQ ? __fsub_rn(f[e], s_mu[g * 8 + e]) : f[e]));
+    }
+    if (!valid)
+        amax = 0.0f;
+    if constexpr (!FINE) {
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1)
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        if (lane == 0)
+            s_amax[quarter] = amax;
+        named_bar_sync(1 + i, 128);
+        amax = fmaxf(fmaxf(s_amax[0], s_amax[1]), fmaxf(s_amax[2], s_amax[3]));
+    }
+    const float scale = __fdiv_rn(amax, 127.0f);
+    const float rcp = scale != 0.0f ? __fdiv_rn(1.0f, scale) : 0.0f;
+    const uint32_t base = smem_u32(tile) + row * D;
+#pragma unroll
+    for (int c = 0; c < D / 16; c++) {      // 16 codes = one 16-byte chunk
+        uint2 w[2];
+#pragma unroll
+        for (int hh = 0; hh < 2; hh++) {
+            const int g = 2 * c + hh;
+            float f[8];
+            unpack8(raw[g], f);
+            float2 x[4];
+#pragma unroll
+            for (int e = 0; e < 4; e++) {
+                x[e] = make_float2(f[2 * e], f[2 * e + 1]);
+                if constexpr (SQ)
+                    x[e] = make_float2(__fsub_rn(x[e].x, s_mu[g * 8 + 2 * e]),
+                                       __fsub_rn(x[e].y, s_mu[g * 8 + 2 * e + 1]));
+            }
+            w[hh] = valid ? int8_codes8(x, scale, rcp) : make_uint2(0u, 0u);
+        }
+        const int sw = D == 128 ? (row & 7) : ((row >> 1) & 3);
+        st_shared_v4(base + ((c ^ sw) << 4), w[0].x, w[0].y, w[1].x, w[1].y);
+    }
+    return valid || !FINE ? scale : 0.0f;
+}
+
 // FINE: one Q scale per query row and one K scale per 32 keys; else one Q scale per
 // 128-row tile and one K scale per 64 keys. SQ: smooth Q, the score of key j gets the
-// compensation mean(Q) K_j^T (p.q_comp), loaded with V into each stage.
-template <int D, bool FP8, int NQT, bool DUMP, bool FINE, bool SQ>
+// compensation mean(Q) K_j^T (p.q_comp), loaded with V into each stage. QIN: the CTA
+// quantizes its own Q tiles from fp16 (p.q16) instead of loading INT8 codes.
+template <int D, bool FP8, int NQT, bool DUMP, bool FINE, bool SQ, bool QIN>
 __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
     attn_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                 const __grid_constant__ CUtensorMap tmV, const KParams p)
@@ -234,7 +310,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
 
     const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
     if (threadIdx.x == 0) {
-        mbar_init(bar_q, 1);
+        mbar_init(bar_q, QIN ? C::kSoftmaxWarps : 1);
         for (int i = 0; i < C::STAGES; i++) {
             mbar_init(&k_full[i], 1);
             mbar_init(&k_empty[i], 1);
@@ -272,9 +348,24 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
         const uint32_t tO = tmem_base + lane_off + NQT * C::BN + i * D;
         const int64_t sh = (int64_t)s * L.H + h;
         // this row's Q scale (one per query tile, or one per token)
-        const int qidx = FINE ? qrow : qt;
-        const bool q_valid = (FINE ? qrow : qt * C::BM) < len;
-        const float qsc = (q_valid ? __ldg(p.q_scale + sh * p.nqb + qidx) : 0.0f) * p.sc_log2;
+        float qsc;
+        if constexpr (QIN) {
+            // quantize this row into Q tile i, then tell the MMA issuer (bar_q counts the
+            // softmax warps)
+            qsc = quantize_q_row<D, FINE, SQ>(
+                      p.q16 + L.offset(s, start, h, qrow < len ? qrow : 0), qrow < len,
+                      SQ ? p.qsum + sh * D : nullptr, len, smem + C::kOffQ + i * C::kQBytes,
+                      row_in_tile, i, reinterpret_cast<float *>(sP + i * C::kPBytes)) *
+                  p.sc_log2;
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0)
+                mbar_arrive(bar_q);
+        } else {
+            const int qidx = FINE ? qrow : qt;
+            const bool q_valid = (FINE ? qrow : qt * C::BM) < len;
+            qsc = (q_valid ? __ldg(p.q_scale + sh * p.nqb + qidx) : 0.0f) * p.sc_log2;
+        }
         constexpr int kKGroups = FINE ? 4 : 2;        // K scales per 128-key tile
         const int kb_valid = (klen + C::BN / kKGroups - 1) / (C::BN / kKGroups);
 
@@ -583,14 +674,17 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
         if constexpr (NQT == 2)
             asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(C::kRegOther) : "memory");
         if (lane == 0) {
-            tma_prefetch_desc(&tmQ);
+            if constexpr (!QIN)
+                tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
             int c1, c2;
-            mbar_arrive_expect_tx(bar_q, NQT * C::kQBytes);
-            for (int i = 0; i < NQT; i++) {
-                tma_coords(L, s, start, h, (qt0 + i) * C::BM, c1, c2);
-                tma_load_3d(sQ + i * C::kQBytes, &tmQ, bar_q, 0, c1, c2);
+            if constexpr (!QIN) {   // (QIN: the softmax warps write the Q tiles)
+                mbar_arrive_expect_tx(bar_q, NQT * C::kQBytes);
+                for (int i = 0; i < NQT; i++) {
+                    tma_coords(L, s, start, h, (qt0 + i) * C::BM, c1, c2);
+                    tma_load_3d(sQ + i * C::kQBytes, &tmQ, bar_q, 0, c1, c2);
+                }
             }
             int issued = 0;
             for (int j = 0; j < nkv; j++) {
@@ -619,7 +713,8 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
                 issued = j + 1;
             }
             // drain: make sure no copy is still landing in shared memory when we leave
-            mbar_wait(bar_q, 0, nullptr, p.status, status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs);
+            if constexpr (!QIN)
+                mbar_wait(bar_q, 0, nullptr, p.status, status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs);
             for (int j = max(0, issued - C::STAGES); j < issued; j++) {
                 const int stg = j % C::STAGES;
                 const uint32_t ph = (j / C::STAGES) & 1;
@@ -786,7 +881,7 @@ bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int elem
     return r == CUDA_SUCCESS;
 }
 
-template <int D, bool FP8, int NQT, bool DUMP, bool FINE, bool SQ>
+template <int D, bool FP8, int NQT, bool DUMP, bool FINE, bool SQ, bool QIN>
 cudaError_t run(const AttnArgs &a, const SeqLayout &L, const SeqLayout &LK, int *status,
                 cudaStream_t st, sage_status_t *host_err)
 {
@@ -796,8 +891,11 @@ cudaError_t run(const AttnArgs &a, const SeqLayout &L, const SeqLayout &LK, int 
         D == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     const CUtensorMapSwizzle v_swz =
         C::kVRowBytes == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
-    bool ok = make_map(&mq, a.q_i8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L, D, C::BM, qk_swz) &&
-              make_map(&mk, a.k_i8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, LK, D, C::BN, qk_swz) &&
+    // (QIN: no Q map; the K map stands in for the unused parameter)
+    bool ok = make_map(&mk, a.k_i8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, LK, D, C::BN, qk_swz) &&
+              (QIN ? (mq = mk, true)
+                   : make_map(&mq, a.q_i8, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, L, D, C::BM,
+                              qk_swz)) &&
               make_map(&mv, a.v,
                        FP8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16,
                        C::kVElem, LK, C::kVRowBytes / C::kVElem, C::BN, v_swz);
@@ -822,8 +920,10 @@ cudaError_t run(const AttnArgs &a, const SeqLayout &L, const SeqLayout &LK, int 
     p.causal = a.causal;
     p.sc_log2 = a.sm_scale * kLog2e;
     p.status = status;
+    p.q16 = a.q16;
+    p.qsum = a.qsum;
 
-    auto kern = attn_kernel<D, FP8, NQT, DUMP, FINE, SQ>;
+    auto kern = attn_kernel<D, FP8, NQT, DUMP, FINE, SQ, QIN>;
     cudaError_t e =
         cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
     if (e != cudaSuccess)
@@ -847,18 +947,34 @@ cudaError_t run(const AttnArgs &a, const SeqLayout &L, const SeqLayout &LK, int 
     return cudaGetLastError();
 }
 
-// The instantiation for the P.V mode, the scale groups and smooth Q.
+// The instantiation for the P.V mode, the scale groups, smooth Q and where Q's codes
+// come from. In-kernel Q quantization is built for smooth Q only, where it measures
+// faster than the separate pass (with plain Q the per-CTA prologue costs more than the
+// pass it saves, most on short causal sequences).
 template <int D>
 cudaError_t dispatch_d(const AttnArgs &a, const SeqLayout &L, const SeqLayout &LK, int *status,
                        cudaStream_t st, sage_status_t *host_err)
 {
     const bool fp8 = a.pv_mode == SAGE_PV_FP8, fine = a.fine != 0, sq = a.q_comp != nullptr;
     auto pick = [&](auto f8, auto fn, auto q) {
-        return run<D, decltype(f8)::value, 2, false, decltype(fn)::value, decltype(q)::value>(
+        return run<D, decltype(f8)::value, 2, false, decltype(fn)::value, decltype(q)::value,
+                   false>(a, L, LK, status, st, host_err);
+    };
+    auto pick_qin = [&](auto f8, auto fn) {
+        return run<D, decltype(f8)::value, 2, false, decltype(fn)::value, true, true>(
             a, L, LK, status, st, host_err);
     };
     using T = std::true_type;
     using F = std::false_type;
+    if (a.q16 != nullptr) {
+        if (!sq || a.qsum == nullptr) {
+            *host_err = SAGE_ERR_INVALID_ARG;
+            return cudaErrorInvalidValue;
+        }
+        if (fp8)
+            return fine ? pick_qin(T{}, T{}) : pick_qin(T{}, F{});
+        return fine ? pick_qin(F{}, T{}) : pick_qin(F{}, F{});
+    }
     if (fp8) {
         if (fine)
             return sq ? pick(T{}, T{}, T{}) : pick(T{}, T{}, F{});
@@ -881,8 +997,8 @@ cudaError_t launch_attention(const AttnArgs &a, const SeqLayout &L, const SeqLay
     }
     if (a.s_dump != nullptr) {
         if (L.d == 128)
-            return run<128, false, 2, true, false, false>(a, L, LK, status, st, host_err);
-        return run<64, false, 2, true, false, false>(a, L, LK, status, st, host_err);
+            return run<128, false, 2, true, false, false, false>(a, L, LK, status, st, host_err);
+        return run<64, false, 2, true, false, false, false>(a, L, LK, status, st, host_err);
     }
     return L.d == 128 ? dispatch_d<128>(a, L, LK, status, st, host_err)
                       : dispatch_d<64>(a, L, LK, status, st, host_err);

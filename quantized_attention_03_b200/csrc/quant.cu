@@ -20,6 +20,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include "quant_codes.cuh"
 #include "sage_common.cuh"
 #include "sm100_ptx.cuh"
 
@@ -30,17 +31,6 @@ namespace {
 constexpr int kColChunk = 512;   // tokens per colstats CTA
 constexpr int kThreads = 256;
 constexpr uint64_t kWaitNs = 2000000000ull;   // bound on the wait for a chunk's bulk copy
-
-__device__ __forceinline__ void unpack8(const uint4 &u, float (&f)[8])
-{
-    const __half2 *h = reinterpret_cast<const __half2 *>(&u);
-#pragma unroll
-    for (int i = 0; i < 4; i++) {
-        const float2 t = __half22float2(h[i]);
-        f[2 * i] = t.x;
-        f[2 * i + 1] = t.y;
-    }
-}
 
 // DO_K: fp64 sums of K; DO_V: max and max of -V, plus fp64 sums of V when cs.vsum is set.
 template <int D, bool DO_K, bool DO_V>
@@ -160,65 +150,6 @@ __global__ void __launch_bounds__(kThreads) colstats_kernel(const __half *__rest
             atomicMax(cs.vneg + o, float_key(__float_as_uint(mn)));
         }
     }
-}
-
-constexpr float kRound = 12582912.0f;            // 1.5 * 2^23: adding it rounds to an integer
-constexpr int kRoundBits = 0x4B400000;
-
-// round-half-even(fl(x / s)) clamped to [-127, 127], where fl(x / s) is the IEEE fp32
-// quotient and r = fl(1 / s). The product x * r is within 2^-15 of fl(x / s) (|x / s| <=
-// 127.5 keeps every ulp <= 2^-17), so both round to the same integer unless the product
-// lies within 2^-15 of a half-integer; those rare elements take the exact division.
-__device__ __forceinline__ int8_t int8_code(float x, float s, float r)
-{
-    if (s == 0.0f)
-        return 0;
-    const float q = x * r;
-    const float b = q + kRound;                    // RNE integer in the low mantissa bits
-    const float d = fabsf(q - (b - kRound));       // distance to that integer, <= 1/2
-    int c = __float_as_int(b) - kRoundBits;
-    if (d > 0.5f - 3.0517578125e-05f)              // near a tie: exact IEEE quotient
-        c = __float2int_rn(__fdiv_rn(x, s));
-    c = max(-127, min(127, c));
-    return (int8_t)c;
-}
-
-// The eight codes int8_code(x, s, r) of x[0..3] (pairs), packed little-endian. The
-// product x * r, rounded to an integer by the 1.5 * 2^23 bias, is computed on packed
-// fp32 pairs; the code is the low byte of the biased float's bits (their integer part
-// is 0x4B400000 + code). No clamp is needed: s = fl(amax / 127) and r = fl(1 / s) give
-// |x r| <= 127 (1 + 2^-22) < 127.5. Elements within 2^-15 of a tie are redone with the
-// exact quotient (rare).
-__device__ __forceinline__ uint2 int8_codes8(const float2 (&x)[4], float s, float r)
-{
-    if (s == 0.0f)
-        return make_uint2(0u, 0u);
-    constexpr float kTie = 0.5f - 3.0517578125e-05f;
-    uint32_t bits[8];
-    bool tie = false;
-#pragma unroll
-    for (int j = 0; j < 4; j++) {
-        const float2 t = mul2(x[j], make_float2(r, r));
-        const float2 b = add2(t, make_float2(kRound, kRound));
-        const float2 n = add2(b, make_float2(-kRound, -kRound));
-        const float2 d = fma2(n, make_float2(-1.0f, -1.0f), t);   // t - round(t), exact
-        tie |= (fabsf(d.x) > kTie) | (fabsf(d.y) > kTie);
-        bits[2 * j] = __float_as_uint(b.x);
-        bits[2 * j + 1] = __float_as_uint(b.y);
-    }
-    if (tie) {
-#pragma unroll
-        for (int j = 0; j < 4; j++) {
-            bits[2 * j] = (uint8_t)int8_code(x[j].x, s, r);
-            bits[2 * j + 1] = (uint8_t)int8_code(x[j].y, s, r);
-        }
-    }
-    uint2 w;
-    w.x = __byte_perm(__byte_perm(bits[0], bits[1], 0x0040), __byte_perm(bits[2], bits[3], 0x0040),
-                      0x5410);
-    w.y = __byte_perm(__byte_perm(bits[4], bits[5], 0x0040), __byte_perm(bits[6], bits[7], 0x0040),
-                      0x5410);
-    return w;
 }
 
 // fl(x / s) for the E4M3 encoder, with r = fl(1 / s): the product x * r differs from the
@@ -382,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 4) quant_kernel(
     int8_t *__restrict__ k_i8, float *__restrict__ k_scale, float *__restrict__ k_mean,
     uint8_t *__restrict__ v_e4m3, float *__restrict__ v_scale, float *__restrict__ v_mean,
     float *__restrict__ q_mean, float *__restrict__ q_comp, SeqLayout Lq, SeqLayout Lk,
-    int with_q, int nkc, int *status)
+    int nqc, int nkc, int *status)
 {
     constexpr int kGpr = D / 8;                      // 16-byte groups per row
     constexpr int kRowStep = kThreads / kGpr;        // rows between a thread's groups
@@ -399,18 +330,17 @@ __global__ void __launch_bounds__(kThreads, 4) quant_kernel(
     __shared__ float s_muq[D];            // Q mean per channel (smooth Q, K chunks)
 
     // 0: Q block, 1: K pair of blocks, 2: V chunk. grid.x spans the parts in order:
-    // [Q chunks of Lq | K chunks of Lk] when with_q, then [V chunks of Lk] if any.
-    const int nqc = (Lq.maxlen + kQBlock - 1) / kQBlock;   // 128-token Q chunks per head
+    // [nqc Q chunks of Lq | nkc K chunks of Lk | V chunks of Lk]; nqc or nkc is 0 when
+    // that part is not quantized here.
     const int nqb = (Lq.maxlen + kQG - 1) / kQG;           // Q scales per head
     const int nkb = (Lk.maxlen + kKG - 1) / kKG;           // K scales per head
     int kind, chunk = (int)blockIdx.x;
-    if (with_q && chunk < nqc) {
+    if (chunk < nqc) {
         kind = 0;
     } else {
-        if (with_q)
-            chunk -= nqc;
-        kind = (with_q && chunk < nkc) ? 1 : 2;
-        if (kind == 2 && with_q)
+        chunk -= nqc;
+        kind = chunk < nkc ? 1 : 2;
+        if (kind == 2)
             chunk -= nkc;
     }
     const SeqLayout &L = kind == 0 ? Lq : Lk;
@@ -704,18 +634,20 @@ cudaError_t launch_colstats(const __half *k, const __half *v, const ColStats &cs
     return cudaGetLastError();
 }
 
-// Quantizes Q and K (q_i8 != nullptr) and/or V (v_e4m3 != nullptr) in one launch.
+// Quantizes Q (q_i8 != nullptr), K (k_i8 != nullptr) and/or V (v_e4m3 != nullptr) in
+// one launch.
 cudaError_t launch_quant(const __half *q, const __half *k, const __half *v, const ColStats &cs,
                          int8_t *q_i8, float *q_scale, int8_t *k_i8, float *k_scale,
                          float *k_mean, uint8_t *v_e4m3, float *v_scale, float *v_mean,
                          float *q_mean, float *q_comp, const SeqLayout &Lq,
                          const SeqLayout &Lk, bool fine, int *status, cudaStream_t st)
 {
-    const int with_q = q_i8 != nullptr ? 1 : 0;
+    const bool with_q = q_i8 != nullptr, with_k = k_i8 != nullptr;
     const bool with_v = v_e4m3 != nullptr;
-    const int nqc = (Lq.maxlen + kQBlock - 1) / kQBlock;     // 128-token chunks
-    const int nkc = (Lk.maxlen + kQBlock - 1) / kQBlock;
-    const int nx = (with_q ? nqc + nkc : 0) + (with_v ? nkc : 0);
+    const int nqc = with_q ? (Lq.maxlen + kQBlock - 1) / kQBlock : 0;   // 128-token chunks
+    const int nkc = with_k ? (Lk.maxlen + kQBlock - 1) / kQBlock : 0;
+    const int nvc = with_v ? (Lk.maxlen + kQBlock - 1) / kQBlock : 0;
+    const int nx = nqc + nkc + nvc;
     if (nx == 0 || Lk.H == 0 || Lk.nseq == 0)
         return cudaSuccess;
     if (with_q && (Lq.nseq != Lk.nseq || Lq.H != Lk.H || Lq.d != Lk.d))
@@ -724,7 +656,7 @@ cudaError_t launch_quant(const __half *q, const __half *k, const __half *v, cons
     auto kern = Lk.d == 128 ? (fine ? quant_kernel<128, true> : quant_kernel<128, false>)
                             : (fine ? quant_kernel<64, true> : quant_kernel<64, false>);
     kern<<<grid, kThreads, 0, st>>>(q, k, v, cs, q_i8, q_scale, k_i8, k_scale, k_mean, v_e4m3,
-                                    v_scale, v_mean, q_mean, q_comp, Lq, Lk, with_q, nkc,
+                                    v_scale, v_mean, q_mean, q_comp, Lq, Lk, nqc, nkc,
                                     status);
     return cudaGetLastError();
 }

@@ -90,13 +90,13 @@ __host__ __device__ inline uint32_t key_bits(uint32_t key)
 // Launchers (quant.cu, attn_sm100.cu). All return cudaSuccess or the launch error.
 cudaError_t launch_colstats(const __half *k, const __half *v, const ColStats &cs,
                             const SeqLayout &L, int *status, cudaStream_t st);
-// Quantizes Q and K (q_i8 != nullptr) and/or V (v_e4m3 != nullptr). K is smoothed when
-// cs.ksum is set, V when cs.vsum is set (its mean goes to v_mean if that is set), Q when
-// cs.qsum is set (its mean goes to q_mean if that is set, and the compensation mean(Q)
-// K^T of every key to q_comp, [nseq, H, comp_stride(maxk)]). Q lives in layout Lq, K
-// and V in Lk (the same layout for self-attention). fine: one Q scale per token and one
-// K scale per 32 tokens (q_scale [nseq,H,maxq], k_scale [nseq,H,ceil(maxk/32)]); else
-// per-block scales (128 Q tokens, 64 K tokens).
+// Quantizes Q (q_i8 != nullptr), K (k_i8 != nullptr) and/or V (v_e4m3 != nullptr). K is
+// smoothed when cs.ksum is set, V when cs.vsum is set (its mean goes to v_mean if that
+// is set), Q when cs.qsum is set (its mean goes to q_mean if that is set, and the
+// compensation mean(Q) K^T of every key to q_comp, [nseq, H, comp_stride(maxk)]). Q
+// lives in layout Lq, K and V in Lk (the same layout for self-attention). fine: one Q
+// scale per token and one K scale per 32 tokens (q_scale [nseq,H,maxq], k_scale
+// [nseq,H,ceil(maxk/32)]); else per-block scales (128 Q tokens, 64 K tokens).
 cudaError_t launch_quant(const __half *q, const __half *k, const __half *v, const ColStats &cs,
                          int8_t *q_i8, float *q_scale, int8_t *k_i8, float *k_scale,
                          float *k_mean, uint8_t *v_e4m3, float *v_scale, float *v_mean,
@@ -122,6 +122,11 @@ struct AttnArgs {
     int pv_mode;
     float sm_scale;
     int fine;             // scales per Q token and per 32 K tokens (else per block)
+    // fp16 Q quantized by the attention kernel itself (each CTA its own query tiles, with
+    // the codes and scales the quantization kernel would give); q_i8 and q_scale are then
+    // unused. With smooth Q, qsum holds Q's fp64 column sums [nseq, H, d]. Else nullptr.
+    const __half *q16 = nullptr;
+    const double *qsum = nullptr;
 };
 // Queries in layout Lq, keys and values in Lk (the same layout for self-attention; with
 // different lengths the causal mask aligns at the bottom right).

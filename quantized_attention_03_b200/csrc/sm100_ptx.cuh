@@ -329,6 +329,13 @@ __device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint
 
 // Make this thread's generic-proxy shared-memory writes visible to the async proxy
 // (tensor-core operand reads) before it signals the MMA issuer.
+// Barrier among the n threads (whole warps) that name barrier `id` (1-15; 0 is
+// __syncthreads'). Every one of them reaches it: it is not a wait on another role.
+__device__ __forceinline__ void named_bar_sync(int id, int n)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
+}
+
 __device__ __forceinline__ void fence_proxy_async_smem()
 {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");

@@ -488,6 +488,50 @@ def test_smooth_q_small_full_compare(Nq, Nk, d, causal, fine, pv):
     assert_vs_fp64(got, exact, pv == "fp8", tag)
 
 
+@pytest.mark.parametrize("N,d,pv,fine", [
+    (700, 128, "fp8", False), (700, 64, "fp16", False), (333, 64, "fp8", True),
+    (129, 128, "fp16", True), (1, 128, "fp16", False), (4096, 128, "fp16", False)])
+def test_smooth_q_in_kernel_q_codes_match_the_quantization_pass(N, d, pv, fine):
+    """With smooth Q the fused entry quantizes Q inside the attention kernel; the result
+    must be bit-identical to Q's codes from the quantization pass (quant_qk) fed to the
+    pre-quantized entry."""
+    B, H = 2, 3
+    w = inputs.Workload("t", 160 + N + d, B, H, N, d, True, 1.0)
+    q, k, v = (t.cuda() for t in inputs.make_dense(w))
+    q = _offset_q(q.cpu(), d, 161 + N).cuda()
+    fused = sage.sageattn(q, k, v, True, True, PV[pv], fine=fine, smooth_q=True)
+    z = sage.quant_qk(q, k, True, fine=fine, smooth_q=True)
+    if pv == "fp8":
+        vv, vs = sage.quant_v_fp8(v)
+    else:
+        vv, vs = v, None
+    split = sage.attn_quantized(z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], vv, vs, True,
+                                PV[pv], fine=fine, q_comp=z["q_comp"])
+    assert sage.sage_get_device_status() == 0
+    assert torch.equal(fused, split)
+
+
+@pytest.mark.parametrize("pv", ["fp16", "fp8"])
+def test_smooth_q_varlen_against_oracle(pv):
+    """Packed sequences with smooth Q (in-kernel Q quantization over the packed rows)."""
+    H, d = 2, 128
+    lens = [130, 1, 257, 640]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T = int(cu[-1])
+    g = torch.Generator().manual_seed(171)
+    q = (torch.randn((T, H, d), generator=g) + torch.rand(d, generator=g) * 8 - 4).half()
+    k = (torch.randn((T, H, d), generator=g) + 2.0).half()
+    v = torch.randn((T, H, d), generator=g).half()
+    cud = torch.from_numpy(cu).cuda()
+    out = sage.sageattn_varlen(q.cuda(), k.cuda(), v.cuda(), cud, max(lens), True, True, PV[pv],
+                               smooth_q=True)
+    assert sage.sage_get_device_status() == 0
+    lay = oracle.Layout.packed(cu.tolist(), H, d)
+    ref = oracle.sage_attention(q.numpy(), k.numpy(), v.numpy(), lay, True, True, PV[pv],
+                                smooth_q=True)
+    assert_vs_oracle(_np(out), ref, f"smooth Q varlen {pv}")
+
+
 def test_smooth_q_quantized_entry_matches_fused():
     B, H, N, d = 2, 3, 700, 128
     w = inputs.Workload("t", 131, B, H, N, d, True, 1.0)

@@ -70,18 +70,24 @@ struct Cfg {
     static constexpr int kKBytes = BN * D;                   // int8 K tile
     static constexpr int kVBytes = BN * D * (FP8 ? 1 : 2);   // V tile
     static constexpr int kPBytes = BM * BN * (FP8 ? 1 : 2);      // P tile (A operand of P.V)
+    // d = 64: TMEM has room for P beside S and O, so P goes there and P.V takes its A
+    // operand from TMEM (at d = 64 an M=128 N=64 P.V with both operands in shared memory
+    // needs more shared-memory bandwidth than its math); d = 128: P in shared memory.
+    static constexpr bool kPTmem = D == 64;
+    static constexpr int kPSmem = kPTmem ? 0 : kPBytes;          // P bytes in shared memory
+    static constexpr int kPCols = kPTmem ? BN * (FP8 ? 1 : 2) / 4 : 0;   // P columns in TMEM
     // smooth Q: each stage also holds the 128 fp32 score compensations of its keys
     static constexpr int kCompBytes = SQ ? BN * 4 : 0;
     static constexpr int kStageBytes = kKBytes + kVBytes + kCompBytes;
     static constexpr int kBudget = 220 * 1024;
-    static constexpr int kStagesFit = (kBudget - NQT * (kQBytes + kPBytes)) / kStageBytes;
+    static constexpr int kStagesFit = (kBudget - NQT * (kQBytes + kPSmem)) / kStageBytes;
     static constexpr int STAGES = kStagesFit > 4 ? 4 : kStagesFit;
     static_assert(STAGES >= 2, "shared-memory ring too shallow");
     static constexpr int kSoftmaxWarps = 4 * NQT;
     static constexpr int kProducerWarp = kSoftmaxWarps;
     static constexpr int kMmaWarp = kSoftmaxWarps + 1;
     static constexpr int kThreads = (kSoftmaxWarps + 4) * 32;
-    static constexpr int kTmemNeed = NQT * (BN + D);
+    static constexpr int kTmemNeed = NQT * (BN + D + kPCols);
     static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128 : kTmemNeed <= 256 ? 256 : 512;
     static_assert(kTmemNeed <= 512, "TMEM budget exceeded");
     // Registers: the kernel launches with kLaunchRegs per thread (65536 / 384, rounded
@@ -98,8 +104,10 @@ struct Cfg {
     static constexpr int kOffK = kOffQ + NQT * kQBytes;
     static constexpr int kOffV = kOffK + STAGES * kKBytes;
     static constexpr int kOffP = kOffV + STAGES * kVBytes;
-    static constexpr int kOffB = kOffP + NQT * kPBytes;
-    static constexpr int kOffBar = kOffB + STAGES * kCompBytes;
+    static constexpr int kOffB = kOffP + NQT * kPSmem;
+    // in-kernel Q quantization: per warpgroup 4 warp maxima + D channel means (fp32)
+    static constexpr int kOffScr = kOffB + STAGES * kCompBytes;
+    static constexpr int kOffBar = kOffScr + NQT * (4 + D) * 4;
     // barriers: q, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[NQT],
     //           p_full[NQT], pv_full[NQT], s_free[NQT], drain
     static constexpr int kNumBars = 1 + 4 * STAGES + 4 * NQT + 1;
@@ -346,6 +354,8 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
         const uint32_t tS = tmem_base + lane_off + i * C::BN;
         const uint32_t tO = tmem_base + lane_off + NQT * C::BN + i * D;
+        [[maybe_unused]] const uint32_t tP =
+            tmem_base + lane_off + NQT * (C::BN + D) + i * C::kPCols;
         const int64_t sh = (int64_t)s * L.H + h;
         // this row's Q scale (one per query tile, or one per token)
         float qsc;
@@ -355,7 +365,8 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
             qsc = quantize_q_row<D, FINE, SQ>(
                       p.q16 + L.offset(s, start, h, qrow < len ? qrow : 0), qrow < len,
                       SQ ? p.qsum + sh * D : nullptr, len, smem + C::kOffQ + i * C::kQBytes,
-                      row_in_tile, i, reinterpret_cast<float *>(sP + i * C::kPBytes)) *
+                      row_in_tile, i,
+                      reinterpret_cast<float *>(smem + C::kOffScr + i * (4 + D) * 4)) *
                   p.sc_log2;
             fence_proxy_async_smem();
             __syncwarp();
@@ -594,10 +605,14 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
 #pragma unroll
                         for (int e = 0; e < 8; e++)
                             w[e] = pack_half2(pe[2 * e], pe[2 * e + 1]);
-                        const uint32_t line = prow + (ch / 4) * C::kPSubBytes;
-                        const uint32_t c0 = (ch % 4) * 2;
-                        st_shared_v4(line + ((c0 ^ sw) << 4), w[0], w[1], w[2], w[3]);
-                        st_shared_v4(line + (((c0 + 1) ^ sw) << 4), w[4], w[5], w[6], w[7]);
+                        if constexpr (C::kPTmem) {
+                            tmem_st8(tP + ch * 8, w);   // keys 16ch.. = columns 8ch..
+                        } else {
+                            const uint32_t line = prow + (ch / 4) * C::kPSubBytes;
+                            const uint32_t c0 = (ch % 4) * 2;
+                            st_shared_v4(line + ((c0 ^ sw) << 4), w[0], w[1], w[2], w[3]);
+                            st_shared_v4(line + (((c0 + 1) ^ sw) << 4), w[4], w[5], w[6], w[7]);
+                        }
                     } else {
                         // 16 keys = one 16-byte chunk of the 128-key line, kept for later
 #pragma unroll
@@ -617,14 +632,21 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
             if constexpr (!kStreamP) {
                 if (!(ok = await_pv_and_rescale()))
                     break;
-                const uint32_t prow = pbuf + row_in_tile * 128;
-                const uint32_t sw = row_in_tile & 7;
+                if constexpr (C::kPTmem) {
+                    tmem_st32(tP, pw);   // 4 E4M3 keys per column
+                } else {
+                    const uint32_t prow = pbuf + row_in_tile * 128;
+                    const uint32_t sw = row_in_tile & 7;
 #pragma unroll
-                for (int c = 0; c < kWords / 4; c++)
-                    st_shared_v4(prow + ((c ^ sw) << 4), pw[4 * c], pw[4 * c + 1], pw[4 * c + 2],
-                                 pw[4 * c + 3]);
+                    for (int c = 0; c < kWords / 4; c++)
+                        st_shared_v4(prow + ((c ^ sw) << 4), pw[4 * c], pw[4 * c + 1],
+                                     pw[4 * c + 2], pw[4 * c + 3]);
+                }
             }
-            fence_proxy_async_smem();
+            if constexpr (C::kPTmem)
+                tmem_st_wait();   // P in TMEM before the MMA issuer is told
+            else
+                fence_proxy_async_smem();
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -753,15 +775,23 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < C::BN / C::kPvK; kk++) {
                     const int key0 = kk * C::kPvK;            // first key of this k-step
-                    const uint64_t a = dP0 + ((i * C::kPBytes + (key0 / C::kPSubKeys) * C::kPSubBytes +
+                    [[maybe_unused]] const uint64_t a = dP0 + ((i * C::kPBytes + (key0 / C::kPSubKeys) * C::kPSubBytes +
                                                (key0 % C::kPSubKeys) * (FP8 ? 1 : 2)) >> 4);
                     const uint64_t b =
                         dV0 + ((stg * C::kVBytes + key0 * C::kVRowBytes) >> 4);
                     const uint32_t acc = (kk > 0 || j > 0) ? 1u : 0u;
-                    if constexpr (FP8)
+                    if constexpr (C::kPTmem) {
+                        // P_i in TMEM: 8 columns (16 f16 or 32 E4M3 keys) per k-step
+                        const uint32_t ta = tmem_base + NQT * (C::BN + D) + i * C::kPCols + kk * 8;
+                        if constexpr (FP8)
+                            mma_f8_ts(dO, ta, b, idesc_pv, acc);
+                        else
+                            mma_f16_ts(dO, ta, b, idesc_pv, acc);
+                    } else if constexpr (FP8) {
                         mma_f8_ss(dO, a, b, idesc_pv, acc);
-                    else
+                    } else {
                         mma_f16_ss(dO, a, b, idesc_pv, acc);
+                    }
                 }
                 mma_commit(&pv_full[i]);
             };

@@ -70,10 +70,17 @@ struct Cfg {
     static constexpr int kKBytes = BN * D;                   // int8 K tile
     static constexpr int kVBytes = BN * D * (FP8 ? 1 : 2);   // V tile
     static constexpr int kPBytes = BM * BN * (FP8 ? 1 : 2);      // P tile (A operand of P.V)
-    // d = 64: TMEM has room for P beside S and O, so P goes there and P.V takes its A
-    // operand from TMEM (at d = 64 an M=128 N=64 P.V with both operands in shared memory
-    // needs more shared-memory bandwidth than its math); d = 128: P in shared memory.
-    static constexpr bool kPTmem = D == 64;
+    // P goes to TMEM and P.V takes its A operand from there: P.V then reads only V from
+    // shared memory, and the P tiles leave shared memory. At d = 64 TMEM has room for P
+    // beside S_0, S_1, O_0, O_1. At d = 128 it has not, so the two query tiles' scores
+    // share one S region (kSharedS): S_1(j) is computed once S_0(j) has been read, S_0(j+1)
+    // once S_1(j) has been read.
+#ifndef SAGE_SHARED_S
+#define SAGE_SHARED_S 1
+#endif
+    static constexpr bool kSharedS = D == 128 && NQT == 2 && SAGE_SHARED_S != 0;
+    static constexpr bool kPTmem = D == 64 || kSharedS;
+    static constexpr int kSCols = kSharedS ? BN : NQT * BN;      // TMEM columns of S
     static constexpr int kPSmem = kPTmem ? 0 : kPBytes;          // P bytes in shared memory
     static constexpr int kPCols = kPTmem ? BN * (FP8 ? 1 : 2) / 4 : 0;   // P columns in TMEM
     // smooth Q: each stage also holds the 128 fp32 score compensations of its keys
@@ -87,7 +94,7 @@ struct Cfg {
     static constexpr int kProducerWarp = kSoftmaxWarps;
     static constexpr int kMmaWarp = kSoftmaxWarps + 1;
     static constexpr int kThreads = (kSoftmaxWarps + 4) * 32;
-    static constexpr int kTmemNeed = NQT * (BN + D + kPCols);
+    static constexpr int kTmemNeed = kSCols + NQT * (D + kPCols);
     static constexpr int kTmemCols = kTmemNeed <= 32 ? 32 : kTmemNeed <= 64 ? 64 : kTmemNeed <= 128 ? 128 : kTmemNeed <= 256 ? 256 : 512;
     static_assert(kTmemNeed <= 512, "TMEM budget exceeded");
     // Registers: the kernel launches with kLaunchRegs per thread (65536 / 384, rounded
@@ -352,10 +359,10 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
         const int row_in_tile = quarter * 32 + lane;
         const int qrow = qt * C::BM + row_in_tile;
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-        const uint32_t tS = tmem_base + lane_off + i * C::BN;
-        const uint32_t tO = tmem_base + lane_off + NQT * C::BN + i * D;
+        const uint32_t tS = tmem_base + lane_off + (C::kSharedS ? 0 : i * C::BN);
+        const uint32_t tO = tmem_base + lane_off + C::kSCols + i * D;
         [[maybe_unused]] const uint32_t tP =
-            tmem_base + lane_off + NQT * (C::BN + D) + i * C::kPCols;
+            tmem_base + lane_off + C::kSCols + NQT * D + i * C::kPCols;
         const int64_t sh = (int64_t)s * L.H + h;
         // this row's Q scale (one per query tile, or one per token)
         float qsc;
@@ -422,7 +429,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(&s_free[i]);
+                mbar_arrive(&s_free[C::kSharedS ? 0 : i]);
             // smooth Q: this tile's score compensations arrive with V(j); the stage is not
             // refilled before P.V(j), which needs this tile's P first
             [[maybe_unused]] const float *bt = sB + (j % C::STAGES) * C::BN;
@@ -760,7 +767,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
             const uint64_t dK0 = smem_desc(smem_u32(sK), 16, C::kQkSbo, C::kQkSwizzle);
             const uint64_t dV0 = smem_desc(smem_u32(sV), C::kVBoxBytes, C::kVSbo, C::kVSwizzle);
             auto issue_s = [&](int i, int stg) {
-                const uint32_t dS = tmem_base + i * C::BN;
+                const uint32_t dS = tmem_base + (C::kSharedS ? 0 : i * C::BN);
 #pragma unroll
                 for (int kk = 0; kk < D / 32; kk++) {
                     const uint64_t a = dQ0 + ((i * C::kQBytes + kk * 32) >> 4);
@@ -771,7 +778,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
             };
             const uint64_t dP0 = smem_desc(smem_u32(sP), 16, 1024, 2 /*128B*/);
             auto issue_pv = [&](int i, int stg, int j) {
-                const uint32_t dO = tmem_base + NQT * C::BN + i * D;
+                const uint32_t dO = tmem_base + C::kSCols + i * D;
 #pragma unroll
                 for (int kk = 0; kk < C::BN / C::kPvK; kk++) {
                     const int key0 = kk * C::kPvK;            // first key of this k-step
@@ -782,7 +789,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
                     const uint32_t acc = (kk > 0 || j > 0) ? 1u : 0u;
                     if constexpr (C::kPTmem) {
                         // P_i in TMEM: 8 columns (16 f16 or 32 E4M3 keys) per k-step
-                        const uint32_t ta = tmem_base + NQT * (C::BN + D) + i * C::kPCols + kk * 8;
+                        const uint32_t ta = tmem_base + C::kSCols + NQT * D + i * C::kPCols + kk * 8;
                         if constexpr (FP8)
                             mma_f8_ts(dO, ta, b, idesc_pv, acc);
                         else
@@ -799,45 +806,91 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
                 return mbar_wait(bar, parity, abort, p.status, status_bit(SAGE_ERR_TIMEOUT),
                                  kTimeoutNs);
             };
-            // S_i(j+1) is issued as soon as the softmax warps have read S_i(j) into
-            // registers, so the next scores are computed while the current tile's
-            // exponentials run; PV_i(j) follows once P_i(j) is in shared memory.
-            bool ok = wait(bar_q, 0) && wait(&k_full[0], 0);
-            if (ok) {
-                tc_fence_after();
-                for (int i = 0; i < NQT; i++)
-                    issue_s(i, 0);
-                mma_commit(&k_empty[0]);
-            }
-            for (int j = 0; j < nkv && ok; j++) {
-                const int stg = j % C::STAGES;
-                const uint32_t ph = (j / C::STAGES) & 1;
-                if (j + 1 < nkv) {
+            if constexpr (C::kSharedS) {
+                // One S region for both query tiles. s_free completes once per read of S,
+                // in the order S_0(0), S_1(0), S_0(1), ...: completion 2j + i is query
+                // tile i's read of S_i(j). Per KV tile: S_0(j+1) once S_1(j) has been
+                // read, P.V_0(j), S_1(j+1) once S_0(j+1) has been read, P.V_1(j).
+                bool ok = wait(bar_q, 0) && wait(&k_full[0], 0);
+                if (ok) {
+                    tc_fence_after();
+                    issue_s(0, 0);
+                }
+                if (ok && (ok = wait(&s_free[0], 0))) {
+                    tc_fence_after();
+                    issue_s(1, 0);
+                    mma_commit(&k_empty[0]);
+                }
+                for (int j = 0; j < nkv && ok; j++) {
+                    const int stg = j % C::STAGES;
+                    const uint32_t ph = (j / C::STAGES) & 1;
+                    const bool more = j + 1 < nkv;
                     const int stg1 = (j + 1) % C::STAGES;
                     const uint32_t ph1 = ((j + 1) / C::STAGES) & 1;
-                    if (!(ok = wait(&k_full[stg1], ph1)))
-                        break;
-                    for (int i = 0; i < NQT && ok; i++) {
-                        if (!(ok = wait(&s_free[i], j & 1)))
+                    if (more) {
+                        if (!(ok = wait(&k_full[stg1], ph1) && wait(&s_free[0], 1)))
                             break;
                         tc_fence_after();
-                        issue_s(i, stg1);
+                        issue_s(0, stg1);
+                    }
+                    if (!(ok = wait(&v_full[stg], ph) && wait(&p_full[0], j & 1)))
+                        break;
+                    tc_fence_after();
+                    issue_pv(0, stg, j);
+                    if (more) {
+                        if (!(ok = wait(&s_free[0], 0)))
+                            break;
+                        tc_fence_after();
+                        issue_s(1, stg1);
+                        mma_commit(&k_empty[stg1]);
+                    }
+                    if (!(ok = wait(&p_full[1], j & 1)))
+                        break;
+                    tc_fence_after();
+                    issue_pv(1, stg, j);
+                    mma_commit(&v_empty[stg]);
+                }
+            } else {
+                // S_i(j+1) is issued as soon as the softmax warps have read S_i(j) into
+                // registers, so the next scores are computed while the current tile's
+                // exponentials run; PV_i(j) follows once P_i(j) is in shared memory.
+                bool ok = wait(bar_q, 0) && wait(&k_full[0], 0);
+                if (ok) {
+                    tc_fence_after();
+                    for (int i = 0; i < NQT; i++)
+                        issue_s(i, 0);
+                    mma_commit(&k_empty[0]);
+                }
+                for (int j = 0; j < nkv && ok; j++) {
+                    const int stg = j % C::STAGES;
+                    const uint32_t ph = (j / C::STAGES) & 1;
+                    if (j + 1 < nkv) {
+                        const int stg1 = (j + 1) % C::STAGES;
+                        const uint32_t ph1 = ((j + 1) / C::STAGES) & 1;
+                        if (!(ok = wait(&k_full[stg1], ph1)))
+                            break;
+                        for (int i = 0; i < NQT && ok; i++) {
+                            if (!(ok = wait(&s_free[i], j & 1)))
+                                break;
+                            tc_fence_after();
+                            issue_s(i, stg1);
+                        }
+                        if (!ok)
+                            break;
+                        mma_commit(&k_empty[stg1]);
+                    }
+                    if (!(ok = wait(&v_full[stg], ph)))
+                        break;
+                    for (int i = 0; i < NQT && ok; i++) {
+                        if (!(ok = wait(&p_full[i], j & 1)))
+                            break;
+                        tc_fence_after();
+                        issue_pv(i, stg, j);
                     }
                     if (!ok)
                         break;
-                    mma_commit(&k_empty[stg1]);
+                    mma_commit(&v_empty[stg]);
                 }
-                if (!(ok = wait(&v_full[stg], ph)))
-                    break;
-                for (int i = 0; i < NQT && ok; i++) {
-                    if (!(ok = wait(&p_full[i], j & 1)))
-                        break;
-                    tc_fence_after();
-                    issue_pv(i, stg, j);
-                }
-                if (!ok)
-                    break;
-                mma_commit(&v_empty[stg]);
             }
             // drain: every MMA issued above has completed before TMEM is released
             mma_commit(bar_drain);

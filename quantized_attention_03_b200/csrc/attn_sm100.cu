@@ -15,20 +15,23 @@
 //                     shared-memory ring (mbarrier full/empty pairs)
 //   warp 9            MMA issuer (one thread) and TMEM owner:
 //                       S_i  = Q_i K^T    tcgen05.mma kind::i8, smem x smem -> TMEM s32
-//                       O_i += P_i V      tcgen05.mma kind::f16 | kind::f8f6f4, P and V
-//                                         from shared memory (V MN-major) -> TMEM f32
+//                       O_i += P_i V      tcgen05.mma kind::f16 | kind::f8f6f4, P from
+//                                         TMEM, V from shared memory (MN-major) -> f32
 //   warps 10-11       idle (complete the warpgroup for the register split)
-// TMEM columns: [S_0 | S_1 | O_0 | O_1] = 2*128 + 2*d <= 512.
+// TMEM columns: d = 128: [S | O_0 | O_1 | P_0 | P_1], the two query tiles taking turns
+// in one S region (S_1(j) is computed once S_0(j) has been read, S_0(j+1) once S_1(j)
+// has); d = 64: [S_0 | S_1 | O_0 | O_1 | P_0 | P_1]. P is 64 columns per tile in FP16
+// mode, 32 in FP8 mode; at most 512 in all.
 //
 // Per tile, a softmax thread reads its 128 scores from TMEM into registers once and
-// releases S_i at once, so the tensor core computes S_i(j+1) while the exponentials of
-// tile j run. It takes the integer max of each 64-key half (the two K blocks carry
-// their own scales), converts S to fp32 exactly with a magic-number bias, forms
+// releases S at once, so the tensor core computes the next scores while the
+// exponentials of this tile run. It takes the integer max of each K scale group (each
+// has its own scale), converts S to fp32 exactly with a magic-number bias, forms
 // p = 2^(S*sc - m) with one packed FFMA + ex2, and writes P (f16, or E4M3 of 448 p)
-// into shared memory in the 128-byte-swizzled K-major layout the MMA reads. O lives in
-// TMEM; a row's O is rescaled in place only when its reference max m moves (in FP16
-// mode only when the max grows by more than 2^8, so P <= 256; in FP8 mode on every
-// increase, so 448 P fits E4M3).
+// into TMEM, where the P.V MMA reads it as its A operand. O lives in TMEM; a row's O is
+// rescaled in place only when its reference max m moves (in FP16 mode only when the
+// max grows by more than 2^8, so P <= 256; in FP8 mode on every increase, so 448 P fits
+// E4M3).
 //
 // Every wait is bounded (global timer); a timeout sets the device status word, all
 // roles drain and the CTA releases TMEM and exits. Nothing traps.
@@ -53,14 +56,6 @@ namespace {
 constexpr uint64_t kTimeoutNs = 2000000000ull;   // 2 s: far above any legitimate wait
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLog2_448 = 8.807354922057604f;  // log2(448): E4M3 P = e4m3(448 p)
-#ifndef SAGE_EXP_EMU_EVERY
-#define SAGE_EXP_EMU_EVERY 0
-#endif
-// FP16 mode: one exponential pair in this many is evaluated by exp2_poly2 on the FMA
-// pipe instead of MUFU ex2 (0: none), so the two units share the work. Its 1e-4 relative
-// error is a fraction of an f16 ulp of P; E4M3 P (FP8 mode) always uses MUFU ex2, whose
-// error is far from the E4M3 rounding boundaries.
-constexpr int kEmuEveryF16 = SAGE_EXP_EMU_EVERY;
 
 
 template <int D, bool FP8, int NQT, bool SQ = false>
@@ -559,45 +554,35 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
             const uint32_t pbuf = smem_u32(sP) + i * C::kPBytes;
 
             // p = 2^(S sc - m): S to fp32 exactly through the magic bias
-            // (|S| <= 127^2 d < 2^22), one packed FFMA, ex2; each 16-key chunk is packed to
-            // f16 / E4M3. The P tile in shared memory is K-major with the 128-byte swizzle:
-            // 16-byte chunk c of row r sits at chunk c ^ (r % 8) of the row's 128-byte line.
+            // (|S| <= 127^2 d < 2^22), one packed FFMA, ex2; each 32-key chunk is packed to
+            // f16 / E4M3. P_i goes to TMEM (row = lane, keys along the columns, the layout
+            // of an A operand in TMEM), or, with the S region not shared at d = 128, to a
+            // K-major 128-byte-swizzled tile in shared memory (16-byte chunk c of row r at
+            // chunk c ^ (r % 8) of the row's 128-byte line).
             auto tile_exp = [&](auto masked) {
                 constexpr bool MASKED = decltype(masked)::value;
                 [[maybe_unused]] const uint32_t prow = pbuf + row_in_tile * 128;
                 [[maybe_unused]] const uint32_t sw = row_in_tile & 7;
                 float2 lsum2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
-                for (int ch = 0; ch < 8; ch++) {
-                    [[maybe_unused]] const float sc = sck[ch * kKGroups / 8];
-                    const uint32_t keep =
-                        MASKED ? chunk_mask(col_lim - kcol0 - ch * 16) & 0xffffu : 0xffffu;
-                    float pe[16];
+                for (int cq = 0; cq < 4; cq++) {   // 32 keys: one TMEM load's worth
+                    [[maybe_unused]] const float sc = sck[cq * kKGroups / 4];
+                    const uint32_t keep = MASKED ? chunk_mask(col_lim - kcol0 - cq * 32) : ~0u;
+                    float pe[32];
 #pragma unroll
-                    for (int e = 0; e < 16; e += 2) {
+                    for (int e = 0; e < 32; e += 2) {
                         float2 t;
                         if constexpr (SQ) {   // u = S sc + comp c is already in sreg
-                            t = add2(make_float2(__uint_as_float(sreg[ch / 2][(ch % 2) * 16 + e]),
-                                                 __uint_as_float(sreg[ch / 2][(ch % 2) * 16 + e + 1])),
+                            t = add2(make_float2(__uint_as_float(sreg[cq][e]),
+                                                 __uint_as_float(sreg[cq][e + 1])),
                                      make_float2(-bias, -bias));
                         } else {
-                            float2 x =
-                                make_float2(magic_biased(sreg[ch / 2][(ch % 2) * 16 + e]),
-                                            magic_biased(sreg[ch / 2][(ch % 2) * 16 + e + 1]));
+                            float2 x = make_float2(magic_biased(sreg[cq][e]),
+                                                   magic_biased(sreg[cq][e + 1]));
                             x = add2(x, make_float2(-kMagic, -kMagic));      // exact S
                             t = fma2(x, make_float2(sc, sc), make_float2(-bias, -bias));
                         }
-                        // one pair in kEmuEvery on the FMA pipe, the rest on MUFU
-                        constexpr int kEmuEvery = FP8 ? 0 : kEmuEveryF16;
-                        float2 pv;
-                        if constexpr (kEmuEvery > 0) {
-                            if ((e / 2) % kEmuEvery == kEmuEvery - 1)
-                                pv = exp2_poly2(t);
-                            else
-                                pv = make_float2(ex2_approx(t.x), ex2_approx(t.y));
-                        } else {
-                            pv = make_float2(ex2_approx(t.x), ex2_approx(t.y));
-                        }
+                        float2 pv = make_float2(ex2_approx(t.x), ex2_approx(t.y));
                         if constexpr (MASKED) {
                             pv.x = ((keep >> e) & 1u) ? pv.x : 0.0f;
                             pv.y = ((keep >> (e + 1)) & 1u) ? pv.y : 0.0f;
@@ -607,24 +592,29 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
                         lsum2[(e >> 1) & 1] = add2(lsum2[(e >> 1) & 1], pv);
                     }
                     if constexpr (!FP8) {
-                        // 16 keys = two 16-byte chunks of the 64-key sub-tile ch / 4
-                        uint32_t w[8];
+                        // 32 keys = 16 columns of P_i in TMEM (two f16 per column), or four
+                        // 16-byte chunks of the 64-key sub-tile cq / 2 in shared memory
+                        uint32_t w[16];
 #pragma unroll
-                        for (int e = 0; e < 8; e++)
+                        for (int e = 0; e < 16; e++)
                             w[e] = pack_half2(pe[2 * e], pe[2 * e + 1]);
                         if constexpr (C::kPTmem) {
-                            tmem_st8(tP + ch * 8, w);   // keys 16ch.. = columns 8ch..
+                            tmem_st16(tP + cq * 16, w);
                         } else {
-                            const uint32_t line = prow + (ch / 4) * C::kPSubBytes;
-                            const uint32_t c0 = (ch % 4) * 2;
-                            st_shared_v4(line + ((c0 ^ sw) << 4), w[0], w[1], w[2], w[3]);
-                            st_shared_v4(line + (((c0 + 1) ^ sw) << 4), w[4], w[5], w[6], w[7]);
+                            const uint32_t line = prow + (cq / 2) * C::kPSubBytes;
+#pragma unroll
+                            for (int q4 = 0; q4 < 4; q4++) {
+                                const uint32_t c0 = (cq % 2) * 4 + q4;
+                                st_shared_v4(line + ((c0 ^ sw) << 4), w[4 * q4], w[4 * q4 + 1],
+                                             w[4 * q4 + 2], w[4 * q4 + 3]);
+                            }
                         }
                     } else {
-                        // 16 keys = one 16-byte chunk of the 128-key line, kept for later
+                        // 32 keys = 8 words of four E4M3 codes, kept for the store after
+                        // the wait for the previous P.V
 #pragma unroll
-                        for (int e = 0; e < 4; e++)
-                            pw[ch * 4 + e] =
+                        for (int e = 0; e < 8; e++)
+                            pw[cq * 8 + e] =
                                 static_cast<uint32_t>(pack_e4m3x2(pe[4 * e], pe[4 * e + 1])) |
                                 (static_cast<uint32_t>(pack_e4m3x2(pe[4 * e + 2], pe[4 * e + 3]))
                                  << 16);

@@ -64,25 +64,20 @@ struct Cfg {
     static constexpr int kQBytes = BM * D;                   // int8 Q tile
     static constexpr int kKBytes = BN * D;                   // int8 K tile
     static constexpr int kVBytes = BN * D * (FP8 ? 1 : 2);   // V tile
-    static constexpr int kPBytes = BM * BN * (FP8 ? 1 : 2);      // P tile (A operand of P.V)
-    // P goes to TMEM and P.V takes its A operand from there: P.V then reads only V from
-    // shared memory, and the P tiles leave shared memory. At d = 64 TMEM has room for P
-    // beside S_0, S_1, O_0, O_1. At d = 128 it has not, so the two query tiles' scores
-    // share one S region (kSharedS): S_1(j) is computed once S_0(j) has been read, S_0(j+1)
-    // once S_1(j) has been read.
-#ifndef SAGE_SHARED_S
-#define SAGE_SHARED_S 1
-#endif
-    static constexpr bool kSharedS = D == 128 && NQT == 2 && SAGE_SHARED_S != 0;
-    static constexpr bool kPTmem = D == 64 || kSharedS;
+    // P lives in TMEM and P.V takes its A operand from there, so P.V reads only V from
+    // shared memory and P never enters it (P in shared memory measured 6% slower in FP16
+    // mode and 13% in FP8 mode). At d = 64 TMEM has room for P beside S_0, S_1, O_0,
+    // O_1. At d = 128 it has not, so the two query tiles' scores share one S region
+    // (kSharedS): S_1(j) is computed once S_0(j) has been read, S_0(j+1) once S_1(j) has.
+    static_assert(NQT == 2, "two query tiles per CTA");
+    static constexpr bool kSharedS = D == 128;
     static constexpr int kSCols = kSharedS ? BN : NQT * BN;      // TMEM columns of S
-    static constexpr int kPSmem = kPTmem ? 0 : kPBytes;          // P bytes in shared memory
-    static constexpr int kPCols = kPTmem ? BN * (FP8 ? 1 : 2) / 4 : 0;   // P columns in TMEM
+    static constexpr int kPCols = BN * (FP8 ? 1 : 2) / 4;        // TMEM columns of a P tile
     // smooth Q: each stage also holds the 128 fp32 score compensations of its keys
     static constexpr int kCompBytes = SQ ? BN * 4 : 0;
     static constexpr int kStageBytes = kKBytes + kVBytes + kCompBytes;
     static constexpr int kBudget = 220 * 1024;
-    static constexpr int kStagesFit = (kBudget - NQT * (kQBytes + kPSmem)) / kStageBytes;
+    static constexpr int kStagesFit = (kBudget - NQT * kQBytes) / kStageBytes;
     static constexpr int STAGES = kStagesFit > 4 ? 4 : kStagesFit;
     static_assert(STAGES >= 2, "shared-memory ring too shallow");
     static constexpr int kSoftmaxWarps = 4 * NQT;
@@ -105,8 +100,7 @@ struct Cfg {
     static constexpr int kOffQ = 0;
     static constexpr int kOffK = kOffQ + NQT * kQBytes;
     static constexpr int kOffV = kOffK + STAGES * kKBytes;
-    static constexpr int kOffP = kOffV + STAGES * kVBytes;
-    static constexpr int kOffB = kOffP + NQT * kPSmem;
+    static constexpr int kOffB = kOffV + STAGES * kVBytes;
     // in-kernel Q quantization: per warpgroup 4 warp maxima + D channel means (fp32)
     static constexpr int kOffScr = kOffB + STAGES * kCompBytes;
     static constexpr int kOffBar = kOffScr + NQT * (4 + D) * 4;
@@ -126,8 +120,6 @@ struct Cfg {
     static constexpr int kQkSbo = 8 * D;                                 // 8 rows
     // P in shared memory, K-major 128-byte swizzle: 64-key (FP16) or 128-key (FP8)
     // sub-tiles of 128 rows x 128 bytes
-    static constexpr int kPSubBytes = BM * 128;
-    static constexpr int kPSubKeys = FP8 ? 128 : 64;
     static constexpr int kVSwizzle = kVRowBytes == 128 ? 2 : 4;
     static constexpr int kVSbo = 8 * kVRowBytes;
     // The reference max of a row is refreshed only when the row max exceeds it by more
@@ -302,7 +294,6 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
     uint8_t *sQ = smem + C::kOffQ;
     uint8_t *sK = smem + C::kOffK;
     uint8_t *sV = smem + C::kOffV;
-    uint8_t *sP = smem + C::kOffP;
     [[maybe_unused]] const float *sB = reinterpret_cast<const float *>(smem + C::kOffB);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBar);
     uint64_t *bar_q = bars;
@@ -540,10 +531,10 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
                 }
                 return true;
             };
-            // FP16 mode streams each chunk of P to shared memory as it is produced (the
-            // P.V wait comes first); FP8 mode, whose P tile is half the size, packs the
-            // whole row in registers and stores it after the wait. (Streaming FP8 P, with
-            // one buffer or with two, measured slower.)
+            // FP16 mode streams each 32-key chunk of P into TMEM as it is produced (the
+            // P.V wait comes first); FP8 mode, whose P row is 32 words, packs it in
+            // registers and stores it after the wait. (Streaming FP8 P measured slower,
+            // into shared memory and into TMEM alike.)
             constexpr bool kStreamP = !FP8;
             if constexpr (kStreamP) {
                 if (!(ok = await_pv_and_rescale()))
@@ -551,18 +542,13 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
             }
             constexpr int kWords = FP8 ? C::BN / 4 : 1;
             uint32_t pw[kWords];
-            const uint32_t pbuf = smem_u32(sP) + i * C::kPBytes;
 
             // p = 2^(S sc - m): S to fp32 exactly through the magic bias
             // (|S| <= 127^2 d < 2^22), one packed FFMA, ex2; each 32-key chunk is packed to
-            // f16 / E4M3. P_i goes to TMEM (row = lane, keys along the columns, the layout
-            // of an A operand in TMEM), or, with the S region not shared at d = 128, to a
-            // K-major 128-byte-swizzled tile in shared memory (16-byte chunk c of row r at
-            // chunk c ^ (r % 8) of the row's 128-byte line).
+            // f16 / E4M3. P_i goes to TMEM: row = lane, keys along the columns (two f16 or
+            // four E4M3 per column), the layout of an A operand in TMEM.
             auto tile_exp = [&](auto masked) {
                 constexpr bool MASKED = decltype(masked)::value;
-                [[maybe_unused]] const uint32_t prow = pbuf + row_in_tile * 128;
-                [[maybe_unused]] const uint32_t sw = row_in_tile & 7;
                 float2 lsum2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
 #pragma unroll
                 for (int cq = 0; cq < 4; cq++) {   // 32 keys: one TMEM load's worth
@@ -592,23 +578,12 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
                         lsum2[(e >> 1) & 1] = add2(lsum2[(e >> 1) & 1], pv);
                     }
                     if constexpr (!FP8) {
-                        // 32 keys = 16 columns of P_i in TMEM (two f16 per column), or four
-                        // 16-byte chunks of the 64-key sub-tile cq / 2 in shared memory
+                        // 32 keys = 16 columns of P_i (two f16 per column)
                         uint32_t w[16];
 #pragma unroll
                         for (int e = 0; e < 16; e++)
                             w[e] = pack_half2(pe[2 * e], pe[2 * e + 1]);
-                        if constexpr (C::kPTmem) {
-                            tmem_st16(tP + cq * 16, w);
-                        } else {
-                            const uint32_t line = prow + (cq / 2) * C::kPSubBytes;
-#pragma unroll
-                            for (int q4 = 0; q4 < 4; q4++) {
-                                const uint32_t c0 = (cq % 2) * 4 + q4;
-                                st_shared_v4(line + ((c0 ^ sw) << 4), w[4 * q4], w[4 * q4 + 1],
-                                             w[4 * q4 + 2], w[4 * q4 + 3]);
-                            }
-                        }
+                        tmem_st16(tP + cq * 16, w);
                     } else {
                         // 32 keys = 8 words of four E4M3 codes, kept for the store after
                         // the wait for the previous P.V
@@ -629,21 +604,9 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
             if constexpr (!kStreamP) {
                 if (!(ok = await_pv_and_rescale()))
                     break;
-                if constexpr (C::kPTmem) {
-                    tmem_st32(tP, pw);   // 4 E4M3 keys per column
-                } else {
-                    const uint32_t prow = pbuf + row_in_tile * 128;
-                    const uint32_t sw = row_in_tile & 7;
-#pragma unroll
-                    for (int c = 0; c < kWords / 4; c++)
-                        st_shared_v4(prow + ((c ^ sw) << 4), pw[4 * c], pw[4 * c + 1],
-                                     pw[4 * c + 2], pw[4 * c + 3]);
-                }
+                tmem_st32(tP, pw);   // 4 E4M3 keys per column
             }
-            if constexpr (C::kPTmem)
-                tmem_st_wait();   // P in TMEM before the MMA issuer is told
-            else
-                fence_proxy_async_smem();
+            tmem_st_wait();   // P in TMEM before the MMA issuer is told
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
@@ -766,29 +729,20 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
                 }
                 mma_commit(&s_full[i]);
             };
-            const uint64_t dP0 = smem_desc(smem_u32(sP), 16, 1024, 2 /*128B*/);
             auto issue_pv = [&](int i, int stg, int j) {
                 const uint32_t dO = tmem_base + C::kSCols + i * D;
 #pragma unroll
                 for (int kk = 0; kk < C::BN / C::kPvK; kk++) {
                     const int key0 = kk * C::kPvK;            // first key of this k-step
-                    [[maybe_unused]] const uint64_t a = dP0 + ((i * C::kPBytes + (key0 / C::kPSubKeys) * C::kPSubBytes +
-                                               (key0 % C::kPSubKeys) * (FP8 ? 1 : 2)) >> 4);
                     const uint64_t b =
                         dV0 + ((stg * C::kVBytes + key0 * C::kVRowBytes) >> 4);
                     const uint32_t acc = (kk > 0 || j > 0) ? 1u : 0u;
-                    if constexpr (C::kPTmem) {
-                        // P_i in TMEM: 8 columns (16 f16 or 32 E4M3 keys) per k-step
-                        const uint32_t ta = tmem_base + C::kSCols + NQT * D + i * C::kPCols + kk * 8;
-                        if constexpr (FP8)
-                            mma_f8_ts(dO, ta, b, idesc_pv, acc);
-                        else
-                            mma_f16_ts(dO, ta, b, idesc_pv, acc);
-                    } else if constexpr (FP8) {
-                        mma_f8_ss(dO, a, b, idesc_pv, acc);
-                    } else {
-                        mma_f16_ss(dO, a, b, idesc_pv, acc);
-                    }
+                    // P_i in TMEM: 8 columns (16 f16 or 32 E4M3 keys) per k-step
+                    const uint32_t ta = tmem_base + C::kSCols + NQT * D + i * C::kPCols + kk * 8;
+                    if constexpr (FP8)
+                        mma_f8_ts(dO, ta, b, idesc_pv, acc);
+                    else
+                        mma_f16_ts(dO, ta, b, idesc_pv, acc);
                 }
                 mma_commit(&pv_full[i]);
             };

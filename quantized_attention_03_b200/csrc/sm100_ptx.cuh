@@ -303,32 +303,6 @@ __device__ __forceinline__ void mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint
         : "memory");
 }
 
-// D(tmem) (+)= A(smem) * B(smem), kind::f16.
-__device__ __forceinline__ void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                           uint32_t idesc, uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// D(tmem) (+)= A(smem) * B(smem), kind::f8f6f4.
-__device__ __forceinline__ void mma_f8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                          uint32_t idesc, uint32_t accumulate)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// Make this thread's generic-proxy shared-memory writes visible to the async proxy
-// (tensor-core operand reads) before it signals the MMA issuer.
 // Barrier among the n threads (whole warps) that name barrier `id` (1-15; 0 is
 // __syncthreads'). Every one of them reaches it: it is not a wait on another role.
 __device__ __forceinline__ void named_bar_sync(int id, int n)
@@ -336,6 +310,8 @@ __device__ __forceinline__ void named_bar_sync(int id, int n)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
+// Make this thread's generic-proxy shared-memory writes visible to the async proxy
+// (tensor-core operand reads) before it signals the MMA issuer.
 __device__ __forceinline__ void fence_proxy_async_smem()
 {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -393,29 +369,6 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b)
         : "=f"(d.x), "=f"(d.y)
         : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
     return d;
-}
-
-// 2^t on the FMA and integer pipes, for pairs (relieves the MUFU ex2 unit).
-// t = n + f with n = round(t) (a 1.5 * 2^23 bias rounds t into the low mantissa bits) and
-// f in [-1/2, 1/2]; 2^f is a degree-3 polynomial, minimax in relative error on
-// [-1/2, 1/2] (max 1.0e-4, coefficients fitted for this library by linear programming);
-// 2^n is added to the exponent field. Inputs are clamped to >= -126 (results below
-// 2^-126 are irrelevant here); valid for t < 128.
-__device__ __forceinline__ float2 exp2_poly2(float2 t)
-{
-    constexpr float c1 = 0.693282961845398f, c2 = 0.2422110140323639f, c3 = 0.05500873923301697f;
-    constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
-    t.x = fmaxf(t.x, -126.0f);
-    t.y = fmaxf(t.y, -126.0f);
-    const float2 y = add2(t, make_float2(kRound, kRound));               // round(t) in low bits
-    const float2 n = add2(y, make_float2(-kRound, -kRound));             // round(t), exact
-    const float2 f = fma2(n, make_float2(-1.0f, -1.0f), t);              // t - n, exact
-    float2 q = fma2(f, make_float2(c3, c3), make_float2(c2, c2));
-    q = fma2(q, f, make_float2(c1, c1));
-    q = fma2(q, f, make_float2(1.0f, 1.0f));
-    // the low bits of y hold n (two's complement); 0x4B400000 << 23 vanishes mod 2^32
-    return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(y.x) << 23)),
-                       __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(y.y) << 23)));
 }
 
 // Exact int32 -> fp32 for |x| < 2^22 without the conversion unit: adding 1.5 * 2^23

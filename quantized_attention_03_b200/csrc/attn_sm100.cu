@@ -18,10 +18,9 @@
 //                       O_i += P_i V      tcgen05.mma kind::f16 | kind::f8f6f4, P from
 //                                         TMEM, V from shared memory (MN-major) -> f32
 //   warps 10-11       idle (complete the warpgroup for the register split)
-// TMEM columns: d = 128: [S | O_0 | O_1 | P_0 | P_1], the two query tiles taking turns
-// in one S region (S_1(j) is computed once S_0(j) has been read, S_0(j+1) once S_1(j)
-// has); d = 64: [S_0 | S_1 | O_0 | O_1 | P_0 | P_1]. P is 64 columns per tile in FP16
-// mode, 32 in FP8 mode; at most 512 in all.
+// TMEM columns: [S | O_0 | O_1 | P_0 | P_1] = 128 + 2d + 2 * (64 | 32) <= 512: the two
+// query tiles take turns in one S region (S_1(j) is computed once S_0(j) has been read,
+// S_0(j+1) once S_1(j) has); P is 64 columns per tile in FP16 mode, 32 in FP8 mode.
 //
 // Per tile, a softmax thread reads its 128 scores from TMEM into registers once and
 // releases S at once, so the tensor core computes the next scores while the
@@ -66,12 +65,12 @@ struct Cfg {
     static constexpr int kVBytes = BN * D * (FP8 ? 1 : 2);   // V tile
     // P lives in TMEM and P.V takes its A operand from there, so P.V reads only V from
     // shared memory and P never enters it (P in shared memory measured 6% slower in FP16
-    // mode and 13% in FP8 mode). At d = 64 TMEM has room for P beside S_0, S_1, O_0,
-    // O_1. At d = 128 it has not, so the two query tiles' scores share one S region
-    // (kSharedS): S_1(j) is computed once S_0(j) has been read, S_0(j+1) once S_1(j) has.
+    // mode and 13% in FP8 mode at d = 128). To make room for P at d = 128, the two query
+    // tiles' scores share one S region: S_1(j) is computed once S_0(j) has been read,
+    // S_0(j+1) once S_1(j) has. That also keeps the two softmax warpgroups half a tile
+    // apart, so it is used at d = 64 as well (1-5% faster there than an S region each).
     static_assert(NQT == 2, "two query tiles per CTA");
-    static constexpr bool kSharedS = D == 128;
-    static constexpr int kSCols = kSharedS ? BN : NQT * BN;      // TMEM columns of S
+    static constexpr int kSCols = BN;                             // TMEM columns of S
     static constexpr int kPCols = BN * (FP8 ? 1 : 2) / 4;        // TMEM columns of a P tile
     // smooth Q: each stage also holds the 128 fp32 score compensations of its keys
     static constexpr int kCompBytes = SQ ? BN * 4 : 0;
@@ -105,8 +104,8 @@ struct Cfg {
     static constexpr int kOffScr = kOffB + STAGES * kCompBytes;
     static constexpr int kOffBar = kOffScr + NQT * (4 + D) * 4;
     // barriers: q, k_full[S], k_empty[S], v_full[S], v_empty[S], s_full[NQT],
-    //           p_full[NQT], pv_full[NQT], s_free[NQT], drain
-    static constexpr int kNumBars = 1 + 4 * STAGES + 4 * NQT + 1;
+    //           p_full[NQT], pv_full[NQT], s_free, drain
+    static constexpr int kNumBars = 1 + 4 * STAGES + 3 * NQT + 2;
     static constexpr int kOffMisc = kOffBar + kNumBars * 8;
     static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + alignment slack
     // V operand geometry (MN-major): bytes per token row inside one swizzle chunk
@@ -304,8 +303,8 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
     uint64_t *s_full = v_empty + C::STAGES;
     uint64_t *p_full = s_full + NQT;
     uint64_t *pv_full = p_full + NQT;
-    uint64_t *s_free = pv_full + NQT;      // S_i read into registers: TMEM free for S_i(j+1)
-    uint64_t *bar_drain = s_free + NQT;
+    uint64_t *s_free = pv_full + NQT;      // S read into registers: the S region is free
+    uint64_t *bar_drain = s_free + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffMisc);
     volatile int *abort = reinterpret_cast<volatile int *>(smem + C::kOffMisc + 4);
 
@@ -322,8 +321,8 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
             mbar_init(&s_full[i], 1);
             mbar_init(&p_full[i], 4);
             mbar_init(&pv_full[i], 1);
-            mbar_init(&s_free[i], 4);
         }
+        mbar_init(s_free, 4);   // the 4 warps of the warpgroup that read S
         mbar_init(bar_drain, 1);
         *abort = 0;
         fence_barrier_init();
@@ -345,7 +344,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
         const int row_in_tile = quarter * 32 + lane;
         const int qrow = qt * C::BM + row_in_tile;
         const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-        const uint32_t tS = tmem_base + lane_off + (C::kSharedS ? 0 : i * C::BN);
+        const uint32_t tS = tmem_base + lane_off;   // the shared S region
         const uint32_t tO = tmem_base + lane_off + C::kSCols + i * D;
         [[maybe_unused]] const uint32_t tP =
             tmem_base + lane_off + C::kSCols + NQT * D + i * C::kPCols;
@@ -411,11 +410,11 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
                             drow[kcol0 + e] = static_cast<int>(sreg[e / 32][e % 32]);
                 }
             }
-            // S_i is in registers: the tensor core may write S_i(j+1) now
+            // S_i is in registers: the tensor core may write the other tile's scores now
             tc_fence_before();
             __syncwarp();
             if (lane == 0)
-                mbar_arrive(&s_free[C::kSharedS ? 0 : i]);
+                mbar_arrive(s_free);
             // smooth Q: this tile's score compensations arrive with V(j); the stage is not
             // refilled before P.V(j), which needs this tile's P first
             [[maybe_unused]] const float *bt = sB + (j % C::STAGES) * C::BN;
@@ -720,7 +719,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
             const uint64_t dK0 = smem_desc(smem_u32(sK), 16, C::kQkSbo, C::kQkSwizzle);
             const uint64_t dV0 = smem_desc(smem_u32(sV), C::kVBoxBytes, C::kVSbo, C::kVSwizzle);
             auto issue_s = [&](int i, int stg) {
-                const uint32_t dS = tmem_base + (C::kSharedS ? 0 : i * C::BN);
+                const uint32_t dS = tmem_base;   // the shared S region
 #pragma unroll
                 for (int kk = 0; kk < D / 32; kk++) {
                     const uint64_t a = dQ0 + ((i * C::kQBytes + kk * 32) >> 4);
@@ -750,91 +749,48 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
                 return mbar_wait(bar, parity, abort, p.status, status_bit(SAGE_ERR_TIMEOUT),
                                  kTimeoutNs);
             };
-            if constexpr (C::kSharedS) {
-                // One S region for both query tiles. s_free completes once per read of S,
-                // in the order S_0(0), S_1(0), S_0(1), ...: completion 2j + i is query
-                // tile i's read of S_i(j). Per KV tile: S_0(j+1) once S_1(j) has been
-                // read, P.V_0(j), S_1(j+1) once S_0(j+1) has been read, P.V_1(j).
-                bool ok = wait(bar_q, 0) && wait(&k_full[0], 0);
-                if (ok) {
-                    tc_fence_after();
-                    issue_s(0, 0);
-                }
-                if (ok && (ok = wait(&s_free[0], 0))) {
-                    tc_fence_after();
-                    issue_s(1, 0);
-                    mma_commit(&k_empty[0]);
-                }
-                for (int j = 0; j < nkv && ok; j++) {
-                    const int stg = j % C::STAGES;
-                    const uint32_t ph = (j / C::STAGES) & 1;
-                    const bool more = j + 1 < nkv;
-                    const int stg1 = (j + 1) % C::STAGES;
-                    const uint32_t ph1 = ((j + 1) / C::STAGES) & 1;
-                    if (more) {
-                        if (!(ok = wait(&k_full[stg1], ph1) && wait(&s_free[0], 1)))
-                            break;
-                        tc_fence_after();
-                        issue_s(0, stg1);
-                    }
-                    if (!(ok = wait(&v_full[stg], ph) && wait(&p_full[0], j & 1)))
+            // One S region for both query tiles. s_free completes once per read of S,
+            // in the order S_0(0), S_1(0), S_0(1), ...: completion 2j + i is query
+            // tile i's read of S_i(j). Per KV tile: S_0(j+1) once S_1(j) has been
+            // read, P.V_0(j), S_1(j+1) once S_0(j+1) has been read, P.V_1(j).
+            bool ok = wait(bar_q, 0) && wait(&k_full[0], 0);
+            if (ok) {
+                tc_fence_after();
+                issue_s(0, 0);
+            }
+            if (ok && (ok = wait(s_free, 0))) {
+                tc_fence_after();
+                issue_s(1, 0);
+                mma_commit(&k_empty[0]);
+            }
+            for (int j = 0; j < nkv && ok; j++) {
+                const int stg = j % C::STAGES;
+                const uint32_t ph = (j / C::STAGES) & 1;
+                const bool more = j + 1 < nkv;
+                const int stg1 = (j + 1) % C::STAGES;
+                const uint32_t ph1 = ((j + 1) / C::STAGES) & 1;
+                if (more) {
+                    if (!(ok = wait(&k_full[stg1], ph1) && wait(s_free, 1)))
                         break;
                     tc_fence_after();
-                    issue_pv(0, stg, j);
-                    if (more) {
-                        if (!(ok = wait(&s_free[0], 0)))
-                            break;
-                        tc_fence_after();
-                        issue_s(1, stg1);
-                        mma_commit(&k_empty[stg1]);
-                    }
-                    if (!(ok = wait(&p_full[1], j & 1)))
+                    issue_s(0, stg1);
+                }
+                if (!(ok = wait(&v_full[stg], ph) && wait(&p_full[0], j & 1)))
+                    break;
+                tc_fence_after();
+                issue_pv(0, stg, j);
+                if (more) {
+                    if (!(ok = wait(s_free, 0)))
                         break;
                     tc_fence_after();
-                    issue_pv(1, stg, j);
-                    mma_commit(&v_empty[stg]);
+                    issue_s(1, stg1);
+                    mma_commit(&k_empty[stg1]);
                 }
-            } else {
-                // S_i(j+1) is issued as soon as the softmax warps have read S_i(j) into
-                // registers, so the next scores are computed while the current tile's
-                // exponentials run; PV_i(j) follows once P_i(j) is in shared memory.
-                bool ok = wait(bar_q, 0) && wait(&k_full[0], 0);
-                if (ok) {
-                    tc_fence_after();
-                    for (int i = 0; i < NQT; i++)
-                        issue_s(i, 0);
-                    mma_commit(&k_empty[0]);
-                }
-                for (int j = 0; j < nkv && ok; j++) {
-                    const int stg = j % C::STAGES;
-                    const uint32_t ph = (j / C::STAGES) & 1;
-                    if (j + 1 < nkv) {
-                        const int stg1 = (j + 1) % C::STAGES;
-                        const uint32_t ph1 = ((j + 1) / C::STAGES) & 1;
-                        if (!(ok = wait(&k_full[stg1], ph1)))
-                            break;
-                        for (int i = 0; i < NQT && ok; i++) {
-                            if (!(ok = wait(&s_free[i], j & 1)))
-                                break;
-                            tc_fence_after();
-                            issue_s(i, stg1);
-                        }
-                        if (!ok)
-                            break;
-                        mma_commit(&k_empty[stg1]);
-                    }
-                    if (!(ok = wait(&v_full[stg], ph)))
-                        break;
-                    for (int i = 0; i < NQT && ok; i++) {
-                        if (!(ok = wait(&p_full[i], j & 1)))
-                            break;
-                        tc_fence_after();
-                        issue_pv(i, stg, j);
-                    }
-                    if (!ok)
-                        break;
-                    mma_commit(&v_empty[stg]);
-                }
+                if (!(ok = wait(&p_full[1], j & 1)))
+                    break;
+                tc_fence_after();
+                issue_pv(1, stg, j);
+                mma_commit(&v_empty[stg]);
             }
             // drain: every MMA issued above has completed before TMEM is released
             mma_commit(bar_drain);

@@ -117,8 +117,6 @@ struct Cfg {
     // Q/K operand geometry (K-major, one swizzle atom wide)
     static constexpr int kQkSwizzle = D == 128 ? 2 : 4;                 // 128B / 64B
     static constexpr int kQkSbo = 8 * D;                                 // 8 rows
-    // P in shared memory, K-major 128-byte swizzle: 64-key (FP16) or 128-key (FP8)
-    // sub-tiles of 128 rows x 128 bytes
     static constexpr int kVSwizzle = kVRowBytes == 128 ? 2 : 4;
     static constexpr int kVSbo = 8 * kVRowBytes;
     // The reference max of a row is refreshed only when the row max exceeds it by more
@@ -500,7 +498,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
             else
                 tile_max(std::false_type{});
 
-            // PV_i(j-1) must be complete before the P buffer is rewritten, and O is
+            // PV_i(j-1) must be complete before P_i is rewritten in TMEM, and O is
             // rescaled in TMEM before this tile's P.V lands on it (the whole warp takes
             // part if any of its rows moved its reference max)
             auto await_pv_and_rescale = [&]() -> bool {

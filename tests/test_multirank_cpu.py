@@ -43,3 +43,12 @@ def test_max_over_ranks_and_weak_scaling():
 def test_single_rank_is_identity():
     assert bench.max_over_ranks(7.5) == 7.5
     assert bench.weak_scaling_tops(1e12, 2, 1, 1000.0) == pytest.approx(2.0)
+
+
+def test_end_to_end_bound_from_the_input_copy():
+    """The e2e ceiling: the step's input bytes over the measured copy time."""
+    b = bench._e2e_bound(8.8e12, 1, 805306368, 14.5)
+    assert b["h2d_gbs"] == pytest.approx(805306368 / 14.5e-3 / 1e9)
+    assert b["h2d_bound"] == pytest.approx(8.8e12 / 14.5e-3 / 1e12)
+    assert bench._e2e_bound(8.8e12, 4, 805306368, 14.5)["h2d_bound"] == pytest.approx(
+        4 * 8.8e12 / 14.5e-3 / 1e12)

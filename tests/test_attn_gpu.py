@@ -511,6 +511,24 @@ def test_smooth_q_in_kernel_q_codes_match_the_quantization_pass(N, d, pv, fine):
     assert torch.equal(fused, split)
 
 
+@pytest.mark.parametrize("fine", [False, True])
+def test_smooth_q_with_smooth_v_fp8(fine):
+    """All three smoothings at once (K, V and Q) in FP8 mode, against the oracle."""
+    B, H, Nq, Nk, d = 2, 2, 300, 700, 128
+    w = inputs.Workload("t", 181, B, H, Nk, d, True, 2.0, nq=Nq)
+    q, k, v = inputs.make_dense(w)
+    q = _offset_q(q, d, 182)
+    v = (v.float() + torch.linspace(-3, 3, d)).half()     # V channel offsets
+    out = sage.sageattn(q.cuda(), k.cuda(), v.cuda(), True, True, sage.SAGE_PV_FP8, fine=fine,
+                        smooth_q=True, smooth_v=True)
+    assert sage.sage_get_device_status() == 0
+    lq, lk = oracle.Layout.dense(B, H, Nq, d), oracle.Layout.dense(B, H, Nk, d)
+    ref = oracle.sage_attention(q.numpy(), k.numpy(), v.numpy(), lq, True, True,
+                                sage.SAGE_PV_FP8, kv_layout=lk, fine=fine, smooth_q=True,
+                                smooth_v=True)
+    assert_vs_oracle(_np(out), ref, f"smooth K+V+Q fine={fine}")
+
+
 @pytest.mark.parametrize("pv", ["fp16", "fp8"])
 def test_smooth_q_varlen_against_oracle(pv):
     """Packed sequences with smooth Q (in-kernel Q quantization over the packed rows)."""

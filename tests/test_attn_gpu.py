@@ -178,6 +178,16 @@ def test_sweep_points_sampled(N, d, causal):
                      [(w.B - 1, 7)], w.name)
 
 
+def test_headline_fp8_sampled():
+    """The headline workload (B2 H32 N16384 d128, non-causal) in FP8 P.V mode."""
+    w = inputs.sweep(16384, 128, False)
+    q, k, v = inputs.make_dense(w)
+    got = _run_dense(q, k, v, False, "fp8")
+    lay = oracle.Layout.dense(w.B, w.H, w.N, w.d)
+    _compare_sampled(got, q.numpy(), k.numpy(), v.numpy(), lay, False, "fp8",
+                     [(0, 5), (w.B - 1, w.H - 1)], "headline fp8")
+
+
 def test_varlen_config_sampled():
     w = inputs.varlen()
     q, k, v, cu = inputs.make_varlen(w)

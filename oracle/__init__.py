@@ -19,7 +19,6 @@ from __future__ import annotations
 
 import ctypes
 import math
-import os
 from dataclasses import dataclass
 from typing import Iterable, List, Optional, Sequence, Tuple
 

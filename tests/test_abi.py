@@ -1,7 +1,6 @@
 """The C-ABI library: it loads, exports every symbol include/sage.h declares, and rejects
 bad arguments on the host before anything is enqueued (no GPU needed: these calls return
 before any CUDA call)."""
-import ctypes
 import os
 import re
 

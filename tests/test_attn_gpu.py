@@ -474,6 +474,7 @@ SQ_CASES = [
     # Nq, Nk, d, causal, fine
     (1, 1, 128, False, False), (300, 300, 64, True, False), (513, 513, 128, False, False),
     (200, 900, 128, True, False), (640, 640, 64, True, True), (129, 129, 128, False, True),
+    (300, 100, 64, True, False),   # more queries than keys: the first 200 rows see none
 ]
 
 

@@ -111,6 +111,11 @@ typedef struct CUstream_st *sage_stream_t;
 SAGE_API size_t sage_workspace_size(int nseq, int H, int max_seqlen, int total_tokens, int d,
                            int pv_mode);
 
+/* sage_workspace_size for the dense layout: the scratch sage_attn_fwd_ws needs for
+ * [B,H,N,d] inputs (= sage_workspace_size(B, H, N, B*N, d, pv_mode); 0 for a negative
+ * size, or when B*N overflows int). */
+SAGE_API size_t sage_attn_workspace_size(int B, int H, int N, int d, int pv_mode);
+
 /* sage_workspace_size for queries and keys of different lengths (the *_kv entry points):
  * max_seqlen_q / total_q for Q and the output, max_seqlen_k / total_k for K and V. */
 SAGE_API size_t sage_workspace_size_kv(int nseq, int H, int max_seqlen_q, int max_seqlen_k,

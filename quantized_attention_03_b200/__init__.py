@@ -47,6 +47,7 @@ _Z = ctypes.c_size_t
 _S = ctypes.c_int  # sage_status_t
 SIGNATURES = {
     "sage_workspace_size": (_Z, [_I, _I, _I, _I, _I, _I]),
+    "sage_attn_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
     "sage_workspace_size_kv": (_Z, [_I, _I, _I, _I, _I, _I, _I, _I]),
     "sage_quant_qk_kv": (_S, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _P, _Z,
                               _P]),
@@ -140,6 +141,10 @@ def _call(name: str, *args):
 
 def sage_workspace_size(nseq, H, max_seqlen, total_tokens, d, pv_mode) -> int:
     return int(lib().sage_workspace_size(nseq, H, max_seqlen, total_tokens, d, pv_mode))
+
+
+def sage_attn_workspace_size(B, H, N, d, pv_mode) -> int:
+    return int(lib().sage_attn_workspace_size(B, H, N, d, pv_mode))
 
 
 def sage_workspace_size_kv(nseq, H, max_seqlen_q, max_seqlen_k, total_q, total_k, d,

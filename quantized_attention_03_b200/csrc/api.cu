@@ -3,6 +3,7 @@
 #include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
+#include <climits>
 #include <cmath>
 #include <cstdint>
 #include <cstdio>
@@ -333,6 +334,14 @@ size_t sage_workspace_size(int nseq, int H, int max_seqlen, int total_tokens, in
 {
     return sage_workspace_size_kv(nseq, H, max_seqlen, max_seqlen, total_tokens, total_tokens, d,
                                   pv_mode);
+}
+
+size_t sage_attn_workspace_size(int B, int H, int N, int d, int pv_mode)
+{
+    const int64_t total = (int64_t)B * N;
+    if (B < 0 || N < 0 || total > INT_MAX)
+        return 0;
+    return sage_workspace_size(B, H, N, (int)total, d, pv_mode);
 }
 
 size_t sage_workspace_size_kv(int nseq, int H, int max_seqlen_q, int max_seqlen_k,

@@ -97,6 +97,12 @@ def test_size_limits(lib):
     assert lib.sage_workspace_size_kv(1, 1, 128, 256, 128, 256, 64, 0) > \
         lib.sage_workspace_size_kv(1, 1, 128, 128, 128, 128, 64, 0)
     assert lib.sage_workspace_size_kv(-1, 1, 128, 256, 128, 256, 64, 0) == 0
+    # the dense-layout form is the general one with total_tokens = B*N
+    for pv in (0, 1):
+        assert lib.sage_attn_workspace_size(2, 4, 300, 128, pv) == \
+            lib.sage_workspace_size(2, 4, 300, 600, 128, pv)
+    assert lib.sage_attn_workspace_size(-1, 4, 300, 128, 0) == 0
+    assert lib.sage_attn_workspace_size(65535, 1, 65536, 64, 0) == 0   # B*N past int32
 
 
 def test_empty_inputs_are_noops(lib):

@@ -134,6 +134,77 @@ def weak_scaling_tops(ops_per_step: float, steps: int, world: int, ms: float) ->
     return world * ops_per_step * steps / (ms * 1e-3) / 1e12
 
 
+# A timed region shorter than this runs at the burst clock (the bf16 GEMM's "burst"
+# figure, best of 10 short runs); a longer one settles under the power cap (the
+# "sustained" figure, a GEMM looped for seconds).
+SUSTAINED_AFTER_S = 2.0
+
+
+def tensor_peaks(peaks: dict, fp8_pv: bool, timed_ms: float):
+    """(mixed peak, INT8 peak, bf16 figure used, which) in TOPS. INT8 and FP8 dense run at
+    2x the bf16 rate, FP16 at 1x (nominal 4.5 : 2.25 PFLOP/s); the kernel does half its
+    operations in the INT8 QK^T and half in the P.V, so its bound is the harmonic mix."""
+    sustained = timed_ms * 1e-3 >= SUSTAINED_AFTER_S and "bf16_tflops_sustained" in peaks
+    which = "sustained" if sustained else "burst"
+    bf16 = peaks["bf16_tflops_sustained" if sustained else "bf16_tflops"]
+    int8_peak = 2.0 * bf16
+    pv_peak = 2.0 * bf16 if fp8_pv else bf16
+    return 1.0 / (0.5 / int8_peak + 0.5 / pv_peak), int8_peak, bf16, which
+
+
+def quant_bytes(B: int, H: int, Nq: int, Nk: int, d: int, fp8_pv: bool, smooth_q: bool) -> dict:
+    """Bytes the quantization step must move at the least (each input read once, each
+    output written once) and the bytes the two-pass form actually moves (the column-sum
+    pass reads K, and V in FP8 mode, and Q with smooth Q, a second time)."""
+    nq, nk = B * H * Nq * d, B * H * Nk * d
+    algorithmic = 3 * nq + 3 * nk + 4 * B * H * d            # fp16 in, int8 out; the K mean
+    algorithmic += 4 * B * H * (math.ceil(Nq / 128) + math.ceil(Nk / 64))   # block scales
+    moved = algorithmic + 2 * nk + (2 * nq if smooth_q else 0)
+    if fp8_pv:
+        algorithmic += 3 * nk + 4 * B * H * d                 # V in, E4M3 out; V scales
+        moved += 3 * nk + 4 * B * H * d + 2 * nk              # V statistics pass
+    return {"algorithmic": algorithmic, "moved": moved}
+
+
+def quant_roofline(B, H, Nq, Nk, d, fp8_pv, smooth_q, quant_ms, peaks, src) -> dict:
+    """The quantization step (K column sums + Q/K codes, + V in FP8 mode) against HBM."""
+    b = quant_bytes(B, H, Nq, Nk, d, fp8_pv, smooth_q)
+    gbs = b["algorithmic"] / (quant_ms * 1e-3) / 1e9
+    return {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": gbs / peaks["hbm_gbs"], "ms": quant_ms,
+            "bytes_algorithmic": b["algorithmic"], "bytes_moved_two_pass": b["moved"],
+            "moved_gbs": b["moved"] / (quant_ms * 1e-3) / 1e9,
+            "peak_note": f"STREAM-style copy bandwidth (of {src})"}
+
+
+def free_port() -> int:
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def torchrun_argv(n: int, script: str, argv, port: int):
+    """One process per GPU on this node, rendezvous on the loopback address."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={n}", "--master-addr", "127.0.0.1", "--master-port", str(port),
+            script, *argv]
+
+
+def maybe_relaunch(gpus, script: str, argv) -> None:
+    """--gpus N outside torchrun re-executes `script` under torchrun with N ranks (this
+    process is replaced); inside torchrun, N must match the world size it set."""
+    world = os.environ.get("WORLD_SIZE")
+    if world is None:
+        if gpus is not None and gpus > 1:
+            cmd = torchrun_argv(gpus, script, argv, free_port())
+            sys.stdout.flush()
+            os.execv(cmd[0], cmd)
+        return
+    if gpus is not None and gpus != int(world):
+        raise SystemExit(f"--gpus {gpus} but torchrun started {world} ranks")
+
+
 def _dist():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -510,19 +581,19 @@ def run_ours(args):
     q_bytes = B * H * Nq * d * 2           # Q or O
 
     peaks, src = _peaks()
-    bf16 = peaks["bf16_tflops_sustained"]
-    int8_peak = 2.0 * bf16            # nominal dense ratio int8 : bf16 = 4.5 : 2.25
-    pv_peak = bf16 if pv == sage.SAGE_PV_FP16 else 2.0 * bf16   # fp16 = bf16; fp8 = int8
-    mixed = 1.0 / (0.5 / int8_peak + 0.5 / pv_peak)
+    mixed, int8_peak, bf16, which = tensor_peaks(peaks, pv == sage.SAGE_PV_FP8, total_ms)
+    quant_avg_ms = sum(quant_ms) / len(quant_ms)
     roofline = {
         "bound": "tensor", "achieved": attn_tops, "peak": mixed, "unit": "TOPS",
         "frac": attn_tops / mixed, "traffic": None,
         "kernel": f"attn_kernel<d={d}, PV={W['pv_mode']}, 2 query tiles per CTA>",
         "peak_note": (f"mixed INT8-QK/{W['pv_mode'].upper()}-PV dense peak from the {src} "
-                      f"sustained bf16 GEMM ({bf16:.1f} TF/s): int8 and fp8 = 2x, fp16 = 1x, "
-                      f"half the operations each (of measured)"),
+                      f"{which} bf16 GEMM ({bf16:.1f} TF/s): int8 and fp8 = 2x, fp16 = 1x, "
+                      f"half the operations each (of {src})"),
         "frac_of_int8_peak": attn_tops / int8_peak,
-        "attn_ms": attn_avg_ms, "quant_ms": sum(quant_ms) / len(quant_ms),
+        "attn_ms": attn_avg_ms, "quant_ms": quant_avg_ms,
+        "quant": quant_roofline(B, H, Nq, N, d, pv == sage.SAGE_PV_FP8, sq, quant_avg_ms,
+                                peaks, src),
     }
     traffic_file = os.path.join(ROOT, "profiles", "attn_traffic.json")
     if os.path.exists(traffic_file):
@@ -636,10 +707,7 @@ def run_varlen(args, W, dist, world, rank, local):
     e2e_value = weak_scaling_tops(ops, e2e_steps, world, e2e_ms) if e2e_steps else None
 
     peaks, src = _peaks()
-    bf16 = peaks["bf16_tflops_sustained"]
-    int8_peak = 2.0 * bf16
-    pv_peak = bf16 if pv == sage.SAGE_PV_FP16 else 2.0 * bf16
-    mixed = 1.0 / (0.5 / int8_peak + 0.5 / pv_peak)
+    mixed, int8_peak, bf16, which = tensor_peaks(peaks, pv == sage.SAGE_PV_FP8, total_ms)
     if rank == 0:
         elem_bytes = q.numel() * 2
         line = {
@@ -654,7 +722,9 @@ def run_varlen(args, W, dist, world, rank, local):
             "roofline": {"bound": "tensor", "achieved": value / world, "peak": mixed,
                          "unit": "TOPS", "frac": value / world / mixed, "traffic": None,
                          "kernel": "whole varlen step (quantization + attention in one call; "
-                                   "the attention kernel is not timed separately)"},
+                                   "the attention kernel is not timed separately)",
+                         "peak_note": f"mixed dense peak from the {src} {which} bf16 GEMM "
+                                      f"({bf16:.1f} TF/s) (of {src})"},
             "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": 3 * elem_bytes,
                     "d2h_bytes_per_step": elem_bytes, "steps": e2e_steps,
                     **(_e2e_bound(ops, world, 3 * elem_bytes, copy_ms) if e2e_steps else {}),
@@ -696,7 +766,8 @@ def _kernel_hash():
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--gpus", type=int, default=None,
+                    help="ranks, one per GPU (outside torchrun, bench.py starts them itself)")
     ap.add_argument("--steps", type=int, default=60)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
@@ -720,6 +791,7 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    maybe_relaunch(args.gpus, os.path.abspath(__file__), sys.argv[1:])
     if args.impl == "reference":
         run_reference(args)
     else:

@@ -264,15 +264,26 @@ def attn_fp64(q, k, v, layout: Layout, causal: bool, sm_scale: float, heads=None
     as in attn_quant."""
     kvl = layout if kv_layout is None else kv_layout
     assert kvl.stride == layout.stride and kvl.nseq == layout.nseq
-    q64 = np.ascontiguousarray(q, np.float64)
-    k64 = np.ascontiguousarray(k, np.float64)
-    v64 = np.ascontiguousarray(v, np.float64)
-    out = np.full(q64.shape, np.nan, np.float64)
+    qf, kf, vf = (np.asarray(x).reshape(-1) for x in (q, k, v))
+    out = np.full(np.shape(q), np.nan, np.float64)
+    of = out.reshape(-1)
     r0, r1 = rows if rows is not None else (0, layout.maxlen)
+    st, d = layout.stride, layout.d
     for (s, h, off, n), (_, _, koff, nk) in zip(layout.heads(heads), kvl.heads(heads)):
-        lib().oracle_head_attn_fp64(_ptr(q64, off), _ptr(k64, koff), _ptr(v64, koff), n, nk,
-                                    layout.stride, layout.d, int(causal), float(sm_scale),
-                                    r0, r1, _ptr(out, off))
+        # only the selected head's span of each tensor is widened to fp64 (the whole
+        # tensors can be GBs); rows outside [r0, r1) stay NaN
+        span_q = (n - 1) * st + d if n > 0 else 0
+        span_k = (nk - 1) * st + d if nk > 0 else 0
+        q64 = np.ascontiguousarray(qf[off:off + span_q], np.float64)
+        k64 = np.ascontiguousarray(kf[koff:koff + span_k], np.float64)
+        v64 = np.ascontiguousarray(vf[koff:koff + span_k], np.float64)
+        o64 = np.full(span_q, np.nan, np.float64)
+        if span_q:
+            lib().oracle_head_attn_fp64(_ptr(q64), _ptr(k64) if span_k else 0,
+                                        _ptr(v64) if span_k else 0, n, nk, st, d,
+                                        int(causal), float(sm_scale), r0, r1, _ptr(o64))
+        seg = of[off:off + span_q]
+        np.copyto(seg, o64, where=~np.isnan(o64))
     return out
 
 

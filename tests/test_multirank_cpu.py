@@ -52,3 +52,45 @@ def test_end_to_end_bound_from_the_input_copy():
     assert b["h2d_bound"] == pytest.approx(8.8e12 / 14.5e-3 / 1e12)
     assert bench._e2e_bound(8.8e12, 4, 805306368, 14.5)["h2d_bound"] == pytest.approx(
         4 * 8.8e12 / 14.5e-3 / 1e12)
+
+
+def test_gpus_flag_starts_its_own_ranks():
+    """`--gpus 2` outside torchrun: the script re-executes itself under torchrun with two
+    ranks, and rank 0 reports the max over ranks (rank 1 is the slow one)."""
+    import json
+    import subprocess
+    import sys
+    probe = os.path.join(os.path.dirname(os.path.abspath(__file__)), "replica_probe.py")
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    r = subprocess.run([sys.executable, probe, "--gpus", "2"], capture_output=True, text=True,
+                       timeout=300, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    out = json.loads(lines[0])
+    assert out["world"] == 2
+    assert out["job_ms"] == pytest.approx(15.0)
+    assert out["tops"] == pytest.approx(2 * 8.8e12 * 3 / 15e-3 / 1e12)
+
+
+def test_gpus_flag_must_match_torchrun_world(monkeypatch):
+    monkeypatch.setenv("WORLD_SIZE", "4")
+    with pytest.raises(SystemExit):
+        bench.maybe_relaunch(2, "bench.py", [])
+    bench.maybe_relaunch(4, "bench.py", [])      # consistent: nothing to do
+    bench.maybe_relaunch(None, "bench.py", [])
+
+
+def test_peaks_and_quant_bytes():
+    peaks = {"bf16_tflops": 1660.9, "bf16_tflops_sustained": 1399.1, "hbm_gbs": 6541.8}
+    mixed, int8, bf16, which = bench.tensor_peaks(peaks, False, 140.0)
+    assert which == "burst" and bf16 == 1660.9
+    assert mixed == pytest.approx(1 / (0.5 / 3321.8 + 0.5 / 1660.9))
+    mixed8, _, _, _ = bench.tensor_peaks(peaks, True, 140.0)
+    assert mixed8 == pytest.approx(3321.8)
+    assert bench.tensor_peaks(peaks, False, 5000.0)[3] == "sustained"
+    b = bench.quant_bytes(2, 32, 16384, 16384, 128, False, False)
+    n = 2 * 32 * 16384 * 128
+    assert b["algorithmic"] == 6 * n + 4 * 2 * 32 * 128 + 4 * 2 * 32 * (128 + 256)
+    assert b["moved"] == b["algorithmic"] + 2 * n

@@ -13,7 +13,8 @@
 //                     (TMEM lane t)
 //   warp 8            TMA producer: Q tiles once, then K/V tiles into a STAGES-deep
 //                     shared-memory ring (mbarrier full/empty pairs)
-//   warp 9            MMA issuer (one thread) and TMEM owner:
+//   warp 9            MMA issuer and TMEM owner (the whole warp runs the issue loop,
+//                     one elected lane issues each MMA):
 //                       S_i  = Q_i K^T    tcgen05.mma kind::i8, smem x smem -> TMEM s32
 //                       O_i += P_i V      tcgen05.mma kind::f16 | kind::f8f6f4, P from
 //                                         TMEM, V from shared memory (MN-major) -> f32
@@ -707,7 +708,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
         // ---------------------------------------------------------------- MMA issuer
         if constexpr (NQT == 2)
             asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(C::kRegOther) : "memory");
-        if (lane == 0) {
+        {
             constexpr uint32_t idesc_qk = instr_desc(2 /*s32*/, 1 /*s8*/, 1 /*s8*/, 0, 0, 128, 128);
             constexpr uint32_t idesc_pv = instr_desc(1 /*f32*/, 0 /*f16|e4m3*/, 0, 0,
                                                      1 /*V MN-major*/, 128, D);
@@ -743,9 +744,12 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
                 }
                 mma_commit(&pv_full[i]);
             };
+            // every lane polls (the warp stays converged); the vote makes a timeout seen
+            // by any lane the whole warp's outcome
             auto wait = [&](uint64_t *bar, uint32_t parity) {
-                return mbar_wait(bar, parity, abort, p.status, status_bit(SAGE_ERR_TIMEOUT),
-                                 kTimeoutNs);
+                return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, p.status,
+                                                         status_bit(SAGE_ERR_TIMEOUT),
+                                                         kTimeoutNs));
             };
             // One S region for both query tiles. s_free completes once per read of S,
             // in the order S_0(0), S_1(0), S_0(1), ...: completion 2j + i is query
@@ -792,7 +796,9 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
             }
             // drain: every MMA issued above has completed before TMEM is released
             mma_commit(bar_drain);
-            mbar_wait(bar_drain, 0, nullptr, p.status, status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs);
+            if (lane == 0)
+                mbar_wait(bar_drain, 0, nullptr, p.status, status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs);
+            __syncwarp();
         }
     } else {
         if constexpr (NQT == 2)

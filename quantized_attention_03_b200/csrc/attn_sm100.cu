@@ -595,10 +595,75 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
                 }
                 l = alpha * l + (lsum2[0].x + lsum2[0].y + lsum2[1].x + lsum2[1].y);
             };
-            if (need_mask)
-                tile_exp(std::true_type{});
-            else
-                tile_exp(std::false_type{});
+            auto tile_exp_il = [&](auto masked) {
+                constexpr bool MASKED = decltype(masked)::value;
+                float2 lsum2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
+                // FP8 mode: two 32-key chunks at a time, their element pairs interleaved, so
+                // that two independent dependency chains are in flight (FP8 +1.5%; FP16, which
+                // streams each chunk of P to TMEM as it is produced, measured 1% slower)
+#pragma unroll
+                for (int cp = 0; cp < 4; cp += 2) {
+                    float pe[2][32];
+#pragma unroll
+                    for (int e = 0; e < 32; e += 2) {
+#pragma unroll
+                        for (int h2 = 0; h2 < 2; h2++) {
+                            const int cq = cp + h2;
+                            [[maybe_unused]] const float sc = sck[cq * kKGroups / 4];
+                            float2 t;
+                            if constexpr (SQ) {
+                                t = add2(make_float2(__uint_as_float(sreg[cq][e]),
+                                                     __uint_as_float(sreg[cq][e + 1])),
+                                         make_float2(-bias, -bias));
+                            } else {
+                                float2 x = make_float2(magic_biased(sreg[cq][e]),
+                                                       magic_biased(sreg[cq][e + 1]));
+                                x = add2(x, make_float2(-kMagic, -kMagic));      // exact S
+                                t = fma2(x, make_float2(sc, sc), make_float2(-bias, -bias));
+                            }
+                            float2 pv = make_float2(ex2_approx(t.x), ex2_approx(t.y));
+                            if constexpr (MASKED) {
+                                const uint32_t keep = chunk_mask(col_lim - kcol0 - cq * 32);
+                                pv.x = ((keep >> e) & 1u) ? pv.x : 0.0f;
+                                pv.y = ((keep >> (e + 1)) & 1u) ? pv.y : 0.0f;
+                            }
+                            pe[h2][e] = pv.x;
+                            pe[h2][e + 1] = pv.y;
+                            lsum2[h2] = add2(lsum2[h2], pv);
+                        }
+                    }
+#pragma unroll
+                    for (int h2 = 0; h2 < 2; h2++) {
+                        const int cq = cp + h2;
+                        if constexpr (!FP8) {
+                            uint32_t w[16];
+#pragma unroll
+                            for (int e = 0; e < 16; e++)
+                                w[e] = pack_half2(pe[h2][2 * e], pe[h2][2 * e + 1]);
+                            tmem_st16(tP + cq * 16, w);
+                        } else {
+#pragma unroll
+                            for (int e = 0; e < 8; e++)
+                                pw[cq * 8 + e] =
+                                    static_cast<uint32_t>(pack_e4m3x2(pe[h2][4 * e], pe[h2][4 * e + 1])) |
+                                    (static_cast<uint32_t>(pack_e4m3x2(pe[h2][4 * e + 2], pe[h2][4 * e + 3]))
+                                     << 16);
+                        }
+                    }
+                }
+                l = alpha * l + (lsum2[0].x + lsum2[0].y + lsum2[1].x + lsum2[1].y);
+            };
+            if constexpr (FP8) {
+                if (need_mask)
+                    tile_exp_il(std::true_type{});
+                else
+                    tile_exp_il(std::false_type{});
+            } else {
+                if (need_mask)
+                    tile_exp(std::true_type{});
+                else
+                    tile_exp(std::false_type{});
+            }
             if constexpr (!kStreamP) {
                 if (!(ok = await_pv_and_rescale()))
                     break;

@@ -12,7 +12,8 @@
 //   warps 0-3 / 4-7   softmax warpgroups, one per query tile; thread t owns row t
 //                     (TMEM lane t)
 //   warp 8            TMA producer: Q tiles once, then K/V tiles into a STAGES-deep
-//                     shared-memory ring (mbarrier full/empty pairs)
+//                     shared-memory ring (mbarrier full/empty pairs); the whole warp
+//                     runs the loop, one elected lane issues each copy
 //   warp 9            MMA issuer and TMEM owner (the whole warp runs the issue loop,
 //                     one elected lane issues each MMA):
 //                       S_i  = Q_i K^T    tcgen05.mma kind::i8, smem x smem -> TMEM s32
@@ -715,19 +716,21 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
         }
     } else if (warp == C::kProducerWarp) {
         // ----------------------------------------------------------------- producer
+        // (like the MMA warp, the whole warp runs the loop and one elected lane issues each
+        // copy: 0.5-1.5% faster than a lane-0 loop, and the warp no longer spills)
         if constexpr (NQT == 2)
             asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(C::kRegOther) : "memory");
-        if (lane == 0) {
+        {
             if constexpr (!QIN)
                 tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmV);
             int c1, c2;
             if constexpr (!QIN) {   // (QIN: the softmax warps write the Q tiles)
-                mbar_arrive_expect_tx(bar_q, NQT * C::kQBytes);
+                mbar_arrive_expect_tx_w(bar_q, NQT * C::kQBytes);
                 for (int i = 0; i < NQT; i++) {
                     tma_coords(L, s, start, h, (qt0 + i) * C::BM, c1, c2);
-                    tma_load_3d(sQ + i * C::kQBytes, &tmQ, bar_q, 0, c1, c2);
+                    tma_load_3d_w(sQ + i * C::kQBytes, &tmQ, bar_q, 0, c1, c2);
                 }
             }
             int issued = 0;
@@ -735,38 +738,42 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
                 const int stg = j % C::STAGES;
                 const uint32_t ph = (j / C::STAGES) & 1;
                 tma_coords(LK, s, kstart, h, j * C::BN, c1, c2);
-                if (!mbar_wait(&k_empty[stg], ph ^ 1, abort, p.status,
-                               status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs))
+                if (!__all_sync(0xffffffffu, mbar_wait(&k_empty[stg], ph ^ 1, abort, p.status,
+                                                       status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs)))
                     break;
-                mbar_arrive_expect_tx(&k_full[stg], C::kKBytes);
-                tma_load_3d(sK + stg * C::kKBytes, &tmK, &k_full[stg], 0, c1, c2);
-                if (!mbar_wait(&v_empty[stg], ph ^ 1, abort, p.status,
-                               status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs)) {
+                mbar_arrive_expect_tx_w(&k_full[stg], C::kKBytes);
+                tma_load_3d_w(sK + stg * C::kKBytes, &tmK, &k_full[stg], 0, c1, c2);
+                if (!__all_sync(0xffffffffu, mbar_wait(&v_empty[stg], ph ^ 1, abort, p.status,
+                                                       status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs))) {
                     issued = j + 1;   // the K load of this tile is in flight
                     break;
                 }
-                mbar_arrive_expect_tx(&v_full[stg], C::kVBytes + C::kCompBytes);
+                mbar_arrive_expect_tx_w(&v_full[stg], C::kVBytes + C::kCompBytes);
                 if constexpr (SQ)   // the stride is whole 128-key tiles: 16-byte aligned
-                    bulk_load_g2s(smem + C::kOffB + stg * C::kCompBytes,
-                                  p.q_comp + ((int64_t)s * L.H + h) * p.ncomp + j * C::BN,
-                                  C::kCompBytes, &v_full[stg]);
+                    bulk_load_g2s_w(smem + C::kOffB + stg * C::kCompBytes,
+                                    p.q_comp + ((int64_t)s * L.H + h) * p.ncomp + j * C::BN,
+                                    C::kCompBytes, &v_full[stg]);
 #pragma unroll
                 for (int cb = 0; cb < C::kVChunks; cb++)
-                    tma_load_3d(sV + stg * C::kVBytes + cb * C::kVBoxBytes, &tmV, &v_full[stg],
-                                cb * (C::kVRowBytes / C::kVElem), c1, c2);
+                    tma_load_3d_w(sV + stg * C::kVBytes + cb * C::kVBoxBytes, &tmV,
+                                  &v_full[stg], cb * (C::kVRowBytes / C::kVElem), c1, c2);
                 issued = j + 1;
             }
             // drain: make sure no copy is still landing in shared memory when we leave
-            if constexpr (!QIN)
-                mbar_wait(bar_q, 0, nullptr, p.status, status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs);
-            for (int j = max(0, issued - C::STAGES); j < issued; j++) {
-                const int stg = j % C::STAGES;
-                const uint32_t ph = (j / C::STAGES) & 1;
-                mbar_wait(&k_full[stg], ph, nullptr, p.status, status_bit(SAGE_ERR_TIMEOUT),
-                          kTimeoutNs);
-                mbar_wait(&v_full[stg], ph, nullptr, p.status, status_bit(SAGE_ERR_TIMEOUT),
-                          kTimeoutNs);
+            if (lane == 0) {
+                if constexpr (!QIN)
+                    mbar_wait(bar_q, 0, nullptr, p.status, status_bit(SAGE_ERR_TIMEOUT),
+                              kTimeoutNs);
+                for (int j = max(0, issued - C::STAGES); j < issued; j++) {
+                    const int stg = j % C::STAGES;
+                    const uint32_t ph = (j / C::STAGES) & 1;
+                    mbar_wait(&k_full[stg], ph, nullptr, p.status, status_bit(SAGE_ERR_TIMEOUT),
+                              kTimeoutNs);
+                    mbar_wait(&v_full[stg], ph, nullptr, p.status, status_bit(SAGE_ERR_TIMEOUT),
+                              kTimeoutNs);
+                }
             }
+            __syncwarp();
         }
     } else if (warp == C::kMmaWarp) {
         // ---------------------------------------------------------------- MMA issuer

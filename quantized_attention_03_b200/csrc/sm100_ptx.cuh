@@ -110,6 +110,36 @@ __device__ __forceinline__ void bulk_load_g2s(void *smem_dst, const void *gmem_s
         : "memory");
 }
 
+// Warp-wide forms of the three calls above: the whole warp executes the call and one
+// elected lane issues it (the warp stays converged and its operands warp-uniform).
+__device__ __forceinline__ void tma_load_3d_w(void *smem_dst, const CUtensorMap *m, uint64_t *bar,
+                                              int c0, int c1, int c2)
+{
+    asm volatile(
+        "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+        "@e cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%3, %4, %5}], [%2];\n\t}" ::"r"(smem_u32(smem_dst)),
+        "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+        : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx_w(uint64_t *bar, uint32_t bytes)
+{
+    asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+                 "@e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n\t}" ::"r"(smem_u32(bar)),
+                 "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_load_g2s_w(void *smem_dst, const void *gmem_src, uint32_t bytes,
+                                                uint64_t *bar)
+{
+    asm volatile(
+        "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+        "@e cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n\t}"
+        ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(gmem_src)), "r"(bytes),
+        "r"(smem_u32(bar))
+        : "memory");
+}
+
 // -------------------------------------------------------------------------- TMEM
 
 // Allocate `ncols` (power of two >= 32) tensor-memory columns; the base address is

@@ -176,6 +176,19 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
                                              status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs));
 }
 
+// A softmax warp's arrival on a barrier (after __syncwarp): one elected lane in FP16 mode;
+// lane 0 under a branch in FP8 mode (same-box A/B: FP16 +1.5-2.5%, FP8 -4% with elect).
+template <bool FP8>
+__device__ __forceinline__ void warp_arrive(uint64_t *bar)
+{
+    if constexpr (FP8) {
+        if ((threadIdx.x & 31) == 0)
+            mbar_arrive(bar);
+    } else {
+        mbar_arrive_w(bar);
+    }
+}
+
 // The INT8 codes and the scale of this thread's query row (QIN): Q is read as fp16, made
 // smooth (x - mean(Q), SQ), and quantized with one scale per 128-row tile (the
 // warpgroup's amax) or per row (FINE) exactly as the quantization kernel does it; the
@@ -361,8 +374,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
                   p.sc_log2;
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0)
-                mbar_arrive(bar_q);
+            warp_arrive<FP8>(bar_q);
         } else {
             const int qidx = FINE ? qrow : qt;
             const bool q_valid = (FINE ? qrow : qt * C::BM) < len;
@@ -412,8 +424,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
             // S_i is in registers: the tensor core may write the other tile's scores now
             tc_fence_before();
             __syncwarp();
-            if (lane == 0)
-                mbar_arrive(s_free);
+            warp_arrive<FP8>(s_free);
             // smooth Q: this tile's score compensations arrive with V(j); the stage is not
             // refilled before P.V(j), which needs this tile's P first
             [[maybe_unused]] const float *bt = sB + (j % C::STAGES) * C::BN;
@@ -672,8 +683,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
             tmem_st_wait();   // P in TMEM before the MMA issuer is told
             tc_fence_before();
             __syncwarp();
-            if (lane == 0)
-                mbar_arrive(&p_full[i]);
+            warp_arrive<FP8>(&p_full[i]);
         }
         // epilogue: the last P.V, normalize, round to fp16, store the row
         if (ok && (ok = warp_wait(&pv_full[i], (nkv - 1) & 1, abort, p.status))) {

@@ -140,6 +140,14 @@ __device__ __forceinline__ void bulk_load_g2s_w(void *smem_dst, const void *gmem
         : "memory");
 }
 
+// Arrive once on `bar` from one elected lane of a converged warp.
+__device__ __forceinline__ void mbar_arrive_w(uint64_t *bar)
+{
+    asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+                 "@e mbarrier.arrive.shared::cta.b64 _, [%0];\n\t}" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
 // -------------------------------------------------------------------------- TMEM
 
 // Allocate `ncols` (power of two >= 32) tensor-memory columns; the base address is

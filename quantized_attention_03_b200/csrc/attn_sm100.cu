@@ -540,16 +540,17 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
                 }
                 return true;
             };
-            // FP16 mode streams each 32-key chunk of P into TMEM as it is produced (the
-            // P.V wait comes first); FP8 mode, whose P row is 32 words, packs it in
-            // registers and stores it after the wait. (Streaming FP8 P measured slower,
-            // into shared memory and into TMEM alike.)
-            constexpr bool kStreamP = !FP8;
+            // FP16 mode at d = 128 streams each 32-key chunk of P into TMEM as it is
+            // produced (the P.V wait comes first). FP8 mode (a P row of 32 words) and FP16
+            // mode at d = 64 (64 words) pack the row in registers and store it after the
+            // wait. Same-box A/B: streaming FP8 P is slower (into shared memory and into
+            // TMEM alike); packing FP16 P is 2% faster at d = 64 and 1.5% slower at d = 128.
+            constexpr bool kStreamP = !FP8 && D != 64;
             if constexpr (kStreamP) {
                 if (!(ok = await_pv_and_rescale()))
                     break;
             }
-            constexpr int kWords = FP8 ? C::BN / 4 : 1;
+            constexpr int kWords = FP8 ? C::BN / 4 : (kStreamP ? 1 : C::BN / 2);
             uint32_t pw[kWords];
 
             // p = 2^(S sc - m): S to fp32 exactly through the magic bias
@@ -609,9 +610,10 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
             auto tile_exp_il = [&](auto masked) {
                 constexpr bool MASKED = decltype(masked)::value;
                 float2 lsum2[2] = {make_float2(0.0f, 0.0f), make_float2(0.0f, 0.0f)};
-                // FP8 mode: two 32-key chunks at a time, their element pairs interleaved, so
-                // that two independent dependency chains are in flight (FP8 +1.5%; FP16, which
-                // streams each chunk of P to TMEM as it is produced, measured 1% slower)
+                // Row kept in registers (FP8; FP16 at d = 64): two 32-key chunks at a time,
+                // their element pairs interleaved, so that two independent dependency chains
+                // are in flight (FP8 +1.5%; FP16 at d = 128, which streams each chunk of P to
+                // TMEM as it is produced, measured 1% slower this way)
 #pragma unroll
                 for (int cp = 0; cp < 4; cp += 2) {
                     float pe[2][32];
@@ -647,11 +649,11 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
                     for (int h2 = 0; h2 < 2; h2++) {
                         const int cq = cp + h2;
                         if constexpr (!FP8) {
-                            uint32_t w[16];
+                            // 32 keys = 16 words of two f16, kept for the store after the
+                            // wait for the previous P.V
 #pragma unroll
                             for (int e = 0; e < 16; e++)
-                                w[e] = pack_half2(pe[h2][2 * e], pe[h2][2 * e + 1]);
-                            tmem_st16(tP + cq * 16, w);
+                                pw[cq * 16 + e] = pack_half2(pe[h2][2 * e], pe[h2][2 * e + 1]);
                         } else {
 #pragma unroll
                             for (int e = 0; e < 8; e++)
@@ -664,7 +666,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
                 }
                 l = alpha * l + (lsum2[0].x + lsum2[0].y + lsum2[1].x + lsum2[1].y);
             };
-            if constexpr (FP8) {
+            if constexpr (!kStreamP) {
                 if (need_mask)
                     tile_exp_il(std::true_type{});
                 else
@@ -678,7 +680,10 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
             if constexpr (!kStreamP) {
                 if (!(ok = await_pv_and_rescale()))
                     break;
-                tmem_st32(tP, pw);   // 4 E4M3 keys per column
+                // 4 E4M3 keys or 2 f16 keys per column
+#pragma unroll
+                for (int c = 0; c < kWords; c += 32)
+                    tmem_st32(tP + c, *reinterpret_cast<uint32_t(*)[32]>(pw + c));
             }
             tmem_st_wait();   // P in TMEM before the MMA issuer is told
             tc_fence_before();

@@ -197,12 +197,13 @@ sage_status_t forward(const void *q, const void *k, const void *v, void *out, co
         cs.vsum = nullptr;
     if (!sq)
         cs.qsum = nullptr;
-    if ((e = launch_colstats(kh, vh, cs, LK, status, st)) != cudaSuccess)
+    bool stats = false;
+    if ((e = launch_colstats(kh, vh, cs, LK, status, st, &stats)) != cudaSuccess)
         return cuda_fail(e);
     if (sq) {                                  // Q column sums (the K-sum path over Q)
         ColStats qs;
         qs.ksum = cs.qsum;
-        if ((e = launch_colstats(qh, nullptr, qs, L, status, st)) != cudaSuccess)
+        if ((e = launch_colstats(qh, nullptr, qs, L, status, st, &stats)) != cudaSuccess)
             return cuda_fail(e);
     }
     // With smooth Q the attention kernel quantizes its own Q tiles from fp16 (measured
@@ -211,7 +212,8 @@ sage_status_t forward(const void *q, const void *k, const void *v, void *out, co
     if ((e = launch_quant(qh, kh, vh, cs, q_in_kernel ? nullptr : w.q_i8,
                           q_in_kernel ? nullptr : w.q_scale, w.k_i8, w.k_scale, w.k_mean,
                           fp8 ? w.v8 : nullptr, w.v_scale, sv ? w.v_mean : nullptr, nullptr,
-                          sq ? w.q_comp : nullptr, L, LK, fine, status, st)) != cudaSuccess)
+                          sq ? w.q_comp : nullptr, L, LK, fine, stats, status, st)) !=
+        cudaSuccess)
         return cuda_fail(e);
     AttnArgs a{w.q_i8,     w.q_scale, w.k_i8, w.k_scale, fp8 ? (const void *)w.v8 : v,
                w.v_scale,  sv ? w.v_mean : nullptr,     sq ? w.q_comp : nullptr,
@@ -438,20 +440,22 @@ sage_status_t quant_qk_entry(const void *q, const void *k, const Shape &sh, int8
         cs.qsum = reinterpret_cast<double *>(sums + sum_bytes);
     if (need)
         e = cudaMemsetAsync(sums, 0, need, st);
+    bool stats = false;
     if (e == cudaSuccess && cs.ksum != nullptr) {
         ColStats kc;
         kc.ksum = cs.ksum;
-        e = launch_colstats(static_cast<const __half *>(k), nullptr, kc, Lk, status, st);
+        e = launch_colstats(static_cast<const __half *>(k), nullptr, kc, Lk, status, st, &stats);
     }
     if (e == cudaSuccess && cs.qsum != nullptr) {
         ColStats qc;
         qc.ksum = cs.qsum;
-        e = launch_colstats(static_cast<const __half *>(q), nullptr, qc, Lq, status, st);
+        e = launch_colstats(static_cast<const __half *>(q), nullptr, qc, Lq, status, st, &stats);
     }
     if (e == cudaSuccess)
         e = launch_quant(static_cast<const __half *>(q), static_cast<const __half *>(k), nullptr,
                          cs, q_i8, q_scale, k_i8, k_scale, k_mean, nullptr, nullptr, nullptr,
-                         sq ? q_mean : nullptr, sq ? q_comp : nullptr, Lq, Lk, fine, status, st);
+                         sq ? q_mean : nullptr, sq ? q_comp : nullptr, Lq, Lk, fine, stats,
+                         status, st);
     if (owned)
         cudaFreeAsync(sums, st);
     return e == cudaSuccess ? SAGE_OK : cuda_fail(e);
@@ -496,12 +500,13 @@ sage_status_t quant_v_entry(const void *v, const int32_t *cu_seqlens, int nseq, 
     cs.vsum = smooth ? static_cast<double *>(p) : nullptr;
     cs.vhi = reinterpret_cast<uint32_t *>(static_cast<char *>(p) + n * 8);
     cs.vneg = cs.vhi + n;
+    bool stats = false;
     if ((e = cudaMemsetAsync(p, 0, bytes, st)) == cudaSuccess &&
-        (e = launch_colstats(nullptr, static_cast<const __half *>(v), cs, L, status, st)) ==
-            cudaSuccess)
+        (e = launch_colstats(nullptr, static_cast<const __half *>(v), cs, L, status, st,
+                             &stats)) == cudaSuccess)
         e = launch_quant(nullptr, nullptr, static_cast<const __half *>(v), cs, nullptr, nullptr,
                          nullptr, nullptr, nullptr, v_e4m3, v_scale, smooth ? v_mean : nullptr,
-                         nullptr, nullptr, L, L, false, status, st);
+                         nullptr, nullptr, L, L, false, stats, status, st);
     if (workspace == nullptr)
         cudaFreeAsync(p, st);
     return e == cudaSuccess ? SAGE_OK : cuda_fail(e);

@@ -41,6 +41,9 @@ __global__ void __launch_bounds__(kThreads) colstats_kernel(const __half *__rest
     constexpr int kGroups = D / 8;              // 16-byte column groups per row
     constexpr int kRowsPerPass = kThreads / kGroups;
     constexpr int kWarps = kThreads / 32;
+    // the quantization kernel that follows may start its Q blocks now (they do not read
+    // the sums; its K and V blocks wait for this grid to complete)
+    griddep_launch_dependents();
     const int s = blockIdx.z, h = blockIdx.y;
     int start, len;
     if (!L.range(s, start, len, status))
@@ -511,6 +514,11 @@ __global__ void __launch_bounds__(kThreads, 4) quant_kernel(
                       D * 2, &s_bar);
 
     // ---- per-channel statistics while the copy is in flight
+    // The sums come from the column-statistics kernel just before this one, which this
+    // launch may overlap (programmatic dependent launch): every block that reads them
+    // waits for that grid first. Plain Q blocks need nothing from it.
+    if (kind != 0 || cs.qsum != nullptr)
+        griddep_wait();
     if (kind == 1 && threadIdx.x < D) {
         const int c = threadIdx.x;
         const float mu = cs.ksum ? (float)(cs.ksum[sh * D + c] / (double)len) : 0.0f;
@@ -639,10 +647,12 @@ __global__ void __launch_bounds__(kThreads, 4) quant_kernel(
 }  // namespace
 
 cudaError_t launch_colstats(const __half *k, const __half *v, const ColStats &cs,
-                            const SeqLayout &L, int *status, cudaStream_t st)
+                            const SeqLayout &L, int *status, cudaStream_t st, bool *launched)
 {
     if ((cs.ksum == nullptr && cs.vhi == nullptr) || L.maxlen == 0 || L.H == 0 || L.nseq == 0)
         return cudaSuccess;
+    if (launched != nullptr)
+        *launched = true;
     dim3 grid((L.maxlen + kColChunk - 1) / kColChunk, L.H, L.nseq);
     const bool dk = cs.ksum != nullptr, dv = cs.vhi != nullptr;
     if (L.d == 128) {
@@ -670,7 +680,8 @@ cudaError_t launch_quant(const __half *q, const __half *k, const __half *v, cons
                          int8_t *q_i8, float *q_scale, int8_t *k_i8, float *k_scale,
                          float *k_mean, uint8_t *v_e4m3, float *v_scale, float *v_mean,
                          float *q_mean, float *q_comp, const SeqLayout &Lq,
-                         const SeqLayout &Lk, bool fine, int *status, cudaStream_t st)
+                         const SeqLayout &Lk, bool fine, bool after_colstats, int *status,
+                         cudaStream_t st)
 {
     const bool with_q = q_i8 != nullptr, with_k = k_i8 != nullptr;
     const bool with_v = v_e4m3 != nullptr;
@@ -689,10 +700,21 @@ cudaError_t launch_quant(const __half *q, const __half *k, const __half *v, cons
                             : (qk_only ? quant_kernel<128, false, true> : quant_kernel<128, false, false>))
                     : (fine ? (qk_only ? quant_kernel<64, true, true> : quant_kernel<64, true, false>)
                             : (qk_only ? quant_kernel<64, false, true> : quant_kernel<64, false, false>));
-    kern<<<grid, kThreads, 0, st>>>(q, k, v, cs, q_i8, q_scale, k_i8, k_scale, k_mean, v_e4m3,
-                                    v_scale, v_mean, q_mean, q_comp, Lq, Lk, nqc, nkc,
-                                    status);
-    return cudaGetLastError();
+    // Right after a column-statistics launch, this one may overlap its tail: the blocks
+    // that read the statistics wait for it in the kernel. Anything else launched before
+    // has completed by then, because the statistics kernel itself started after it.
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = after_colstats ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, q, k, v, cs, q_i8, q_scale, k_i8, k_scale, k_mean,
+                              v_e4m3, v_scale, v_mean, q_mean, q_comp, Lq, Lk, nqc, nkc, status);
 }
 
 }  // namespace sage

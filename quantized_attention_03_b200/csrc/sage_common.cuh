@@ -88,8 +88,10 @@ __host__ __device__ inline uint32_t key_bits(uint32_t key)
 }
 
 // Launchers (quant.cu, attn_sm100.cu). All return cudaSuccess or the launch error.
+// launch_colstats sets *launched (when given) if it launched a kernel.
 cudaError_t launch_colstats(const __half *k, const __half *v, const ColStats &cs,
-                            const SeqLayout &L, int *status, cudaStream_t st);
+                            const SeqLayout &L, int *status, cudaStream_t st,
+                            bool *launched = nullptr);
 // Quantizes Q (q_i8 != nullptr), K (k_i8 != nullptr) and/or V (v_e4m3 != nullptr). K is
 // smoothed when cs.ksum is set, V when cs.vsum is set (its mean goes to v_mean if that
 // is set), Q when cs.qsum is set (its mean goes to q_mean if that is set, and the
@@ -97,11 +99,14 @@ cudaError_t launch_colstats(const __half *k, const __half *v, const ColStats &cs
 // lives in layout Lq, K and V in Lk (the same layout for self-attention). fine: one Q
 // scale per token and one K scale per 32 tokens (q_scale [nseq,H,maxq], k_scale
 // [nseq,H,ceil(maxk/32)]); else per-block scales (128 Q tokens, 64 K tokens).
+// after_colstats: the previous launch on the stream is launch_colstats (the one that
+// produced cs); this launch may then overlap its tail.
 cudaError_t launch_quant(const __half *q, const __half *k, const __half *v, const ColStats &cs,
                          int8_t *q_i8, float *q_scale, int8_t *k_i8, float *k_scale,
                          float *k_mean, uint8_t *v_e4m3, float *v_scale, float *v_mean,
                          float *q_mean, float *q_comp, const SeqLayout &Lq,
-                         const SeqLayout &Lk, bool fine, int *status, cudaStream_t st);
+                         const SeqLayout &Lk, bool fine, bool after_colstats, int *status,
+                         cudaStream_t st);
 
 // Row stride of the smooth-Q compensation array: the key count rounded up to whole
 // 128-key tiles, so that every tile's 512 bytes start 16-byte aligned.

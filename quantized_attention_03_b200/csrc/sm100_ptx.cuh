@@ -20,6 +20,20 @@ __device__ __forceinline__ uint64_t globaltimer_ns()
 
 // ------------------------------------------------------------------------ mbarrier
 
+// Programmatic dependent launch. A kernel launched with programmatic stream
+// serialization may start once every CTA of the kernel before it in the stream has
+// called griddep_launch_dependents() (or exited); griddep_wait() then blocks until that
+// kernel has completed and its memory writes are visible. Without the launch attribute
+// both are no-ops.
+__device__ __forceinline__ void griddep_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait()
+{
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count)
 {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count)

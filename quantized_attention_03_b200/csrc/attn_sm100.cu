@@ -55,6 +55,10 @@ namespace sage {
 namespace {
 
 constexpr uint64_t kTimeoutNs = 2000000000ull;   // 2 s: far above any legitimate wait
+// The producer and MMA warps poll with a 1 us suspend hint: they share SM sub-partitions
+// 0 and 1 with softmax warps, whose issue slots a hot poll takes (same-box A/B: FP16
+// +1.5%, FP8 +0.9% at the headline; 100 us measured no better).
+constexpr uint32_t kPollSleepNs = 1000;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLog2_448 = 8.807354922057604f;  // log2(448): E4M3 P = e4m3(448 p)
 
@@ -754,12 +758,14 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
                 const uint32_t ph = (j / C::STAGES) & 1;
                 tma_coords(LK, s, kstart, h, j * C::BN, c1, c2);
                 if (!__all_sync(0xffffffffu, mbar_wait(&k_empty[stg], ph ^ 1, abort, p.status,
-                                                       status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs)))
+                                                       status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs,
+                                                       kPollSleepNs)))
                     break;
                 mbar_arrive_expect_tx_w(&k_full[stg], C::kKBytes);
                 tma_load_3d_w(sK + stg * C::kKBytes, &tmK, &k_full[stg], 0, c1, c2);
                 if (!__all_sync(0xffffffffu, mbar_wait(&v_empty[stg], ph ^ 1, abort, p.status,
-                                                       status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs))) {
+                                                       status_bit(SAGE_ERR_TIMEOUT), kTimeoutNs,
+                                                       kPollSleepNs))) {
                     issued = j + 1;   // the K load of this tile is in flight
                     break;
                 }
@@ -835,7 +841,7 @@ __global__ void __launch_bounds__(Cfg<D, FP8, NQT, SQ>::kThreads, 1)
             auto wait = [&](uint64_t *bar, uint32_t parity) {
                 return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, p.status,
                                                          status_bit(SAGE_ERR_TIMEOUT),
-                                                         kTimeoutNs));
+                                                         kTimeoutNs, kPollSleepNs));
             };
             // One S region for both query tiles. s_free completes once per read of S,
             // in the order S_0(0), S_1(0), S_0(1), ...: completion 2j + i is query

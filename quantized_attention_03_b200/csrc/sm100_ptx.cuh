@@ -70,18 +70,37 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity)
     return ok != 0;
 }
 
+// The same test, but the thread may be suspended for up to `hint_ns` until the phase
+// completes (instead of the hardware's default limit).
+__device__ __forceinline__ bool mbar_try_wait_sleep(uint64_t *bar, uint32_t parity, uint32_t hint_ns)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for the phase of `parity` to complete, giving up after `timeout_ns` of global
 // time or as soon as another thread of the CTA raised `*abort` (if non-null). On a timeout this
 // thread raises `*abort` and ORs `code` into the device status word. Returns false if
 // the wait did not complete.
+// sleep_ns > 0: each poll after the first may suspend the thread for up to sleep_ns
+// until the phase completes, so a warp that only waits takes fewer issue slots from the
+// warps that share its SM sub-partition.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                          int *status, int code, uint64_t timeout_ns)
+                                          int *status, int code, uint64_t timeout_ns,
+                                          uint32_t sleep_ns = 0)
 {
     if (mbar_try_wait(bar, parity))
         return true;
     const uint64_t t0 = globaltimer_ns();
     while (true) {
-        if (mbar_try_wait(bar, parity))
+        if (sleep_ns != 0 ? mbar_try_wait_sleep(bar, parity, sleep_ns) : mbar_try_wait(bar, parity))
             return true;
         if (abort != nullptr && *abort)
             return false;

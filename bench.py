@@ -52,71 +52,109 @@ def _ops(B, H, N, d, causal):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    """SM clocks and throttle reasons sampled while running: through NVML every 10 ms
+    (enough samples inside a timed region of a tenth of a second), else from nvidia-smi
+    every 200 ms. Only reads; it changes no setting of the GPU."""
 
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
     def __init__(self, index: int):
         self.index = index
-        self.lines = []
+        self.samples = []          # (time, sm MHz, max sm MHz, set of active reasons)
         self.proc = None
         self.thread = None
+        self.stop = threading.Event()
+        self.source = None
 
     def __enter__(self):
+        if self._start_nvml():
+            return self
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "200"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread = threading.Thread(target=self._read_smi, daemon=True)
             self.thread.start()
+            self.source = "nvidia-smi"
         except OSError:
             self.proc = None
         return self
 
-    def _read(self):
+    def _start_nvml(self) -> bool:
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            handle = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            max_sm = float(pynvml.nvmlDeviceGetMaxClockInfo(handle, pynvml.NVML_CLOCK_SM))
+            reasons_fn = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            bits = {"hw_slowdown": pynvml.nvmlClocksEventReasonHwSlowdown,
+                    "hw_thermal_slowdown": pynvml.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": pynvml.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": pynvml.nvmlClocksEventReasonSwPowerCap}
+        except Exception:
+            return False
+
+        def poll():
+            while not self.stop.is_set():
+                try:
+                    sm = float(pynvml.nvmlDeviceGetClockInfo(handle, pynvml.NVML_CLOCK_SM))
+                    r = int(reasons_fn(handle))
+                    self.samples.append((time.time(), sm, max_sm,
+                                         {n for n, bit in bits.items() if r & bit}))
+                except Exception:
+                    pass
+                self.stop.wait(0.01)
+
+        self.thread = threading.Thread(target=poll, daemon=True)
+        self.thread.start()
+        self.source = "nvml"
+        return True
+
+    def _read_smi(self):
         for line in self.proc.stdout:
-            self.lines.append((time.time(), line.strip()))
+            parts = [x.strip() for x in line.strip().split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm, mx = float(parts[0]), float(parts[1])
+            except ValueError:
+                continue
+            self.samples.append((time.time(), sm, mx, {n for n, v in zip(self.REASONS, parts[4:8])
+                                                       if v.lower() == "active"}))
 
     def mark(self, name):
         setattr(self, name, time.time())
 
     def __exit__(self, *exc):
+        self.stop.set()
         if self.proc is not None:
             self.proc.terminate()
             try:
                 self.proc.wait(timeout=5)
             except subprocess.TimeoutExpired:
                 self.proc.kill()
+        if self.thread is not None:
             self.thread.join(timeout=2)
 
     def summary(self):
         """Samples taken between mark('t0') and mark('t1') (the timed region)."""
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        t0 = getattr(self, "t0", 0.0) - 0.1
-        t1 = getattr(self, "t1", float("inf")) + 0.1
-        for ts, ln in self.lines:
-            if not (t0 <= ts <= t1):
-                continue
-            parts = [x.strip() for x in ln.split(",")]
-            if len(parts) < 8:
-                continue
-            try:
-                sm.append(float(parts[0]))
-                mx.append(float(parts[1]))
-            except ValueError:
-                continue
-            for n, v in zip(names, parts[4:8]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        busy = [s for s in sm if s > 0.5 * max(sm)] or sm
-        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(mx),
-                "reasons": sorted(reasons), "samples": len(sm)}
+        pad = 0.01 if self.source == "nvml" else 0.1     # half a sampling period or so
+        t0 = getattr(self, "t0", 0.0) - pad
+        t1 = getattr(self, "t1", float("inf")) + pad
+        inside = [x for x in self.samples if t0 <= x[0] <= t1]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "source": self.source}
+        sm = [x[1] for x in inside]
+        reasons = set().union(*(x[3] for x in inside))
+        busy = [v for v in sm if v > 0.5 * max(sm)] or sm
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": max(x[2] for x in inside),
+                "reasons": sorted(reasons), "samples": len(sm), "source": self.source}
 
 
 def max_over_ranks(ms: float, dist=None, device=None) -> float:

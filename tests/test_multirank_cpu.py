@@ -94,3 +94,20 @@ def test_peaks_and_quant_bytes():
     n = 2 * 32 * 16384 * 128
     assert b["algorithmic"] == 6 * n + 4 * 2 * 32 * 128 + 4 * 2 * 32 * (128 + 256)
     assert b["moved"] == b["algorithmic"] + 2 * n
+
+
+def test_clock_summary_keeps_the_timed_region_only():
+    # samples as the NVML poller records them: (time, SM MHz, max SM MHz, active reasons)
+    c = bench.ClockSampler(0)
+    c.source = "nvml"
+    c.samples = [(0.90, 1965.0, 1965.0, {"hw_slowdown"}),      # before the timed region
+                 (1.00, 1965.0, 1965.0, set()),
+                 (1.05, 1800.0, 1965.0, {"sw_power_cap"}),
+                 (1.10, 1850.0, 1965.0, set()),
+                 (1.50, 210.0, 1965.0, set())]                  # after it
+    c.t0, c.t1 = 1.0, 1.1
+    s = c.summary()
+    assert s["samples"] == 3 and s["sm_mhz"] == 1850.0 and s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"] and s["source"] == "nvml"
+    c.t0, c.t1 = 2.0, 2.1                                       # no sample inside
+    assert c.summary()["samples"] == 0 and c.summary()["sm_mhz"] is None

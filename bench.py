@@ -472,6 +472,90 @@ def _e2e_bound(ops, world, h2d_bytes, copy_ms):
             "h2d_bound": weak_scaling_tops(ops, 1, world, copy_ms)}
 
 
+def decode_bytes(B: int, H: int, Nq: int, Nk: int, d: int) -> int:
+    """Algorithmic HBM bytes of one decode step: every K code (1 byte) and V element
+    (2 bytes) read once, the query codes read and the output written (2 bytes), and the
+    scales."""
+    return B * H * (3 * Nk * d + 3 * Nq * d + 4 * (Nq + (Nk + 63) // 64))
+
+
+def run_decode(args, dist, world, rank, local):
+    """A decode step (Nq = 1 new query per sequence against its 32768 quantized cached keys,
+    B=8 H=32 d=128) through sage_attn_decode_quantized; the K codes and V stay resident
+    between steps, as a KV cache does. The line's roofline is HBM bandwidth."""
+    import torch
+    import quantized_attention_03_b200 as sage
+    from quantized_attention_03_b200 import inputs
+
+    w = inputs.decode()
+    B, H, Nq, Nk, d = w.B, w.H, w.nq, w.N, w.d
+    qc, kc, vc = inputs.make_dense(w)
+    q, k, v = qc.cuda(), kc.cuda(), vc.cuda()
+    z = sage.quant_qk(q, k, True)                  # the cache's codes, made once
+    out = torch.empty_like(q)
+    ws = torch.empty(sage.sage_attn_decode_workspace_size(B, H, Nq, Nk, d), dtype=torch.uint8,
+                     device=q.device)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        rc = sage.sage_attn_decode_quantized(z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], v,
+                                             out, B, H, Nq, Nk, d, w.causal, 0.0, 0, ws,
+                                             ws.numel(), stream)
+        if rc != sage.SAGE_OK:
+            raise RuntimeError(sage.status_string(rc))
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.__enter__()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks.mark("t0")
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks.mark("t1")
+    clocks.__exit__(None, None, None)
+    status = sage.sage_get_device_status()
+    if status != sage.SAGE_OK:
+        raise RuntimeError(f"device status {sage.status_string(status)}")
+    ms = max_over_ranks(e0.elapsed_time(e1), dist, q.device)
+    ms_step = ms / args.steps
+    ops = inputs.attention_ops_kv(B, H, Nq, Nk, d, w.causal)
+    nbytes = decode_bytes(B, H, Nq, Nk, d)
+    gbs = nbytes / (ms_step * 1e-3) / 1e9
+    peaks, peak_src = _peaks()
+    line = {
+        "metric": METRIC, "value": weak_scaling_tops(ops, args.steps, world, ms),
+        "unit": "TOPS", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "s8+f16", "data": "synthetic",
+        "config": {"workload": f"decode B={B} H={H} Nq={Nq} Nk={Nk} d={d} causal PV=fp16 "
+                               "(per GPU; K codes and V resident)",
+                   "B": B, "H": H, "Nq": Nq, "Nk": Nk, "d": d, "causal": w.causal,
+                   "pv_mode": "fp16", "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (K codes 1.07 GB, V 2.15 GB); no flush"},
+        "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": gbs / peaks["hbm_gbs"], "traffic": None,
+                     "kernel": "decode_partial + decode_combine (split-K over the keys)",
+                     "bytes_per_step": nbytes,
+                     "peak_note": f"STREAM-style copy bandwidth (of {peak_src})"},
+        "e2e": {"value": None, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0,
+                "note": "a decode step's inputs are the resident K/V cache; not measured"},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks.summary(),
+    }
+    if rank == 0:
+        print(json.dumps(line))
+    if dist is not None:
+        dist.destroy_process_group()
+
+
 def run_ours(args):
     import torch
     import quantized_attention_03_b200 as sage
@@ -485,6 +569,8 @@ def run_ours(args):
         from datetime import timedelta
         dist.init_process_group("nccl", timeout=timedelta(seconds=120))
 
+    if args.workload == "decode":
+        return run_decode(args, dist, world, rank, local)
     W = _workload(args)
     if args.workload == "varlen":
         return run_varlen(args, W, dist, world, rank, local)
@@ -815,7 +901,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="headline",
                     choices=["headline", "llm_prefill", "video_dit", "sweep", "varlen",
-                             "prefill_kv"],
+                             "prefill_kv", "decode"],
                     help="headline: B2 H32 N16384 d128 non-causal FP16 PV (the metric's point)")
     ap.add_argument("--ref-rows", type=int, default=64)
     ap.add_argument("--cpu-seconds", type=float, default=15.0)

@@ -292,6 +292,35 @@ SAGE_API sage_status_t sage_attn_fwd_quantized_kv(const int8_t *q_i8, const floa
                                                   int flags, sage_stream_t stream);
 
 /*
+ * Decode: steps 2-3 for a few queries (1 <= Nq <= SAGE_DECODE_MAX_Q) against many keys,
+ * FP16 P.V mode, dense layout: q_i8 [B,H,Nq,d], k_i8 [B,H,Nk,d] and the scales as
+ * produced by sage_quant_qk_kv (flags 0: q_scale [B,H,1], k_scale [B,H,ceil(Nk/64)];
+ * flags SAGE_QK_FINE: q_scale [B,H,Nq], k_scale [B,H,ceil(Nk/32)]), v fp16 [B,H,Nk,d],
+ * out fp16 [B,H,Nq,d]. The method is that of sage_attn_fwd_quantized_kv
+ * (「SageAttention：低比特量化Attention，实现推理加速」, 技术方案: INT8 scores dequantized by
+ * the two scales, online softmax, FP16 P times FP16 V): causal masks bottom-right (query
+ * i sees keys j <= i + Nk - Nq; the decode step of 「如何将SageAttention量化注意力机制集成到
+ * 你的AI项目中获得2-5倍速度提升」, 语言模型推理加速). The keys are split over many CTAs and
+ * the splits' partial softmax results merged, so P is taken relative to each split's
+ * maximum; the result agrees with the tile walk of sage_attn_fwd_quantized_kv to FP16
+ * rounding. A query that sees no key is written as zeros.
+ *
+ * workspace: device memory of at least sage_attn_decode_workspace_size(B, H, Nq, Nk, d)
+ * bytes, 16-byte aligned, owned by the caller (nothing is allocated). Returns
+ * SAGE_ERR_UNSUPPORTED for Nq > SAGE_DECODE_MAX_Q, SAGE_ERR_WORKSPACE for a short
+ * workspace, SAGE_ERR_INVALID_ARG / SAGE_ERR_MISALIGNED as the other entry points;
+ * every check happens before anything is enqueued. sm_scale <= 0 means 1/sqrt(d).
+ */
+#define SAGE_DECODE_MAX_Q 16
+SAGE_API size_t sage_attn_decode_workspace_size(int B, int H, int Nq, int Nk, int d);
+SAGE_API sage_status_t sage_attn_decode_quantized(const int8_t *q_i8, const float *q_scale,
+                                                  const int8_t *k_i8, const float *k_scale,
+                                                  const void *v, void *out, int B, int H,
+                                                  int Nq, int Nk, int d, int causal,
+                                                  float sm_scale, int flags, void *workspace,
+                                                  size_t ws_bytes, sage_stream_t stream);
+
+/*
  * Debug: the integer score tiles S = q_i8 k_i8^T (int32, [B,H,N,N]) exactly as the
  * attention kernel's tensor-core pass produces them, dumped from tensor memory. Meant
  * for small N (the output is N^2 per head). Uses stream-ordered scratch for a dummy

@@ -38,6 +38,7 @@ SAGE_QK_FINE = 8
 
 Q_BLOCK = 128
 K_BLOCK = 64
+DECODE_MAX_Q = 16   # SAGE_DECODE_MAX_Q: most queries sage_attn_decode_quantized takes
 
 # name -> (restype, argtypes) as declared in include/sage.h
 _P = ctypes.c_void_p
@@ -56,6 +57,9 @@ SIGNATURES = {
                                      _I, _F, _P, _Z, _P]),
     "sage_attn_fwd_quantized_kv": (_S, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I,
                                         _I, _I, _F, _I, _P]),
+    "sage_attn_decode_workspace_size": (_Z, [_I, _I, _I, _I, _I]),
+    "sage_attn_decode_quantized": (_S, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _F, _I,
+                                        _P, _Z, _P]),
     "sage_quant_qk": (_S, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P]),
     "sage_quant_qk_ws": (_S, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _P, _Z, _P]),
     "sage_quant_qk_varlen": (_S, [_P, _P, _P, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P, _I, _P]),
@@ -174,6 +178,17 @@ def sage_attn_varlen_fwd_kv(q, k, v, out, cu_seqlens_q, cu_seqlens_k, nseq, tota
                  _ptr(cu_seqlens_q), _ptr(cu_seqlens_k), nseq, total_q, total_k, max_seqlen_q,
                  max_seqlen_k, H, d, int(causal), int(smooth_k), int(pv_mode), float(sm_scale),
                  _ptr(workspace), int(ws_bytes), _stream(stream))
+
+
+def sage_attn_decode_workspace_size(B, H, Nq, Nk, d) -> int:
+    return int(lib().sage_attn_decode_workspace_size(B, H, Nq, Nk, d))
+
+
+def sage_attn_decode_quantized(q_i8, q_scale, k_i8, k_scale, v, out, B, H, Nq, Nk, d, causal,
+                               sm_scale, flags, workspace, ws_bytes, stream=None):
+    return _call("sage_attn_decode_quantized", _ptr(q_i8), _ptr(q_scale), _ptr(k_i8),
+                 _ptr(k_scale), _ptr(v), _ptr(out), B, H, Nq, Nk, d, int(causal),
+                 float(sm_scale), int(flags), _ptr(workspace), int(ws_bytes), _stream(stream))
 
 
 def sage_attn_fwd_quantized_kv(q_i8, q_scale, k_i8, k_scale, v, v_scale, v_mean, q_comp, out, B,
@@ -471,6 +486,25 @@ def attn_quantized(q_i8, q_scale, k_i8, k_scale, v, v_scale, causal: bool = Fals
         return out
     sage_attn_fwd_quantized(q_i8, q_scale, k_i8, k_scale, v, v_scale, out, B, H, N, d, causal,
                             pv_mode, sm_scale, stream)
+    return out
+
+
+def attn_decode(q_i8, q_scale, k_i8, k_scale, v, causal: bool = False, sm_scale: float = 0.0,
+                out=None, stream=None, fine: bool = False, workspace=None):
+    """Step 3 for a few queries (Nq <= DECODE_MAX_Q) on pre-quantized operands, FP16 P.V,
+    split over the keys (sage_attn_decode_quantized); the workspace is allocated here
+    unless given."""
+    import torch
+    B, H, Nq, d = q_i8.shape
+    Nk = k_i8.shape[2]
+    if out is None:
+        out = torch.empty(q_i8.shape, dtype=torch.float16, device=q_i8.device)
+    need = sage_attn_decode_workspace_size(B, H, Nq, Nk, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q_i8.device)
+    sage_attn_decode_quantized(q_i8, q_scale, k_i8, k_scale, v, out, B, H, Nq, Nk, d, causal,
+                               sm_scale, SAGE_QK_FINE if fine else 0, workspace,
+                               workspace.numel() * workspace.element_size(), stream)
     return out
 
 

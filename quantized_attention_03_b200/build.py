@@ -9,7 +9,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libsage.so")
-SOURCES = ["api.cu", "quant.cu", "attn_sm100.cu", "selftest.cu"]
+SOURCES = ["api.cu", "quant.cu", "attn_sm100.cu", "decode.cu", "selftest.cu"]
 HEADERS = ["sage_common.cuh", "sm100_ptx.cuh", "quant_codes.cuh"]
 
 NVCC_FLAGS = [

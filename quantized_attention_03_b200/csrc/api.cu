@@ -735,6 +735,49 @@ sage_status_t sage_attn_fwd_quantized_kv(const int8_t *q_i8, const float *q_scal
                            reinterpret_cast<cudaStream_t>(stream));
 }
 
+size_t sage_attn_decode_workspace_size(int B, int H, int Nq, int Nk, int d)
+{
+    if (B <= 0 || H <= 0 || Nq <= 0 || Nq > kDecodeMaxQ || Nk <= 0 || (d != 64 && d != 128))
+        return 0;
+    return decode_partial_floats(B, H, Nq, Nk, d) * sizeof(float);
+}
+
+sage_status_t sage_attn_decode_quantized(const int8_t *q_i8, const float *q_scale,
+                                         const int8_t *k_i8, const float *k_scale, const void *v,
+                                         void *out, int B, int H, int Nq, int Nk, int d,
+                                         int causal, float sm_scale, int flags, void *workspace,
+                                         size_t ws_bytes, sage_stream_t stream)
+{
+    sage_status_t r = check_shape(B, H, Nq, d);
+    if (r != SAGE_OK)
+        return r;
+    if (Nk < 0 || (flags & ~SAGE_QK_FINE))
+        return SAGE_ERR_INVALID_ARG;
+    if (Nq > kDecodeMaxQ)
+        return SAGE_ERR_UNSUPPORTED;
+    if (B == 0 || H == 0 || Nq == 0)
+        return SAGE_OK;
+    if (!q_i8 || !q_scale || !out || (Nk > 0 && (!k_i8 || !k_scale || !v || !workspace)))
+        return SAGE_ERR_INVALID_ARG;
+    if (!dense_fits(B, Nq) || !dense_fits(B, Nk))
+        return SAGE_ERR_UNSUPPORTED;
+    if (!aligned16(q_i8) || !aligned16(k_i8) || !aligned16(v) || !aligned16(out) ||
+        !aligned16(workspace))
+        return SAGE_ERR_MISALIGNED;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    if (Nk == 0) {   // no keys: every query sees none
+        cudaError_t e = cudaMemsetAsync(out, 0, (size_t)B * H * Nq * d * 2, st);
+        return e == cudaSuccess ? SAGE_OK : cuda_fail(e);
+    }
+    if (ws_bytes < sage_attn_decode_workspace_size(B, H, Nq, Nk, d))
+        return SAGE_ERR_WORKSPACE;
+    DecodeArgs a{q_i8, q_scale, k_i8, k_scale, static_cast<const __half *>(v),
+                 static_cast<__half *>(out), static_cast<float *>(workspace), B, H, Nq, Nk, d,
+                 causal ? 1 : 0, (flags & SAGE_QK_FINE) ? 1 : 0, resolve_scale(sm_scale, d)};
+    cudaError_t e = launch_decode(a, st);
+    return e == cudaSuccess ? SAGE_OK : cuda_fail(e);
+}
+
 sage_status_t sage_attn_fwd_quantized_smooth_v(const int8_t *q_i8, const float *q_scale,
                                                const int8_t *k_i8, const float *k_scale,
                                                const uint8_t *v_e4m3, const float *v_scale,

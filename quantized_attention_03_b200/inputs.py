@@ -71,6 +71,13 @@ def prefill_kv() -> Workload:
                     128, True, 1.0, nq=2048)
 
 
+def decode() -> Workload:
+    """One decode step: one new query per sequence attending to 32768 cached keys, B=8 H=32
+    d=128 (causal, which for the last position is every key)."""
+    return Workload("LLM decode B8 H32 Nq1 Nk32768 d128 causal", 1006, 8, 32, 32768, 128, True,
+                    1.0, nq=1)
+
+
 def varlen() -> Workload:
     return Workload("packed varlen causal 8 seqs H32 d128", 1004, 0, 32, 0, 128, True, 2.0,
                     pv_modes=("fp8",), nseq=8)

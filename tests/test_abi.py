@@ -138,3 +138,38 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(sage, "_lib", None)
     with pytest.raises(RuntimeError, match="no fallback"):
         sage.lib()
+
+
+def _dec(lib, q=FAKE, o=FAKE, ws=FAKE, ws_bytes=1 << 30, B=1, H=2, Nq=1, Nk=700, d=128,
+         flags=0):
+    return lib.sage_attn_decode_quantized(q, FAKE, FAKE, FAKE, FAKE, o, B, H, Nq, Nk, d, 1, 0.0,
+                                          flags, ws, ws_bytes, None)
+
+
+def test_decode_host_validation(lib):
+    # a few queries only, FP16 P.V, d 64 or 128; every check before anything is enqueued
+    assert _dec(lib, Nq=17) == sage.SAGE_ERR_UNSUPPORTED
+    assert _dec(lib, d=96) == sage.SAGE_ERR_UNSUPPORTED
+    assert _dec(lib, Nk=-1) == sage.SAGE_ERR_INVALID_ARG
+    assert _dec(lib, flags=sage.SAGE_SMOOTH_Q) == sage.SAGE_ERR_INVALID_ARG
+    assert _dec(lib, q=0) == sage.SAGE_ERR_INVALID_ARG
+    assert _dec(lib, ws=0) == sage.SAGE_ERR_INVALID_ARG
+    assert _dec(lib, o=MIS) == sage.SAGE_ERR_MISALIGNED
+    assert _dec(lib, ws=MIS) == sage.SAGE_ERR_MISALIGNED
+    need = lib.sage_attn_decode_workspace_size(1, 2, 1, 700, 128)
+    assert _dec(lib, ws_bytes=need - 1) == sage.SAGE_ERR_WORKSPACE
+    assert _dec(lib, B=0) == sage.SAGE_OK and _dec(lib, Nq=0) == sage.SAGE_OK
+
+
+def test_decode_workspace_size(lib):
+    # per (sequence, head, split, query): the split's max, its sum and d output sums (fp32);
+    # whole 128-key splits, so the size is a multiple of (2 + d) * 4 * B * H * Nq
+    for B, H, Nq, Nk, d in ((1, 2, 1, 700, 128), (8, 32, 1, 32768, 128), (2, 3, 16, 4100, 64)):
+        n = lib.sage_attn_decode_workspace_size(B, H, Nq, Nk, d)
+        unit = (2 + d) * 4 * B * H * Nq
+        assert n > 0 and n % unit == 0
+        nsplit = n // unit
+        assert 1 <= nsplit <= -(-Nk // 128)
+    assert lib.sage_attn_decode_workspace_size(1, 1, 17, 100, 64) == 0
+    assert lib.sage_attn_decode_workspace_size(1, 1, 1, 0, 64) == 0
+    assert lib.sage_attn_decode_workspace_size(1, 1, 1, 100, 96) == 0

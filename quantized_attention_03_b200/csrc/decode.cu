@@ -16,7 +16,10 @@
 // result carries the same rounding error as the tile walk's.
 //
 // The pass is bound by HBM: every K code (1 byte) and every V element (2 bytes) is read
-// once; the arithmetic (Nq dp4a per 4 key bytes) is small.
+// once, and at one query the arithmetic (Nq dp4a per 4 key bytes, Nq FMA pairs per V
+// pair) is small: B8 H32 Nk32768 d128 reads at the copy bandwidth, 1.8x the tensor-core
+// kernel. The arithmetic grows with Nq; from about 8 queries the tensor-core kernel,
+// whose tile holds them all, is the faster one.
 #include <cuda_fp16.h>
 #include <math.h>
 

@@ -10,7 +10,7 @@ CSRC = os.path.join(HERE, "csrc")
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libsage.so")
 SOURCES = ["api.cu", "quant.cu", "attn_sm100.cu", "decode.cu", "selftest.cu"]
-HEADERS = ["sage_common.cuh", "sm100_ptx.cuh", "quant_codes.cuh"]
+HEADERS = ["sage_common.cuh", "sm100_ptx.cuh", "quant_codes.cuh", "decode.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -10,6 +10,7 @@
 #include <cstdlib>
 #include <mutex>
 
+#include "decode.cuh"
 #include "sage_common.cuh"
 
 namespace sage {

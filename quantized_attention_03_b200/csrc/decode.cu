@@ -25,6 +25,7 @@
 
 #include <algorithm>
 
+#include "decode.cuh"
 #include "sage_common.cuh"
 #include "sm100_ptx.cuh"
 

@@ -650,3 +650,67 @@ def test_int8_scores_beat_e4m3_scores():
     err_i8 = np.abs(s_i8 - exact).mean()
     err_f8 = np.abs(s_f8 - exact).mean()
     assert err_i8 < 0.6 * err_f8
+
+
+# ------------------------------------------------------------ split-K merge (R21, decode)
+
+
+def _split_merge(z, v, nq, nk, d, causal, sm, split, round_p=True, weighted=True):
+    """The decode path's arithmetic in fp64 from the oracle's codes (one head): keys in
+    splits, P = f16(2^(t - m_split)), O_s = P V, l_s = sum p, merged with the weights
+    2^(m_s - M). round_p=False keeps p unrounded; weighted=False drops the merge weights
+    (a planted mistake)."""
+    qi = z["q_i8"][0, 0].astype(np.int64)
+    ki = z["k_i8"][0, 0].astype(np.int64)
+    qs = np.float64(z["q_scale"][0, 0, 0])
+    ks = z["k_scale"][0, 0].astype(np.float64)
+    c = sm * math.log2(math.e)
+    t = (qi @ ki.T).astype(np.float64) * qs * np.repeat(ks, 64)[:nk][None, :] * c
+    if causal:
+        vis = np.arange(nk)[None, :] <= np.arange(nq)[:, None] + nk - nq
+        t = np.where(vis, t, -np.inf)
+    vv = v[0, 0].astype(np.float64)
+    out = np.zeros((nq, d))
+    for i in range(nq):
+        parts = []
+        for k0 in range(0, nk, split):
+            ts = t[i, k0:k0 + split]
+            m = ts.max()
+            if m == -np.inf:
+                continue
+            p = np.exp2(ts - m)
+            pr = p.astype(np.float16).astype(np.float64) if round_p else p
+            parts.append((m, p.sum(), pr @ vv[k0:k0 + split]))
+        if not parts:
+            continue
+        M = max(m for m, _, _ in parts)
+        w = [2.0 ** (m - M) if weighted else 1.0 for m, _, _ in parts]
+        l = sum(wi * ls for wi, (_, ls, _) in zip(w, parts))
+        out[i] = sum(wi * os_ for wi, (_, _, os_) in zip(w, parts)) / l
+    return out
+
+
+@pytest.mark.parametrize("nq,causal", [(1, True), (4, True), (3, False)])
+def test_split_merge_matches_the_tile_walk(nq, causal):
+    # R21: splitting the keys and merging (m_s, l_s, O_s) is the online softmax regrouped;
+    # with p unrounded it equals one softmax exactly (fp64), and with P = f16(p) relative
+    # to the split's maximum it stays within the bounds the GPU is held to against the
+    # oracle's tile walk. Dropping the merge weights fails those bounds.
+    nk, d = 1100, 64
+    q = _rand16((1, 1, nq, d), 31 + nq)
+    k = _rand16((1, 1, nk, d), 41 + nq)
+    k = (k.astype(np.float32) + _rand16((1, 1, 1, d), 51, 2.0).astype(np.float32)).astype(np.float16)
+    v = _rand16((1, 1, nk, d), 61 + nq)
+    lq, lk = Layout.dense(1, 1, nq, d), Layout.dense(1, 1, nk, d)
+    sm = 1.0 / math.sqrt(d)
+    z = oracle.quant_qk(q, k, lq, True, kv_layout=lk)
+    walk = oracle.attn_quant(z["q_i8"], z["q_scale"], z["k_i8"], z["k_scale"], v, None, lq,
+                             causal, PV_FP16, sm, kv_layout=lk)[0, 0].astype(np.float64)
+    one = _split_merge(z, v, nq, nk, d, causal, sm, split=nk, round_p=False)
+    for split in (128, 256, 1024):
+        exact = _split_merge(z, v, nq, nk, d, causal, sm, split, round_p=False)
+        assert np.abs(exact - one).max() < 1e-12
+        got = _split_merge(z, v, nq, nk, d, causal, sm, split)
+        assert _cos(got, walk) >= 0.9999 and np.abs(got - walk).max() <= 1e-2, split
+        bad = _split_merge(z, v, nq, nk, d, causal, sm, split, weighted=False)
+        assert np.abs(bad - walk).max() > 1e-2, split

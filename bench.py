@@ -368,6 +368,8 @@ def _workload(args):
         w = inputs.varlen()
     elif args.workload == "prefill_kv":
         w = inputs.prefill_kv()
+    elif args.workload == "decode":
+        w = inputs.decode()
     elif args.workload == "sweep":
         n = args.N or 16384
         w = inputs.sweep(n, args.d or 128, args.causal)
